@@ -1,0 +1,221 @@
+"""Seeded synthetic workloads for the dynamic short convolution hot path.
+
+This module only draws numbers and describes shapes; it holds none of the
+method's arithmetic.  It is the single source of inputs shared by the fp64
+oracle, the CUDA path, the tests and the benchmark.
+
+Generator definition (one counter-based stream per tensor):
+
+* ``splitmix64`` (Steele, Lea & Flood, "Fast splittable pseudorandom number
+  generators", OOPSLA 2014) applied to the counter ``key + (i + 1) * GOLDEN``
+  gives 64 random bits for draw ``i``.  ``key`` is derived from the workload
+  seed and a per-tensor tag.
+* Two uniforms ``u1 = (a >> 11 + 1) / 2**53`` (in (0, 1]) and
+  ``u2 = (b >> 11) / 2**53`` feed the Box-Muller transform
+  ``sqrt(-2 ln u1) * cos(2 pi u2)``, giving N(0, 1) in fp64.
+* The draw is scaled by the tensor's standard deviation, then rounded once to
+  the storage dtype: fp64 -> fp32 (round to nearest even) -> bf16 (round to
+  nearest even) for bf16 workloads, fp64 -> fp32 for fp32 workloads.  The
+  oracle receives exactly these rounded values, widened back to fp64.
+
+Workload shapes follow the five configurations of the dynamic short
+convolution benchmark (dynamic filters on Q/K/V at 150M scale, head-wise on
+2B-scale GQA, after every linear of a 2B block, packed variable-length
+documents), see "Dynamic Short Convolutions Improve Transformers", gist.science
+technical summary, sections "Placement" and "Language Modeling".
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+
+GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+LOWRANK = "lowrank"
+HEADWISE = "headwise"
+
+
+def _mix(x: np.ndarray) -> np.ndarray:
+    """splitmix64 output function on a uint64 array (wrapping arithmetic)."""
+    with np.errstate(over="ignore"):
+        z = x.copy()
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+        return z ^ (z >> np.uint64(31))
+
+
+def _key(seed: int, tag: str) -> np.uint64:
+    """Stream key for one tensor: splitmix64 of the seed folded with the tag bytes."""
+    k = np.array([seed & 0xFFFFFFFFFFFFFFFF], dtype=np.uint64)
+    for ch in tag.encode():
+        with np.errstate(over="ignore"):
+            k = _mix(k ^ np.uint64(ch)) + GOLDEN
+    return k[0]
+
+
+def raw_bits(seed: int, tag: str, count: int, offset: int = 0) -> np.ndarray:
+    """``count`` 64-bit draws of the stream (seed, tag), starting at draw ``offset``."""
+    i = np.arange(offset, offset + count, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        ctr = _key(seed, tag) + (i + np.uint64(1)) * GOLDEN
+    return _mix(ctr)
+
+
+def uniform(seed: int, tag: str, count: int) -> np.ndarray:
+    """Uniform fp64 draws in (0, 1]."""
+    b = raw_bits(seed, tag, count)
+    return ((b >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+
+
+def normal(seed: int, tag: str, count: int, std: float = 1.0) -> np.ndarray:
+    """N(0, std^2) fp64 draws by Box-Muller on two interleaved uniform streams."""
+    b = raw_bits(seed, tag, 2 * count)
+    u1 = ((b[0::2] >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+    u2 = (b[1::2] >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    return std * np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+
+
+def round_to_storage(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round fp64 values to the storage dtype and return them widened to fp64."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.float32)
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16).to(torch.float32)
+    elif dtype != "f32":
+        raise ValueError(f"unknown storage dtype {dtype!r}")
+    return t.to(torch.float64).numpy()
+
+
+def geometric_doc_lengths(seed: int, total: int, mean: float, lo: int, hi: int) -> List[int]:
+    """Packed-document lengths: Geometric(p = 1/mean) on {1, 2, ...} by inverse CDF,
+    clipped to [lo, hi], appended while the running sum is below ``total``; the
+    last document takes the remainder, and a remainder below ``lo`` is merged
+    into the previous document."""
+    p = 1.0 / mean
+    lengths: List[int] = []
+    s = 0
+    us = uniform(seed, "doclen", total // max(lo, 1) + 2)
+    draw = 0
+    while s < total:
+        u = us[draw]
+        draw += 1
+        L = int(math.ceil(math.log(u) / math.log1p(-p))) if u < 1.0 else 1
+        L = max(lo, min(hi, max(L, 1)))
+        if s + L >= total:
+            rem = total - s
+            if rem < lo and lengths:
+                lengths[-1] += rem
+            else:
+                lengths.append(rem)
+            s = total
+        else:
+            lengths.append(L)
+            s += L
+    return lengths
+
+
+@dataclasses.dataclass(frozen=True)
+class Layer:
+    """One dynamic short convolution call: C channels filtered from a d-wide hidden state."""
+
+    name: str
+    d_model: int
+    channels: int
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str                    # LOWRANK or HEADWISE
+    dtype: str                   # "f32" or "bf16" (storage; accumulation is fp32)
+    batch: int
+    seqlen: int
+    ksize: int
+    rank: int                    # low-rank r (0 for head-wise)
+    head_dim: int                # head-wise channels per head (0 for low-rank)
+    layers: tuple                # tuple[Layer, ...]
+    seed: int
+    a_std: Optional[float] = None  # None: 1/sqrt(d)
+    b_std: Optional[float] = None  # None: 1/sqrt(r)
+    varlen: bool = False
+    doc_mean: float = 2048.0
+    doc_lo: int = 16
+    doc_hi: int = 16384
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+def _cfg() -> Dict[str, Workload]:
+    return {
+        "c1_fp32_lowrank": Workload(
+            "c1_fp32_lowrank", LOWRANK, "f32", 2, 128, 3, 4, 0,
+            (Layer("conv", 64, 64),), seed=0, a_std=1.0 / 8.0, b_std=0.5),
+        "c2_qkv_150m_lowrank": Workload(
+            "c2_qkv_150m_lowrank", LOWRANK, "bf16", 8, 2048, 3, 32, 0,
+            (Layer("qkv", 768, 2304),), seed=1),
+        "c3_qkv_2b_headwise_gqa": Workload(
+            "c3_qkv_2b_headwise_gqa", HEADWISE, "bf16", 4, 4096, 4, 0, 128,
+            (Layer("qkv", 2048, 3072),), seed=2),
+        "c4_all_linear_2b_block": Workload(
+            "c4_all_linear_2b_block", LOWRANK, "bf16", 4, 4096, 3, 64, 0,
+            (Layer("qkv", 2048, 3072), Layer("o", 2048, 2048),
+             Layer("gate_up", 2048, 11264), Layer("down", 5632, 2048)), seed=3),
+        "c5_varlen_packed": Workload(
+            "c5_varlen_packed", LOWRANK, "bf16", 1, 65536, 4, 64, 0,
+            (Layer("conv", 4096, 4096),), seed=4, varlen=True),
+    }
+
+
+CONFIGS: Dict[str, Workload] = _cfg()
+CONFIG_ORDER = list(CONFIGS)
+
+
+def scaled(w: Workload, batch: int, seqlen: int, layers=None, name=None) -> Workload:
+    """The same workload recipe at a smaller token count (and optionally other layers)."""
+    return dataclasses.replace(w, batch=batch, seqlen=seqlen,
+                               layers=tuple(layers) if layers is not None else w.layers,
+                               name=name or f"{w.name}_B{batch}T{seqlen}")
+
+
+def cu_seqlens_for(w: Workload) -> np.ndarray:
+    """int32 document offsets [n_docs + 1]: uniform sequences for dense batches,
+    Geometric document lengths for packed workloads."""
+    if w.varlen:
+        lens = geometric_doc_lengths(w.seed, w.tokens, w.doc_mean, w.doc_lo, w.doc_hi)
+    else:
+        lens = [w.seqlen] * w.batch
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+
+def make_inputs(w: Workload, layer: Layer, layer_index: int = 0) -> Dict[str, np.ndarray]:
+    """Seeded inputs for one layer call, already rounded to the storage dtype (fp64 arrays).
+
+    Keys: u [N,C], h [N,d], g [N,C] (upstream gradient), and A [d,r] + B [r,C*K]
+    (low-rank) or W [d,(C/head_dim)*K] (head-wise), cu_seqlens int32.
+    """
+    N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
+    s = w.seed * 1000 + layer_index
+    out: Dict[str, np.ndarray] = {}
+    out["u"] = round_to_storage(normal(s, "u", N * C).reshape(N, C), w.dtype)
+    out["h"] = round_to_storage(normal(s, "h", N * d).reshape(N, d), w.dtype)
+    out["g"] = round_to_storage(normal(s, "g", N * C).reshape(N, C), w.dtype)
+    if w.kind == LOWRANK:
+        r = w.rank
+        a_std = w.a_std if w.a_std is not None else 1.0 / math.sqrt(d)
+        b_std = w.b_std if w.b_std is not None else 1.0 / math.sqrt(r)
+        out["A"] = round_to_storage(normal(s, "A", d * r, a_std).reshape(d, r), w.dtype)
+        out["B"] = round_to_storage(normal(s, "B", r * C * K, b_std).reshape(r, C * K), w.dtype)
+    else:
+        H = C // w.head_dim
+        out["W"] = round_to_storage(
+            normal(s, "W", d * H * K, 1.0 / math.sqrt(d)).reshape(d, H * K), w.dtype)
+    out["cu_seqlens"] = cu_seqlens_for(w)
+    return out
