@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark: dynamic short convolution forward + backward tokens/s on B200.
+
+One step = one forward and one backward pass of every layer of the workload
+(the hot path: filter generation, causal conv + residual, du, dz/dwh, dA/dB or
+dW, dh) over one batch of seeded synthetic inputs already resident in HBM.
+The default workload is the 150M-scale QKV placement (B=8, T=2048, d=768,
+C=2304, K=3, low-rank r=32, bf16).
+
+Prints ONE JSON line (rank 0).  Under torchrun each rank runs its own replica
+on its own seeded shard (weak scaling, no data-path collective); the timing
+is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dyn-conv fwd+bwd tokens/s at 1 B200; achieved HBM GB/s vs ~8 TB/s roofline"
+DEFAULT_CONFIG = "c2_qkv_150m_lowrank"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cores_used() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- algorithmic traffic
+def layer_bytes(w, layer):
+    """Algorithmic HBM bytes of one forward+backward of one layer call: every tensor
+    the op must read or write, once (bf16 storage s bytes, fp32 parameter grads):
+    fwd reads u, h, writes y, z; bwd reads g, u, h, z, writes du, dh; parameters
+    A, B (or W) read in both passes; dA, dB (or dW) written once.  The [N,C,K]
+    filter is never materialised, so it counts zero."""
+    s = 2 if w.dtype == "bf16" else 4
+    N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
+    per_tok = s * (2 * C + d) + s * (3 * C + d) + s * d   # fwd u,y,h ; bwd g,u,du,h ; dh
+    if w.kind == "lowrank":
+        r = w.rank
+        per_tok += 2 * s * r                               # z written in fwd, read in bwd
+        params = 2 * s * (d * r + r * C * K) + 4 * (d * r + r * C * K)
+    else:
+        H = C // w.head_dim
+        params = 2 * s * d * H * K + 4 * d * H * K
+    return N * per_tok + params
+
+
+def layer_flops(w, layer):
+    """Tensor-core FLOPs of one forward+backward: low-rank 2rCK per token for each of
+    w (fwd), w (bwd recompute), dz and dB, plus 2dr for z, dA and dh; head-wise
+    2dHK for the filters, dW and dh."""
+    N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
+    if w.kind == "lowrank":
+        return N * (8 * w.rank * C * K + 6 * d * w.rank)
+    H = C // w.head_dim
+    return N * 6 * d * H * K
+
+
+def kernel_bytes(name, w, layer):
+    """Algorithmic bytes of ONE launch of a library kernel on one layer call
+    (inputs read once, outputs written once, at the kernel's interface)."""
+    s = 2 if w.dtype == "bf16" else 4
+    N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
+    if w.kind == "lowrank":
+        R, P = w.rank, d * w.rank
+        BW = w.rank * C * K
+    else:
+        R = (C // w.head_dim) * K
+        P = d * R
+        BW = 0
+    table = {
+        "simt_gen": N * d * s + P * s + N * R * (4 + (s if w.kind == "lowrank" else 0)),
+        "simt_widen": N * R * (s + 4),
+        "simt_conv_fwd": N * C * 2 * s + N * R * 4 + BW * s,
+        "simt_conv_bwd": N * C * 3 * s + N * R * 8 + BW * s,
+        "simt_dB": N * R * 4 + N * C * 2 * s + BW * 4,
+        "simt_hTX": N * d * s + N * R * 4 + P * 4,
+        "simt_dh": N * R * 4 + P * s + N * d * s,
+        "tc_gen": N * d * s + P * s + N * R * s,
+        "tc_lowrank_fwd": N * C * 2 * s + N * R * s + BW * s,
+        "tc_lowrank_bwd": N * C * 3 * s + N * R * s + BW * s,
+        "tc_gen_bwd": N * d * 2 * s + N * R * s + P * (s + 4),
+        "tc_headwise_fwd": N * C * 2 * s + N * d * s + P * s,
+        "tc_headwise_bwd": N * C * 3 * s + N * R * 4,
+    }
+    return table.get(name)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML every 20 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+
+            N.nvmlInit()
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = N.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self.N = N
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h) \
+                    if hasattr(N, "nvmlDeviceGetCurrentClocksEventReasons") \
+                    else N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                util = N.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((sm, rs, util))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "err", "no NVML")}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, rs, _ in busy:
+            for bit, nm in self.REASONS.items():
+                if rs & bit and nm != "gpu_idle":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+class OracleSample:
+    """The fp64 oracle (as it stands) on a bounded sample of the workload: forward,
+    per-token backward and parameter gradients of every layer on the first T
+    tokens of one sequence.  Inputs are drawn once, outside the timing."""
+
+    def __init__(self, w, T):
+        from dynamic_short_convolutions_b200 import workloads as W
+        from oracle import oracle as O
+
+        O.build()
+        self.O = O
+        self.T = T
+        ws = W.scaled(w, 1, T, name="oracle_sample")
+        self.calls = []
+        for li, layer in enumerate(ws.layers):
+            x = W.make_inputs(ws, layer, li)
+            p = O.Problem(O.LOWRANK if ws.kind == W.LOWRANK else O.HEADWISE, T, layer.d_model, layer.channels,
+                          ws.ksize, [0, T], rank=ws.rank, head_dim=ws.head_dim)
+            self.calls.append((p, x, x.get("A"), x["B"] if ws.kind == W.LOWRANK else x["W"]))
+
+    def run(self) -> float:
+        O = self.O
+        t0 = time.perf_counter()
+        for p, x, A, BW in self.calls:
+            O.forward(p, x["u"], x["h"], A, BW)
+            O.backward_rows(p, x["g"], x["u"], x["h"], A, BW)
+            O.param_grads(p, x["g"], x["u"], x["h"], A, BW)
+        return time.perf_counter() - t0
+
+
+def oracle_tokens_for(w, budget_s: float, max_tokens: int) -> int:
+    """Sample size whose oracle run takes about budget_s seconds (calibrated on 16 tokens)."""
+    cal = OracleSample(w, 16)
+    cal.run()
+    per_tok = max(cal.run() / 16, 1e-7)
+    return int(max(16, min(max_tokens, budget_s / per_tok)))
+
+
+def oracle_sample_rate(w, budget_s: float, max_tokens: int):
+    """(tokens/s, T, seconds) of one oracle run sized to about budget_s seconds."""
+    T = oracle_tokens_for(w, budget_s, max_tokens)
+    secs = OracleSample(w, T).run()
+    return T / secs, T, secs
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from dynamic_short_convolutions_b200 import _lib as L, ops, workloads as W
+
+    L.load()  # fails loudly if the CUDA library is missing
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.CONFIGS[args.config]
+    if rank:
+        import dataclasses
+        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)   # each rank: its own shard
+    kind = L.LOWRANK if w.kind == W.LOWRANK else L.HEADWISE
+    dt = W.storage_dtype(w)
+    layers = []
+    for li, layer in enumerate(w.layers):
+        t = W.make_inputs(w, layer, li, device=dev)
+        batch, seqlen = (1, w.tokens) if w.varlen else (w.batch, w.seqlen)
+        plan = ops.DynConvPlan(kind, dt, batch, seqlen, layer.d_model, layer.channels, w.ksize, w.rank,
+                               w.head_dim, algo=args.algo, device=dev)
+        A = t.get("A")
+        BW = t["B"] if kind == L.LOWRANK else t["W"]
+        N = w.tokens
+        bufs = dict(y=torch.empty((N, layer.channels), dtype=dt, device=dev),
+                    z=torch.empty((N, w.rank), dtype=dt, device=dev) if kind == L.LOWRANK else None,
+                    out={"du": torch.empty((N, layer.channels), dtype=dt, device=dev),
+                         "dh": torch.empty((N, layer.d_model), dtype=dt, device=dev),
+                         "dA": torch.empty(tuple(A.shape), dtype=torch.float32, device=dev) if A is not None else None,
+                         "dBW": torch.empty(tuple(BW.shape), dtype=torch.float32, device=dev)})
+        cu = t["cu_seqlens"] if w.varlen else None
+        layers.append((layer, t, plan, A, BW, cu, bufs))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for layer, t, plan, A, BW, cu, b in layers:
+            plan.forward(t["u"], t["h"], A, BW, cu, y=b["y"], z_save=b["z"])
+            plan.backward(t["g"], t["u"], t["h"], A, BW, cu, z_saved=b["z"], out=b["out"])
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for _, _, plan, *_ in layers:
+        assert L.dynconv_device_status(plan.ws) == 0, L.dynconv_last_error()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    L.dynconv_profile_read(reset=True)
+    L.dynconv_profile_enable(True)
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    L.dynconv_profile_enable(False)
+    prof = L.dynconv_profile_read(reset=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax.item())
+    tokens_all = w.tokens * world * args.steps
+    value = tokens_all / (total_ms / 1e3)
+
+    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
+    host = []
+    h2d = d2h = 0
+    for layer, t, plan, A, BW, cu, b in layers:
+        hin = {k: v.to("cpu").pin_memory() for k, v in t.items() if k in ("u", "h", "g", "A", "B", "W")}
+        hout = {"y": torch.empty_like(b["y"], device="cpu").pin_memory(),
+                "du": torch.empty_like(b["out"]["du"], device="cpu").pin_memory(),
+                "dh": torch.empty_like(b["out"]["dh"], device="cpu").pin_memory(),
+                "dBW": torch.empty_like(b["out"]["dBW"], device="cpu").pin_memory()}
+        if b["out"]["dA"] is not None:
+            hout["dA"] = torch.empty_like(b["out"]["dA"], device="cpu").pin_memory()
+        h2d += sum(v.numel() * v.element_size() for v in hin.values())
+        d2h += sum(v.numel() * v.element_size() for v in hout.values())
+        host.append((hin, hout))
+
+    def e2e_step():
+        for (layer, t, plan, A, BW, cu, b), (hin, hout) in zip(layers, host):
+            for k, v in hin.items():
+                t[k].copy_(v, non_blocking=True)
+            plan.forward(t["u"], t["h"], t.get("A"), t["B"] if "B" in t else t["W"], cu, y=b["y"], z_save=b["z"])
+            plan.backward(t["g"], t["u"], t["h"], t.get("A"), t["B"] if "B" in t else t["W"], cu,
+                          z_saved=b["z"], out=b["out"])
+            hout["y"].copy_(b["y"], non_blocking=True)
+            for k in ("du", "dh", "dBW", "dA"):
+                if k in hout:
+                    hout[k].copy_(b["out"][k], non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = w.tokens * world * e2e_steps / (float(e2e_ms.item()) / 1e3)
+
+    # ---- roofline of the dominant kernel (live CUDA-event timing from the library's tracer)
+    pk, pk_src = peaks()
+    launches = sum(v[0] for v in prof.values())
+    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    roof = None
+    kernels = {}
+    for name, (n_l, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
+        kernels[name] = {"launches": n_l, "ms_total": round(ms, 4), "share": round(ms / max(total_ms, 1e-9), 4)}
+    if dom is not None:
+        name, (n_l, ms) = dom
+        per_launch_bytes = sum(kernel_bytes(name, w, layer) or 0 for layer in w.layers) / len(w.layers)
+        avg_s = ms / n_l / 1e3
+        achieved = per_launch_bytes / avg_s / 1e9
+        roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "peak_source": pk_src, "avg_launch_us": round(avg_s * 1e6, 2),
+                "algorithmic_bytes_per_launch": int(per_launch_bytes)}
+    step_bytes = sum(layer_bytes(w, layer) for layer in w.layers)
+    step_flops = sum(layer_flops(w, layer) for layer in w.layers)
+    ms_per_step = total_ms / args.steps
+    t_hbm = step_bytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = step_flops / (pk["bf16_tflops_sustained"] * 1e12)
+    step_roof = {"algorithmic_bytes": int(step_bytes), "tensor_flops": int(step_flops),
+                 "achieved_gbs": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
+                 "roofline_us": round(max(t_hbm, t_tc) * 1e6, 2),
+                 "frac_of_roofline": round(max(t_hbm, t_tc) / (ms_per_step / 1e3), 4),
+                 "vs_8TBps_frac": round(step_bytes / 8e12 / (ms_per_step / 1e3), 4), "peak_source": pk_src}
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "kind": w.kind, "batch": w.batch, "seq_len": w.seqlen,
+                       "tokens_per_gpu": w.tokens, "ksize": w.ksize, "rank": w.rank, "head_dim": w.head_dim,
+                       "layers": [[l.name, l.d_model, l.channels] for l in w.layers],
+                       "varlen": w.varlen, "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                       "algo": {0: "auto", 1: "simt", 2: "tc"}[args.algo]},
+            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
+            "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+            "gpu_launches": int(launches), "clocks": clk.summary()}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--algo", type=int, default=0, help="0 auto, 1 CUDA-core kernels, 2 tensor-core kernels")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from dynamic_short_convolutions_b200 import workloads as W
+
+    w = W.CONFIGS[args.config]
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        # The reference arm is the fp64 oracle as it stands, on this host's cores:
+        # each step is a bounded sample of the workload (first T tokens, every layer).
+        per_step_budget = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+        T = oracle_tokens_for(w, per_step_budget, w.seqlen)
+        sample = OracleSample(w, T)
+        for _ in range(args.warmup):
+            sample.run()
+        secs = [sample.run() for _ in range(args.steps)]
+        value = T * args.steps / sum(secs)
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(secs) / len(secs), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": w.name, "sample_tokens_per_step": T},
+                "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores_used(),
+                                 "kind": "oracle",
+                                 "sample": f"fp64 oracle fwd+bwd on the first {T} tokens of one sequence of "
+                                           f"{w.name}, every layer, per step"},
+                "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            rate, T, secs = oracle_sample_rate(w, args.cpu_budget, w.seqlen)
+            line["cpu_baseline"] = {"value": round(rate, 2), "unit": "tokens/s", "cores": cores_used(),
+                                    "kind": "oracle",
+                                    "sample": f"fp64 oracle fwd+bwd on the first {T} tokens of one sequence "
+                                              f"of {w.name}, every layer ({secs:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,41 @@
+// common.cuh -- small device helpers shared by the dynamic short convolution kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace dynconv {
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// First token of the sequence / packed document holding token n.
+//  cu == nullptr: dense batch of sequences of length seqlen.
+//  otherwise:     largest s with cu[s] <= n, by binary search over cu[0..n_docs].
+// The result is clamped to [0, n] so that a malformed cu_seqlens can never send
+// a tap outside the tensor (the pre-check kernel reports it instead).
+__device__ __forceinline__ int64_t seg_start(int64_t n, const int32_t* __restrict__ cu, int64_t n_docs,
+                                             int64_t seqlen) {
+    int64_t s;
+    if (cu == nullptr) {
+        s = (n / seqlen) * seqlen;
+    } else {
+        int64_t lo = 0, hi = n_docs;
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if ((int64_t)__ldg(cu + mid) <= n) lo = mid; else hi = mid;
+        }
+        s = (int64_t)__ldg(cu + lo);
+    }
+    s = s < 0 ? 0 : s;
+    return s > n ? n : s;
+}
+
+}  // namespace dynconv

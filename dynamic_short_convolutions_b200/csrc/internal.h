@@ -1,0 +1,64 @@
+// internal.h -- host-side structures shared by the C ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dynconv {
+
+// Bits of the device error word kept at the start of the workspace.
+enum : uint32_t {
+    kErrBadSeqlens = 1u,   // cu_seqlens not 0 ... N, non-decreasing
+    kErrWaitTimeout = 2u,  // an mbarrier wait ran out of its iteration limit
+};
+
+// A validated problem: all sizes resolved, strides filled in.
+struct Prob {
+    int kind;           // 0 low-rank, 1 head-wise
+    int dtype;          // 0 fp32, 1 bf16
+    int64_t batch, seqlen, N;
+    int64_t d, C, K;
+    int64_t r;          // low-rank rank
+    int64_t hd, H;      // head-wise head_dim and head count
+    int64_t R;          // generator width: r (low-rank) or H*K (head-wise)
+    int64_t us, hs;     // row strides of u and h, in elements
+    const int32_t* cu;  // device cu_seqlens or nullptr (dense batch)
+    int64_t n_docs;
+    int deterministic;
+};
+
+// Workspace carve-up (byte offsets; every region 256-byte aligned).
+struct WsLayout {
+    size_t err;         // uint32 device error word
+    size_t gen;         // fp32 [N, R]: z (low-rank) or head-wise filters (SIMT path)
+    size_t dgen;        // fp32 [N, R]: dz or dwh
+    size_t tc;          // start of the tensor-core path's private region
+    size_t tc_bytes;
+    size_t total;
+};
+
+WsLayout ws_layout(const Prob& p);
+size_t tc_workspace_bytes(const Prob& p);
+bool tc_supported(const Prob& p);
+
+// Generic CUDA-core kernels (any shape, fp32 or bf16 storage).
+cudaError_t simt_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW,
+                         void* y, void* z_save, void* ws, cudaStream_t st);
+cudaError_t simt_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
+                          const void* BW, const void* z_saved, void* du, void* dh, float* dA, float* dBW,
+                          void* ws, cudaStream_t st);
+
+// tcgen05 / TMA kernels (bf16 storage, shapes accepted by tc_supported).
+cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW,
+                       void* y, void* z_save, void* ws, cudaStream_t st);
+cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
+                        const void* BW, const void* z_saved, void* du, void* dh, float* dA, float* dBW,
+                        void* ws, cudaStream_t st);
+
+cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st);
+
+// Text for the thread-local error message.
+void set_error(const char* fmt, ...);
+
+}  // namespace dynconv

@@ -195,27 +195,89 @@ def cu_seqlens_for(w: Workload) -> np.ndarray:
     return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
 
 
-def make_inputs(w: Workload, layer: Layer, layer_index: int = 0) -> Dict[str, np.ndarray]:
-    """Seeded inputs for one layer call, already rounded to the storage dtype (fp64 arrays).
+def _mix_t(x):
+    """splitmix64 output function on an int64 torch tensor (two's-complement
+    wrapping; logical right shifts by masking), bit-identical to ``_mix``."""
+    M1 = int(_M1) - (1 << 64)
+    M2 = int(_M2) - (1 << 64)
+    x = x ^ ((x >> 30) & ((1 << 34) - 1))
+    x = x * M1
+    x = x ^ ((x >> 27) & ((1 << 37) - 1))
+    x = x * M2
+    return x ^ ((x >> 31) & ((1 << 33) - 1))
+
+
+def normal_torch(seed: int, tag: str, count: int, std: float = 1.0, device="cpu", chunk: int = 1 << 24):
+    """The same recipe as ``normal`` evaluated with torch ops on ``device`` (fp64).
+    The bits are identical to ``normal``; the fp64 log/cos may differ from
+    numpy's in the last ulp, which the storage rounding almost always absorbs.
+    Each test or benchmark uses one realisation for both sides of a comparison."""
+    import torch
+
+    key = int(_key(seed, tag))
+    key = key - (1 << 64) if key >= (1 << 63) else key
+    G = int(GOLDEN) - (1 << 64)
+    out = torch.empty(count, dtype=torch.float64, device=device)
+    for a in range(0, count, chunk):
+        b = min(count, a + chunk)
+        i = torch.arange(2 * a, 2 * b, dtype=torch.int64, device=device)
+        bits = _mix_t(key + (i + 1) * G)
+        m53 = (1 << 53) - 1
+        u1 = (((bits[0::2] >> 11) & m53).to(torch.float64) + 1.0) * (2.0 ** -53)
+        u2 = ((bits[1::2] >> 11) & m53).to(torch.float64) * (2.0 ** -53)
+        out[a:b] = std * torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * math.pi * u2)
+    return out
+
+
+def storage_dtype(w: "Workload"):
+    import torch
+
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def make_inputs(w: Workload, layer: Layer, layer_index: int = 0, device=None) -> Dict[str, object]:
+    """Seeded inputs for one layer call.
+
+    device None: fp64 numpy arrays holding values already rounded to the
+    storage dtype (small problems, CPU-only tests).  device given: torch
+    tensors in the storage dtype on that device (same recipe, drawn there).
 
     Keys: u [N,C], h [N,d], g [N,C] (upstream gradient), and A [d,r] + B [r,C*K]
-    (low-rank) or W [d,(C/head_dim)*K] (head-wise), cu_seqlens int32.
+    (low-rank) or W [d,(C/head_dim)*K] (head-wise), cu_seqlens int32 [docs+1].
     """
     N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
     s = w.seed * 1000 + layer_index
-    out: Dict[str, np.ndarray] = {}
-    out["u"] = round_to_storage(normal(s, "u", N * C).reshape(N, C), w.dtype)
-    out["h"] = round_to_storage(normal(s, "h", N * d).reshape(N, d), w.dtype)
-    out["g"] = round_to_storage(normal(s, "g", N * C).reshape(N, C), w.dtype)
+    shapes = {"u": ((N, C), 1.0), "h": ((N, d), 1.0), "g": ((N, C), 1.0)}
     if w.kind == LOWRANK:
         r = w.rank
         a_std = w.a_std if w.a_std is not None else 1.0 / math.sqrt(d)
         b_std = w.b_std if w.b_std is not None else 1.0 / math.sqrt(r)
-        out["A"] = round_to_storage(normal(s, "A", d * r, a_std).reshape(d, r), w.dtype)
-        out["B"] = round_to_storage(normal(s, "B", r * C * K, b_std).reshape(r, C * K), w.dtype)
+        shapes["A"] = ((d, r), a_std)
+        shapes["B"] = ((r, C * K), b_std)
     else:
         H = C // w.head_dim
-        out["W"] = round_to_storage(
-            normal(s, "W", d * H * K, 1.0 / math.sqrt(d)).reshape(d, H * K), w.dtype)
-    out["cu_seqlens"] = cu_seqlens_for(w)
+        shapes["W"] = ((d, H * K), 1.0 / math.sqrt(d))
+    out: Dict[str, object] = {}
+    for name, (shape, std) in shapes.items():
+        cnt = int(np.prod(shape))
+        if device is None:
+            out[name] = round_to_storage(normal(s, name, cnt, std).reshape(shape), w.dtype)
+        else:
+            out[name] = normal_torch(s, name, cnt, std, device=device).to(
+                __import__("torch").float32).to(storage_dtype(w)).reshape(shape)
+    cu = cu_seqlens_for(w)
+    if device is None:
+        out["cu_seqlens"] = cu
+    else:
+        import torch
+        out["cu_seqlens"] = torch.from_numpy(cu).to(device)
     return out
+
+
+def to_f64(x) -> np.ndarray:
+    """Host fp64 copy of a torch tensor or numpy array (for the oracle)."""
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.float64)
+    import torch
+
+    return x.detach().to("cpu", torch.float64).contiguous().numpy()

@@ -1,0 +1,171 @@
+/*
+ * dynconv.h -- C ABI of the B200 (sm_100a) dynamic short convolution library.
+ *
+ * The operation ("Dynamic Short Convolutions Improve Transformers",
+ * gist.science technical summary, section "Dynamic Short Convolutions"):
+ * every token n generates its own depthwise causal filter of K taps from its
+ * hidden state h[n,:] by a learned linear map, factored either
+ *
+ *   low-rank  (Parameterization 1):  z[n,:] = h[n,:] A            A: [d, r]
+ *                                    w[n,c,j] = sum_k z[n,k] B[k, c*K + j]
+ *                                                                 B: [r, C*K]
+ *   head-wise (Parameterization 2):  w[n,c,j] = sum_i h[n,i] W[i, (c/head_dim)*K + j]
+ *                                                                 W: [d, H*K]
+ *
+ * and applies it with the residual of the "Placement" paragraph
+ * (X = X + dynamicShortConv(X)) and the "Mechanism" formula, tap 0 being the
+ * current token:
+ *
+ *   y[n,c] = u[n,c] + sum_{j<K, n-j >= s(n)} w[n,c,j] u[n-j,c]
+ *
+ * where s(n) is the first token of n's sequence (dense batch) or packed
+ * document (cu_seqlens); taps before it read zero.  The filter tensor
+ * w [N,C,K] is never written to memory by the tensor-core path.
+ *
+ * Conventions shared by every entry point
+ *   - Layout: token-major, channels contiguous.  u is [N, C] with row stride
+ *     desc->u_row_stride elements (0 means C), so u may be a column slice of
+ *     a fused QKV output; h is [N, d] with row stride desc->h_row_stride
+ *     (0 means d).  y, g, du are dense [N, C]; dh is dense [N, d]; A is
+ *     [d, r]; B is [r, C*K] (column c*K + j); W is [d, H*K] (column q*K + j).
+ *     N = batch * seqlen tokens.
+ *   - Storage dtype desc->dtype (fp32 or bf16) for u, h, A, B/W, y, z, g, du,
+ *     dh; accumulation is always fp32; parameter gradients dA, dB/dW are fp32
+ *     and OVERWRITTEN (not accumulated).
+ *   - Ownership: the caller allocates every buffer, including the workspace
+ *     (size from dynconv_workspace_bytes).  All pointers are device pointers
+ *     (a host pointer is rejected with DYNCONV_ERR_INVALID: there is no CPU
+ *     path).  Pointers must be 16-byte aligned and row strides multiples of
+ *     8 elements for bf16 / 4 for fp32.  The library allocates nothing.
+ *   - Stream: `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *     work is enqueued asynchronously on it; nothing synchronises.
+ *   - Errors: arguments are validated before any launch; a failed launch
+ *     returns DYNCONV_ERR_CUDA.  dynconv_last_error() gives a thread-local
+ *     message for the last failure.  Nothing traps on the device.
+ */
+#ifndef DYNCONV_H
+#define DYNCONV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DYNCONV_API __attribute__((visibility("default")))
+#else
+#define DYNCONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DYNCONV_OK = 0,
+    DYNCONV_ERR_INVALID = 1,      /* bad argument: null/host/misaligned pointer, bad shape */
+    DYNCONV_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. ksize > 4) */
+    DYNCONV_ERR_WORKSPACE = 3,    /* ws_bytes below dynconv_workspace_bytes() */
+    DYNCONV_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed */
+    DYNCONV_ERR_DEVICE_CHECK = 5  /* a device-side check failed (bad cu_seqlens, barrier timeout) */
+} dynconv_status;
+
+typedef enum { DYNCONV_F32 = 0, DYNCONV_BF16 = 1 } dynconv_dtype;
+typedef enum { DYNCONV_LOWRANK = 0, DYNCONV_HEADWISE = 1 } dynconv_kind;
+
+/* Kernel family.  AUTO picks the tcgen05/TMA tensor-core kernels for bf16
+ * shapes they cover and the generic CUDA-core kernels otherwise (always for
+ * fp32, which must not be rounded to a tensor-core input type). */
+typedef enum { DYNCONV_ALGO_AUTO = 0, DYNCONV_ALGO_SIMT = 1, DYNCONV_ALGO_TC = 2 } dynconv_algo;
+
+typedef struct {
+    int32_t kind;           /* dynconv_kind */
+    int32_t dtype;          /* dynconv_dtype */
+    int64_t batch;          /* B sequences of seqlen tokens (varlen: 1) */
+    int64_t seqlen;         /* T (varlen: total packed tokens N) */
+    int64_t d_model;        /* d: width of the hidden state h feeding the generator */
+    int64_t channels;       /* C: channels of u being filtered */
+    int64_t ksize;          /* K: taps, 1..4 */
+    int64_t rank;           /* low-rank r (1..128); head-wise: 0 */
+    int64_t head_dim;       /* head-wise channels per head (C % head_dim == 0); low-rank: 0 */
+    int64_t u_row_stride;   /* elements between tokens of u; 0 = channels */
+    int64_t h_row_stride;   /* elements between tokens of h; 0 = d_model */
+    int32_t deterministic;  /* 1: every reduction in a fixed order, no float atomics */
+    int32_t algo;           /* dynconv_algo */
+} dynconv_desc;
+
+/* Workspace needed by dynconv_fwd / dynconv_fwd_varlen / dynconv_bwd for this
+ * descriptor (one size serves all three).  Returns 0 for an invalid desc.
+ * The first 256 bytes hold the device error word: zero them once before the
+ * workspace's first use (the library clears the word when it reports it).
+ * One workspace must not be used by two calls that overlap on the device. */
+DYNCONV_API size_t dynconv_workspace_bytes(const dynconv_desc *desc);
+
+/* Forward, dense batch: y = u + dynamic causal conv(u), filters from h.
+ *   u      [N, C] (u_row_stride), h [N, d] (h_row_stride)
+ *   A      [d, r] (low-rank) or NULL (head-wise)
+ *   B_or_W [r, C*K] (low-rank) or [d, H*K] (head-wise)
+ *   y      [N, C] output, dense
+ *   z_save nullable; low-rank only: receives z = h A as [N, r] (storage dtype)
+ *          for the backward pass to reuse. */
+DYNCONV_API dynconv_status dynconv_fwd(const dynconv_desc *desc, const void *u, const void *h, const void *A,
+                           const void *B_or_W, void *y, void *z_save, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* Forward over packed documents: desc->batch must be 1 and desc->seqlen the
+ * total token count N.  cu_seqlens is a DEVICE int32 array [n_docs + 1] with
+ * cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_docs] = N; the filter never
+ * reaches across a document start.  A malformed cu_seqlens is caught by a
+ * device pre-check that raises a flag read by dynconv_device_status(); the
+ * results of that call are then undefined, but every access stays inside the
+ * tensors (each tap's source index is clamped into the token range). */
+DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const int32_t *cu_seqlens, int64_t n_docs,
+                                  const void *u, const void *h, const void *A, const void *B_or_W,
+                                  void *y, void *z_save, void *ws, size_t ws_bytes, void *stream);
+
+/* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch).
+ *   g        [N, C] upstream gradient dL/dy, dense
+ *   z_saved  nullable: z from the forward pass (low-rank); NULL recomputes it
+ *   du       [N, C] output dL/du, dense
+ *   dh       nullable [N, d] output dL/dh, dense
+ *   dA       [d, r] fp32 output (low-rank; ignored for head-wise)
+ *   dB_or_dW [r, C*K] or [d, H*K] fp32 output */
+DYNCONV_API dynconv_status dynconv_bwd(const dynconv_desc *desc, const int32_t *cu_seqlens, int64_t n_docs,
+                           const void *g, const void *u, const void *h, const void *A,
+                           const void *B_or_W, const void *z_saved, void *du, void *dh, float *dA,
+                           float *dB_or_dW, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream` and reports device-side check failures raised by the
+ * calls that used this workspace since the last query (then clears them):
+ * DYNCONV_ERR_DEVICE_CHECK for a malformed cu_seqlens or a pipeline wait that
+ * ran out of its iteration limit, else DYNCONV_OK. */
+DYNCONV_API dynconv_status dynconv_device_status(void *ws, size_t ws_bytes, void *stream);
+
+/* Thread-local text of the last failure in this thread ("" if none). */
+DYNCONV_API const char *dynconv_last_error(void);
+
+/* Name of a status code. */
+DYNCONV_API const char *dynconv_status_string(dynconv_status status);
+
+/* Per-kernel device timing (tracing).  When enabled, every kernel launch of
+ * the library is bracketed by two CUDA events recorded on its launch stream.
+ * dynconv_profile_enable returns the previous state.  dynconv_profile_read
+ * waits for the recorded events, writes up to max_entries rows (kernel name,
+ * launches, summed device milliseconds) for kernels launched since the last
+ * reset, and returns how many kernels have rows; reset != 0 clears the sums.
+ * Not for use inside CUDA graph capture. */
+typedef struct {
+    char name[48];
+    int64_t launches;
+    double total_ms;
+} dynconv_profile_entry;
+
+DYNCONV_API int dynconv_profile_enable(int enable);
+DYNCONV_API int dynconv_profile_read(dynconv_profile_entry *entries, int max_entries, int reset);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+DYNCONV_API int dynconv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYNCONV_H */

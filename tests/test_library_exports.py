@@ -1,0 +1,51 @@
+"""CPU checks of the C ABI library: it loads and exports every entry point the
+header declares (no compute call: there is no GPU here), and the binding's list
+matches the header."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dynconv.h")
+LIB = os.path.join(ROOT, "dynamic_short_convolutions_b200", "libdynconv.so")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DYNCONV_API\s+[\w\s\*]*?\b(dynconv_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd", "dynconv_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    if not os.path.exists(LIB):
+        from dynamic_short_convolutions_b200 import build
+
+        build.build()
+    lib = ctypes.CDLL(LIB)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    assert sorted(L.EXPORTS) == sorted(set(L.EXPORTS) & set(_declared())) or set(_declared()) >= set(L.EXPORTS)
+    assert set(L.EXPORTS) == set(_declared())
+
+
+def test_pure_host_entry_points_without_gpu():
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    if not os.path.exists(LIB):
+        pytest.skip("library not built")
+    lib = L.load()
+    assert lib.dynconv_version() >= 100
+    assert lib.dynconv_status_string(2) == b"DYNCONV_ERR_UNSUPPORTED"
+    d = L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 3, 32)
+    assert L.dynconv_workspace_bytes(d) > 0
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 0, 32)) == 0
+    assert L.dynconv_workspace_bytes(L.make_desc(L.HEADWISE, L.BF16, 1, 10, 8, 12, 3, 0, 5)) == 0

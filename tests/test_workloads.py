@@ -50,3 +50,22 @@ def test_config_shapes():
     assert c["c2_qkv_150m_lowrank"].tokens == 16384
     assert sum(l.channels for l in c["c4_all_linear_2b_block"].layers) == 3072 + 2048 + 11264 + 2048
     assert c["c3_qkv_2b_headwise_gqa"].layers[0].channels // 128 == 24
+
+
+def test_torch_generator_matches_numpy_bits_and_values():
+    import torch
+
+    a = W.normal(5, "u", 4097)
+    b = W.normal_torch(5, "u", 4097, chunk=1000).numpy()
+    assert np.max(np.abs(a - b)) <= 1e-12 * max(1.0, np.abs(a).max())
+    bits_np = W._mix(np.arange(1, 100, dtype=np.uint64) * W.GOLDEN)
+    bits_t = W._mix_t(torch.arange(1, 100, dtype=torch.int64) * (int(W.GOLDEN) - (1 << 64))).numpy()
+    assert np.array_equal(bits_np.view(np.int64), bits_t)
+
+
+def test_make_inputs_numpy_and_torch_agree_after_rounding():
+    w = W.scaled(W.CONFIGS["c2_qkv_150m_lowrank"], 1, 64)
+    a = W.make_inputs(w, w.layers[0])
+    b = W.make_inputs(w, w.layers[0], device="cpu")
+    for k in ("u", "h", "g", "A", "B"):
+        assert np.array_equal(a[k], W.to_f64(b[k])), k
