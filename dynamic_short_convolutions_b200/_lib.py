@@ -27,7 +27,7 @@ ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 # Every entry point the header declares (checked against the library's exports by the tests).
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
-           "dynconv_profile_enable", "dynconv_profile_read")
+           "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma")
 
 
 class DynConvError(RuntimeError):
@@ -79,6 +79,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_profile_enable.restype = ctypes.c_int
     lib.dynconv_profile_read.argtypes = [ctypes.POINTER(dynconv_profile_entry), ctypes.c_int, ctypes.c_int]
     lib.dynconv_profile_read.restype = ctypes.c_int
+    lib.dynconv_selftest_umma.argtypes = [ctypes.c_int, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
+    lib.dynconv_selftest_umma.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -152,3 +154,9 @@ def dynconv_profile_read(reset: bool = True):
     arr = (dynconv_profile_entry * 64)()
     n = lib.dynconv_profile_read(arr, 64, int(bool(reset)))
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(min(n, 64))}
+
+
+def dynconv_selftest_umma(variant: int, A, B, D, N: int, Kd: int, err_word, stream=None) -> int:
+    """Diagnostic tile D = A B^T through TMA + tcgen05 (see include/dynconv_diag.h); returns the status."""
+    return int(load().dynconv_selftest_umma(variant, _ptr(A), _ptr(B), _ptr(D), N, Kd, _ptr(err_word),
+                                            _stream(stream, A)))

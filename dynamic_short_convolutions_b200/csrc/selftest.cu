@@ -1,0 +1,122 @@
+// selftest.cu -- self-test of the tensor-core building blocks: one 128-row tile of
+// D = A * B^T loaded by TMA (128-byte swizzle) and multiplied by tcgen05.mma with
+// the same descriptor helpers the product kernels use, for the operand layouts
+// they use.  It exists so that a layout or descriptor mistake shows up as a
+// plain wrong number on a small case.
+#include <cstdio>
+
+#include "../../include/dynconv.h"
+#include "../../include/dynconv_diag.h"
+#include "tc_common.cuh"
+#include "tmap.h"
+
+namespace dynconv {
+namespace {
+
+using namespace tc;
+
+constexpr int kSelftestSmem = 1024 + 49152 + 98304;
+
+// variant 0: A [128][Kd] and B [N][Kd], both K-major, Kd in {64, 128, 192}.
+// variant 1: A stored [Kd][128] and B stored [Kd][N], both MN-major, Kd in {16, ..., 128}.
+__global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ CUtensorMap ta,
+                                                       const __grid_constant__ CUtensorMap tb, int variant, int N,
+                                                       int Kd, float* __restrict__ D, uint32_t* err) {
+    extern __shared__ uint8_t raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sa = sm;
+    uint8_t* sb = sm + 49152;
+    __shared__ uint64_t bar_load, bar_mma;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_mma, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        if (variant == 0) {
+            const int na = Kd / 64;
+            mbar_arrive_expect_tx(&bar_load, uint32_t(na * (128 * 128 + N * 128)));
+            for (int a = 0; a < na; ++a) tma_load_2d(sa + a * 16384, &ta, &bar_load, 64 * a, 0);
+            for (int a = 0; a < na; ++a) tma_load_2d(sb + a * N * 128, &tb, &bar_load, 64 * a, 0);
+        } else {
+            const int nb = (N + 63) / 64;
+            mbar_arrive_expect_tx(&bar_load, uint32_t((2 + nb) * Kd * 128));
+            for (int a = 0; a < 2; ++a) tma_load_2d(sa + a * Kd * 128, &ta, &bar_load, 64 * a, 0);
+            for (int a = 0; a < nb; ++a) tma_load_2d(sb + a * Kd * 128, &tb, &bar_load, 64 * a, 0);
+        }
+        ok = mbar_wait(&bar_load, 0, &abort_flag, err);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, N, variant == 1, variant == 1);
+            const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+            if (variant == 0) {
+                for (int kb = 0; kb < Kd / 64; ++kb)
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16(tbase, kmajor_desc(a0 + kb * 16384, k), kmajor_desc(b0 + kb * N * 128, k), idesc,
+                                  (kb | k) != 0);
+            } else {
+                for (int ks = 0; ks < Kd / 16; ++ks)
+                    umma_bf16(tbase, mnmajor_desc(a0, Kd * 128, ks * 16), mnmajor_desc(b0, Kd * 128, ks * 16),
+                              idesc, ks != 0);
+            }
+            umma_commit(&bar_mma);
+        }
+    }
+    __syncwarp();
+    if (mbar_wait(&bar_mma, 0, &abort_flag, err)) {
+        tc_fence_after();
+        const int row = warp * 32 + lane;
+        for (int c = 0; c < N; c += 8) {
+            uint32_t r[8];
+            tmem_ld8(tbase + (uint32_t(warp * 32) << 16) + c, r);
+            tmem_wait_ld();
+            for (int i = 0; i < 8; ++i) D[row * N + c + i] = __uint_as_float(r[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 256);
+    }
+}
+
+}  // namespace
+}  // namespace dynconv
+
+using namespace dynconv;
+
+extern "C" DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const void* A, const void* B, float* D,
+                                                            int N, int Kd, void* err_word, void* stream) {
+    if (variant == 0 && !(Kd == 64 || Kd == 128 || Kd == 192)) return DYNCONV_ERR_INVALID;
+    if (variant == 1 && !(Kd >= 16 && Kd <= 128 && Kd % 16 == 0)) return DYNCONV_ERR_INVALID;
+    if (variant != 0 && variant != 1) return DYNCONV_ERR_INVALID;
+    if (N < 16 || N > 256 || N % 16) return DYNCONV_ERR_INVALID;
+    if (!A || !B || !D || !err_word) return DYNCONV_ERR_INVALID;
+    CUtensorMap ta, tb;
+    bool ok;
+    if (variant == 0)
+        ok = make_tmap_bf16(&ta, A, Kd, 128, Kd, 64, 128) && make_tmap_bf16(&tb, B, Kd, N, Kd, 64, N);
+    else
+        ok = make_tmap_bf16(&ta, A, 128, Kd, 128, 64, Kd) && make_tmap_bf16(&tb, B, N, Kd, N, 64, Kd);
+    if (!ok) return DYNCONV_ERR_CUDA;
+    if (cudaFuncSetAttribute(selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelftestSmem) !=
+        cudaSuccess)
+        return DYNCONV_ERR_CUDA;
+    selftest_kernel<<<1, 128, kSelftestSmem, static_cast<cudaStream_t>(stream)>>>(
+        ta, tb, variant, N, Kd, D, static_cast<uint32_t*>(err_word));
+    return cudaGetLastError() == cudaSuccess ? DYNCONV_OK : DYNCONV_ERR_CUDA;
+}

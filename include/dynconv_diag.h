@@ -1,0 +1,32 @@
+/*
+ * dynconv_diag.h -- diagnostics of libdynconv.so (no counterpart in the pages:
+ * these check the library's own sm_100a building blocks, not the method).
+ */
+#ifndef DYNCONV_DIAG_H
+#define DYNCONV_DIAG_H
+
+#include "dynconv.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One 128-row tile of D = A * B^T (bf16 in, fp32 out) through TMA loads with
+ * 128-byte swizzle and one CTA's tcgen05.mma, using the descriptor helpers of
+ * the product kernels.
+ *   variant 0: A is [128, Kd] and B is [N, Kd], row-major (both K-major);
+ *              Kd in {64, 128, 192}.
+ *   variant 1: A is stored [Kd, 128] and B is stored [Kd, N] (both MN-major);
+ *              Kd a multiple of 16 up to 128.
+ *   N: multiple of 16, 16..256.  D: [128, N] fp32, row-major.
+ * All pointers are device pointers (16-byte aligned); err_word is a device
+ * uint32 that receives the wait-timeout bit if the tile never completes.
+ * Asynchronous on `stream`; returns DYNCONV_ERR_INVALID for other shapes. */
+DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const void *A, const void *B, float *D, int N, int Kd,
+                                                 void *err_word, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYNCONV_DIAG_H */

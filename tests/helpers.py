@@ -7,8 +7,9 @@ from dynamic_short_convolutions_b200 import workloads as W
 
 # Tolerances: fp32 storage rel-L2 <= 1e-5; bf16 storage rel-L2 <= 2e-2 and
 # max-abs <= 5e-2, the max-abs read on the scale of the tensor: max|err| /
-# max(1, rms(ref)) (literal for O(1) outputs such as y and du; relative for
-# gradients that are sums over thousands of tokens).
+# max(1, max|ref|) (literal for tensors bounded by 1; relative above that,
+# since the bf16 rounding of one stored value of magnitude v is already up to
+# 2^-9 v, i.e. above 5e-2 for |v| > 25).
 TOL = {"f32": dict(rel_l2=1e-5, max_abs=None), "bf16": dict(rel_l2=2e-2, max_abs=5e-2)}
 
 
@@ -22,8 +23,7 @@ def scaled_max_abs(a, ref):
     a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
     if a.size == 0:
         return 0.0
-    rms = float(np.sqrt(np.mean(ref * ref)))
-    return float(np.max(np.abs(a - ref)) / max(1.0, rms))
+    return float(np.max(np.abs(a - ref)) / max(1.0, float(np.max(np.abs(ref)))))
 
 
 def assert_close(name, a, ref, dtype):

@@ -8,12 +8,13 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "dynconv.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 LIB = os.path.join(ROOT, "dynamic_short_convolutions_b200", "libdynconv.so")
 
 
 def _declared():
-    text = open(HEADER).read()
+    text = "\n".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"DYNCONV_API\s+[\w\s\*]*?\b(dynconv_\w+)\s*\(", text)))
 
 
