@@ -182,22 +182,27 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle leg
 class OracleSample:
     """The fp64 oracle (as it stands) on a bounded sample of the workload: forward,
-    per-token backward and parameter gradients of every layer on the first T
-    tokens of one sequence.  Inputs are drawn once, outside the timing."""
+    per-token backward and parameter gradients of every layer on the first
+    `seqs` sequences of the batch, truncated to T tokens each.  Inputs are drawn
+    once, outside the timing."""
 
-    def __init__(self, w, T):
+    def __init__(self, w, seqs, T):
         from dynamic_short_convolutions_b200 import workloads as W
         from oracle import oracle as O
 
         O.build()
         self.O = O
-        self.T = T
-        ws = W.scaled(w, 1, T, name="oracle_sample")
+        self.tokens = seqs * T
+        ws = W.scaled(w, seqs, T, name="oracle_sample")
+        if ws.varlen:   # a prefix of the packed stream, with its own document boundaries
+            import dataclasses
+            ws = dataclasses.replace(ws, varlen=False)
+        cu = [i * T for i in range(seqs + 1)]
         self.calls = []
         for li, layer in enumerate(ws.layers):
             x = W.make_inputs(ws, layer, li)
-            p = O.Problem(O.LOWRANK if ws.kind == W.LOWRANK else O.HEADWISE, T, layer.d_model, layer.channels,
-                          ws.ksize, [0, T], rank=ws.rank, head_dim=ws.head_dim)
+            p = O.Problem(O.LOWRANK if ws.kind == W.LOWRANK else O.HEADWISE, seqs * T, layer.d_model,
+                          layer.channels, ws.ksize, cu, rank=ws.rank, head_dim=ws.head_dim)
             self.calls.append((p, x, x.get("A"), x["B"] if ws.kind == W.LOWRANK else x["W"]))
 
     def run(self) -> float:
@@ -210,19 +215,24 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
-def oracle_tokens_for(w, budget_s: float, max_tokens: int) -> int:
-    """Sample size whose oracle run takes about budget_s seconds (calibrated on 16 tokens)."""
-    cal = OracleSample(w, 16)
-    cal.run()
-    per_tok = max(cal.run() / 16, 1e-7)
-    return int(max(16, min(max_tokens, budget_s / per_tok)))
+def oracle_sample_shape(w, budget_s: float):
+    """(sequences, tokens per sequence) of a sample whose oracle run takes about
+    budget_s seconds: whole sequences while they fit, else a prefix of one."""
+    n_cal = min(256, w.seqlen)
+    cal = OracleSample(w, 1, n_cal)
+    per_tok = max(cal.run() / n_cal, 1e-7)
+    want = max(16, int(budget_s / per_tok))
+    if want <= w.seqlen:
+        return 1, want
+    return max(1, min(w.batch, want // w.seqlen)), w.seqlen
 
 
-def oracle_sample_rate(w, budget_s: float, max_tokens: int):
-    """(tokens/s, T, seconds) of one oracle run sized to about budget_s seconds."""
-    T = oracle_tokens_for(w, budget_s, max_tokens)
-    secs = OracleSample(w, T).run()
-    return T / secs, T, secs
+def oracle_sample_rate(w, budget_s: float):
+    """(tokens/s, description, seconds) of one oracle run sized to about budget_s seconds."""
+    seqs, T = oracle_sample_shape(w, budget_s)
+    smp = OracleSample(w, seqs, T)
+    secs = smp.run()
+    return smp.tokens / secs, f"{seqs} sequence(s) x {T} tokens", secs
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -408,20 +418,20 @@ def main():
         # The reference arm is the fp64 oracle as it stands, on this host's cores:
         # each step is a bounded sample of the workload (first T tokens, every layer).
         per_step_budget = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-        T = oracle_tokens_for(w, per_step_budget, w.seqlen)
-        sample = OracleSample(w, T)
+        seqs, T = oracle_sample_shape(w, per_step_budget)
+        sample = OracleSample(w, seqs, T)
         for _ in range(args.warmup):
             sample.run()
         secs = [sample.run() for _ in range(args.steps)]
-        value = T * args.steps / sum(secs)
+        value = sample.tokens * args.steps / sum(secs)
         line = {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(secs) / len(secs), 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "impl": "reference",
-                "config": {"workload": w.name, "sample_tokens_per_step": T},
+                "config": {"workload": w.name, "sample_tokens_per_step": sample.tokens},
                 "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores_used(),
                                  "kind": "oracle",
-                                 "sample": f"fp64 oracle fwd+bwd on the first {T} tokens of one sequence of "
+                                 "sample": f"fp64 oracle fwd+bwd on {seqs} sequence(s) x {T} tokens of "
                                            f"{w.name}, every layer, per step"},
                 "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -441,11 +451,11 @@ def main():
             dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            rate, T, secs = oracle_sample_rate(w, args.cpu_budget, w.seqlen)
+            rate, desc, secs = oracle_sample_rate(w, args.cpu_budget)
             line["cpu_baseline"] = {"value": round(rate, 2), "unit": "tokens/s", "cores": cores_used(),
                                     "kind": "oracle",
-                                    "sample": f"fp64 oracle fwd+bwd on the first {T} tokens of one sequence "
-                                              f"of {w.name}, every layer ({secs:.1f} s)"}
+                                    "sample": f"fp64 oracle fwd+bwd on {desc} of {w.name}, every layer "
+                                              f"({secs:.1f} s)"}
         print(json.dumps(line), flush=True)
     return 0
 

@@ -93,7 +93,8 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream, ref: torch.Tensor):
     if stream is not None:
         return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
-    return ctypes.c_void_p(torch.cuda.current_stream(ref.device).cuda_stream)
+    dev = ref.device if ref is not None and ref.device.type == "cuda" else None
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
 def _check(status: int):

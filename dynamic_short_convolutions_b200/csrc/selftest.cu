@@ -19,6 +19,7 @@ constexpr int kSelftestSmem = 1024 + 49152 + 98304;
 
 // variant 0: A [128][Kd] and B [N][Kd], both K-major, Kd in {64, 128, 192}.
 // variant 1: A stored [Kd][128] and B stored [Kd][N], both MN-major, Kd in {16, ..., 128}.
+// variant 2: A [128][64] K-major and B stored [64][N] MN-major (Kd = 64).
 __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ CUtensorMap ta,
                                                        const __grid_constant__ CUtensorMap tb, int variant, int N,
                                                        int Kd, float* __restrict__ D, uint32_t* err) {
@@ -51,6 +52,11 @@ __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ C
             mbar_arrive_expect_tx(&bar_load, uint32_t(na * (128 * 128 + N * 128)));
             for (int a = 0; a < na; ++a) tma_load_2d(sa + a * 16384, &ta, &bar_load, 64 * a, 0);
             for (int a = 0; a < na; ++a) tma_load_2d(sb + a * N * 128, &tb, &bar_load, 64 * a, 0);
+        } else if (variant == 2) {
+            const int nb = (N + 63) / 64;
+            mbar_arrive_expect_tx(&bar_load, uint32_t(128 * 128 + nb * 64 * 128));
+            tma_load_2d(sa, &ta, &bar_load, 0, 0);
+            for (int a = 0; a < nb; ++a) tma_load_2d(sb + a * 64 * 128, &tb, &bar_load, 64 * a, 0);
         } else {
             const int nb = (N + 63) / 64;
             mbar_arrive_expect_tx(&bar_load, uint32_t((2 + nb) * Kd * 128));
@@ -60,13 +66,16 @@ __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ C
         ok = mbar_wait(&bar_load, 0, &abort_flag, err);
         if (ok) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, N, variant == 1, variant == 1);
+            const uint32_t idesc = idesc_bf16(128, N, variant == 1, variant >= 1);
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             if (variant == 0) {
                 for (int kb = 0; kb < Kd / 64; ++kb)
                     for (int k = 0; k < 4; ++k)
                         umma_bf16(tbase, kmajor_desc(a0 + kb * 16384, k), kmajor_desc(b0 + kb * N * 128, k), idesc,
                                   (kb | k) != 0);
+            } else if (variant == 2) {
+                for (int k = 0; k < 4; ++k)
+                    umma_bf16(tbase, kmajor_desc(a0, k), mnmajor_desc(b0, 64 * 128, k * 16), idesc, k != 0);
             } else {
                 for (int ks = 0; ks < Kd / 16; ++ks)
                     umma_bf16(tbase, mnmajor_desc(a0, Kd * 128, ks * 16), mnmajor_desc(b0, Kd * 128, ks * 16),
@@ -103,13 +112,16 @@ extern "C" DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const v
                                                             int N, int Kd, void* err_word, void* stream) {
     if (variant == 0 && !(Kd == 64 || Kd == 128 || Kd == 192)) return DYNCONV_ERR_INVALID;
     if (variant == 1 && !(Kd >= 16 && Kd <= 128 && Kd % 16 == 0)) return DYNCONV_ERR_INVALID;
-    if (variant != 0 && variant != 1) return DYNCONV_ERR_INVALID;
+    if (variant == 2 && Kd != 64) return DYNCONV_ERR_INVALID;
+    if (variant < 0 || variant > 2) return DYNCONV_ERR_INVALID;
     if (N < 16 || N > 256 || N % 16) return DYNCONV_ERR_INVALID;
     if (!A || !B || !D || !err_word) return DYNCONV_ERR_INVALID;
     CUtensorMap ta, tb;
     bool ok;
     if (variant == 0)
         ok = make_tmap_bf16(&ta, A, Kd, 128, Kd, 64, 128) && make_tmap_bf16(&tb, B, Kd, N, Kd, 64, N);
+    else if (variant == 2)
+        ok = make_tmap_bf16(&ta, A, 64, 128, 64, 64, 128) && make_tmap_bf16(&tb, B, N, 64, N, 64, 64);
     else
         ok = make_tmap_bf16(&ta, A, 128, Kd, 128, 64, Kd) && make_tmap_bf16(&tb, B, N, Kd, N, 64, Kd);
     if (!ok) return DYNCONV_ERR_CUDA;

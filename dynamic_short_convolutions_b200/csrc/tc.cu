@@ -1,13 +1,444 @@
-// tc.cu -- tcgen05 / TMA tensor-core kernels (bf16 storage).  Placeholder until written.
+// tc.cu -- tensor-core (tcgen05 + TMA) kernels for bf16 dynamic short convolutions.
+//
+// Forward, low-rank ("Dynamic Short Convolutions Improve Transformers",
+// gist.science technical summary: "Parameterization" 1 and the "Fused Low-Rank
+// Kernel" paragraph of "Efficient Training Implementation"):
+//   gen_kernel         z = h A                        (M = 128 tokens, N = r, K = d)
+//   lowrank_fwd_kernel per (128-token tile, 64-channel chunk):
+//                      W = z B_chunk  -> TMEM        (M = 128, N = 64 K, K = r)
+//                      y = u + sum_j W[:, c K + j] u[t - j, c]  (epilogue, CUDA cores)
+//                      the [N, C, K] filter lives only in TMEM and registers.
+//
+// Every kernel here is warp-specialised: warp 0 issues TMA loads, warp 1 issues
+// tcgen05.mma (one elected thread) and owns the tensor memory, warps 2-5 are the
+// epilogue (thread = token row = TMEM lane).  Shared-memory stages and TMEM
+// accumulators are handed over with mbarriers; every wait is bounded.
+#include <algorithm>
+#include <cstdio>
+
+#include "common.cuh"
 #include "internal.h"
+#include "prof.h"
+#include "tc_common.cuh"
+#include "tmap.h"
 
 namespace dynconv {
-bool tc_supported(const Prob&) { return false; }
-size_t tc_workspace_bytes(const Prob&) { return 0; }
-cudaError_t tc_forward(const Prob&, const void*, const void*, const void*, const void*, void*, void*, void*,
-                       cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t tc_backward(const Prob&, const void*, const void*, const void*, const void*, const void*,
-                        const void*, void*, void*, float*, float*, void*, cudaStream_t) {
-    return cudaErrorNotSupported;
+namespace {
+
+using namespace tc;
+
+constexpr int kTcThreads = 192;   // 6 warps
+
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Barrier over the 128 epilogue threads that also ORs a predicate across them, so
+// that a bounded wait giving up in one warp makes every epilogue warp leave its
+// loop at the same point (no thread is left waiting at a named barrier).
+__device__ __forceinline__ bool epi_bar_any(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, 2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred))
+        : "memory");
+    return r != 0;
 }
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+__host__ __device__ inline uint32_t tmem_cols_for(int cols) {
+    uint32_t c = 32;
+    while (c < (uint32_t)cols) c <<= 1;
+    return c;
+}
+
+// =====================================================================================
+// gen_kernel: X[N, R] = h[N, d] . P[d, R]   (z = h A; bf16 out), R <= 256.
+//   A operand: h tile [128 tokens][64 of d], K-major (TMA box {64, 128}).
+//   B operand: P tile [64 rows of d][64 of R] per 64-wide atom, MN-major (box {64, 64}).
+// =====================================================================================
+constexpr int kGenStages = 4;
+
+struct GenArgs {
+    int64_t N, d;
+    int R, NB, NMMA;   // output width, P atoms per stage, MMA N
+    int64_t out_ld;
+    uint32_t* err;
+};
+
+template <typename OutT>
+__global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constant__ CUtensorMap tm_h,
+                                                            const __grid_constant__ CUtensorMap tm_p,
+                                                            OutT* __restrict__ out, GenArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    const uint32_t stage_bytes = 16384u + a.NB * 8192u;
+    __shared__ uint64_t full[kGenStages], empty[kGenStages], tfull[2], tempty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_tiles = (a.N + 127) / 128;
+    const int nk = (int)((a.d + 63) / 64);
+    const uint32_t tcols = tmem_cols_for(2 * a.NMMA);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGenStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch(&tm_h);
+        tma_prefetch(&tm_p);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kGenStages;
+                    const uint32_t ph = (it / kGenStages) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, a.err)) break;
+                    uint8_t* st = sm + s * stage_bytes;
+                    mbar_arrive_expect_tx(&full[s], stage_bytes);
+                    tma_load_2d(st, &tm_h, &full[s], 64 * kb, (int32_t)(tile * 128));
+                    for (int b = 0; b < a.NB; ++b) tma_load_2d(st + 16384 + b * 8192, &tm_p, &full[s], 64 * b, 64 * kb);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, a.NMMA, false, true);
+            uint32_t it = 0, t = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++t) {
+                const int b = t & 1;
+                if (!mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                tc_fence_after();
+                const uint32_t dcol = tbase + b * a.NMMA;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kGenStages;
+                    const uint32_t ph = (it / kGenStages) & 1;
+                    if (!mbar_wait(&full[s], ph, &abort_flag, a.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(sm + s * stage_bytes);
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16(dcol, kmajor_desc(st, k), mnmajor_desc(st + 16384, 8192, 16 * k), idesc,
+                                  (kb | k) != 0);
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&tfull[b]);
+            }
+        }
+    } else {
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;
+        uint32_t t = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++t) {
+            const int b = t & 1;
+            if (!mbar_wait(&tfull[b], (t >> 1) & 1, &abort_flag, a.err)) break;
+            tc_fence_after();
+            const int64_t n = tile * 128 + row;
+            const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * a.NMMA;
+            for (int c = 0; c < a.R; c += 8) {
+                uint32_t v[8];
+                tmem_ld8(taddr + c, v);
+                tmem_wait_ld();
+                if (n < a.N) {
+                    if constexpr (sizeof(OutT) == 2) {
+                        uint4 pk;
+                        pk.x = pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                        pk.y = pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                        pk.z = pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                        pk.w = pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                        *reinterpret_cast<uint4*>(out + n * a.out_ld + c) = pk;
+                    } else {
+                        float4* o = reinterpret_cast<float4*>(out + n * a.out_ld + c);
+                        o[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                           __uint_as_float(v[3]));
+                        o[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                           __uint_as_float(v[7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, tcols);
+    }
+}
+
+// =====================================================================================
+// lowrank_fwd_kernel<K>: one work item = (128-token tile m0, 64-channel chunk c0).
+//   stage smem: z tile [128][64] (K-major A) | B chunk as K atoms [64 r-rows][64] (MN-major B)
+//               | u tile [136 rows = m0-8 .. m0+127][64 channels]
+//   TMEM: W[128 tokens][64 K] fp32, column c K + j = w[m0 + row, c0 + c, j]; two buffers.
+//   epilogue: y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c] -> bf16 staging
+//             (128-byte swizzled) -> TMA store.
+// =====================================================================================
+struct FwdArgs {
+    int64_t N, C, seqlen, n_docs;
+    const int32_t* cu;
+    uint32_t* err;
+};
+
+constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
+
+template <int K>
+constexpr uint32_t fwd_stage_bytes() { return kZBytes + K * 8192 + kUBytes; }
+template <int K>
+constexpr uint32_t fwd_smem_bytes() { return 1024 + 2 * fwd_stage_bytes<K>() + 2 * kYBytes; }
+
+template <int K>
+__global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                                    const __grid_constant__ CUtensorMap tm_b,
+                                                                    const __grid_constant__ CUtensorMap tm_u,
+                                                                    const __grid_constant__ CUtensorMap tm_y,
+                                                                    FwdArgs a) {
+    constexpr uint32_t SB = fwd_stage_bytes<K>();
+    constexpr int NMMA = 64 * K;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    uint8_t* ystage = sm + 2 * SB;
+    __shared__ uint64_t full[2], empty[2], tfull[2], tempty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_tiles = (a.N + 127) / 128, n_chunks = a.C / 64;
+    const int64_t n_items = n_tiles * n_chunks;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 4);
+            mbar_init(&tfull[s], 1);
+            mbar_init(&tempty[s], 4);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch(&tm_z);
+        tma_prefetch(&tm_b);
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++it) {
+                const int64_t chunk = item / n_tiles, tile = item % n_tiles;
+                const int s = it & 1;
+                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                uint8_t* st = sm + s * SB;
+                mbar_arrive_expect_tx(&full[s], SB);
+                const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
+                tma_load_2d(st, &tm_z, &full[s], 0, m0);
+                for (int j = 0; j < K; ++j) tma_load_2d(st + kZBytes + j * 8192, &tm_b, &full[s], c0 * K + 64 * j, 0);
+                tma_load_2d(st + kZBytes + K * 8192, &tm_u, &full[s], c0, m0 - 8);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, NMMA, false, true);
+            uint32_t it = 0;
+            for (int64_t item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++it) {
+                const int s = it & 1;
+                const uint32_t ph = (it >> 1) & 1;
+                if (!mbar_wait(&tempty[s], ph ^ 1, &abort_flag, a.err)) break;
+                if (!mbar_wait(&full[s], ph, &abort_flag, a.err)) break;
+                tc_fence_after();
+                const uint32_t st = smem_u32(sm + s * SB);
+                for (int k = 0; k < 4; ++k)
+                    umma_bf16(tbase + s * 256, kmajor_desc(st, k), mnmajor_desc(st + kZBytes, 8192, 16 * k), idesc,
+                              k != 0);
+                umma_commit(&tfull[s]);
+                umma_commit(&empty[s]);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int et = threadIdx.x - 64;        // 0..127 epilogue thread index
+        uint32_t it = 0;
+        for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+            const int64_t chunk = item / n_tiles, tile = item % n_tiles;
+            const int s = it & 1;
+            const uint32_t ph = (it >> 1) & 1;
+            const bool ok = mbar_wait(&tfull[s], ph, &abort_flag, a.err) && mbar_wait(&full[s], ph, &abort_flag, a.err);
+            if (et == 0) tma_store_wait_read_le1();     // the store that last used this staging buffer
+            if (epi_bar_any(!ok)) break;
+            tc_fence_after();
+            const int64_t n = tile * 128 + row;
+            const int64_t pos = n < a.N ? n - seg_start(n, a.cu, a.n_docs, a.seqlen) : 0;
+            const uint8_t* us = sm + s * SB + kZBytes + K * 8192;
+            uint8_t* ys = ystage + s * kYBytes;
+            const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + s * 256;
+#pragma unroll 1
+            for (int g = 0; g < 8; ++g) {                 // 8 channels per group
+                uint32_t wv[8 * K];
+#pragma unroll
+                for (int i = 0; i < K; ++i) tmem_ld8(taddr + g * 8 * K + 8 * i, *reinterpret_cast<uint32_t(*)[8]>(wv + 8 * i));
+                uint4 uj[K];
+#pragma unroll
+                for (int j = 0; j < K; ++j)
+                    uj[j] = *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g));
+                tmem_wait_ld();
+                float acc[8];
+                const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    acc[c] = bf16_lo(u0[c >> 1]);
+                    acc[c + 1] = bf16_hi(u0[c >> 1]);
+                }
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    if (j <= pos) {
+                        const uint32_t* uu = reinterpret_cast<const uint32_t*>(&uj[j]);
+#pragma unroll
+                        for (int c = 0; c < 8; c += 2) {
+                            acc[c] = fmaf(__uint_as_float(wv[c * K + j]), bf16_lo(uu[c >> 1]), acc[c]);
+                            acc[c + 1] = fmaf(__uint_as_float(wv[(c + 1) * K + j]), bf16_hi(uu[c >> 1]), acc[c + 1]);
+                        }
+                    }
+                }
+                uint4 pk;
+                pk.x = pack_bf16(acc[0], acc[1]);
+                pk.y = pack_bf16(acc[2], acc[3]);
+                pk.z = pack_bf16(acc[4], acc[5]);
+                pk.w = pack_bf16(acc[6], acc[7]);
+                *reinterpret_cast<uint4*>(ys + sw128_off(row, g)) = pk;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&tempty[s]);
+                mbar_arrive(&empty[s]);
+            }
+            fence_async_smem();
+            epi_bar_sync();
+            if (et == 0) {
+                tma_store_2d(&tm_y, ys, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                tma_store_commit();
+            }
+        }
+        if (et == 0) tma_store_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+template <int K>
+cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
+                               const CUtensorMap& ty, const FwdArgs& fa, int64_t items, cudaStream_t st) {
+    constexpr uint32_t smem = fwd_smem_bytes<K>();
+    cudaError_t e = cudaFuncSetAttribute(lowrank_fwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)std::min<int64_t>(items, num_sms());
+    DC_LAUNCH(kTcLowrankFwd, st, lowrank_fwd_kernel<K><<<grid, kTcThreads, smem, st>>>(tz, tb, tu, ty, fa));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gen_bf16(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
+                            int64_t out_ld, uint32_t* err, cudaStream_t st) {
+    CUtensorMap th, tp;
+    if (!make_tmap_bf16(&th, h, d, N, hs, 64, 128) || !make_tmap_bf16(&tp, P, R, d, R, 64, 64))
+        return cudaErrorInvalidValue;
+    GenArgs ga{N, d, R, (R + 63) / 64, (R + 15) / 16 * 16, out_ld, err};
+    const int smem = 1024 + kGenStages * (16384 + ga.NB * 8192);
+    cudaError_t e = cudaFuncSetAttribute(gen_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t n_tiles = (N + 127) / 128;
+    const unsigned grid = (unsigned)std::min<int64_t>(n_tiles, num_sms());
+    DC_LAUNCH(kTcGen, st, gen_kernel<__nv_bfloat16><<<grid, kTcThreads, smem, st>>>(
+        th, tp, static_cast<__nv_bfloat16*>(out), ga));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const Prob& p) {
+    if (p.dtype != 1 || p.kind != 0) return false;
+    if (p.r % 8 != 0 || p.r > 64) return false;
+    if (p.C % 64 != 0 || p.d % 8 != 0) return false;
+    if (p.K < 1 || p.K > 4) return false;
+    return tensor_map_encoder() != nullptr;
+}
+
+size_t tc_workspace_bytes(const Prob& p) {
+    return (size_t)p.N * p.r * 2 + 256;   // z scratch when the caller passes no z buffer
+}
+
+cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
+                       void* z_save, void* ws, cudaStream_t st) {
+    const WsLayout L = ws_layout(p);
+    uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
+    void* z = z_save ? z_save : static_cast<void*>(static_cast<char*>(ws) + L.tc);
+    cudaError_t e = launch_gen_bf16(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tz, tb, tu, ty;
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
+        return cudaErrorInvalidValue;
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err};
+    const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
+    switch (p.K) {
+        case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);
+        case 2: return launch_lowrank_fwd<2>(tz, tb, tu, ty, fa, items, st);
+        case 3: return launch_lowrank_fwd<3>(tz, tb, tu, ty, fa, items, st);
+        default: return launch_lowrank_fwd<4>(tz, tb, tu, ty, fa, items, st);
+    }
+}
+
+cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A, const void* BW,
+                        const void* z_saved, void* du, void* dh, float* dA, float* dBW, void* ws, cudaStream_t st) {
+    // The tensor-core backward kernels are not written yet: the generic kernels run it.
+    return simt_backward(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, ws, st);
+}
+
 }  // namespace dynconv

@@ -18,6 +18,8 @@ extern "C" {
  *              Kd in {64, 128, 192}.
  *   variant 1: A is stored [Kd, 128] and B is stored [Kd, N] (both MN-major);
  *              Kd a multiple of 16 up to 128.
+ *   variant 2: A is [128, 64] (K-major) and B is stored [64, N] (MN-major);
+ *              Kd = 64.
  *   N: multiple of 16, 16..256.  D: [128, N] fp32, row-major.
  * All pointers are device pointers (16-byte aligned); err_word is a device
  * uint32 that receives the wait-timeout bit if the tile never completes.

@@ -61,36 +61,50 @@ def _compare(w, gpu, ref, skip=()):
         assert_close(f"{w.name}:z", gpu["z"], ref["z"], w.dtype)
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+def _run_or_skip(w, layer, t, algo, **kw):
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    try:
+        return gpu_run(w, layer, t, algo=algo, **kw)
+    except L.DynConvError as e:
+        if algo == 2 and e.status == 2:
+            pytest.skip("shape outside the tensor-core kernels' coverage")
+        raise
+
+
+ALGOS = pytest.mark.parametrize("algo", [1, 0, 2], ids=["simt", "auto", "tc"])
+
+
+@ALGOS
 @pytest.mark.parametrize("case", SMALL, ids=[c[0].name for c in SMALL])
 def test_small_parity(case, algo):
     w, li = case
     layer = w.layers[li]
     x = W.make_inputs(w, layer, li)
-    gpu = gpu_run(w, layer, _to_device(x, w), algo=algo)
+    gpu = _run_or_skip(w, layer, _to_device(x, w), algo)
     _compare(w, gpu, oracle_all(w, layer, x))
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+@ALGOS
 def test_varlen_parity(algo):
     w = _varlen_case()
     layer = w.layers[0]
     x = W.make_inputs(w, layer)
     x["cu_seqlens"] = np.array(VARLEN_CU, dtype=np.int32)
-    gpu = gpu_run(w, layer, _to_device(x, w), algo=algo)
+    gpu = _run_or_skip(w, layer, _to_device(x, w), algo)
     _compare(w, gpu, oracle_all(w, layer, x))
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+@ALGOS
 def test_recompute_z_and_no_dh(algo):
     w = _case("c2_qkv_150m_lowrank", 2, 140, "no_zsave")
     layer = w.layers[0]
     x = W.make_inputs(w, layer)
-    gpu = gpu_run(w, layer, _to_device(x, w), algo=algo, z_roundtrip=False, want_dh=False)
+    gpu = _run_or_skip(w, layer, _to_device(x, w), algo, z_roundtrip=False, want_dh=False)
     _compare(w, gpu, oracle_all(w, layer, x), skip=("dh",))
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+@ALGOS
 def test_strided_u_and_h(algo):
     """u and h as column slices of wider (fused-projection) tensors."""
     w = _case("c2_qkv_150m_lowrank", 2, 150, "strided")
@@ -103,11 +117,11 @@ def test_strided_u_and_h(algo):
     big_h = torch.zeros((N, d + 8), dtype=torch.bfloat16, device="cuda")
     big_h[:, :d] = t["h"]
     t["u"], t["h"] = big_u[:, 64:], big_h[:, :d]
-    gpu = gpu_run(w, layer, t, algo=algo)
+    gpu = _run_or_skip(w, layer, t, algo)
     _compare(w, gpu, oracle_all(w, layer, x))
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+@ALGOS
 def test_causality_and_isolation_on_gpu(algo):
     """Perturbing token t* leaves every earlier output bitwise unchanged; perturbing a
     document changes nothing outside it."""
@@ -118,7 +132,7 @@ def test_causality_and_isolation_on_gpu(algo):
     cu = np.array([0, 7, 300, 301, 600], dtype=np.int32)
     x["cu_seqlens"] = cu
     t = _to_device(x, w)
-    y0 = gpu_run(w, layer, t, algo=algo)["y"]
+    y0 = _run_or_skip(w, layer, t, algo)["y"]
     t2 = {k: v.clone() for k, v in t.items()}
     ts = 333
     t2["u"][ts] += 1.0
@@ -134,12 +148,12 @@ def test_causality_and_isolation_on_gpu(algo):
     assert np.array_equal(y3[outside], y0[outside])
 
 
-@pytest.mark.parametrize("algo", [1, 0], ids=["simt", "auto"])
+@ALGOS
 def test_deterministic_mode_is_bitwise_repeatable(algo):
     w = _case("c2_qkv_150m_lowrank", 2, 260, "det")
     layer = w.layers[0]
     t = _to_device(W.make_inputs(w, layer), w)
-    a = gpu_run(w, layer, t, algo=algo, deterministic=True)
+    a = _run_or_skip(w, layer, t, algo, deterministic=True)
     b = gpu_run(w, layer, t, algo=algo, deterministic=True)
     for k in a:
         if a[k] is not None:

@@ -6,7 +6,8 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 CASES = [(0, 64, 64), (0, 192, 64), (0, 256, 64), (0, 96, 64), (0, 192, 192), (0, 64, 128),
-         (1, 64, 64), (1, 64, 16), (1, 96, 128), (1, 256, 128), (1, 128, 32)]
+         (1, 64, 64), (1, 64, 16), (1, 96, 128), (1, 256, 128), (1, 128, 32),
+         (2, 64, 64), (2, 192, 64), (2, 256, 64), (2, 96, 64)]
 
 
 @pytest.mark.parametrize("variant,N,Kd", CASES)
@@ -18,6 +19,10 @@ def test_umma_tile(variant, N, Kd):
         A = torch.randn(128, Kd, device="cuda", generator=g).bfloat16()
         B = torch.randn(N, Kd, device="cuda", generator=g).bfloat16()
         ref = A.double() @ B.double().T
+    elif variant == 2:
+        A = torch.randn(128, Kd, device="cuda", generator=g).bfloat16()
+        B = torch.randn(Kd, N, device="cuda", generator=g).bfloat16()
+        ref = A.double() @ B.double()
     else:
         A = torch.randn(Kd, 128, device="cuda", generator=g).bfloat16()
         B = torch.randn(Kd, N, device="cuda", generator=g).bfloat16()
