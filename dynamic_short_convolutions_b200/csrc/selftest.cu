@@ -20,6 +20,9 @@ constexpr int kSelftestSmem = 1024 + 49152 + 98304;
 // variant 0: A [128][Kd] and B [N][Kd], both K-major, Kd in {64, 128, 192}.
 // variant 1: A stored [Kd][128] and B stored [Kd][N], both MN-major, Kd in {16, ..., 128}.
 // variant 2: A [128][64] K-major and B stored [64][N] MN-major (Kd = 64).
+// variant 3/4: A [136][64] K-major loaded as one 136-row tile, the operand starting
+//   `Kd` rows (1..7) into it (D = A[Kd : Kd+128] B^T), B [N][64] K-major; variant 3
+//   leaves the descriptor's base-offset field 0, variant 4 sets it from the start address.
 __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ CUtensorMap ta,
                                                        const __grid_constant__ CUtensorMap tb, int variant, int N,
                                                        int Kd, float* __restrict__ D, uint32_t* err) {
@@ -52,6 +55,10 @@ __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ C
             mbar_arrive_expect_tx(&bar_load, uint32_t(na * (128 * 128 + N * 128)));
             for (int a = 0; a < na; ++a) tma_load_2d(sa + a * 16384, &ta, &bar_load, 64 * a, 0);
             for (int a = 0; a < na; ++a) tma_load_2d(sb + a * N * 128, &tb, &bar_load, 64 * a, 0);
+        } else if (variant >= 3) {
+            mbar_arrive_expect_tx(&bar_load, uint32_t(136 * 128 + N * 128));
+            tma_load_2d(sa, &ta, &bar_load, 0, 0);
+            tma_load_2d(sb, &tb, &bar_load, 0, 0);
         } else if (variant == 2) {
             const int nb = (N + 63) / 64;
             mbar_arrive_expect_tx(&bar_load, uint32_t(128 * 128 + nb * 64 * 128));
@@ -66,13 +73,20 @@ __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ C
         ok = mbar_wait(&bar_load, 0, &abort_flag, err);
         if (ok) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, N, variant == 1, variant >= 1);
+            const uint32_t idesc = idesc_bf16(128, N, variant == 1, variant == 1 || variant == 2);
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             if (variant == 0) {
                 for (int kb = 0; kb < Kd / 64; ++kb)
                     for (int k = 0; k < 4; ++k)
                         umma_bf16(tbase, kmajor_desc(a0 + kb * 16384, k), kmajor_desc(b0 + kb * N * 128, k), idesc,
                                   (kb | k) != 0);
+            } else if (variant >= 3) {
+                const uint32_t start = a0 + 128u * Kd;
+                for (int k = 0; k < 4; ++k) {
+                    uint64_t da = kmajor_desc(start, k);
+                    if (variant == 4) da |= uint64_t(((start + 32u * k) >> 7) & 7u) << 49;
+                    umma_bf16(tbase, da, kmajor_desc(b0, k), idesc, k != 0);
+                }
             } else if (variant == 2) {
                 for (int k = 0; k < 4; ++k)
                     umma_bf16(tbase, kmajor_desc(a0, k), mnmajor_desc(b0, 64 * 128, k * 16), idesc, k != 0);
@@ -113,7 +127,8 @@ extern "C" DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const v
     if (variant == 0 && !(Kd == 64 || Kd == 128 || Kd == 192)) return DYNCONV_ERR_INVALID;
     if (variant == 1 && !(Kd >= 16 && Kd <= 128 && Kd % 16 == 0)) return DYNCONV_ERR_INVALID;
     if (variant == 2 && Kd != 64) return DYNCONV_ERR_INVALID;
-    if (variant < 0 || variant > 2) return DYNCONV_ERR_INVALID;
+    if (variant >= 3 && !(Kd >= 1 && Kd <= 7)) return DYNCONV_ERR_INVALID;
+    if (variant < 0 || variant > 4) return DYNCONV_ERR_INVALID;
     if (N < 16 || N > 256 || N % 16) return DYNCONV_ERR_INVALID;
     if (!A || !B || !D || !err_word) return DYNCONV_ERR_INVALID;
     CUtensorMap ta, tb;
@@ -122,6 +137,8 @@ extern "C" DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const v
         ok = make_tmap_bf16(&ta, A, Kd, 128, Kd, 64, 128) && make_tmap_bf16(&tb, B, Kd, N, Kd, 64, N);
     else if (variant == 2)
         ok = make_tmap_bf16(&ta, A, 64, 128, 64, 64, 128) && make_tmap_bf16(&tb, B, N, 64, N, 64, 64);
+    else if (variant >= 3)
+        ok = make_tmap_bf16(&ta, A, 64, 136, 64, 64, 136) && make_tmap_bf16(&tb, B, 64, N, 64, 64, N);
     else
         ok = make_tmap_bf16(&ta, A, 128, Kd, 128, 64, Kd) && make_tmap_bf16(&tb, B, N, Kd, N, 64, Kd);
     if (!ok) return DYNCONV_ERR_CUDA;

@@ -20,6 +20,10 @@ extern "C" {
  *              Kd a multiple of 16 up to 128.
  *   variant 2: A is [128, 64] (K-major) and B is stored [64, N] (MN-major);
  *              Kd = 64.
+ *   variants 3, 4: A is [136, 64] and B is [N, 64] (both K-major); the A
+ *              operand starts Kd rows (1..7) into the 136-row tile, so
+ *              D = A[Kd:Kd+128] B^T.  Variant 3 leaves the descriptor's
+ *              base-offset field 0, variant 4 sets it from the start address.
  *   N: multiple of 16, 16..256.  D: [128, N] fp32, row-major.
  * All pointers are device pointers (16-byte aligned); err_word is a device
  * uint32 that receives the wait-timeout bit if the tile never completes.
