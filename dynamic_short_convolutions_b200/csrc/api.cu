@@ -192,8 +192,8 @@ dynconv_status dynconv_bwd(const dynconv_desc* desc, const int32_t* cu_seqlens, 
         p.cu = cu_seqlens;
         p.n_docs = n_docs;
     }
-    if (desc->algo == DYNCONV_ALGO_TC && !tc_supported(p)) {
-        set_error("the tensor-core kernels do not cover this shape/dtype");
+    if (desc->algo == DYNCONV_ALGO_TC && !tc_supported_bwd(p)) {
+        set_error("the tensor-core kernels do not cover this shape/dtype/mode");
         return DYNCONV_ERR_UNSUPPORTED;
     }
     if ((s = check_ptr(dA, "dA", p.kind == 0)) || (s = check_ptr(dB_or_dW, "dB_or_dW", true))) return s;
@@ -215,7 +215,7 @@ dynconv_status dynconv_bwd(const dynconv_desc* desc, const int32_t* cu_seqlens, 
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
     if (cu_seqlens && (s = cuda_status(launch_check_seqlens(cu_seqlens, n_docs, p.N, err, st), "cu_seqlens check")))
         return s;
-    cudaError_t e = use_tc(p, desc->algo)
+    cudaError_t e = (desc->algo != DYNCONV_ALGO_SIMT && tc_supported_bwd(p))
                         ? tc_backward(p, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or_dW, ws, st)
                         : simt_backward(p, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or_dW, ws, st);
     return cuda_status(e, "backward launch");

@@ -38,4 +38,25 @@ __device__ __forceinline__ int64_t seg_start(int64_t n, const int32_t* __restric
     return s > n ? n : s;
 }
 
+// Start s (first token) and end e (one past the last token) of the sequence /
+// packed document holding token n < N, clamped so that s <= n < e <= N whatever
+// cu_seqlens holds.
+__device__ __forceinline__ void seg_bounds(int64_t n, const int32_t* __restrict__ cu, int64_t n_docs,
+                                           int64_t seqlen, int64_t N, int64_t& s, int64_t& e) {
+    if (cu == nullptr) {
+        s = (n / seqlen) * seqlen;
+        e = s + seqlen;
+    } else {
+        int64_t lo = 0, hi = n_docs;
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if ((int64_t)__ldg(cu + mid) <= n) lo = mid; else hi = mid;
+        }
+        s = (int64_t)__ldg(cu + lo);
+        e = (int64_t)__ldg(cu + lo + 1);
+    }
+    s = s < 0 ? 0 : (s > n ? n : s);
+    e = e <= n ? n + 1 : (e > N ? N : e);
+}
+
 }  // namespace dynconv

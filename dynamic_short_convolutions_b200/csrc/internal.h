@@ -40,7 +40,8 @@ struct WsLayout {
 
 WsLayout ws_layout(const Prob& p);
 size_t tc_workspace_bytes(const Prob& p);
-bool tc_supported(const Prob& p);
+bool tc_supported(const Prob& p);      // forward
+bool tc_supported_bwd(const Prob& p);  // backward
 
 // Generic CUDA-core kernels (any shape, fp32 or bf16 storage).
 cudaError_t simt_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW,

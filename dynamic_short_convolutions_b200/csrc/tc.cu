@@ -29,45 +29,6 @@ using namespace tc;
 
 constexpr int kTcThreads = 192;   // 6 warps
 
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// Barrier over the 128 epilogue threads that also ORs a predicate across them, so
-// that a bounded wait giving up in one warp makes every epilogue warp leave its
-// loop at the same point (no thread is left waiting at a named barrier).
-__device__ __forceinline__ bool epi_bar_any(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.or.pred q, 2, 128, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(uint32_t(pred))
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
-__host__ __device__ inline uint32_t tmem_cols_for(int cols) {
-    uint32_t c = 32;
-    while (c < (uint32_t)cols) c <<= 1;
-    return c;
-}
-
 // =====================================================================================
 // gen_kernel: X[N, R] = h[N, d] . P[d, R]   (z = h A; bf16 out), R <= 256.
 //   A operand: h tile [128 tokens][64 of d], K-major (TMA box {64, 128}).
@@ -384,8 +345,10 @@ cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, con
     return cudaGetLastError();
 }
 
-cudaError_t launch_gen_bf16(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
-                            int64_t out_ld, uint32_t* err, cudaStream_t st) {
+}  // namespace
+
+cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
+                          int64_t out_ld, uint32_t* err, cudaStream_t st) {
     CUtensorMap th, tp;
     if (!make_tmap_bf16(&th, h, d, N, hs, 64, 128) || !make_tmap_bf16(&tp, P, R, d, R, 64, 64))
         return cudaErrorInvalidValue;
@@ -400,7 +363,15 @@ cudaError_t launch_gen_bf16(const void* h, int64_t hs, const void* P, int64_t N,
     return cudaGetLastError();
 }
 
-}  // namespace
+struct TcBwdLayout {
+    size_t zs, bp, dz, dzb, dbpart, dpart, total;
+    int64_t per_cta, n_items, n_tiles;
+    int pieces, grid, n_dblk, n_split;
+};
+TcBwdLayout tc_bwd_layout(const Prob& p);
+cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
+                                const void* B, const void* z_saved, void* du, void* dh, float* dA, float* dB,
+                                char* tcws, uint32_t* err, cudaStream_t st);
 
 bool tc_supported(const Prob& p) {
     if (p.dtype != 1 || p.kind != 0) return false;
@@ -410,16 +381,20 @@ bool tc_supported(const Prob& p) {
     return tensor_map_encoder() != nullptr;
 }
 
-size_t tc_workspace_bytes(const Prob& p) {
-    return (size_t)p.N * p.r * 2 + 256;   // z scratch when the caller passes no z buffer
+bool tc_supported_bwd(const Prob& p) {
+    // The backward reduces dz over channel chunks with fp32 atomics; the
+    // deterministic mode takes the generic kernels instead.
+    return tc_supported(p) && !p.deterministic;
 }
+
+size_t tc_workspace_bytes(const Prob& p) { return tc_bwd_layout(p).total; }
 
 cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
                        void* z_save, void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
     void* z = z_save ? z_save : static_cast<void*>(static_cast<char*>(ws) + L.tc);
-    cudaError_t e = launch_gen_bf16(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
+    cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
     if (e != cudaSuccess) return e;
     CUtensorMap tz, tb, tu, ty;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
@@ -437,8 +412,9 @@ cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* 
 
 cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A, const void* BW,
                         const void* z_saved, void* du, void* dh, float* dA, float* dBW, void* ws, cudaStream_t st) {
-    // The tensor-core backward kernels are not written yet: the generic kernels run it.
-    return simt_backward(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, ws, st);
+    const WsLayout L = ws_layout(p);
+    uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
+    return tc_lowrank_backward(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, static_cast<char*>(ws) + L.tc, err, st);
 }
 
 }  // namespace dynconv

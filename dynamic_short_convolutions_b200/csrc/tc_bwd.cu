@@ -1,0 +1,652 @@
+// tc_bwd.cu -- tensor-core (tcgen05 + TMA) backward of the low-rank dynamic short
+// convolution, bf16 storage, fp32 accumulation.
+//
+// The adjoint of y[t,c] = u[t,c] + sum_{j<K, t-j >= s(t)} w[t,c,j] u[t-j,c] with
+// w[t,c,j] = sum_k z[t,k] B[k,c K + j] and z = h A ("Dynamic Short Convolutions
+// Improve Transformers", gist.science technical summary, "Dynamic Short
+// Convolutions": Mechanism, Parameterization 1, Placement), for upstream g = dL/dy:
+//   du[t,c]    = g[t,c] + sum_{j<K, t+j < e(t)} w[t+j,c,j] g[t+j,c]
+//   dw[t,c,j]  = g[t,c] u[t-j,c]                      (t-j >= s(t), else 0)
+//   dz[t,k]    = sum_{c,j} dw[t,c,j] B[k,c K + j]
+//   dB[k,cK+j] = sum_t z[t,k] dw[t,c,j]
+//   dA = h^T dz,  dh = dz A^T
+// where s(t) / e(t) are the first / one-past-last token of t's sequence or document.
+//
+// Kernels
+//   permute_b_kernel   B [r, C K] -> Bp [r, K C] tap-major (Bp[k, j C + c] = B[k, c K + j]).
+//   lowrank_bwd_kernel one CTA per contiguous run of (64-channel chunk, 128-token tile)
+//                      work items, chunk-major, so the chunk's Bp stays in shared memory
+//                      and dB for the chunk accumulates in TMEM across the run:
+//       MMA1  Wd_j[t, c] = sum_k z[t+j, k] Bp[k, j C + c]   (the filter of token t+j:
+//             the z tile is loaded with 8 rows of look-ahead and the A operand starts
+//             j rows into it), so du needs no exchange between threads;
+//       epi A du (-> TMA store) and dw (-> bf16 tile in shared memory, 64 channels per tap);
+//       MMA2  dz  = dW Bp_chunk^T      (M = 128 tokens, N = r, K = 64 K)
+//       MMA3  dBt += dW^T z            (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
+//       epi B dz -> fp32 atomic add into a [N, r] buffer (reduction over chunks);
+//       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
+//   reduce_dB_kernel   sums the partials of each chunk in run order -> dB [r, C K] fp32.
+//   dz_to_bf16_kernel  fp32 dz -> bf16 operand for the generator backward.
+//   gen_bwd_kernel     dh = dz A^T (M = 128 tokens, N = 256 of d, K = r) and
+//                      dA += h^T dz (M = 128 of d, N = r, K = 128 tokens) per (256-wide d
+//                      block, token range); reduce_dA_kernel sums the token ranges.
+#include <algorithm>
+#include <cstdio>
+
+#include "common.cuh"
+#include "internal.h"
+#include "prof.h"
+#include "tc_common.cuh"
+#include "tmap.h"
+
+namespace dynconv {
+
+cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
+                          int64_t out_ld, uint32_t* err, cudaStream_t st);
+
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 192;
+constexpr uint32_t kRowTile = 136 * 128;     // 136-row, 64-column bf16 tile
+constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
+
+__global__ void permute_b_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat16* __restrict__ Bp, int64_t r,
+                                 int64_t C, int64_t K) {
+    const int64_t total = r * C * K;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t k = e / (C * K), col = e % (C * K), c = col / K, j = col % K;
+        Bp[k * C * K + j * C + c] = B[e];
+    }
+}
+
+struct BwdArgs {
+    int64_t N, C, seqlen, n_docs;
+    const int32_t* cu;
+    int r, ndz;               // rank, MMA N for dz / dB (r rounded up to 16)
+    int64_t n_tiles, n_items, per_cta;
+    int pieces;               // partial slots per chunk
+    float* dz_acc;            // [N, r] fp32, zero on entry
+    float* dB_part;           // [n_chunks][pieces][64 K][r]
+    uint32_t* err;
+};
+
+template <int K>
+struct BwdSmem {
+    static constexpr int NA = 2 * ((K + 1) / 2);            // dW atoms (padded to whole 128-row MMA blocks)
+    static constexpr uint32_t stage = 3 * kRowTile;         // z | g | u
+    static constexpr uint32_t bp = 2 * stage;
+    static constexpr uint32_t dw = bp + K * 8192;
+    static constexpr uint32_t dust = dw + NA * kAtom128;
+    static constexpr uint32_t total = dust + kAtom128 + 1024;
+};
+
+template <int K>
+__global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                                  const __grid_constant__ CUtensorMap tm_g,
+                                                                  const __grid_constant__ CUtensorMap tm_u,
+                                                                  const __grid_constant__ CUtensorMap tm_bp,
+                                                                  const __grid_constant__ CUtensorMap tm_du,
+                                                                  BwdArgs a) {
+    using S = BwdSmem<K>;
+    constexpr int NBLK = S::NA / 2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dzfull;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t i0 = (int64_t)blockIdx.x * a.per_cta;
+    const int64_t i1 = min(i0 + a.per_cta, a.n_items);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 4);
+        }
+        mbar_init(&bfull, 1);
+        mbar_init(&bempty, 1);
+        mbar_init(&wfull, 1);
+        mbar_init(&wempty, 4);
+        mbar_init(&dzfull, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch(&tm_z);
+        tma_prefetch(&tm_g);
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_bp);
+        tma_prefetch(&tm_du);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp >= 2) {
+        // dW atoms past the last tap stay zero for the whole kernel (they pad the
+        // last 128-row block of the dB MMA).
+        const int row = (warp & 3) * 32 + lane;
+        for (int at = K; at < S::NA; ++at)
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4*>(sm + S::dw + at * kAtom128 + sw128_off(row, q)) = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+    constexpr uint32_t kColDz = 256, kColDb = 320;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t prev = -1;
+            uint32_t cc = 0, it = 0;
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
+                const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
+                if (chunk != prev) {
+                    if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
+                    mbar_arrive_expect_tx(&bfull, K * 8192);
+                    for (int j = 0; j < K; ++j)
+                        tma_load_2d(sm + S::bp + j * 8192, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0);
+                    ++cc;
+                    prev = chunk;
+                }
+                const int s = it & 1;
+                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                uint8_t* st = sm + s * S::stage;
+                const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
+                mbar_arrive_expect_tx(&full[s], S::stage);
+                tma_load_2d(st, &tm_z, &full[s], 0, m0);
+                tma_load_2d(st + kRowTile, &tm_g, &full[s], c0, m0);
+                tma_load_2d(st + 2 * kRowTile, &tm_u, &full[s], c0, m0 - 8);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
+            const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
+            const uint32_t idesc_db = idesc_bf16(128, a.ndz, true, true);
+            const uint32_t bp0 = smem_u32(sm + S::bp), dw0 = smem_u32(sm + S::dw);
+            int64_t prev = -1;
+            uint32_t cc = 0, it = 0;
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
+                const int64_t chunk = item / a.n_tiles;
+                const bool first = chunk != prev;
+                const bool last = (item + 1 == i1) || ((item + 1) / a.n_tiles != chunk);
+                if (first) {
+                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
+                    ++cc;
+                    prev = chunk;
+                }
+                const int s = it & 1;
+                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) break;
+                if (!mbar_wait(&wempty, (it & 1) ^ 1, &abort_flag, a.err)) break;   // Wd free
+                tc_fence_after();
+                const uint32_t z0 = smem_u32(sm + s * S::stage);
+                // MMA1: Wd_j = z[j : j + 128] . Bp_j  (K-major A starting j rows in; MN-major B)
+#pragma unroll
+                for (int j = 0; j < K; ++j)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k), mnmajor_desc(bp0 + j * 8192, 8192, 16 * k),
+                                  idesc_w, k != 0);
+                umma_commit(&wfull);
+                if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;         // dW(it) written
+                tc_fence_after();
+                // MMA2: dz = dW . Bp^T  (both K-major, K = (tap, channel))
+#pragma unroll
+                for (int j = 0; j < K; ++j)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16(tbase + kColDz, kmajor_desc(dw0 + j * kAtom128, k), kmajor_desc(bp0 + j * 8192, k),
+                                  idesc_dz, (j | k) != 0);
+                // MMA3: dBt[blk] += dW^T . z  (both MN-major, K = 128 tokens)
+#pragma unroll
+                for (int b = 0; b < NBLK; ++b)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tbase + kColDb + 64 * b, mnmajor_desc(dw0 + 2 * b * kAtom128, kAtom128, 16 * ks),
+                                  mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
+                umma_commit(&dzfull);
+                umma_commit(&empty[s]);
+                if (last) umma_commit(&bempty);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int et = threadIdx.x - 64;
+        const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
+        uint8_t* dws = sm + S::dw;
+        uint8_t* dus = sm + S::dust;
+        uint32_t it = 0;
+        for (int64_t item = i0; item < i1; ++item, ++it) {
+            const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
+            const bool last = (item + 1 == i1) || ((item + 1) / a.n_tiles != chunk);
+            const int s = it & 1;
+            bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
+                      mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err);
+            if (et == 0) tma_store_wait_all();       // du staging and dW are free again
+            if (epi_bar_any(!ok)) break;
+            tc_fence_after();
+            const int64_t n = tile * 128 + row;
+            int64_t pos = -1, epos = -1;             // valid past / future taps of this row
+            if (n < a.N) {
+                int64_t sb, eb;
+                seg_bounds(n, a.cu, a.n_docs, a.seqlen, a.N, sb, eb);
+                pos = n - sb;
+                epos = eb - 1 - n;
+            }
+            const uint8_t* zt = sm + s * S::stage;
+            const uint8_t* gt = zt + kRowTile;
+            const uint8_t* ut = zt + 2 * kRowTile;
+            (void)zt;
+#pragma unroll 1
+            for (int g8 = 0; g8 < 8; ++g8) {
+                uint32_t wv[K][8];
+#pragma unroll
+                for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * g8, wv[j]);
+                uint4 gg[K], uu[K];
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    gg[j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g8));
+                    uu[j] = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
+                }
+                tmem_wait_ld();
+                const uint32_t* g0 = reinterpret_cast<const uint32_t*>(&gg[0]);
+                float gv[8], acc[8];
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    gv[c] = bf16_lo(g0[c >> 1]);
+                    gv[c + 1] = bf16_hi(g0[c >> 1]);
+                    acc[c] = gv[c];
+                    acc[c + 1] = gv[c + 1];
+                }
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    if (j <= epos) {
+                        const uint32_t* gj = reinterpret_cast<const uint32_t*>(&gg[j]);
+#pragma unroll
+                        for (int c = 0; c < 8; c += 2) {
+                            acc[c] = fmaf(__uint_as_float(wv[j][c]), bf16_lo(gj[c >> 1]), acc[c]);
+                            acc[c + 1] = fmaf(__uint_as_float(wv[j][c + 1]), bf16_hi(gj[c >> 1]), acc[c + 1]);
+                        }
+                    }
+                }
+                uint4 pk;
+                pk.x = pack_bf16(acc[0], acc[1]);
+                pk.y = pack_bf16(acc[2], acc[3]);
+                pk.z = pack_bf16(acc[4], acc[5]);
+                pk.w = pack_bf16(acc[6], acc[7]);
+                *reinterpret_cast<uint4*>(dus + sw128_off(row, g8)) = pk;
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    const bool v = j <= pos;
+                    const uint32_t* uj = reinterpret_cast<const uint32_t*>(&uu[j]);
+                    float d[8];
+#pragma unroll
+                    for (int c = 0; c < 8; c += 2) {
+                        d[c] = v ? gv[c] * bf16_lo(uj[c >> 1]) : 0.f;
+                        d[c + 1] = v ? gv[c + 1] * bf16_hi(uj[c >> 1]) : 0.f;
+                    }
+                    uint4 dk;
+                    dk.x = pack_bf16(d[0], d[1]);
+                    dk.y = pack_bf16(d[2], d[3]);
+                    dk.z = pack_bf16(d[4], d[5]);
+                    dk.w = pack_bf16(d[6], d[7]);
+                    *reinterpret_cast<uint4*>(dws + j * kAtom128 + sw128_off(row, g8)) = dk;
+                }
+            }
+            tc_fence_before();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&wempty);
+                mbar_arrive(&empty[s]);
+            }
+            epi_bar_sync();
+            if (et == 0) {
+                tma_store_2d(&tm_du, dus, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                tma_store_commit();
+            }
+            ok = mbar_wait(&dzfull, it & 1, &abort_flag, a.err);
+            if (epi_bar_any(!ok)) break;
+            tc_fence_after();
+            // epilogue B: dz rows -> fp32 atomic add (reduction over channel chunks)
+            for (int c = 0; c < a.r; c += 8) {
+                uint32_t v[8];
+                tmem_ld8(lane_base + kColDz + c, v);
+                tmem_wait_ld();
+                if (n < a.N) {
+                    float4* dst = reinterpret_cast<float4*>(a.dz_acc + n * a.r + c);
+                    atomicAdd(dst, make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                               __uint_as_float(v[3])));
+                    atomicAdd(dst + 1, make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]),
+                                                   __uint_as_float(v[6]), __uint_as_float(v[7])));
+                }
+            }
+            // epilogue C: the run for this chunk ends here -> dB partial of this run
+            if (last) {
+                const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
+                float* part = a.dB_part + ((chunk * a.pieces + piece) * (64 * K)) * a.r;
+#pragma unroll
+                for (int b = 0; b < NBLK; ++b) {
+                    const int m = b * 128 + row;     // (tap, channel) row = j * 64 + c
+                    for (int c = 0; c < a.r; c += 8) {
+                        uint32_t v[8];
+                        tmem_ld8(lane_base + kColDb + 64 * b + c, v);
+                        tmem_wait_ld();
+                        if (m < 64 * K) {
+                            float4* dst = reinterpret_cast<float4*>(part + (int64_t)m * a.r + c);
+                            dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                                 __uint_as_float(v[3]));
+                            dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                                 __uint_as_float(v[7]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+        if (et == 0) tma_store_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+// dB[k, c K + j] = sum over the runs covering chunk c/64, in run order.
+__global__ void reduce_dB_kernel(const float* __restrict__ part, float* __restrict__ dB, int64_t r, int64_t C,
+                                 int64_t K, int64_t n_tiles, int64_t per_cta, int pieces) {
+    const int64_t total = r * C * K;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t k = e / (C * K), col = e % (C * K), c = col / K, j = col % K;
+        const int64_t chunk = c / 64, m = j * 64 + (c % 64);
+        const int64_t first = (chunk * n_tiles) / per_cta, lastc = ((chunk + 1) * n_tiles - 1) / per_cta;
+        float acc = 0.f;
+        for (int64_t p = 0; p <= lastc - first; ++p)
+            acc += part[((chunk * pieces + p) * (64 * K) + m) * r + k];
+        dB[e] = acc;
+    }
+}
+
+__global__ void dz_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t count) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+// =====================================================================================
+// gen_bwd_kernel: per (256-wide block db of d, token range):
+//   dh[t, db*256 + i] = sum_k X[t, k] P[db*256 + i, k]          (X = dz or dwh, P = A or W)
+//   dPpart[split][db*256 + i, k] = sum_{t in range} h[t, db*256 + i] X[t, k]
+// smem: stage = X tile [128][64] (K-major A of dh; MN-major B of dP) + h tile 4 atoms
+//       [128 tokens][64 of d] (MN-major A of dP); P block [256 of d][64] resident (K-major B of dh).
+// TMEM: dh [128][256] at column 0, dP blocks [128][R] at 256 and 320... (two blocks of 128 rows of d).
+// =====================================================================================
+struct GenBwdArgs {
+    int64_t N, d;
+    int R, ndz;
+    int64_t hs;
+    int n_dblk, n_split;
+    int64_t n_tiles;
+    __nv_bfloat16* dh;        // nullable
+    float* dP_part;           // [n_split][d][R]
+    uint32_t* err;
+};
+
+constexpr uint32_t kGbStage = kAtom128 + 4 * kAtom128;     // X tile + 4 h atoms
+constexpr uint32_t kGbSmem = 2 * kGbStage + 256 * 128 + 1024;   // + resident P block (256 rows x 128 B)
+
+__global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                              const __grid_constant__ CUtensorMap tm_h,
+                                                              const __grid_constant__ CUtensorMap tm_p,
+                                                              GenBwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    uint8_t* pblk = sm + 2 * kGbStage;                       // 256 rows x 128 B = 32 KB
+    __shared__ uint64_t full[2], empty[2], pfull, hfull, hempty, dpfull;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int db = blockIdx.x % a.n_dblk, split = blockIdx.x / a.n_dblk;
+    const int64_t t0 = (a.n_tiles * split) / a.n_split, t1 = (a.n_tiles * (split + 1)) / a.n_split;
+    const bool want_dh = a.dh != nullptr;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&pfull, 1);
+        mbar_init(&hfull, 1);
+        mbar_init(&hempty, 4);
+        mbar_init(&dpfull, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch(&tm_x);
+        tma_prefetch(&tm_h);
+        tma_prefetch(&tm_p);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+    constexpr uint32_t kColDp = 256;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&pfull, 256 * 128);
+            tma_load_2d(pblk, &tm_p, &pfull, 0, db * 256);
+            uint32_t it = 0;
+            for (int64_t tile = t0; tile < t1 && !abort_flag; ++tile, ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                uint8_t* st = sm + s * kGbStage;
+                mbar_arrive_expect_tx(&full[s], kGbStage);
+                tma_load_2d(st, &tm_x, &full[s], 0, (int32_t)(tile * 128));
+                for (int at = 0; at < 4; ++at)
+                    tma_load_2d(st + kAtom128 * (1 + at), &tm_h, &full[s], db * 256 + 64 * at, (int32_t)(tile * 128));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc_dh = idesc_bf16(128, 256, false, false);
+            const uint32_t idesc_dp = idesc_bf16(128, a.ndz, true, true);
+            const uint32_t p0 = smem_u32(pblk);
+            bool ok = mbar_wait(&pfull, 0, &abort_flag, a.err);
+            uint32_t it = 0;
+            for (int64_t tile = t0; ok && tile < t1 && !abort_flag; ++tile, ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) break;
+                tc_fence_after();
+                const uint32_t x0 = smem_u32(sm + s * kGbStage), h0 = x0 + kAtom128;
+                if (want_dh) {
+                    if (!mbar_wait(&hempty, (it & 1) ^ 1, &abort_flag, a.err)) break;
+                    tc_fence_after();
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16(tbase, kmajor_desc(x0, k), kmajor_desc(p0, k), idesc_dh, k != 0);
+                    umma_commit(&hfull);
+                }
+                for (int b = 0; b < 2; ++b)
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tbase + kColDp + 64 * b, mnmajor_desc(h0 + 2 * b * kAtom128, kAtom128, 16 * ks),
+                                  mnmajor_desc(x0, kAtom128, 16 * ks), idesc_dp, !(tile == t0 && ks == 0));
+                umma_commit(&empty[s]);
+            }
+            umma_commit(&dpfull);     // every dP MMA of this CTA has completed
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
+        uint32_t it = 0;
+        bool ok = true;
+        if (want_dh) {
+            for (int64_t tile = t0; tile < t1; ++tile, ++it) {
+                ok = mbar_wait(&hfull, it & 1, &abort_flag, a.err);
+                if (epi_bar_any(!ok)) break;
+                tc_fence_after();
+                const int64_t n = tile * 128 + row;
+                for (int c = 0; c < 256; c += 8) {
+                    uint32_t v[8];
+                    tmem_ld8(lane_base + c, v);
+                    tmem_wait_ld();
+                    const int64_t col = (int64_t)db * 256 + c;
+                    if (n < a.N && col < a.d) {
+                        uint4 pk;
+                        pk.x = pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                        pk.y = pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                        pk.z = pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                        pk.w = pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                        *reinterpret_cast<uint4*>(a.dh + n * a.d + col) = pk;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&hempty);
+            }
+        }
+        if (ok && t1 > t0) ok = mbar_wait(&dpfull, 0, &abort_flag, a.err);
+        if (!epi_bar_any(!ok) && t1 > t0) {
+            tc_fence_after();
+            float* part = a.dP_part + (int64_t)split * a.d * a.R;
+            for (int b = 0; b < 2; ++b) {
+                const int64_t drow = (int64_t)db * 256 + b * 128 + row;
+                for (int c = 0; c < a.R; c += 8) {
+                    uint32_t v[8];
+                    tmem_ld8(lane_base + kColDp + 64 * b + c, v);
+                    tmem_wait_ld();
+                    if (drow < a.d) {
+                        float4* dst = reinterpret_cast<float4*>(part + drow * a.R + c);
+                        dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                             __uint_as_float(v[3]));
+                        dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                             __uint_as_float(v[7]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+__global__ void reduce_splits_kernel(const float* __restrict__ part, float* __restrict__ out, int64_t count,
+                                     int n_split) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < n_split; ++s) acc += part[s * count + i];
+        out[i] = acc;
+    }
+}
+
+inline unsigned grid_for(int64_t n, int threads = 256) {
+    const int64_t b = (n + threads - 1) / threads;
+    return (unsigned)std::max<int64_t>(1, std::min<int64_t>(b, 148 * 16));
+}
+
+template <int K>
+cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
+                       const CUtensorMap& tdu, const BwdArgs& ba, unsigned grid, cudaStream_t st) {
+    constexpr uint32_t smem = BwdSmem<K>::total;
+    cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    DC_LAUNCH(kTcLowrankBwd, st, lowrank_bwd_kernel<K><<<grid, kThreads, smem, st>>>(tz, tg, tu, tbp, tdu, ba));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Workspace of the tensor-core backward (after the z scratch), byte offsets.
+struct TcBwdLayout {
+    size_t zs, bp, dz, dzb, dbpart, dpart, total;
+    int64_t per_cta, n_items, n_tiles;
+    int pieces, grid, n_dblk, n_split;
+};
+
+static inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+TcBwdLayout tc_bwd_layout(const Prob& p) {
+    TcBwdLayout L{};
+    const int sms = 148;   // sizing only; the launch uses at most this many CTAs
+    L.n_tiles = (p.N + 127) / 128;
+    const int64_t n_chunks = p.C / 64;
+    L.n_items = L.n_tiles * n_chunks;
+    L.per_cta = std::max<int64_t>(1, (L.n_items + sms - 1) / sms);
+    L.grid = (int)((L.n_items + L.per_cta - 1) / L.per_cta);
+    L.pieces = (int)(L.n_tiles / L.per_cta + 2);
+    L.n_dblk = (int)((p.d + 255) / 256);
+    L.n_split = std::max<int>(1, std::min<int>(sms / L.n_dblk, (int)L.n_tiles));
+    size_t off = 0;
+    L.zs = off;      off = al256(off + (size_t)p.N * p.r * 2);                     // z scratch (bf16)
+    L.bp = off;      off = al256(off + (size_t)p.r * p.C * p.K * 2);               // tap-major B
+    L.dz = off;      off = al256(off + (size_t)p.N * p.r * 4);                     // dz fp32 accumulator
+    L.dzb = off;     off = al256(off + (size_t)p.N * p.r * 2);                     // dz bf16
+    L.dbpart = off;  off = al256(off + (size_t)n_chunks * L.pieces * 64 * p.K * p.r * 4);
+    L.dpart = off;   off = al256(off + (size_t)L.n_split * p.d * p.r * 4);
+    L.total = off;
+    return L;
+}
+
+cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
+                                const void* B, const void* z_saved, void* du, void* dh, float* dA, float* dB,
+                                char* tcws, uint32_t* err, cudaStream_t st) {
+    const TcBwdLayout L = tc_bwd_layout(p);
+    const void* z = z_saved;
+    if (!z) {
+        void* zs = tcws + L.zs;
+        cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, zs, p.r, err, st);
+        if (e != cudaSuccess) return e;
+        z = zs;
+    }
+    __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(tcws + L.bp);
+    float* dz = reinterpret_cast<float*>(tcws + L.dz);
+    __nv_bfloat16* dzb = reinterpret_cast<__nv_bfloat16*>(tcws + L.dzb);
+    float* dbpart = reinterpret_cast<float*>(tcws + L.dbpart);
+    float* dpart = reinterpret_cast<float*>(tcws + L.dpart);
+    DC_LAUNCH(kTcPrep, st, permute_b_kernel<<<grid_for(p.r * p.C * p.K), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(B), bp, p.r, p.C, p.K));
+    cudaError_t e = cudaMemsetAsync(dz, 0, (size_t)p.N * p.r * 4, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tz, tg, tu, tbp, tdu;
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
+        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+        !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128))
+        return cudaErrorInvalidValue;
+    BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
+               L.per_cta, L.pieces, dz, dbpart, err};
+    switch (p.K) {
+        case 1: e = launch_bwd<1>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
+        case 2: e = launch_bwd<2>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
+        case 3: e = launch_bwd<3>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
+        default: e = launch_bwd<4>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
+    }
+    if (e != cudaSuccess) return e;
+    DC_LAUNCH(kTcReduce, st, reduce_dB_kernel<<<grid_for(p.r * p.C * p.K), 256, 0, st>>>(
+        dbpart, dB, p.r, p.C, p.K, L.n_tiles, L.per_cta, L.pieces));
+    DC_LAUNCH(kTcReduce, st, dz_to_bf16_kernel<<<grid_for(p.N * p.r), 256, 0, st>>>(dz, dzb, p.N * p.r));
+    // generator backward: dA = h^T dz, dh = dz A^T
+    CUtensorMap tx, th, tp;
+    if (!make_tmap_bf16(&tx, dzb, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&th, h, p.d, p.N, p.hs, 64, 128) ||
+        !make_tmap_bf16(&tp, A, p.r, p.d, p.r, 64, 256))
+        return cudaErrorInvalidValue;
+    GenBwdArgs ga{p.N, p.d, (int)p.r, (int)((p.r + 15) / 16 * 16), p.hs, L.n_dblk, L.n_split, L.n_tiles,
+                  static_cast<__nv_bfloat16*>(dh), dpart, err};
+    e = cudaFuncSetAttribute(gen_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGbSmem);
+    if (e != cudaSuccess) return e;
+    DC_LAUNCH(kTcGenBwd, st, gen_bwd_kernel<<<L.n_dblk * L.n_split, kThreads, kGbSmem, st>>>(tx, th, tp, ga));
+    DC_LAUNCH(kTcReduce, st, reduce_splits_kernel<<<grid_for(p.d * p.r), 256, 0, st>>>(
+        dpart, dA, p.d * p.r, L.n_split));
+    return cudaGetLastError();
+}
+
+}  // namespace dynconv

@@ -45,4 +45,16 @@ inline bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, ui
                         box_rows, true);
 }
 
+// Streaming multiprocessors of the current device (cached).
+inline int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
 }  // namespace dynconv
