@@ -27,7 +27,7 @@ ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 # Every entry point the header declares (checked against the library's exports by the tests).
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
-           "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma")
+           "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc")
 
 
 class DynConvError(RuntimeError):
@@ -69,6 +69,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_fwd_varlen.argtypes = [D, vp, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dynconv_bwd.argtypes = [D, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dynconv_device_status.argtypes = [vp, sz, vp]
+    lib.dynconv_fwd_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp]
+    lib.dynconv_fwd_noalloc.restype = ctypes.c_int
     for f in (lib.dynconv_fwd, lib.dynconv_fwd_varlen, lib.dynconv_bwd, lib.dynconv_device_status):
         f.restype = ctypes.c_int
     lib.dynconv_last_error.restype = ctypes.c_char_p
@@ -130,6 +132,12 @@ def dynconv_bwd(desc, cu_seqlens, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or
     _check(load().dynconv_bwd(ctypes.byref(desc), _ptr(cu_seqlens), n_docs, _ptr(g), _ptr(u), _ptr(h), _ptr(A),
                               _ptr(B_or_W), _ptr(z_saved), _ptr(du), _ptr(dh), _ptr(dA), _ptr(dB_or_dW),
                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream, g)))
+
+
+def dynconv_fwd_noalloc(desc, u, h, A, B, y, z_save=None, stream=None):
+    """Forward with no workspace argument (scratch built into the library); see include/dynconv.h."""
+    _check(load().dynconv_fwd_noalloc(ctypes.byref(desc), _ptr(u), _ptr(h), _ptr(A), _ptr(B), _ptr(y), _ptr(z_save),
+                                      _stream(stream, u)))
 
 
 def dynconv_device_status(ws, stream=None) -> int:

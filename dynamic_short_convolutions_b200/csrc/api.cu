@@ -131,6 +131,10 @@ dynconv_status forward_common(const dynconv_desc* desc, const int32_t* cu, int64
 
 }  // namespace
 
+dynconv_status validate_desc(const dynconv_desc* d, Prob* p) { return make_prob(d, p); }
+
+dynconv_status validate_ptr(const void* ptr, const char* name, bool required) { return check_ptr(ptr, name, required); }
+
 void set_error(const char* fmt, ...) {
     va_list ap;
     va_start(ap, fmt);

@@ -410,6 +410,26 @@ cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* 
     }
 }
 
+// Forward on the tensor cores with caller-chosen scratch: z (bf16 [N, r]) and the
+// device error word; used by the entry point that allocates nothing.
+cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
+                               void* z, uint32_t* err, cudaStream_t st) {
+    cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tz, tb, tu, ty;
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
+        return cudaErrorInvalidValue;
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err};
+    const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
+    switch (p.K) {
+        case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);
+        case 2: return launch_lowrank_fwd<2>(tz, tb, tu, ty, fa, items, st);
+        case 3: return launch_lowrank_fwd<3>(tz, tb, tu, ty, fa, items, st);
+        default: return launch_lowrank_fwd<4>(tz, tb, tu, ty, fa, items, st);
+    }
+}
+
 cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A, const void* BW,
                         const void* z_saved, void* du, void* dh, float* dA, float* dBW, void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(p);
