@@ -27,18 +27,23 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTcThreads = 192;   // 6 warps
+constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quarter
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kTcThreads = 64 + kEpiThreads;       // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
 
 // =====================================================================================
 // gen_kernel: X[N, R] = h[N, d] . P[d, R]   (z = h A; bf16 out), R <= 256.
 //   A operand: h tile [128 tokens][64 of d], K-major (TMA box {64, 128}).
 //   B operand: P tile [64 rows of d][64 of R] per 64-wide atom, MN-major (box {64, 64}).
+//   A ring of up to kGenMaxStages shared stages keeps most of a tile's d-loop in flight.
 // =====================================================================================
-constexpr int kGenStages = 4;
+constexpr int kGenMaxStages = 8;
+constexpr uint32_t kGenSmemBudget = 196608;
 
 struct GenArgs {
     int64_t N, d;
     int R, NB, NMMA;   // output width, P atoms per stage, MMA N
+    int stages;
     int64_t out_ld;
     uint32_t* err;
 };
@@ -50,7 +55,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     const uint32_t stage_bytes = 16384u + a.NB * 8192u;
-    __shared__ uint64_t full[kGenStages], empty[kGenStages], tfull[2], tempty[2];
+    const int S = a.stages;
+    __shared__ uint64_t full[kGenMaxStages], empty[kGenMaxStages], tfull[2], tempty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -58,13 +64,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
     const int nk = (int)((a.d + 63) / 64);
     const uint32_t tcols = tmem_cols_for(2 * a.NMMA);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGenStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], kEpiWarps);
         }
         abort_flag = 0;
         fence_mbar_init();
@@ -85,8 +91,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
             uint32_t it = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kGenStages;
-                    const uint32_t ph = (it / kGenStages) & 1;
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, a.err)) break;
                     uint8_t* st = sm + s * stage_bytes;
                     mbar_arrive_expect_tx(&full[s], stage_bytes);
@@ -106,8 +112,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
                 const uint32_t dcol = tbase + b * a.NMMA;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kGenStages;
-                    const uint32_t ph = (it / kGenStages) & 1;
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&full[s], ph, &abort_flag, a.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_u32(sm + s * stage_bytes);
@@ -122,6 +128,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
         }
     } else {
         const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;        // which columns of the row this warp converts
         const int row = q * 32 + lane;
         uint32_t t = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++t) {
@@ -130,7 +137,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
             tc_fence_after();
             const int64_t n = tile * 128 + row;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * a.NMMA;
-            for (int c = 0; c < a.R; c += 8) {
+            for (int c = 8 * half; c < a.R; c += 16) {
                 uint32_t v[8];
                 tmem_ld8(taddr + c, v);
                 tmem_wait_ld();
@@ -169,7 +176,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 //   stage smem: z tile [128][64] (K-major A) | B chunk as K atoms [64 r-rows][64] (MN-major B)
 //               | u tile [136 rows = m0-8 .. m0+127][64 channels]
 //   TMEM: W[128 tokens][64 K] fp32, column c K + j = w[m0 + row, c0 + c, j]; two buffers.
-//   epilogue: y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c] -> bf16 staging
+//   epilogue (8 warps: a lane quarter and half of the 64 channels each):
+//             y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c] -> bf16 staging
 //             (128-byte swizzled) -> TMA store.
 // =====================================================================================
 struct FwdArgs {
@@ -184,6 +192,36 @@ template <int K>
 constexpr uint32_t fwd_stage_bytes() { return kZBytes + K * 8192 + kUBytes; }
 template <int K>
 constexpr uint32_t fwd_smem_bytes() { return 1024 + 2 * fwd_stage_bytes<K>() + 2 * kYBytes; }
+
+// y for 8 channels of one row from the K filter taps (wv[j*8 + c] = W[t, (g8*8 + c) K + j] is
+// loaded as K x8 column runs starting at column g8*8*K, i.e. wv[i] = column g8*8*K + i).
+template <int K>
+__device__ __forceinline__ uint4 conv8(const uint32_t* wv, const uint4* uj, int64_t pos) {
+    float acc[8];
+    const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+        acc[c] = bf16_lo(u0[c >> 1]);
+        acc[c + 1] = bf16_hi(u0[c >> 1]);
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if (j <= pos) {
+            const uint32_t* uu = reinterpret_cast<const uint32_t*>(&uj[j]);
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                acc[c] = fmaf(__uint_as_float(wv[c * K + j]), bf16_lo(uu[c >> 1]), acc[c]);
+                acc[c + 1] = fmaf(__uint_as_float(wv[(c + 1) * K + j]), bf16_hi(uu[c >> 1]), acc[c + 1]);
+            }
+        }
+    }
+    uint4 pk;
+    pk.x = pack_bf16(acc[0], acc[1]);
+    pk.y = pack_bf16(acc[2], acc[3]);
+    pk.z = pack_bf16(acc[4], acc[5]);
+    pk.w = pack_bf16(acc[6], acc[7]);
+    return pk;
+}
 
 template <int K>
 __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
@@ -205,9 +243,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + 4);
+            mbar_init(&empty[s], 1 + kEpiWarps);
             mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], 4);
+            mbar_init(&tempty[s], kEpiWarps);
         }
         abort_flag = 0;
         fence_mbar_init();
@@ -260,8 +298,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
         }
     } else {
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;      // channel groups 4*half .. 4*half+3
         const int row = q * 32 + lane;
-        const int et = threadIdx.x - 64;        // 0..127 epilogue thread index
+        const int et = threadIdx.x - 64;       // 0 .. kEpiThreads-1
         uint32_t it = 0;
         for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
             const int64_t chunk = item / n_tiles, tile = item % n_tiles;
@@ -269,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
             const uint32_t ph = (it >> 1) & 1;
             const bool ok = mbar_wait(&tfull[s], ph, &abort_flag, a.err) && mbar_wait(&full[s], ph, &abort_flag, a.err);
             if (et == 0) tma_store_wait_read_le1();     // the store that last used this staging buffer
-            if (epi_bar_any(!ok)) break;
+            if (epi_bar_any<kEpiThreads>(!ok)) break;
             tc_fence_after();
             const int64_t n = tile * 128 + row;
             const int64_t pos = n < a.N ? n - seg_start(n, a.cu, a.n_docs, a.seqlen) : 0;
@@ -277,39 +316,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
             uint8_t* ys = ystage + s * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + s * 256;
 #pragma unroll 1
-            for (int g = 0; g < 8; ++g) {                 // 8 channels per group
-                uint32_t wv[8 * K];
+            for (int gp = 0; gp < 2; ++gp) {            // two groups of 8 channels per batch
+                const int g0 = 4 * half + 2 * gp;
+                uint32_t wv[2][8 * K];
 #pragma unroll
-                for (int i = 0; i < K; ++i) tmem_ld8(taddr + g * 8 * K + 8 * i, *reinterpret_cast<uint32_t(*)[8]>(wv + 8 * i));
-                uint4 uj[K];
+                for (int x = 0; x < 2; ++x)
 #pragma unroll
-                for (int j = 0; j < K; ++j)
-                    uj[j] = *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g));
+                    for (int i = 0; i < K; ++i)
+                        tmem_ld8(taddr + (g0 + x) * 8 * K + 8 * i, *reinterpret_cast<uint32_t(*)[8]>(wv[x] + 8 * i));
+                uint4 uj[2][K];
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                    for (int j = 0; j < K; ++j)
+                        uj[x][j] = *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g0 + x));
                 tmem_wait_ld();
-                float acc[8];
-                const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    acc[c] = bf16_lo(u0[c >> 1]);
-                    acc[c + 1] = bf16_hi(u0[c >> 1]);
-                }
-#pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    if (j <= pos) {
-                        const uint32_t* uu = reinterpret_cast<const uint32_t*>(&uj[j]);
-#pragma unroll
-                        for (int c = 0; c < 8; c += 2) {
-                            acc[c] = fmaf(__uint_as_float(wv[c * K + j]), bf16_lo(uu[c >> 1]), acc[c]);
-                            acc[c + 1] = fmaf(__uint_as_float(wv[(c + 1) * K + j]), bf16_hi(uu[c >> 1]), acc[c + 1]);
-                        }
-                    }
-                }
-                uint4 pk;
-                pk.x = pack_bf16(acc[0], acc[1]);
-                pk.y = pack_bf16(acc[2], acc[3]);
-                pk.z = pack_bf16(acc[4], acc[5]);
-                pk.w = pack_bf16(acc[6], acc[7]);
-                *reinterpret_cast<uint4*>(ys + sw128_off(row, g)) = pk;
+                for (int x = 0; x < 2; ++x)
+                    *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = conv8<K>(wv[x], uj[x], pos);
             }
             tc_fence_before();
             __syncwarp();
@@ -318,7 +342,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
                 mbar_arrive(&empty[s]);
             }
             fence_async_smem();
-            epi_bar_sync();
+            epi_bar_sync<kEpiThreads>();
             if (et == 0) {
                 tma_store_2d(&tm_y, ys, (int32_t)(chunk * 64), (int32_t)(tile * 128));
                 tma_store_commit();
@@ -352,8 +376,11 @@ cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, i
     CUtensorMap th, tp;
     if (!make_tmap_bf16(&th, h, d, N, hs, 64, 128) || !make_tmap_bf16(&tp, P, R, d, R, 64, 64))
         return cudaErrorInvalidValue;
-    GenArgs ga{N, d, R, (R + 63) / 64, (R + 15) / 16 * 16, out_ld, err};
-    const int smem = 1024 + kGenStages * (16384 + ga.NB * 8192);
+    const int NB = (R + 63) / 64;
+    const int stage_bytes = 16384 + NB * 8192;
+    const int stages = std::max(2, std::min<int>(kGenMaxStages, (int)(kGenSmemBudget / stage_bytes)));
+    GenArgs ga{N, d, R, NB, (R + 15) / 16 * 16, stages, out_ld, err};
+    const int smem = 1024 + stages * stage_bytes;
     cudaError_t e = cudaFuncSetAttribute(gen_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int64_t n_tiles = (N + 127) / 128;

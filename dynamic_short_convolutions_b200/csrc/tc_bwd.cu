@@ -48,7 +48,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quarter
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;         // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
 constexpr uint32_t kRowTile = 136 * 128;     // 136-row, 64-column bf16 tile
 constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
 
@@ -102,12 +104,12 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + 4);
+            mbar_init(&empty[s], 1 + kEpiWarps);
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
         mbar_init(&wfull, 1);
-        mbar_init(&wempty, 4);
+        mbar_init(&wempty, kEpiWarps);
         mbar_init(&dzfull, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -124,9 +126,9 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
     if (warp >= 2) {
         // dW atoms past the last tap stay zero for the whole kernel (they pad the
         // last 128-row block of the dB MMA).
-        const int row = (warp & 3) * 32 + lane;
+        const int row = (warp & 3) * 32 + lane, half = (warp - 2) >> 2;
         for (int at = K; at < S::NA; ++at)
-            for (int q = 0; q < 8; ++q)
+            for (int q = 4 * half; q < 4 * half + 4; ++q)
                 *reinterpret_cast<uint4*>(sm + S::dw + at * kAtom128 + sw128_off(row, q)) = make_uint4(0, 0, 0, 0);
         fence_async_smem();
     }
@@ -213,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
         }
     } else {
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;      // channel groups 4*half..4*half+3; dz/dB columns 8*half + 16 i
         const int row = q * 32 + lane;
         const int et = threadIdx.x - 64;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
                       mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err);
             if (et == 0) tma_store_wait_all();       // du staging and dW are free again
-            if (epi_bar_any(!ok)) break;
+            if (epi_bar_any<kEpiThreads>(!ok)) break;
             tc_fence_after();
             const int64_t n = tile * 128 + row;
             int64_t pos = -1, epos = -1;             // valid past / future taps of this row
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
             const uint8_t* ut = zt + 2 * kRowTile;
             (void)zt;
 #pragma unroll 1
-            for (int g8 = 0; g8 < 8; ++g8) {
+            for (int g8 = 4 * half; g8 < 4 * half + 4; ++g8) {
                 uint32_t wv[K][8];
 #pragma unroll
                 for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * g8, wv[j]);
@@ -303,16 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
                 mbar_arrive(&wempty);
                 mbar_arrive(&empty[s]);
             }
-            epi_bar_sync();
+            epi_bar_sync<kEpiThreads>();
             if (et == 0) {
                 tma_store_2d(&tm_du, dus, (int32_t)(chunk * 64), (int32_t)(tile * 128));
                 tma_store_commit();
             }
             ok = mbar_wait(&dzfull, it & 1, &abort_flag, a.err);
-            if (epi_bar_any(!ok)) break;
+            if (epi_bar_any<kEpiThreads>(!ok)) break;
             tc_fence_after();
             // epilogue B: dz rows -> fp32 atomic add (reduction over channel chunks)
-            for (int c = 0; c < a.r; c += 8) {
+            for (int c = 8 * half; c < a.r; c += 16) {
                 uint32_t v[8];
                 tmem_ld8(lane_base + kColDz + c, v);
                 tmem_wait_ld();
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
 #pragma unroll
                 for (int b = 0; b < NBLK; ++b) {
                     const int m = b * 128 + row;     // (tap, channel) row = j * 64 + c
-                    for (int c = 0; c < a.r; c += 8) {
+                    for (int c = 8 * half; c < a.r; c += 16) {
                         uint32_t v[8];
                         tmem_ld8(lane_base + kColDb + 64 * b + c, v);
                         tmem_wait_ld();
@@ -357,24 +360,51 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
     }
 }
 
-// dB[k, c K + j] = sum over the runs covering chunk c/64, in run order.
-__global__ void reduce_dB_kernel(const float* __restrict__ part, float* __restrict__ dB, int64_t r, int64_t C,
-                                 int64_t K, int64_t n_tiles, int64_t per_cta, int pieces) {
-    const int64_t total = r * C * K;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t k = e / (C * K), col = e % (C * K), c = col / K, j = col % K;
-        const int64_t chunk = c / 64, m = j * 64 + (c % 64);
-        const int64_t first = (chunk * n_tiles) / per_cta, lastc = ((chunk + 1) * n_tiles - 1) / per_cta;
+// dB[k, c K + j] = sum over the runs covering chunk c/64, in run order (one thread per entry).
+template <int K>
+__global__ void reduce_dB_kernel(const float* __restrict__ part, float* __restrict__ dB, int r, int C, int n_tiles,
+                                 int per_cta, int pieces) {
+    const int total = r * C * K;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        const int k = e / (C * K), col = e - k * (C * K), c = col / K, j = col - c * K;
+        const int chunk = c >> 6, m = j * 64 + (c & 63);
+        const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
+        const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
+        const float* src = part + ((int64_t)chunk * pieces * (64 * K) + m) * r + k;
         float acc = 0.f;
-        for (int64_t p = 0; p <= lastc - first; ++p)
-            acc += part[((chunk * pieces + p) * (64 * K) + m) * r + k];
+        for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * (64 * K) * r];
         dB[e] = acc;
     }
 }
 
-__global__ void dz_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t count) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
-        dst[i] = __float2bfloat16_rn(src[i]);
+__global__ void dz_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t count4) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = src[i];
+        dst[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    }
+}
+
+// out[i] = sum_s part[s][i] for i < count (count a multiple of 4): one warp per 4 outputs, lane l
+// sums splits l, l + 32, ... in order, then a fixed butterfly combines the lanes (deterministic).
+__global__ void reduce_splits_kernel(const float* __restrict__ part, float* __restrict__ out, int64_t count,
+                                     int n_split) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; w * 4 < count; w += warps) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = lane; s < n_split; s += 32) {
+            const float4 v = *reinterpret_cast<const float4*>(part + s * count + w * 4);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+        }
+        if (lane == 0) *reinterpret_cast<float4*>(out + w * 4) = acc;
+    }
 }
 
 // =====================================================================================
@@ -420,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         }
         mbar_init(&pfull, 1);
         mbar_init(&hfull, 1);
-        mbar_init(&hempty, 4);
+        mbar_init(&hempty, kEpiWarps);
         mbar_init(&dpfull, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -482,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         }
     } else {
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;      // dh columns 128*half .. +127; dP columns 8*half + 16 i
         const int row = q * 32 + lane;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint32_t it = 0;
@@ -489,21 +520,26 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         if (want_dh) {
             for (int64_t tile = t0; tile < t1; ++tile, ++it) {
                 ok = mbar_wait(&hfull, it & 1, &abort_flag, a.err);
-                if (epi_bar_any(!ok)) break;
+                if (epi_bar_any<kEpiThreads>(!ok)) break;
                 tc_fence_after();
                 const int64_t n = tile * 128 + row;
-                for (int c = 0; c < 256; c += 8) {
-                    uint32_t v[8];
-                    tmem_ld8(lane_base + c, v);
+#pragma unroll 1
+                for (int c = 128 * half; c < 128 * half + 128; c += 32) {
+                    uint32_t v[4][8];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) tmem_ld8(lane_base + c + 8 * x, v[x]);
                     tmem_wait_ld();
-                    const int64_t col = (int64_t)db * 256 + c;
-                    if (n < a.N && col < a.d) {
-                        uint4 pk;
-                        pk.x = pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1]));
-                        pk.y = pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3]));
-                        pk.z = pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5]));
-                        pk.w = pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7]));
-                        *reinterpret_cast<uint4*>(a.dh + n * a.d + col) = pk;
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int64_t col = (int64_t)db * 256 + c + 8 * x;
+                        if (n < a.N && col < a.d) {
+                            uint4 pk;
+                            pk.x = pack_bf16(__uint_as_float(v[x][0]), __uint_as_float(v[x][1]));
+                            pk.y = pack_bf16(__uint_as_float(v[x][2]), __uint_as_float(v[x][3]));
+                            pk.z = pack_bf16(__uint_as_float(v[x][4]), __uint_as_float(v[x][5]));
+                            pk.w = pack_bf16(__uint_as_float(v[x][6]), __uint_as_float(v[x][7]));
+                            *reinterpret_cast<uint4*>(a.dh + n * a.d + col) = pk;
+                        }
                     }
                 }
                 tc_fence_before();
@@ -512,12 +548,12 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
             }
         }
         if (ok && t1 > t0) ok = mbar_wait(&dpfull, 0, &abort_flag, a.err);
-        if (!epi_bar_any(!ok) && t1 > t0) {
+        if (!epi_bar_any<kEpiThreads>(!ok) && t1 > t0) {
             tc_fence_after();
             float* part = a.dP_part + (int64_t)split * a.d * a.R;
             for (int b = 0; b < 2; ++b) {
                 const int64_t drow = (int64_t)db * 256 + b * 128 + row;
-                for (int c = 0; c < a.R; c += 8) {
+                for (int c = 8 * half; c < a.R; c += 16) {
                     uint32_t v[8];
                     tmem_ld8(lane_base + kColDp + 64 * b + c, v);
                     tmem_wait_ld();
@@ -537,15 +573,6 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, 512);
-    }
-}
-
-__global__ void reduce_splits_kernel(const float* __restrict__ part, float* __restrict__ out, int64_t count,
-                                     int n_split) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < n_split; ++s) acc += part[s * count + i];
-        out[i] = acc;
     }
 }
 
@@ -631,9 +658,20 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         default: e = launch_bwd<4>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcReduce, st, reduce_dB_kernel<<<grid_for(p.r * p.C * p.K), 256, 0, st>>>(
-        dbpart, dB, p.r, p.C, p.K, L.n_tiles, L.per_cta, L.pieces));
-    DC_LAUNCH(kTcReduce, st, dz_to_bf16_kernel<<<grid_for(p.N * p.r), 256, 0, st>>>(dz, dzb, p.N * p.r));
+    switch (p.K) {
+#define DC_REDUCE_DB(KK)                                                                                       \
+    case KK:                                                                                                    \
+        DC_LAUNCH(kTcReduce, st, reduce_dB_kernel<KK><<<grid_for(p.r * p.C * p.K), 256, 0, st>>>(              \
+            dbpart, dB, (int)p.r, (int)p.C, (int)L.n_tiles, (int)L.per_cta, L.pieces));                         \
+        break;
+        DC_REDUCE_DB(1)
+        DC_REDUCE_DB(2)
+        DC_REDUCE_DB(3)
+        DC_REDUCE_DB(4)
+#undef DC_REDUCE_DB
+    }
+    DC_LAUNCH(kTcReduce, st, dz_to_bf16_kernel<<<grid_for(p.N * p.r / 4), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb), p.N * p.r / 4));
     // generator backward: dA = h^T dz, dh = dz A^T
     CUtensorMap tx, th, tp;
     if (!make_tmap_bf16(&tx, dzb, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&th, h, p.d, p.N, p.hs, 64, 128) ||
@@ -644,7 +682,7 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     e = cudaFuncSetAttribute(gen_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGbSmem);
     if (e != cudaSuccess) return e;
     DC_LAUNCH(kTcGenBwd, st, gen_bwd_kernel<<<L.n_dblk * L.n_split, kThreads, kGbSmem, st>>>(tx, th, tp, ga));
-    DC_LAUNCH(kTcReduce, st, reduce_splits_kernel<<<grid_for(p.d * p.r), 256, 0, st>>>(
+    DC_LAUNCH(kTcReduce, st, reduce_splits_kernel<<<grid_for(p.d * p.r / 4 * 32), 256, 0, st>>>(
         dpart, dA, p.d * p.r, L.n_split));
     return cudaGetLastError();
 }

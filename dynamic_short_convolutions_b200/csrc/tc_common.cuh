@@ -175,21 +175,24 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Named barrier over the 128 epilogue threads (warps 2-5 of a 6-warp CTA).
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier 1 over the NT epilogue threads (the warps after the producer
+// and MMA warps).
+template <int NT>
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 
-// Barrier over the 128 epilogue threads that also ORs a predicate across them, so
-// that a bounded wait giving up in one warp makes every epilogue warp leave its
-// loop at the same point (no thread is left waiting at a named barrier).
+// Barrier 2 over the NT epilogue threads that also ORs a predicate across them,
+// so that a bounded wait giving up in one warp makes every epilogue warp leave
+// its loop at the same point (no thread is left waiting at a named barrier).
+template <int NT>
 __device__ __forceinline__ bool epi_bar_any(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.or.pred q, 2, 128, p;\n\t"
+        "barrier.cta.red.or.pred q, 2, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(uint32_t(pred))
+        : "r"(uint32_t(pred)), "n"(NT)
         : "memory");
     return r != 0;
 }
