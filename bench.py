@@ -261,7 +261,8 @@ def run_ours(args, rank, world, local_rank):
         BW = t["B"] if kind == L.LOWRANK else t["W"]
         N = w.tokens
         bufs = dict(y=torch.empty((N, layer.channels), dtype=dt, device=dev),
-                    z=torch.empty((N, w.rank), dtype=dt, device=dev) if kind == L.LOWRANK else None,
+                    z=torch.empty((N, w.rank if kind == L.LOWRANK else (layer.channels // w.head_dim) * w.ksize),
+                                  dtype=dt, device=dev),
                     out={"du": torch.empty((N, layer.channels), dtype=dt, device=dev),
                          "dh": torch.empty((N, layer.d_model), dtype=dt, device=dev),
                          "dA": torch.empty(tuple(A.shape), dtype=torch.float32, device=dev) if A is not None else None,

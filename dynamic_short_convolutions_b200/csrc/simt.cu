@@ -196,7 +196,7 @@ cudaError_t forward_t(const Prob& p, const void* u, const void* h, const void* A
     float* X = reinterpret_cast<float*>(static_cast<char*>(ws) + L.gen);
     const T* P = static_cast<const T*>(p.kind == 0 ? A : BW);
     DC_LAUNCH(kSimtGen, st, gen_kernel<T><<<(unsigned)p.N, kThreads, 0, st>>>(
-        static_cast<const T*>(h), p.hs, P, p.d, p.R, X, p.kind == 0 ? static_cast<T*>(z_save) : nullptr));
+        static_cast<const T*>(h), p.hs, P, p.d, p.R, X, static_cast<T*>(z_save)));
     const size_t smem = sizeof(float) * (size_t)p.R;
     if (p.kind == 0)
         DC_LAUNCH(kSimtConvFwd, st, conv_fwd_kernel<T, 0><<<(unsigned)p.N, kThreads, smem, st>>>(
@@ -217,7 +217,7 @@ cudaError_t backward_t(const Prob& p, const void* g, const void* u, const void* 
     float* X = reinterpret_cast<float*>(static_cast<char*>(ws) + L.gen);
     float* DG = reinterpret_cast<float*>(static_cast<char*>(ws) + L.dgen);
     const T* P = static_cast<const T*>(p.kind == 0 ? A : BW);
-    if (p.kind == 0 && z_saved) {
+    if (z_saved) {
         const int64_t cnt = p.N * p.R;
         const unsigned nb = (unsigned)(cnt < 148 * 64 * kThreads ? blocks_for(cnt) : 148 * 64);
         DC_LAUNCH(kSimtWiden, st, widen_kernel<T><<<nb, kThreads, 0, st>>>(static_cast<const T*>(z_saved), X, cnt));

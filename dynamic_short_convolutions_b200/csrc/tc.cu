@@ -396,11 +396,22 @@ struct TcBwdLayout {
     int pieces, grid, n_dblk, n_split;
 };
 TcBwdLayout tc_bwd_layout(const Prob& p);
+struct TcHwLayout {
+    size_t wh, dwh, dpart, total;
+};
+TcHwLayout tc_hw_layout(const Prob& p);
+bool tc_headwise_supported(const Prob& p);
+cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, const void* W, void* y, void* z_save,
+                                char* tcws, uint32_t* err, cudaStream_t st);
+cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, const void* h, const void* W,
+                                 const void* z_saved, void* du, void* dh, float* dW, char* tcws, uint32_t* err,
+                                 cudaStream_t st);
 cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
                                 const void* B, const void* z_saved, void* du, void* dh, float* dA, float* dB,
                                 char* tcws, uint32_t* err, cudaStream_t st);
 
 bool tc_supported(const Prob& p) {
+    if (p.kind == 1) return tc_headwise_supported(p) && tensor_map_encoder() != nullptr;
     if (p.dtype != 1 || p.kind != 0) return false;
     if (p.r % 8 != 0 || p.r > 64) return false;
     if (p.C % 64 != 0 || p.d % 8 != 0) return false;
@@ -409,17 +420,19 @@ bool tc_supported(const Prob& p) {
 }
 
 bool tc_supported_bwd(const Prob& p) {
-    // The backward reduces dz over channel chunks with fp32 atomics; the
-    // deterministic mode takes the generic kernels instead.
-    return tc_supported(p) && !p.deterministic;
+    // The low-rank backward reduces dz over channel chunks with fp32 atomics, so its
+    // deterministic mode takes the generic kernels; the head-wise backward has no
+    // atomics (warp-shuffle and fixed-order split reductions).
+    return tc_supported(p) && (p.kind == 1 || !p.deterministic);
 }
 
-size_t tc_workspace_bytes(const Prob& p) { return tc_bwd_layout(p).total; }
+size_t tc_workspace_bytes(const Prob& p) { return p.kind == 1 ? tc_hw_layout(p).total : tc_bwd_layout(p).total; }
 
 cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
                        void* z_save, void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
+    if (p.kind == 1) return tc_headwise_forward(p, u, h, BW, y, z_save, static_cast<char*>(ws) + L.tc, err, st);
     void* z = z_save ? z_save : static_cast<void*>(static_cast<char*>(ws) + L.tc);
     cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
     if (e != cudaSuccess) return e;
@@ -461,6 +474,8 @@ cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void*
                         const void* z_saved, void* du, void* dh, float* dA, float* dBW, void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
+    if (p.kind == 1)
+        return tc_headwise_backward(p, g, u, h, BW, z_saved, du, dh, dBW, static_cast<char*>(ws) + L.tc, err, st);
     return tc_lowrank_backward(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, static_cast<char*>(ws) + L.tc, err, st);
 }
 

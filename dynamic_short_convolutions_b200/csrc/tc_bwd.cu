@@ -408,16 +408,18 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, float* __re
 }
 
 // =====================================================================================
-// gen_bwd_kernel: per (256-wide block db of d, token range):
-//   dh[t, db*256 + i] = sum_k X[t, k] P[db*256 + i, k]          (X = dz or dwh, P = A or W)
-//   dPpart[split][db*256 + i, k] = sum_{t in range} h[t, db*256 + i] X[t, k]
-// smem: stage = X tile [128][64] (K-major A of dh; MN-major B of dP) + h tile 4 atoms
-//       [128 tokens][64 of d] (MN-major A of dP); P block [256 of d][64] resident (K-major B of dh).
-// TMEM: dh [128][256] at column 0, dP blocks [128][R] at 256 and 320... (two blocks of 128 rows of d).
+// gen_bwd_kernel<XA>: per (DB-wide block db of d, token range), X = dz (low-rank) or the
+// head-wise filter gradient dwh, P = A or W, with R = X's width:
+//   dh[t, db*DB + i] = sum_k X[t, k] P[db*DB + i, k]
+//   dPpart[split][db*DB + i, k] = sum_{t in range} h[t, db*DB + i] X[t, k]
+// XA = 64-wide atoms of X (1: R <= 64, DB = 256; 2: R <= 128, DB = 128).
+// smem: stage = X tile [128 tokens][XA atoms] (K-major A of dh; MN-major B of dP) + h tile
+//       [128 tokens][DB/64 atoms] (MN-major A of dP); P block [DB rows of d][XA atoms] resident
+//       (K-major B of dh).  TMEM: dh [128][DB] at column 0, dP blocks [128 rows of d][R] after it.
 // =====================================================================================
 struct GenBwdArgs {
     int64_t N, d;
-    int R, ndz;
+    int R, ndz, ksteps;       // X width, dP MMA N (R rounded up to 16), dh K steps (R / 16 rounded up)
     int64_t hs;
     int n_dblk, n_split;
     int64_t n_tiles;
@@ -426,16 +428,26 @@ struct GenBwdArgs {
     uint32_t* err;
 };
 
-constexpr uint32_t kGbStage = kAtom128 + 4 * kAtom128;     // X tile + 4 h atoms
-constexpr uint32_t kGbSmem = 2 * kGbStage + 256 * 128 + 1024;   // + resident P block (256 rows x 128 B)
+template <int XA>
+struct GbCfg {
+    static constexpr int DB = XA == 1 ? 256 : 128;          // d columns per CTA
+    static constexpr int HA = DB / 64;                      // h atoms per stage
+    static constexpr uint32_t stage = (XA + HA) * kAtom128;
+    static constexpr uint32_t pblk = 2 * stage;
+    static constexpr uint32_t smem = pblk + DB * 128 * XA + 1024;
+    static constexpr uint32_t col_dp = DB;                  // TMEM column of the first dP block
+    static constexpr uint32_t dp_stride = XA == 1 ? 64 : 128;
+};
 
+template <int XA>
 __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_h,
                                                               const __grid_constant__ CUtensorMap tm_p,
                                                               GenBwdArgs a) {
+    using G = GbCfg<XA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* pblk = sm + 2 * kGbStage;                       // 256 rows x 128 B = 32 KB
+    uint8_t* pblk = sm + G::pblk;
     __shared__ uint64_t full[2], empty[2], pfull, hfull, hempty, dpfull;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -466,26 +478,25 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base;
-    constexpr uint32_t kColDp = 256;
 
     if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(&pfull, 256 * 128);
-            tma_load_2d(pblk, &tm_p, &pfull, 0, db * 256);
+            mbar_arrive_expect_tx(&pfull, G::DB * 128 * XA);
+            for (int xa = 0; xa < XA; ++xa) tma_load_2d(pblk + xa * G::DB * 128, &tm_p, &pfull, 64 * xa, db * G::DB);
             uint32_t it = 0;
             for (int64_t tile = t0; tile < t1 && !abort_flag; ++tile, ++it) {
                 const int s = it & 1;
                 if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
-                uint8_t* st = sm + s * kGbStage;
-                mbar_arrive_expect_tx(&full[s], kGbStage);
-                tma_load_2d(st, &tm_x, &full[s], 0, (int32_t)(tile * 128));
-                for (int at = 0; at < 4; ++at)
-                    tma_load_2d(st + kAtom128 * (1 + at), &tm_h, &full[s], db * 256 + 64 * at, (int32_t)(tile * 128));
+                uint8_t* st = sm + s * G::stage;
+                mbar_arrive_expect_tx(&full[s], G::stage);
+                for (int xa = 0; xa < XA; ++xa) tma_load_2d(st + xa * kAtom128, &tm_x, &full[s], 64 * xa, (int32_t)(tile * 128));
+                for (int at = 0; at < G::HA; ++at)
+                    tma_load_2d(st + kAtom128 * (XA + at), &tm_h, &full[s], db * G::DB + 64 * at, (int32_t)(tile * 128));
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc_dh = idesc_bf16(128, 256, false, false);
+            const uint32_t idesc_dh = idesc_bf16(128, G::DB, false, false);
             const uint32_t idesc_dp = idesc_bf16(128, a.ndz, true, true);
             const uint32_t p0 = smem_u32(pblk);
             bool ok = mbar_wait(&pfull, 0, &abort_flag, a.err);
@@ -494,17 +505,19 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                 const int s = it & 1;
                 if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
-                const uint32_t x0 = smem_u32(sm + s * kGbStage), h0 = x0 + kAtom128;
+                const uint32_t x0 = smem_u32(sm + s * G::stage), h0 = x0 + XA * kAtom128;
                 if (want_dh) {
                     if (!mbar_wait(&hempty, (it & 1) ^ 1, &abort_flag, a.err)) break;
                     tc_fence_after();
-                    for (int k = 0; k < 4; ++k)
-                        umma_bf16(tbase, kmajor_desc(x0, k), kmajor_desc(p0, k), idesc_dh, k != 0);
+                    for (int k = 0; k < a.ksteps; ++k)
+                        umma_bf16(tbase, kmajor_desc(x0 + (k >> 2) * kAtom128, k & 3),
+                                  kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3), idesc_dh, k != 0);
                     umma_commit(&hfull);
                 }
-                for (int b = 0; b < 2; ++b)
+                for (int b = 0; b < G::DB / 128; ++b)
                     for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tbase + kColDp + 64 * b, mnmajor_desc(h0 + 2 * b * kAtom128, kAtom128, 16 * ks),
+                        umma_bf16(tbase + G::col_dp + G::dp_stride * b,
+                                  mnmajor_desc(h0 + 2 * b * kAtom128, kAtom128, 16 * ks),
                                   mnmajor_desc(x0, kAtom128, 16 * ks), idesc_dp, !(tile == t0 && ks == 0));
                 umma_commit(&empty[s]);
             }
@@ -512,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;      // dh columns 128*half .. +127; dP columns 8*half + 16 i
+        const int half = (warp - 2) >> 2;      // dh columns half*DB/2 ..; dP columns 8*half + 16 i
         const int row = q * 32 + lane;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint32_t it = 0;
@@ -524,14 +537,14 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                 tc_fence_after();
                 const int64_t n = tile * 128 + row;
 #pragma unroll 1
-                for (int c = 128 * half; c < 128 * half + 128; c += 32) {
+                for (int c = (G::DB / 2) * half; c < (G::DB / 2) * (half + 1); c += 32) {
                     uint32_t v[4][8];
 #pragma unroll
                     for (int x = 0; x < 4; ++x) tmem_ld8(lane_base + c + 8 * x, v[x]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const int64_t col = (int64_t)db * 256 + c + 8 * x;
+                        const int64_t col = (int64_t)db * G::DB + c + 8 * x;
                         if (n < a.N && col < a.d) {
                             uint4 pk;
                             pk.x = pack_bf16(__uint_as_float(v[x][0]), __uint_as_float(v[x][1]));
@@ -551,11 +564,11 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         if (!epi_bar_any<kEpiThreads>(!ok) && t1 > t0) {
             tc_fence_after();
             float* part = a.dP_part + (int64_t)split * a.d * a.R;
-            for (int b = 0; b < 2; ++b) {
-                const int64_t drow = (int64_t)db * 256 + b * 128 + row;
+            for (int b = 0; b < G::DB / 128; ++b) {
+                const int64_t drow = (int64_t)db * G::DB + b * 128 + row;
                 for (int c = 8 * half; c < a.R; c += 16) {
                     uint32_t v[8];
-                    tmem_ld8(lane_base + kColDp + 64 * b + c, v);
+                    tmem_ld8(lane_base + G::col_dp + G::dp_stride * b + c, v);
                     tmem_wait_ld();
                     if (drow < a.d) {
                         float4* dst = reinterpret_cast<float4*>(part + drow * a.R + c);
@@ -593,6 +606,41 @@ cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUten
 
 }  // namespace
 
+// Generator backward on the tensor cores: dP = h^T X (fp32, overwritten) and, when dh is
+// non-null, dh = X P^T (bf16), for X [N, R] bf16 (R <= 128, multiple of 8), P [d, R] bf16.
+// dP_part must hold n_split * d * R floats (gen_bwd_splits()).
+int gen_bwd_dblk(int64_t d, int R) { return (int)((d + (R <= 64 ? 256 : 128) - 1) / (R <= 64 ? 256 : 128)); }
+int gen_bwd_splits(int64_t N, int64_t d, int R) {
+    const int64_t n_tiles = (N + 127) / 128;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(148 / std::max(1, gen_bwd_dblk(d, R)), n_tiles));
+}
+
+cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
+                            void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st) {
+    const int n_dblk = gen_bwd_dblk(d, R), n_split = gen_bwd_splits(N, d, R);
+    const int XA = R <= 64 ? 1 : 2;
+    const int DB = XA == 1 ? 256 : 128;
+    CUtensorMap tx, th, tp;
+    if (!make_tmap_bf16(&tx, X, R, N, R, 64, 128) || !make_tmap_bf16(&th, h, d, N, hs, 64, 128) ||
+        !make_tmap_bf16(&tp, P, R, d, R, 64, DB))
+        return cudaErrorInvalidValue;
+    GenBwdArgs ga{N, d, R, (R + 15) / 16 * 16, (R + 15) / 16, hs, n_dblk, n_split, (N + 127) / 128,
+                  static_cast<__nv_bfloat16*>(dh), dP_part, err};
+    cudaError_t e;
+    if (XA == 1) {
+        e = cudaFuncSetAttribute(gen_bwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, GbCfg<1>::smem);
+        if (e != cudaSuccess) return e;
+        DC_LAUNCH(kTcGenBwd, st, gen_bwd_kernel<1><<<n_dblk * n_split, kThreads, GbCfg<1>::smem, st>>>(tx, th, tp, ga));
+    } else {
+        e = cudaFuncSetAttribute(gen_bwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, GbCfg<2>::smem);
+        if (e != cudaSuccess) return e;
+        DC_LAUNCH(kTcGenBwd, st, gen_bwd_kernel<2><<<n_dblk * n_split, kThreads, GbCfg<2>::smem, st>>>(tx, th, tp, ga));
+    }
+    DC_LAUNCH(kTcReduce, st, reduce_splits_kernel<<<grid_for(d * R / 4 * 32), 256, 0, st>>>(
+        dP_part, dP, d * R, n_split));
+    return cudaGetLastError();
+}
+
 // Workspace of the tensor-core backward (after the z scratch), byte offsets.
 struct TcBwdLayout {
     size_t zs, bp, dz, dzb, dbpart, dpart, total;
@@ -611,8 +659,8 @@ TcBwdLayout tc_bwd_layout(const Prob& p) {
     L.per_cta = std::max<int64_t>(1, (L.n_items + sms - 1) / sms);
     L.grid = (int)((L.n_items + L.per_cta - 1) / L.per_cta);
     L.pieces = (int)(L.n_tiles / L.per_cta + 2);
-    L.n_dblk = (int)((p.d + 255) / 256);
-    L.n_split = std::max<int>(1, std::min<int>(sms / L.n_dblk, (int)L.n_tiles));
+    L.n_dblk = gen_bwd_dblk(p.d, (int)p.r);
+    L.n_split = gen_bwd_splits(p.N, p.d, (int)p.r);
     size_t off = 0;
     L.zs = off;      off = al256(off + (size_t)p.N * p.r * 2);                     // z scratch (bf16)
     L.bp = off;      off = al256(off + (size_t)p.r * p.C * p.K * 2);               // tap-major B
@@ -673,18 +721,7 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     DC_LAUNCH(kTcReduce, st, dz_to_bf16_kernel<<<grid_for(p.N * p.r / 4), 256, 0, st>>>(
         reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb), p.N * p.r / 4));
     // generator backward: dA = h^T dz, dh = dz A^T
-    CUtensorMap tx, th, tp;
-    if (!make_tmap_bf16(&tx, dzb, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&th, h, p.d, p.N, p.hs, 64, 128) ||
-        !make_tmap_bf16(&tp, A, p.r, p.d, p.r, 64, 256))
-        return cudaErrorInvalidValue;
-    GenBwdArgs ga{p.N, p.d, (int)p.r, (int)((p.r + 15) / 16 * 16), p.hs, L.n_dblk, L.n_split, L.n_tiles,
-                  static_cast<__nv_bfloat16*>(dh), dpart, err};
-    e = cudaFuncSetAttribute(gen_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGbSmem);
-    if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcGenBwd, st, gen_bwd_kernel<<<L.n_dblk * L.n_split, kThreads, kGbSmem, st>>>(tx, th, tp, ga));
-    DC_LAUNCH(kTcReduce, st, reduce_splits_kernel<<<grid_for(p.d * p.r / 4 * 32), 256, 0, st>>>(
-        dpart, dA, p.d * p.r, L.n_split));
-    return cudaGetLastError();
+    return tc_gen_backward(dzb, (int)p.r, h, p.hs, A, p.N, p.d, dh, dA, dpart, err, st);
 }
 
 }  // namespace dynconv

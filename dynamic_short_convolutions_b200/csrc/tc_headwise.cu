@@ -1,0 +1,216 @@
+// tc_headwise.cu -- the head-wise dynamic short convolution, bf16 storage, fp32 accumulation.
+//
+// Parameterization 2 of "Dynamic Short Convolutions Improve Transformers"
+// (gist.science technical summary, "Dynamic Short Convolutions"): one K-tap filter
+// per head, shared by the head's head_dim consecutive channels,
+//   wh[n, q*K + j] = sum_i h[n, i] W[i, q*K + j]                      (tensor cores)
+//   y[n, c]  = u[n, c] + sum_{j <= n - s(n)} wh[n, (c/hd)*K + j] u[n-j, c]
+// and the adjoint
+//   du[m, c] = g[m, c] + sum_{j < e(m) - m} wh[m+j, (c/hd)*K + j] g[m+j, c]
+//   dwh[n, q*K + j] = sum_{c in head q} [j <= n - s(n)] g[n, c] u[n-j, c]   (warp shuffles)
+//   dW = h^T dwh,  dh = dwh W^T                                        (tensor cores)
+// The conv kernels are memory-bound CUDA-core kernels: a block covers 64 tokens x 256
+// channels, a thread 8 channels of one token per step (16-byte loads and stores along
+// C); the K-1 earlier/later rows a token needs were just read by the block's other
+// warps and come from L1/L2.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "prof.h"
+#include "tc_common.cuh"
+#include "tmap.h"
+
+namespace dynconv {
+
+cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
+                          int64_t out_ld, uint32_t* err, cudaStream_t st);
+cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
+                            void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st);
+int gen_bwd_splits(int64_t N, int64_t d, int R);
+
+namespace {
+
+using namespace tc;
+
+constexpr int kTokPerBlock = 64;
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16_lo(w[i]);
+        f[2 * i + 1] = bf16_hi(w[i]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+}
+
+__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+template <int K>
+__global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
+                                                          const __nv_bfloat16* __restrict__ wh, int R, int hd,
+                                                          int64_t N, int64_t C, int64_t seqlen,
+                                                          const int32_t* __restrict__ cu, int64_t n_docs,
+                                                          __nv_bfloat16* __restrict__ y) {
+    const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
+    const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
+    const int q = (int)(c / hd);
+    const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
+    const int64_t n1 = min(N, n0 + kTokPerBlock);
+    for (int64_t n = n0 + tl; n < n1; n += 8) {
+        const int64_t pos = n - seg_start(n, cu, n_docs, seqlen);
+        float acc[8], uf[8];
+        unpack8(*reinterpret_cast<const uint4*>(u + n * us + c), acc);
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            if (j <= pos) {
+                const float w = ldbf(wh + n * R + q * K + j);
+                unpack8(*reinterpret_cast<const uint4*>(u + (n - j) * us + c), uf);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, uf[i], acc[i]);
+            }
+        }
+        *reinterpret_cast<uint4*>(y + n * C + c) = pack8(acc);
+    }
+}
+
+// L = head_dim / 8 lanes hold one head's channels (a power of two <= 32, aligned in the warp).
+template <int K>
+__global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* __restrict__ g,
+                                                          const __nv_bfloat16* __restrict__ u, int64_t us,
+                                                          const __nv_bfloat16* __restrict__ wh, int R, int hd,
+                                                          int64_t N, int64_t C, int64_t seqlen,
+                                                          const int32_t* __restrict__ cu, int64_t n_docs,
+                                                          __nv_bfloat16* __restrict__ du,
+                                                          __nv_bfloat16* __restrict__ dwh) {
+    const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
+    const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
+    const int q = (int)(c / hd);
+    const int L = hd >> 3;
+    const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
+    const int64_t n1 = min(N, n0 + kTokPerBlock);
+    for (int64_t n = n0 + tl; n < n1; n += 8) {
+        int64_t sb, eb;
+        seg_bounds(n, cu, n_docs, seqlen, N, sb, eb);
+        const int64_t pos = n - sb, epos = eb - 1 - n;
+        float gn[8], acc[8], tmp[8];
+        unpack8(*reinterpret_cast<const uint4*>(g + n * C + c), gn);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = gn[i];
+        float part[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            if (j <= epos) {                        // du: the filter of token n+j, tap j
+                const float w = ldbf(wh + (n + j) * R + q * K + j);
+                unpack8(*reinterpret_cast<const uint4*>(g + (n + j) * C + c), tmp);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, tmp[i], acc[i]);
+            }
+            float pj = 0.f;                         // dwh partial over this thread's 8 channels
+            if (j <= pos) {
+                unpack8(*reinterpret_cast<const uint4*>(u + (n - j) * us + c), tmp);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pj = fmaf(gn[i], tmp[i], pj);
+            }
+            part[j] = pj;
+        }
+        *reinterpret_cast<uint4*>(du + n * C + c) = pack8(acc);
+        // sum over the head's L lanes (fixed butterfly: deterministic)
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            for (int off = L >> 1; off > 0; off >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
+        if ((gl & (L - 1)) == 0)
+#pragma unroll
+            for (int j = 0; j < K; ++j) dwh[n * R + q * K + j] = __float2bfloat16_rn(part[j]);
+    }
+}
+
+inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+// Workspace of the head-wise tensor-core path (inside the tensor-core region).
+struct TcHwLayout {
+    size_t wh, dwh, dpart, total;
+};
+
+TcHwLayout tc_hw_layout(const Prob& p) {
+    TcHwLayout L{};
+    size_t off = 0;
+    L.wh = off;     off = al256(off + (size_t)p.N * p.R * 2);
+    L.dwh = off;    off = al256(off + (size_t)p.N * p.R * 2);
+    L.dpart = off;  off = al256(off + (size_t)gen_bwd_splits(p.N, p.d, (int)p.R) * p.d * p.R * 4);
+    L.total = off;
+    return L;
+}
+
+bool tc_headwise_supported(const Prob& p) {
+    if (p.dtype != 1 || p.kind != 1) return false;
+    if (p.R > 128 || p.R % 8 != 0) return false;
+    if (p.hd < 8 || p.hd > 256 || (p.hd & (p.hd - 1)) != 0) return false;
+    if (p.C % 256 != 0 || p.d % 8 != 0) return false;
+    return p.K >= 1 && p.K <= 4;
+}
+
+template <int K>
+static void launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, cudaStream_t st) {
+    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
+    DC_LAUNCH(kTcHeadwiseFwd, st, hw_conv_fwd_kernel<K><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
+        p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
+}
+
+template <int K>
+static void launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
+                          cudaStream_t st) {
+    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
+    DC_LAUNCH(kTcHeadwiseBwd, st, hw_conv_bwd_kernel<K><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
+        static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, p.cu, p.n_docs,
+        static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
+}
+
+cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, const void* W, void* y, void* z_save,
+                                char* tcws, uint32_t* err, cudaStream_t st) {
+    const TcHwLayout L = tc_hw_layout(p);
+    void* wh = z_save ? z_save : static_cast<void*>(tcws + L.wh);
+    cudaError_t e = tc_gen_launch(h, p.hs, W, p.N, p.d, (int)p.R, wh, p.R, err, st);
+    if (e != cudaSuccess) return e;
+    switch (p.K) {
+        case 1: launch_hw_fwd<1>(p, u, wh, y, st); break;
+        case 2: launch_hw_fwd<2>(p, u, wh, y, st); break;
+        case 3: launch_hw_fwd<3>(p, u, wh, y, st); break;
+        default: launch_hw_fwd<4>(p, u, wh, y, st); break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, const void* h, const void* W,
+                                 const void* z_saved, void* du, void* dh, float* dW, char* tcws, uint32_t* err,
+                                 cudaStream_t st) {
+    const TcHwLayout L = tc_hw_layout(p);
+    const void* wh = z_saved;
+    if (!wh) {
+        void* whs = tcws + L.wh;
+        cudaError_t e = tc_gen_launch(h, p.hs, W, p.N, p.d, (int)p.R, whs, p.R, err, st);
+        if (e != cudaSuccess) return e;
+        wh = whs;
+    }
+    void* dwh = tcws + L.dwh;
+    switch (p.K) {
+        case 1: launch_hw_bwd<1>(p, g, u, wh, du, dwh, st); break;
+        case 2: launch_hw_bwd<2>(p, g, u, wh, du, dwh, st); break;
+        case 3: launch_hw_bwd<3>(p, g, u, wh, du, dwh, st); break;
+        default: launch_hw_bwd<4>(p, g, u, wh, du, dwh, st); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return tc_gen_backward(dwh, (int)p.R, h, p.hs, W, p.N, p.d, dh, dW, reinterpret_cast<float*>(tcws + L.dpart),
+                           err, st);
+}
+
+}  // namespace dynconv

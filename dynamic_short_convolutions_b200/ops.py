@@ -76,7 +76,8 @@ class DynamicShortConv(torch.autograd.Function):
         seqlen = N // batch
         plan = DynConvPlan(kind, u.dtype, batch, seqlen, d, C, ksize, rank, head_dim, u.stride(0), h.stride(0),
                            algo=algo, device=u.device)
-        z = torch.empty((N, rank), dtype=u.dtype, device=u.device) if A is not None else None
+        R = rank if A is not None else (C // head_dim) * ksize
+        z = torch.empty((N, R), dtype=u.dtype, device=u.device)    # generator output, reused by backward
         y = plan.forward(u, h, A, B_or_W, cu_seqlens, z_save=z)
         ctx.plan = plan
         ctx.save_for_backward(u, h, A, B_or_W, cu_seqlens, z)

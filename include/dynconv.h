@@ -104,8 +104,9 @@ DYNCONV_API size_t dynconv_workspace_bytes(const dynconv_desc *desc);
  *   A      [d, r] (low-rank) or NULL (head-wise)
  *   B_or_W [r, C*K] (low-rank) or [d, H*K] (head-wise)
  *   y      [N, C] output, dense
- *   z_save nullable; low-rank only: receives z = h A as [N, r] (storage dtype)
- *          for the backward pass to reuse. */
+ *   z_save nullable; receives the generator output [N, R] in the storage
+ *          dtype, R = r (low-rank: z = h A) or H*K (head-wise: the per-head
+ *          filters h W), for the backward pass to reuse. */
 DYNCONV_API dynconv_status dynconv_fwd(const dynconv_desc *desc, const void *u, const void *h, const void *A,
                            const void *B_or_W, void *y, void *z_save, void *ws, size_t ws_bytes,
                            void *stream);
@@ -123,7 +124,8 @@ DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const in
 
 /* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch).
  *   g        [N, C] upstream gradient dL/dy, dense
- *   z_saved  nullable: z from the forward pass (low-rank); NULL recomputes it
+ *   z_saved  nullable: the generator output saved by the forward ([N, r] or
+ *            [N, H*K]); NULL recomputes it
  *   du       [N, C] output dL/du, dense
  *   dh       nullable [N, d] output dL/dh, dense
  *   dA       [d, r] fp32 output (low-rank; ignored for head-wise)

@@ -71,12 +71,12 @@ def gpu_run(w, layer, t, algo=0, varlen=None, z_roundtrip=True, want_dh=True, de
     A = t.get("A")
     BW = t["B"] if w.kind == W.LOWRANK else t["W"]
     cu = t["cu_seqlens"] if varlen else None
-    z = torch.empty((N, w.rank), dtype=W.storage_dtype(w), device=t["u"].device) \
-        if (kind == L.LOWRANK and z_roundtrip) else None
+    R = w.rank if kind == L.LOWRANK else (C // w.head_dim) * w.ksize
+    z = torch.empty((N, R), dtype=W.storage_dtype(w), device=t["u"].device) if z_roundtrip else None
     y = plan.forward(t["u"], t["h"], A, BW, cu, z_save=z)
     out = plan.backward(t["g"], t["u"], t["h"], A, BW, cu, z_saved=z, want_dh=want_dh)
     st = L.dynconv_device_status(plan.ws)
     assert st == 0, L.dynconv_last_error()
     torch.cuda.synchronize()
-    res = dict(y=y, z=z, du=out["du"], dh=out["dh"], dA=out["dA"], dBW=out["dBW"])
+    res = dict(y=y, z=z if kind == L.LOWRANK else None, du=out["du"], dh=out["dh"], dA=out["dA"], dBW=out["dBW"])
     return {k: (W.to_f64(v) if v is not None else None) for k, v in res.items()}

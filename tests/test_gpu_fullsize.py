@@ -37,7 +37,8 @@ def _run_layer(w, layer, li):
     A = t.get("A")
     BW = t["B"] if kind == L.LOWRANK else t["W"]
     cu = t["cu_seqlens"] if w.varlen else None
-    z = torch.empty((w.tokens, w.rank), dtype=W.storage_dtype(w), device="cuda") if kind == L.LOWRANK else None
+    R = w.rank if kind == L.LOWRANK else (layer.channels // w.head_dim) * w.ksize
+    z = torch.empty((w.tokens, R), dtype=W.storage_dtype(w), device="cuda")
     y = plan.forward(t["u"], t["h"], A, BW, cu, z_save=z)
     out = plan.backward(t["g"], t["u"], t["h"], A, BW, cu, z_saved=z)
     assert L.dynconv_device_status(plan.ws) == 0, L.dynconv_last_error()
@@ -66,7 +67,7 @@ def test_full_size_sampled(name):
         assert_close(tag + ":y", W.to_f64(y)[rows], yr, w.dtype)
         assert_close(tag + ":du", W.to_f64(out["du"])[rows], dur, w.dtype)
         assert_close(tag + ":dh", W.to_f64(out["dh"])[rows], dhr, w.dtype)
-        if z is not None:
+        if zr is not None:
             assert_close(tag + ":z", W.to_f64(z)[rows], zr, w.dtype)
         d, C, K = layer.d_model, layer.channels, w.ksize
         if w.kind == W.LOWRANK:
