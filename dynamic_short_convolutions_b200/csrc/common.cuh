@@ -38,6 +38,44 @@ __device__ __forceinline__ int64_t seg_start(int64_t n, const int32_t* __restric
     return s > n ? n : s;
 }
 
+// seg_start for token indices below 2^31 (32-bit arithmetic: the tensor-core
+// kernels require N < 2^31).
+__device__ __forceinline__ int32_t seg_start32(int32_t n, const int32_t* __restrict__ cu, int32_t n_docs,
+                                               int32_t seqlen) {
+    int32_t s;
+    if (cu == nullptr) {
+        s = n - (int32_t)((uint32_t)n % (uint32_t)seqlen);
+    } else {
+        int32_t lo = 0, hi = n_docs;
+        while (hi - lo > 1) {
+            const int32_t mid = (lo + hi) >> 1;
+            if (__ldg(cu + mid) <= n) lo = mid; else hi = mid;
+        }
+        s = __ldg(cu + lo);
+    }
+    s = s < 0 ? 0 : s;
+    return s > n ? n : s;
+}
+
+// seg_bounds for token indices below 2^31 (32-bit arithmetic).
+__device__ __forceinline__ void seg_bounds32(int32_t n, const int32_t* __restrict__ cu, int32_t n_docs,
+                                             int32_t seqlen, int32_t N, int32_t& s, int32_t& e) {
+    if (cu == nullptr) {
+        s = n - (int32_t)((uint32_t)n % (uint32_t)seqlen);
+        e = s + seqlen;
+    } else {
+        int32_t lo = 0, hi = n_docs;
+        while (hi - lo > 1) {
+            const int32_t mid = (lo + hi) >> 1;
+            if (__ldg(cu + mid) <= n) lo = mid; else hi = mid;
+        }
+        s = __ldg(cu + lo);
+        e = __ldg(cu + lo + 1);
+    }
+    s = s < 0 ? 0 : (s > n ? n : s);
+    e = e <= n ? n + 1 : (e > N ? N : e);
+}
+
 // Start s (first token) and end e (one past the last token) of the sequence /
 // packed document holding token n < N, clamped so that s <= n < e <= N whatever
 // cu_seqlens holds.

@@ -172,31 +172,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 }
 
 // =====================================================================================
-// lowrank_fwd_kernel<K>: one work item = (128-token tile m0, 64-channel chunk c0).
-//   stage smem: z tile [128][64] (K-major A) | B chunk as K atoms [64 r-rows][64] (MN-major B)
-//               | u tile [136 rows = m0-8 .. m0+127][64 channels]
+// lowrank_fwd_kernel<K>: work items (128-token tile m0, 64-channel chunk c0) in contiguous
+// chunk-major runs, one run per CTA, so the chunk's B stays in shared memory.
+//   stage smem (ring of kFwdStages): z tile [128][64] (K-major A) | u tile [136 rows =
+//               m0-8 .. m0+127][64 channels]
+//   resident:   B chunk as K atoms [64 r-rows][64] (MN-major B), reloaded when the chunk changes
 //   TMEM: W[128 tokens][64 K] fp32, column c K + j = w[m0 + row, c0 + c, j]; two buffers.
-//   epilogue (8 warps: a lane quarter and half of the 64 channels each):
-//             y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c] -> bf16 staging
-//             (128-byte swizzled) -> TMA store.
+//   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3..10 epilogue (a TMEM lane quarter and half of
+//   the channels each): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c]
+//   -> bf16 staging (128-byte swizzled) -> TMA store by warp 2.
 // =====================================================================================
 struct FwdArgs {
     int64_t N, C, seqlen, n_docs;
     const int32_t* cu;
     uint32_t* err;
+    int64_t per_cta;         // work items per CTA (contiguous run)
+    int ksteps;              // 16-wide K steps of the filter MMA: r / 16 rounded up
 };
 
+constexpr int kFwdStages = 4;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
+constexpr uint32_t kFwdStage = kZBytes + kUBytes;
+constexpr int kFwdThreads = 96 + kEpiThreads;      // producer, MMA, store warps + epilogue
 
 template <int K>
-constexpr uint32_t fwd_stage_bytes() { return kZBytes + K * 8192 + kUBytes; }
-template <int K>
-constexpr uint32_t fwd_smem_bytes() { return 1024 + 2 * fwd_stage_bytes<K>() + 2 * kYBytes; }
+struct FwdSmem {
+    static constexpr uint32_t bres = kFwdStages * kFwdStage;
+    static constexpr uint32_t ys = bres + K * 8192;
+    static constexpr uint32_t total = ys + 2 * kYBytes + 1024;
+};
 
-// y for 8 channels of one row from the K filter taps (wv[j*8 + c] = W[t, (g8*8 + c) K + j] is
-// loaded as K x8 column runs starting at column g8*8*K, i.e. wv[i] = column g8*8*K + i).
+// y for 8 channels of one row from the K filter taps (wv[c K + j] = W[t, (g*8 + c) K + j]).
 template <int K>
-__device__ __forceinline__ uint4 conv8(const uint32_t* wv, const uint4* uj, int64_t pos) {
+__device__ __forceinline__ uint4 conv8(const uint32_t* wv, const uint4* uj, int32_t pos) {
     float acc[8];
     const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
 #pragma unroll
@@ -224,28 +232,33 @@ __device__ __forceinline__ uint4 conv8(const uint32_t* wv, const uint4* uj, int6
 }
 
 template <int K>
-__global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
-                                                                    const __grid_constant__ CUtensorMap tm_b,
-                                                                    const __grid_constant__ CUtensorMap tm_u,
-                                                                    const __grid_constant__ CUtensorMap tm_y,
-                                                                    FwdArgs a) {
-    constexpr uint32_t SB = fwd_stage_bytes<K>();
+__global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                                     const __grid_constant__ CUtensorMap tm_b,
+                                                                     const __grid_constant__ CUtensorMap tm_u,
+                                                                     const __grid_constant__ CUtensorMap tm_y,
+                                                                     FwdArgs a) {
+    using S = FwdSmem<K>;
     constexpr int NMMA = 64 * K;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* ystage = sm + 2 * SB;
-    __shared__ uint64_t full[2], empty[2], tfull[2], tempty[2];
+    __shared__ uint64_t full[kFwdStages], empty[kFwdStages], bfull, bempty, tfull[2], tempty[2], yfull[2], yempty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n_tiles = (a.N + 127) / 128, n_chunks = a.C / 64;
-    const int64_t n_items = n_tiles * n_chunks;
+    const int64_t n_tiles = (a.N + 127) / 128, n_items = n_tiles * (a.C / 64);
+    const int64_t i0 = (int64_t)blockIdx.x * a.per_cta, i1 = min(i0 + a.per_cta, n_items);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kFwdStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + kEpiWarps);
-            mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], kEpiWarps);
+        }
+        mbar_init(&bfull, 1);
+        mbar_init(&bempty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&yfull[b], kEpiWarps);
+            mbar_init(&yempty[b], 1);
         }
         abort_flag = 0;
         fence_mbar_init();
@@ -265,56 +278,84 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
 
     if (warp == 0) {
         if (lane == 0) {
-            uint32_t it = 0;
-            for (int64_t item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++it) {
+            int64_t prev = -1;
+            uint32_t cc = 0, it = 0;
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
                 const int64_t chunk = item / n_tiles, tile = item % n_tiles;
-                const int s = it & 1;
-                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
-                uint8_t* st = sm + s * SB;
-                mbar_arrive_expect_tx(&full[s], SB);
                 const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
+                if (chunk != prev) {
+                    if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
+                    mbar_arrive_expect_tx(&bfull, K * 8192);
+                    for (int j = 0; j < K; ++j) tma_load_2d(sm + S::bres + j * 8192, &tm_b, &bfull, c0 * K + 64 * j, 0);
+                    ++cc;
+                    prev = chunk;
+                }
+                const int s = it % kFwdStages;
+                if (!mbar_wait(&empty[s], ((it / kFwdStages) & 1) ^ 1, &abort_flag, a.err)) break;
+                uint8_t* st = sm + s * kFwdStage;
+                mbar_arrive_expect_tx(&full[s], kFwdStage);
                 tma_load_2d(st, &tm_z, &full[s], 0, m0);
-                for (int j = 0; j < K; ++j) tma_load_2d(st + kZBytes + j * 8192, &tm_b, &full[s], c0 * K + 64 * j, 0);
-                tma_load_2d(st + kZBytes + K * 8192, &tm_u, &full[s], c0, m0 - 8);
+                tma_load_2d(st + kZBytes, &tm_u, &full[s], c0, m0 - 8);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, NMMA, false, true);
-            uint32_t it = 0;
-            for (int64_t item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++it) {
-                const int s = it & 1;
-                const uint32_t ph = (it >> 1) & 1;
-                if (!mbar_wait(&tempty[s], ph ^ 1, &abort_flag, a.err)) break;
-                if (!mbar_wait(&full[s], ph, &abort_flag, a.err)) break;
+            const uint32_t b0 = smem_u32(sm + S::bres);
+            int64_t prev = -1;
+            uint32_t cc = 0, it = 0;
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
+                const int64_t chunk = item / n_tiles;
+                const bool last = (item + 1 == i1) || ((item + 1) / n_tiles != chunk);
+                if (chunk != prev) {
+                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
+                    ++cc;
+                    prev = chunk;
+                }
+                const int s = it % kFwdStages, b = it & 1;
+                if (!mbar_wait(&tempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                if (!mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
-                const uint32_t st = smem_u32(sm + s * SB);
-                for (int k = 0; k < 4; ++k)
-                    umma_bf16(tbase + s * 256, kmajor_desc(st, k), mnmajor_desc(st + kZBytes, 8192, 16 * k), idesc,
-                              k != 0);
-                umma_commit(&tfull[s]);
+                const uint32_t st = smem_u32(sm + s * kFwdStage);
+                for (int k = 0; k < a.ksteps; ++k)
+                    umma_bf16(tbase + b * 256, kmajor_desc(st, k), mnmajor_desc(b0, 8192, 16 * k), idesc, k != 0);
+                umma_commit(&tfull[b]);
                 umma_commit(&empty[s]);
+                if (last) umma_commit(&bempty);
             }
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t item = i0; item < i1; ++item, ++it) {
+                const int64_t chunk = item / n_tiles, tile = item % n_tiles;
+                const int b = it & 1;
+                if (!mbar_wait(&yfull[b], (it >> 1) & 1, &abort_flag, a.err)) break;
+                tma_store_2d(&tm_y, sm + S::ys + b * kYBytes, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                tma_store_commit();
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                mbar_arrive(&yempty[b]);
+            }
+            tma_store_wait_all();
         }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;      // channel groups 4*half .. 4*half+3
+        const int half = (warp - 3) >> 2;      // channel groups 4*half .. 4*half+3
         const int row = q * 32 + lane;
-        const int et = threadIdx.x - 64;       // 0 .. kEpiThreads-1
         uint32_t it = 0;
-        for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
-            const int64_t chunk = item / n_tiles, tile = item % n_tiles;
-            const int s = it & 1;
-            const uint32_t ph = (it >> 1) & 1;
-            const bool ok = mbar_wait(&tfull[s], ph, &abort_flag, a.err) && mbar_wait(&full[s], ph, &abort_flag, a.err);
-            if (et == 0) tma_store_wait_read_le1();     // the store that last used this staging buffer
+        for (int64_t item = i0; item < i1; ++item, ++it) {
+            const int64_t tile = item % n_tiles;
+            const int s = it % kFwdStages, b = it & 1;
+            const bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, &abort_flag, a.err) &&
+                            mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err) &&
+                            mbar_wait(&yempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err);
             if (epi_bar_any<kEpiThreads>(!ok)) break;
             tc_fence_after();
-            const int64_t n = tile * 128 + row;
-            const int64_t pos = n < a.N ? n - seg_start(n, a.cu, a.n_docs, a.seqlen) : 0;
-            const uint8_t* us = sm + s * SB + kZBytes + K * 8192;
-            uint8_t* ys = ystage + s * kYBytes;
-            const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + s * 256;
+            const int32_t n = (int32_t)(tile * 128) + row;
+            const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
+            const uint8_t* us = sm + s * kFwdStage + kZBytes;
+            uint8_t* ys = sm + S::ys + b * kYBytes;
+            const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
 #pragma unroll 1
             for (int gp = 0; gp < 2; ++gp) {            // two groups of 8 channels per batch
                 const int g0 = 4 * half + 2 * gp;
@@ -336,19 +377,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
                     *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = conv8<K>(wv[x], uj[x], pos);
             }
             tc_fence_before();
+            fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&tempty[s]);
+                mbar_arrive(&tempty[b]);
                 mbar_arrive(&empty[s]);
-            }
-            fence_async_smem();
-            epi_bar_sync<kEpiThreads>();
-            if (et == 0) {
-                tma_store_2d(&tm_y, ys, (int32_t)(chunk * 64), (int32_t)(tile * 128));
-                tma_store_commit();
+                mbar_arrive(&yfull[b]);
             }
         }
-        if (et == 0) tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -360,12 +396,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) lowrank_fwd_kernel(const __grid
 
 template <int K>
 cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
-                               const CUtensorMap& ty, const FwdArgs& fa, int64_t items, cudaStream_t st) {
-    constexpr uint32_t smem = fwd_smem_bytes<K>();
+                               const CUtensorMap& ty, FwdArgs fa, int64_t items, cudaStream_t st) {
+    constexpr uint32_t smem = FwdSmem<K>::total;
     cudaError_t e = cudaFuncSetAttribute(lowrank_fwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)std::min<int64_t>(items, num_sms());
-    DC_LAUNCH(kTcLowrankFwd, st, lowrank_fwd_kernel<K><<<grid, kTcThreads, smem, st>>>(tz, tb, tu, ty, fa));
+    fa.per_cta = (items + num_sms() - 1) / num_sms();
+    const unsigned grid = (unsigned)((items + fa.per_cta - 1) / fa.per_cta);
+    DC_LAUNCH(kTcLowrankFwd, st, lowrank_fwd_kernel<K><<<grid, kFwdThreads, smem, st>>>(tz, tb, tu, ty, fa));
     return cudaGetLastError();
 }
 
@@ -416,6 +453,7 @@ bool tc_supported(const Prob& p) {
     if (p.r % 8 != 0 || p.r > 64) return false;
     if (p.C % 64 != 0 || p.d % 8 != 0) return false;
     if (p.K < 1 || p.K > 4) return false;
+    if (p.N >= (int64_t(1) << 31)) return false;
     return tensor_map_encoder() != nullptr;
 }
 
@@ -440,7 +478,7 @@ cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* 
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
         !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
         return cudaErrorInvalidValue;
-    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err};
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16)};
     const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
     switch (p.K) {
         case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);
@@ -460,7 +498,7 @@ cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, cons
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
         !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
         return cudaErrorInvalidValue;
-    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err};
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16)};
     const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
     switch (p.K) {
         case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);

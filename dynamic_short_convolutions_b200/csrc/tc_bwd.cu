@@ -51,15 +51,24 @@ using namespace tc;
 constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quarter
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;         // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
+constexpr int kBwdThreads = 96 + kEpiThreads;      // + warp 2 for TMA stores; epilogue warps 3..
 constexpr uint32_t kRowTile = 136 * 128;     // 136-row, 64-column bf16 tile
 constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
 
-__global__ void permute_b_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat16* __restrict__ Bp, int64_t r,
-                                 int64_t C, int64_t K) {
-    const int64_t total = r * C * K;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t k = e / (C * K), col = e % (C * K), c = col / K, j = col % K;
-        Bp[k * C * K + j * C + c] = B[e];
+// Backward set-up in one launch: zero the fp32 dz accumulator (float4 stores) and write
+// the tap-major copy Bp[k, j C + c] = B[k, c K + j] (coalesced over the output index).
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat16* __restrict__ Bp, int r, int C,
+                                int K, float4* __restrict__ dz4, int64_t n_dz4) {
+    const int64_t n_b = (int64_t)r * C * K;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_dz4 + n_b;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        if (e < n_dz4) {
+            dz4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            const int o = (int)(e - n_dz4);
+            const int k = o / (C * K), rem = o - k * (C * K), j = rem / C, c = rem - j * C;
+            Bp[o] = B[(int64_t)k * C * K + (int64_t)c * K + j];
+        }
     }
 }
 
@@ -72,6 +81,7 @@ struct BwdArgs {
     float* dz_acc;            // [N, r] fp32, zero on entry
     float* dB_part;           // [n_chunks][pieces][64 K][r]
     uint32_t* err;
+    int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
 };
 
 template <int K>
@@ -85,7 +95,7 @@ struct BwdSmem {
 };
 
 template <int K>
-__global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+__global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                   const __grid_constant__ CUtensorMap tm_g,
                                                                   const __grid_constant__ CUtensorMap tm_u,
                                                                   const __grid_constant__ CUtensorMap tm_bp,
@@ -95,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
     constexpr int NBLK = S::NA / 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dzfull;
+    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dzfull, dufull, duempty;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -111,6 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
         mbar_init(&wfull, 1);
         mbar_init(&wempty, kEpiWarps);
         mbar_init(&dzfull, 1);
+        mbar_init(&dufull, kEpiWarps);
+        mbar_init(&duempty, 1);
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_z);
@@ -123,10 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp >= 2) {
+    if (warp >= 3) {
         // dW atoms past the last tap stay zero for the whole kernel (they pad the
         // last 128-row block of the dB MMA).
-        const int row = (warp & 3) * 32 + lane, half = (warp - 2) >> 2;
+        const int row = (warp & 3) * 32 + lane, half = (warp - 3) >> 2;
         for (int at = K; at < S::NA; ++at)
             for (int q = 4 * half; q < 4 * half + 4; ++q)
                 *reinterpret_cast<uint4*>(sm + S::dw + at * kAtom128 + sw128_off(row, q)) = make_uint4(0, 0, 0, 0);
@@ -187,8 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
                 // MMA1: Wd_j = z[j : j + 128] . Bp_j  (K-major A starting j rows in; MN-major B)
 #pragma unroll
                 for (int j = 0; j < K; ++j)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
+                    for (int k = 0; k < a.ksteps; ++k)
                         umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k), mnmajor_desc(bp0 + j * 8192, 8192, 16 * k),
                                   idesc_w, k != 0);
                 umma_commit(&wfull);
@@ -213,11 +224,23 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
                 if (last) umma_commit(&bempty);
             }
         }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t item = i0; item < i1; ++item, ++it) {
+                const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
+                if (!mbar_wait(&dufull, it & 1, &abort_flag, a.err)) break;
+                tma_store_2d(&tm_du, sm + S::dust, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                tma_store_commit();
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                mbar_arrive(&duempty);
+            }
+            tma_store_wait_all();
+        }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;      // channel groups 4*half..4*half+3; dz/dB columns 8*half + 16 i
+        const int half = (warp - 3) >> 2;      // channel groups 4*half..4*half+3; dz/dB columns 8*half + 16 i
         const int row = q * 32 + lane;
-        const int et = threadIdx.x - 64;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint8_t* dws = sm + S::dw;
         uint8_t* dus = sm + S::dust;
@@ -227,15 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
             const bool last = (item + 1 == i1) || ((item + 1) / a.n_tiles != chunk);
             const int s = it & 1;
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
-                      mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err);
-            if (et == 0) tma_store_wait_all();       // du staging and dW are free again
+                      mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err) &&
+                      mbar_wait(&duempty, (it & 1) ^ 1, &abort_flag, a.err);   // du staging free again
             if (epi_bar_any<kEpiThreads>(!ok)) break;
             tc_fence_after();
-            const int64_t n = tile * 128 + row;
-            int64_t pos = -1, epos = -1;             // valid past / future taps of this row
+            const int32_t n = (int32_t)(tile * 128) + row;
+            int32_t pos = -1, epos = -1;             // valid past / future taps of this row
             if (n < a.N) {
-                int64_t sb, eb;
-                seg_bounds(n, a.cu, a.n_docs, a.seqlen, a.N, sb, eb);
+                int32_t sb, eb;
+                seg_bounds32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen, (int32_t)a.N, sb, eb);
                 pos = n - sb;
                 epos = eb - 1 - n;
             }
@@ -305,11 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
             if (lane == 0) {
                 mbar_arrive(&wempty);
                 mbar_arrive(&empty[s]);
-            }
-            epi_bar_sync<kEpiThreads>();
-            if (et == 0) {
-                tma_store_2d(&tm_du, dus, (int32_t)(chunk * 64), (int32_t)(tile * 128));
-                tma_store_commit();
+                mbar_arrive(&dufull);
             }
             ok = mbar_wait(&dzfull, it & 1, &abort_flag, a.err);
             if (epi_bar_any<kEpiThreads>(!ok)) break;
@@ -320,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
                 tmem_ld8(lane_base + kColDz + c, v);
                 tmem_wait_ld();
                 if (n < a.N) {
-                    float4* dst = reinterpret_cast<float4*>(a.dz_acc + n * a.r + c);
+                    float4* dst = reinterpret_cast<float4*>(a.dz_acc + (int64_t)n * a.r + c);
                     atomicAdd(dst, make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
                                                __uint_as_float(v[3])));
                     atomicAdd(dst + 1, make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]),
@@ -350,7 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1) lowrank_bwd_kernel(const __grid_c
             }
             tc_fence_before();
         }
-        if (et == 0) tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -600,7 +618,7 @@ cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUten
     constexpr uint32_t smem = BwdSmem<K>::total;
     cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcLowrankBwd, st, lowrank_bwd_kernel<K><<<grid, kThreads, smem, st>>>(tz, tg, tu, tbp, tdu, ba));
+    DC_LAUNCH(kTcLowrankBwd, st, lowrank_bwd_kernel<K><<<grid, kBwdThreads, smem, st>>>(tz, tg, tu, tbp, tdu, ba));
     return cudaGetLastError();
 }
 
@@ -688,9 +706,10 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     __nv_bfloat16* dzb = reinterpret_cast<__nv_bfloat16*>(tcws + L.dzb);
     float* dbpart = reinterpret_cast<float*>(tcws + L.dbpart);
     float* dpart = reinterpret_cast<float*>(tcws + L.dpart);
-    DC_LAUNCH(kTcPrep, st, permute_b_kernel<<<grid_for(p.r * p.C * p.K), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(B), bp, p.r, p.C, p.K));
-    cudaError_t e = cudaMemsetAsync(dz, 0, (size_t)p.N * p.r * 4, st);
+    DC_LAUNCH(kTcPrep, st, bwd_prep_kernel<<<grid_for(p.N * p.r / 4 + p.r * p.C * p.K), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, reinterpret_cast<float4*>(dz),
+        p.N * p.r / 4));
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap tz, tg, tu, tbp, tdu;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
@@ -698,7 +717,7 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128))
         return cudaErrorInvalidValue;
     BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
-               L.per_cta, L.pieces, dz, dbpart, err};
+               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16)};
     switch (p.K) {
         case 1: e = launch_bwd<1>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
         case 2: e = launch_bwd<2>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;

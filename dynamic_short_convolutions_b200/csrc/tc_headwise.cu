@@ -51,6 +51,31 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 __device__ __forceinline__ float ldbf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 template <int K>
+__device__ __forceinline__ void hw_fwd_token(const __nv_bfloat16* __restrict__ u, int64_t us,
+                                             const __nv_bfloat16* __restrict__ wh, int R, int q, int64_t n,
+                                             int64_t c, int64_t C, int64_t seqlen, const int32_t* __restrict__ cu,
+                                             int64_t n_docs, __nv_bfloat16* __restrict__ y) {
+    const int32_t pos = (int32_t)n - seg_start32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen);
+    uint4 uv[K];
+    float w[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {          // issue every load of the token first
+        const bool v = j <= pos;
+        uv[j] = v ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
+        w[j] = v ? ldbf(wh + n * R + q * K + j) : 0.f;
+    }
+    float acc[8], uf[8];
+    unpack8(uv[0], acc);
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        unpack8(uv[j], uf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], uf[i], acc[i]);
+    }
+    *reinterpret_cast<uint4*>(y + n * C + c) = pack8(acc);
+}
+
+template <int K>
 __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
                                                           const __nv_bfloat16* __restrict__ wh, int R, int hd,
                                                           int64_t N, int64_t C, int64_t seqlen,
@@ -61,20 +86,9 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
     const int q = (int)(c / hd);
     const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
     const int64_t n1 = min(N, n0 + kTokPerBlock);
-    for (int64_t n = n0 + tl; n < n1; n += 8) {
-        const int64_t pos = n - seg_start(n, cu, n_docs, seqlen);
-        float acc[8], uf[8];
-        unpack8(*reinterpret_cast<const uint4*>(u + n * us + c), acc);
-#pragma unroll
-        for (int j = 0; j < K; ++j) {
-            if (j <= pos) {
-                const float w = ldbf(wh + n * R + q * K + j);
-                unpack8(*reinterpret_cast<const uint4*>(u + (n - j) * us + c), uf);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, uf[i], acc[i]);
-            }
-        }
-        *reinterpret_cast<uint4*>(y + n * C + c) = pack8(acc);
+    for (int64_t n = n0 + tl; n < n1; n += 16) {       // two tokens per step: more loads in flight
+        hw_fwd_token<K>(u, us, wh, R, q, n, c, C, seqlen, cu, n_docs, y);
+        if (n + 8 < n1) hw_fwd_token<K>(u, us, wh, R, q, n + 8, c, C, seqlen, cu, n_docs, y);
     }
 }
 
