@@ -108,28 +108,32 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
     const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
     const int64_t n1 = min(N, n0 + kTokPerBlock);
     for (int64_t n = n0 + tl; n < n1; n += 8) {
-        int64_t sb, eb;
-        seg_bounds(n, cu, n_docs, seqlen, N, sb, eb);
-        const int64_t pos = n - sb, epos = eb - 1 - n;
+        int32_t sb, eb;
+        seg_bounds32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb, eb);
+        const int32_t pos = (int32_t)n - sb, epos = eb - 1 - (int32_t)n;
+        uint4 gv[K], uv[K];
+        float w[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {          // issue every load of the token first
+            const bool f = j <= epos, p = j <= pos;
+            gv[j] = f ? *reinterpret_cast<const uint4*>(g + (n + j) * C + c) : make_uint4(0, 0, 0, 0);
+            w[j] = f ? ldbf(wh + (n + j) * R + q * K + j) : 0.f;     // du: filter of token n+j, tap j
+            uv[j] = p ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
+        }
         float gn[8], acc[8], tmp[8];
-        unpack8(*reinterpret_cast<const uint4*>(g + n * C + c), gn);
+        unpack8(gv[0], gn);
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = gn[i];
         float part[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {
-            if (j <= epos) {                        // du: the filter of token n+j, tap j
-                const float w = ldbf(wh + (n + j) * R + q * K + j);
-                unpack8(*reinterpret_cast<const uint4*>(g + (n + j) * C + c), tmp);
+            unpack8(gv[j], tmp);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, tmp[i], acc[i]);
-            }
-            float pj = 0.f;                         // dwh partial over this thread's 8 channels
-            if (j <= pos) {
-                unpack8(*reinterpret_cast<const uint4*>(u + (n - j) * us + c), tmp);
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], tmp[i], acc[i]);
+            unpack8(uv[j], tmp);                // dwh partial over this thread's 8 channels
+            float pj = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) pj = fmaf(gn[i], tmp[i], pj);
-            }
+            for (int i = 0; i < 8; ++i) pj = fmaf(gn[i], tmp[i], pj);
             part[j] = pj;
         }
         *reinterpret_cast<uint4*>(du + n * C + c) = pack8(acc);
