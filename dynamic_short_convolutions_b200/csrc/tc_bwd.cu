@@ -51,7 +51,6 @@ using namespace tc;
 constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quarter
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;         // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
-constexpr int kBwdThreads = 96 + kEpiThreads;      // + warp 2 for TMA stores; epilogue warps 3..
 constexpr uint32_t kRowTile = 136 * 128;     // 136-row, 64-column bf16 tile
 constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
 
@@ -94,18 +93,28 @@ struct BwdSmem {
     static constexpr uint32_t total = dust + kAtom128 + 1024;
 };
 
+// Warp roles of lowrank_bwd_kernel: 0 TMA loads, 1 MMA issue (and TMEM owner), 2 TMA stores of
+// du, 3..10 the du / dw epilogue (GA: a TMEM lane quarter and half of the channels each),
+// 11..14 the dz / dB readout (GB: one TMEM lane quarter each).
+constexpr int kGaWarps = 8, kGbWarps = 4;
+constexpr int kBwdPipeThreads = 32 * (3 + kGaWarps + kGbWarps);
+
+// TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
+constexpr uint32_t kColDz = 256, kColDb = 384;
+
 template <int K>
-__global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
-                                                                  const __grid_constant__ CUtensorMap tm_g,
-                                                                  const __grid_constant__ CUtensorMap tm_u,
-                                                                  const __grid_constant__ CUtensorMap tm_bp,
-                                                                  const __grid_constant__ CUtensorMap tm_du,
-                                                                  BwdArgs a) {
+__global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                                         const __grid_constant__ CUtensorMap tm_g,
+                                                                         const __grid_constant__ CUtensorMap tm_u,
+                                                                         const __grid_constant__ CUtensorMap tm_bp,
+                                                                         const __grid_constant__ CUtensorMap tm_du,
+                                                                         BwdArgs a) {
     using S = BwdSmem<K>;
     constexpr int NBLK = S::NA / 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dzfull, dufull, duempty;
+    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dwready, dwfree, dzfull[2], dzempty[2],
+        dbfree, dufull, duempty;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,14 +123,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kEpiWarps);
+            mbar_init(&empty[s], 1 + kGaWarps);
+            mbar_init(&dzfull[s], 1);
+            mbar_init(&dzempty[s], kGbWarps);
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
         mbar_init(&wfull, 1);
-        mbar_init(&wempty, kEpiWarps);
-        mbar_init(&dzfull, 1);
-        mbar_init(&dufull, kEpiWarps);
+        mbar_init(&wempty, kGaWarps);
+        mbar_init(&dwready, kGaWarps);
+        mbar_init(&dwfree, 1);
+        mbar_init(&dbfree, kGbWarps);
+        mbar_init(&dufull, kGaWarps);
         mbar_init(&duempty, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -135,7 +148,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp >= 3) {
+    if (warp >= 3 && warp < 3 + kGaWarps) {
         // dW atoms past the last tap stay zero for the whole kernel (they pad the
         // last 128-row block of the dB MMA).
         const int row = (warp & 3) * 32 + lane, half = (warp - 3) >> 2;
@@ -148,14 +161,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base;
-    constexpr uint32_t kColDz = 256, kColDb = 320;
+    auto chunk_of = [&](int64_t item) { return item / a.n_tiles; };
 
     if (warp == 0) {
         if (lane == 0) {
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
             for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
-                const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
+                const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
                 if (chunk != prev) {
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * 8192);
@@ -180,55 +193,75 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
             const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
             const uint32_t idesc_db = idesc_bf16(128, a.ndz, true, true);
             const uint32_t bp0 = smem_u32(sm + S::bp), dw0 = smem_u32(sm + S::dw);
-            int64_t prev = -1;
-            uint32_t cc = 0, it = 0;
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
-                const int64_t chunk = item / a.n_tiles;
-                const bool first = chunk != prev;
-                const bool last = (item + 1 == i1) || ((item + 1) / a.n_tiles != chunk);
-                if (first) {
-                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
-                    ++cc;
-                    prev = chunk;
-                }
+            const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
+            uint32_t cc = 0;          // B loads consumed
+            uint32_t m = 0;           // chunks whose dB accumulation has started
+            // Filter MMA of item `it`: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows in).
+            auto mma1 = [&](uint32_t it) -> bool {
                 const int s = it & 1;
-                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) break;
-                if (!mbar_wait(&wempty, (it & 1) ^ 1, &abort_flag, a.err)) break;   // Wd free
+                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) return false;
                 tc_fence_after();
                 const uint32_t z0 = smem_u32(sm + s * S::stage);
-                // MMA1: Wd_j = z[j : j + 128] . Bp_j  (K-major A starting j rows in; MN-major B)
 #pragma unroll
                 for (int j = 0; j < K; ++j)
                     for (int k = 0; k < a.ksteps; ++k)
                         umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k), mnmajor_desc(bp0 + j * 8192, 8192, 16 * k),
                                   idesc_w, k != 0);
                 umma_commit(&wfull);
-                if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;         // dW(it) written
+                return true;
+            };
+            bool ok = nit > 0 && mbar_wait(&bfull, 0, &abort_flag, a.err);
+            if (ok) {
+                cc = 1;
+                ok = mma1(0);
+            }
+            for (uint32_t it = 0; ok && it < nit && !abort_flag; ++it) {
+                const int64_t item = i0 + it, chunk = chunk_of(item);
+                const bool first = it == 0 || chunk_of(item - 1) != chunk;
+                const bool has_next = it + 1 < nit;
+                const bool next_same = has_next && chunk_of(item + 1) == chunk;
+                const int s = it & 1, b = it & 1;
+                if (next_same) {          // the next filter MMA as soon as Wd has been read
+                    if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
+                    if (!mma1(it + 1)) break;
+                }
+                if (!mbar_wait(&dwready, it & 1, &abort_flag, a.err)) break;
+                if (!mbar_wait(&dzempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                if (first && m > 0 && !mbar_wait(&dbfree, (m - 1) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
-                // MMA2: dz = dW . Bp^T  (both K-major, K = (tap, channel))
+                const uint32_t z0 = smem_u32(sm + s * S::stage);
+                // dz = dW . Bp^T  (both K-major, K = (tap, channel))
 #pragma unroll
                 for (int j = 0; j < K; ++j)
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        umma_bf16(tbase + kColDz, kmajor_desc(dw0 + j * kAtom128, k), kmajor_desc(bp0 + j * 8192, k),
-                                  idesc_dz, (j | k) != 0);
-                // MMA3: dBt[blk] += dW^T . z  (both MN-major, K = 128 tokens)
+                        umma_bf16(tbase + kColDz + 64 * b, kmajor_desc(dw0 + j * kAtom128, k),
+                                  kmajor_desc(bp0 + j * 8192, k), idesc_dz, (j | k) != 0);
+                // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
 #pragma unroll
-                for (int b = 0; b < NBLK; ++b)
+                for (int bb = 0; bb < NBLK; ++bb)
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tbase + kColDb + 64 * b, mnmajor_desc(dw0 + 2 * b * kAtom128, kAtom128, 16 * ks),
+                        umma_bf16(tbase + kColDb + 64 * bb, mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks),
                                   mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
-                umma_commit(&dzfull);
+                if (first) ++m;
+                umma_commit(&dzfull[b]);
+                umma_commit(&dwfree);
                 umma_commit(&empty[s]);
-                if (last) umma_commit(&bempty);
+                if (has_next && !next_same) {      // chunk changes: B is reloaded after these MMAs
+                    umma_commit(&bempty);
+                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
+                    ++cc;
+                    if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
+                    if (!mma1(it + 1)) break;
+                }
             }
         }
     } else if (warp == 2) {
         if (lane == 0) {
             uint32_t it = 0;
             for (int64_t item = i0; item < i1; ++item, ++it) {
-                const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
+                const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
                 if (!mbar_wait(&dufull, it & 1, &abort_flag, a.err)) break;
                 tma_store_2d(&tm_du, sm + S::dust, (int32_t)(chunk * 64), (int32_t)(tile * 128));
                 tma_store_commit();
@@ -237,22 +270,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
             }
             tma_store_wait_all();
         }
-    } else {
+    } else if (warp < 3 + kGaWarps) {
+        // ---- GA: du (A1) and dw (A2) of each item
         const int q = warp & 3;
-        const int half = (warp - 3) >> 2;      // channel groups 4*half..4*half+3; dz/dB columns 8*half + 16 i
+        const int half = (warp - 3) >> 2;      // channel groups 4*half .. 4*half+3
         const int row = q * 32 + lane;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint8_t* dws = sm + S::dw;
         uint8_t* dus = sm + S::dust;
         uint32_t it = 0;
         for (int64_t item = i0; item < i1; ++item, ++it) {
-            const int64_t chunk = item / a.n_tiles, tile = item % a.n_tiles;
-            const bool last = (item + 1 == i1) || ((item + 1) / a.n_tiles != chunk);
+            const int64_t tile = item % a.n_tiles;
             const int s = it & 1;
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
                       mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err) &&
-                      mbar_wait(&duempty, (it & 1) ^ 1, &abort_flag, a.err);   // du staging free again
-            if (epi_bar_any<kEpiThreads>(!ok)) break;
+                      mbar_wait(&duempty, (it & 1) ^ 1, &abort_flag, a.err);
+            if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
             tc_fence_after();
             const int32_t n = (int32_t)(tile * 128) + row;
             int32_t pos = -1, epos = -1;             // valid past / future taps of this row
@@ -262,30 +295,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
                 pos = n - sb;
                 epos = eb - 1 - n;
             }
-            const uint8_t* zt = sm + s * S::stage;
-            const uint8_t* gt = zt + kRowTile;
-            const uint8_t* ut = zt + 2 * kRowTile;
-            (void)zt;
+            const uint8_t* gt = sm + s * S::stage + kRowTile;
+            const uint8_t* ut = gt + kRowTile;
+            // A1: du[t, c] = g[t, c] + sum_{j <= epos} Wd_j[t, c] g[t + j, c]
 #pragma unroll 1
             for (int g8 = 4 * half; g8 < 4 * half + 4; ++g8) {
                 uint32_t wv[K][8];
 #pragma unroll
                 for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * g8, wv[j]);
-                uint4 gg[K], uu[K];
+                uint4 gg[K];
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    gg[j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g8));
-                    uu[j] = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
-                }
+                for (int j = 0; j < K; ++j) gg[j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g8));
                 tmem_wait_ld();
+                float acc[8];
                 const uint32_t* g0 = reinterpret_cast<const uint32_t*>(&gg[0]);
-                float gv[8], acc[8];
 #pragma unroll
                 for (int c = 0; c < 8; c += 2) {
-                    gv[c] = bf16_lo(g0[c >> 1]);
-                    gv[c + 1] = bf16_hi(g0[c >> 1]);
-                    acc[c] = gv[c];
-                    acc[c + 1] = gv[c + 1];
+                    acc[c] = bf16_lo(g0[c >> 1]);
+                    acc[c + 1] = bf16_hi(g0[c >> 1]);
                 }
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
@@ -298,12 +325,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
                         }
                     }
                 }
-                uint4 pk;
-                pk.x = pack_bf16(acc[0], acc[1]);
-                pk.y = pack_bf16(acc[2], acc[3]);
-                pk.z = pack_bf16(acc[4], acc[5]);
-                pk.w = pack_bf16(acc[6], acc[7]);
-                *reinterpret_cast<uint4*>(dus + sw128_off(row, g8)) = pk;
+                *reinterpret_cast<uint4*>(dus + sw128_off(row, g8)) =
+                    make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                               pack_bf16(acc[6], acc[7]));
+            }
+            tc_fence_before();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&wempty);
+                mbar_arrive(&dufull);
+            }
+            // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16, one 64-channel atom per tap) once the
+            // dz / dB MMAs of the previous item have finished reading the dW tile
+            ok = mbar_wait(&dwfree, (it & 1) ^ 1, &abort_flag, a.err);
+            if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
+#pragma unroll 1
+            for (int g8 = 4 * half; g8 < 4 * half + 4; ++g8) {
+                uint4 uu[K];
+                const uint4 gv = *reinterpret_cast<const uint4*>(gt + sw128_off(row, g8));
+#pragma unroll
+                for (int j = 0; j < K; ++j) uu[j] = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
+                const uint32_t* g0 = reinterpret_cast<const uint32_t*>(&gv);
+                float gf[8];
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    gf[c] = bf16_lo(g0[c >> 1]);
+                    gf[c + 1] = bf16_hi(g0[c >> 1]);
+                }
 #pragma unroll
                 for (int j = 0; j < K; ++j) {
                     const bool v = j <= pos;
@@ -311,51 +360,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
                     float d[8];
 #pragma unroll
                     for (int c = 0; c < 8; c += 2) {
-                        d[c] = v ? gv[c] * bf16_lo(uj[c >> 1]) : 0.f;
-                        d[c + 1] = v ? gv[c + 1] * bf16_hi(uj[c >> 1]) : 0.f;
+                        d[c] = v ? gf[c] * bf16_lo(uj[c >> 1]) : 0.f;
+                        d[c + 1] = v ? gf[c + 1] * bf16_hi(uj[c >> 1]) : 0.f;
                     }
-                    uint4 dk;
-                    dk.x = pack_bf16(d[0], d[1]);
-                    dk.y = pack_bf16(d[2], d[3]);
-                    dk.z = pack_bf16(d[4], d[5]);
-                    dk.w = pack_bf16(d[6], d[7]);
-                    *reinterpret_cast<uint4*>(dws + j * kAtom128 + sw128_off(row, g8)) = dk;
+                    *reinterpret_cast<uint4*>(dws + j * kAtom128 + sw128_off(row, g8)) =
+                        make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
+                                   pack_bf16(d[6], d[7]));
                 }
             }
-            tc_fence_before();
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&wempty);
+                mbar_arrive(&dwready);
                 mbar_arrive(&empty[s]);
-                mbar_arrive(&dufull);
             }
-            ok = mbar_wait(&dzfull, it & 1, &abort_flag, a.err);
-            if (epi_bar_any<kEpiThreads>(!ok)) break;
+        }
+    } else {
+        // ---- GB: dz readout (fp32 atomic add, reduction over chunks) and dB partials
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
+        uint32_t it = 0;
+        for (int64_t item = i0; item < i1; ++item, ++it) {
+            const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
+            const bool last = (item + 1 == i1) || (chunk_of(item + 1) != chunk);
+            const int b = it & 1;
+            const bool ok = mbar_wait(&dzfull[b], (it >> 1) & 1, &abort_flag, a.err);
+            if (named_bar_any<3, 32 * kGbWarps>(!ok)) break;
             tc_fence_after();
-            // epilogue B: dz rows -> fp32 atomic add (reduction over channel chunks)
-            for (int c = 8 * half; c < a.r; c += 16) {
-                uint32_t v[8];
-                tmem_ld8(lane_base + kColDz + c, v);
+            const int32_t n = (int32_t)(tile * 128) + row;
+            for (int c = 0; c < a.r; c += 16) {
+                uint32_t v[2][8];
+                tmem_ld8(lane_base + kColDz + 64 * b + c, v[0]);
+                if (c + 8 < a.r) tmem_ld8(lane_base + kColDz + 64 * b + c + 8, v[1]);
                 tmem_wait_ld();
                 if (n < a.N) {
                     float4* dst = reinterpret_cast<float4*>(a.dz_acc + (int64_t)n * a.r + c);
-                    atomicAdd(dst, make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
-                                               __uint_as_float(v[3])));
-                    atomicAdd(dst + 1, make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]),
-                                                   __uint_as_float(v[6]), __uint_as_float(v[7])));
+                    atomicAdd(dst, make_float4(__uint_as_float(v[0][0]), __uint_as_float(v[0][1]),
+                                               __uint_as_float(v[0][2]), __uint_as_float(v[0][3])));
+                    atomicAdd(dst + 1, make_float4(__uint_as_float(v[0][4]), __uint_as_float(v[0][5]),
+                                                   __uint_as_float(v[0][6]), __uint_as_float(v[0][7])));
+                    if (c + 8 < a.r) {
+                        atomicAdd(dst + 2, make_float4(__uint_as_float(v[1][0]), __uint_as_float(v[1][1]),
+                                                       __uint_as_float(v[1][2]), __uint_as_float(v[1][3])));
+                        atomicAdd(dst + 3, make_float4(__uint_as_float(v[1][4]), __uint_as_float(v[1][5]),
+                                                       __uint_as_float(v[1][6]), __uint_as_float(v[1][7])));
+                    }
                 }
             }
-            // epilogue C: the run for this chunk ends here -> dB partial of this run
-            if (last) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dzempty[b]);
+            if (last) {                            // the run for this chunk ends: its dB partial
                 const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
                 float* part = a.dB_part + ((chunk * a.pieces + piece) * (64 * K)) * a.r;
 #pragma unroll
-                for (int b = 0; b < NBLK; ++b) {
-                    const int m = b * 128 + row;     // (tap, channel) row = j * 64 + c
-                    for (int c = 8 * half; c < a.r; c += 16) {
+                for (int bb = 0; bb < NBLK; ++bb) {
+                    const int m = bb * 128 + row;     // (tap, channel) row = j * 64 + c
+                    for (int c = 0; c < a.r; c += 8) {
                         uint32_t v[8];
-                        tmem_ld8(lane_base + kColDb + 64 * b + c, v);
+                        tmem_ld8(lane_base + kColDb + 64 * bb + c, v);
                         tmem_wait_ld();
                         if (m < 64 * K) {
                             float4* dst = reinterpret_cast<float4*>(part + (int64_t)m * a.r + c);
@@ -366,8 +430,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) lowrank_bwd_kernel(const __gri
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dbfree);
             }
-            tc_fence_before();
         }
     }
     tc_fence_before();
@@ -618,7 +684,7 @@ cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUten
     constexpr uint32_t smem = BwdSmem<K>::total;
     cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcLowrankBwd, st, lowrank_bwd_kernel<K><<<grid, kBwdThreads, smem, st>>>(tz, tg, tu, tbp, tdu, ba));
+    DC_LAUNCH(kTcLowrankBwd, st, lowrank_bwd_kernel<K><<<grid, kBwdPipeThreads, smem, st>>>(tz, tg, tu, tbp, tdu, ba));
     return cudaGetLastError();
 }
 

@@ -197,6 +197,21 @@ __device__ __forceinline__ bool epi_bar_any(bool pred) {
     return r != 0;
 }
 
+// Reducing named barrier `ID` over NT threads (same contract as epi_bar_any).
+template <int ID, int NT>
+__device__ __forceinline__ bool named_bar_any(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred)), "n"(ID), "n"(NT)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
