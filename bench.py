@@ -287,8 +287,6 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    L.dynconv_profile_read(reset=True)
-    L.dynconv_profile_enable(True)
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
@@ -296,12 +294,21 @@ def run_ours(args, rank, world, local_rank):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    L.dynconv_profile_enable(False)
-    prof = L.dynconv_profile_read(reset=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in ev]
+    # Per-kernel device times: the same steps again with the library's launch tracer on
+    # (events on the launch stream around every launch; these serialise the launches, so
+    # the step time above is measured with the tracer off).
+    L.dynconv_profile_read(reset=True)
+    L.dynconv_profile_enable(True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    L.dynconv_profile_enable(False)
+    prof = L.dynconv_profile_read(reset=True)
     total_ms = float(sum(step_ms))
     tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -354,12 +361,13 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel (live CUDA-event timing from the library's tracer)
     pk, pk_src = peaks()
-    launches = sum(v[0] for v in prof.values())
+    launches = sum(v[0] for v in prof.values())   # our kernels in the timed steps (same launches per step)
     dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
     roof = None
     kernels = {}
     for name, (n_l, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
-        kernels[name] = {"launches": n_l, "ms_total": round(ms, 4), "share": round(ms / max(total_ms, 1e-9), 4)}
+        kernels[name] = {"launches": n_l, "ms_total": round(ms, 4), "us_per_launch": round(1e3 * ms / n_l, 2),
+                         "share": round(ms / max(total_ms, 1e-9), 4)}
     if dom is not None:
         name, (n_l, ms) = dom
         per_launch_bytes = sum(kernel_bytes(name, w, layer) or 0 for layer in w.layers) / len(w.layers)

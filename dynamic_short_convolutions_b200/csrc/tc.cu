@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base;
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -275,6 +277,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base;
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -402,8 +406,8 @@ cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, con
     if (e != cudaSuccess) return e;
     fa.per_cta = (items + num_sms() - 1) / num_sms();
     const unsigned grid = (unsigned)((items + fa.per_cta - 1) / fa.per_cta);
-    DC_LAUNCH(kTcLowrankFwd, st, lowrank_fwd_kernel<K><<<grid, kFwdThreads, smem, st>>>(tz, tb, tu, ty, fa));
-    return cudaGetLastError();
+    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K>, dim3(grid), dim3(kFwdThreads), smem, st, tz, tb, tu, ty, fa));
+    return e;
 }
 
 }  // namespace
@@ -422,9 +426,9 @@ cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, i
     if (e != cudaSuccess) return e;
     const int64_t n_tiles = (N + 127) / 128;
     const unsigned grid = (unsigned)std::min<int64_t>(n_tiles, num_sms());
-    DC_LAUNCH(kTcGen, st, gen_kernel<__nv_bfloat16><<<grid, kTcThreads, smem, st>>>(
-        th, tp, static_cast<__nv_bfloat16*>(out), ga));
-    return cudaGetLastError();
+    DC_LAUNCH(kTcGen, st, e = launch_pdl(gen_kernel<__nv_bfloat16>, dim3(grid), dim3(kTcThreads), (size_t)smem, st, th, tp,
+                                         static_cast<__nv_bfloat16*>(out), ga));
+    return e;
 }
 
 struct TcBwdLayout {
@@ -434,7 +438,7 @@ struct TcBwdLayout {
 };
 TcBwdLayout tc_bwd_layout(const Prob& p);
 struct TcHwLayout {
-    size_t wh, dwh, dpart, total;
+    size_t wh, dwh, dpart, cnt, total;
 };
 TcHwLayout tc_hw_layout(const Prob& p);
 bool tc_headwise_supported(const Prob& p);

@@ -32,6 +32,14 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels launched with launch_pdl() may start while the previous kernel on the stream is
+// still finishing; each kernel runs its prologue (barriers, TMEM, tensor-map prefetch),
+// then pdl_wait() before touching global memory, which returns once the previous grid has
+// completed and its writes are visible.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -26,8 +26,9 @@ namespace dynconv {
 cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
                           int64_t out_ld, uint32_t* err, cudaStream_t st);
 cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
-                            void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st);
+                            void* dh, float* dP, float* dP_part, int* cnt_dblk, uint32_t* err, cudaStream_t st);
 int gen_bwd_splits(int64_t N, int64_t d, int R);
+int gen_bwd_dblk(int64_t d, int R);
 
 namespace {
 
@@ -81,6 +82,8 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
                                                           int64_t N, int64_t C, int64_t seqlen,
                                                           const int32_t* __restrict__ cu, int64_t n_docs,
                                                           __nv_bfloat16* __restrict__ y) {
+    pdl_trigger();
+    pdl_wait();
     const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
     const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
     const int q = (int)(c / hd);
@@ -101,6 +104,8 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
                                                           const int32_t* __restrict__ cu, int64_t n_docs,
                                                           __nv_bfloat16* __restrict__ du,
                                                           __nv_bfloat16* __restrict__ dwh) {
+    pdl_trigger();
+    pdl_wait();
     const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
     const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
     const int q = (int)(c / hd);
@@ -153,7 +158,7 @@ inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Workspace of the head-wise tensor-core path (inside the tensor-core region).
 struct TcHwLayout {
-    size_t wh, dwh, dpart, total;
+    size_t wh, dwh, dpart, cnt, total;
 };
 
 TcHwLayout tc_hw_layout(const Prob& p) {
@@ -162,6 +167,7 @@ TcHwLayout tc_hw_layout(const Prob& p) {
     L.wh = off;     off = al256(off + (size_t)p.N * p.R * 2);
     L.dwh = off;    off = al256(off + (size_t)p.N * p.R * 2);
     L.dpart = off;  off = al256(off + (size_t)gen_bwd_splits(p.N, p.d, (int)p.R) * p.d * p.R * 4);
+    L.cnt = off;    off = al256(off + (size_t)gen_bwd_dblk(p.d, (int)p.R) * 4);
     L.total = off;
     return L;
 }
@@ -175,21 +181,25 @@ bool tc_headwise_supported(const Prob& p) {
 }
 
 template <int K>
-static void launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, cudaStream_t st) {
+static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, cudaStream_t st) {
     const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
-    DC_LAUNCH(kTcHeadwiseFwd, st, hw_conv_fwd_kernel<K><<<grid, 256, 0, st>>>(
+    cudaError_t e;
+    DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
         p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
+    (void)e;
 }
 
 template <int K>
-static void launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
+static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
                           cudaStream_t st) {
     const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
-    DC_LAUNCH(kTcHeadwiseBwd, st, hw_conv_bwd_kernel<K><<<grid, 256, 0, st>>>(
+    cudaError_t e;
+    DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
         static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, p.cu, p.n_docs,
         static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
+    return e;
 }
 
 cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, const void* W, void* y, void* z_save,
@@ -199,12 +209,11 @@ cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, con
     cudaError_t e = tc_gen_launch(h, p.hs, W, p.N, p.d, (int)p.R, wh, p.R, err, st);
     if (e != cudaSuccess) return e;
     switch (p.K) {
-        case 1: launch_hw_fwd<1>(p, u, wh, y, st); break;
-        case 2: launch_hw_fwd<2>(p, u, wh, y, st); break;
-        case 3: launch_hw_fwd<3>(p, u, wh, y, st); break;
-        default: launch_hw_fwd<4>(p, u, wh, y, st); break;
+        case 1: return launch_hw_fwd<1>(p, u, wh, y, st);
+        case 2: return launch_hw_fwd<2>(p, u, wh, y, st);
+        case 3: return launch_hw_fwd<3>(p, u, wh, y, st);
+        default: return launch_hw_fwd<4>(p, u, wh, y, st);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, const void* h, const void* W,
@@ -219,16 +228,16 @@ cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, co
         wh = whs;
     }
     void* dwh = tcws + L.dwh;
+    cudaError_t e;
     switch (p.K) {
-        case 1: launch_hw_bwd<1>(p, g, u, wh, du, dwh, st); break;
-        case 2: launch_hw_bwd<2>(p, g, u, wh, du, dwh, st); break;
-        case 3: launch_hw_bwd<3>(p, g, u, wh, du, dwh, st); break;
-        default: launch_hw_bwd<4>(p, g, u, wh, du, dwh, st); break;
+        case 1: e = launch_hw_bwd<1>(p, g, u, wh, du, dwh, st); break;
+        case 2: e = launch_hw_bwd<2>(p, g, u, wh, du, dwh, st); break;
+        case 3: e = launch_hw_bwd<3>(p, g, u, wh, du, dwh, st); break;
+        default: e = launch_hw_bwd<4>(p, g, u, wh, du, dwh, st); break;
     }
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return tc_gen_backward(dwh, (int)p.R, h, p.hs, W, p.N, p.d, dh, dW, reinterpret_cast<float*>(tcws + L.dpart),
-                           err, st);
+                           reinterpret_cast<int*>(tcws + L.cnt), err, st);
 }
 
 }  // namespace dynconv
