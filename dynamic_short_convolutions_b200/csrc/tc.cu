@@ -438,7 +438,7 @@ struct TcBwdLayout {
 };
 TcBwdLayout tc_bwd_layout(const Prob& p);
 struct TcHwLayout {
-    size_t wh, dwh, dpart, cnt, total;
+    size_t wh, dwh, dpart, total;
 };
 TcHwLayout tc_hw_layout(const Prob& p);
 bool tc_headwise_supported(const Prob& p);

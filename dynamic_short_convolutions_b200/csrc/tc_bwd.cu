@@ -25,12 +25,11 @@
 //       MMA3  dBt += dW^T z            (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
 //       epi B dz -> fp32 atomic add into a [N, r] buffer (reduction over chunks);
 //       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
-//       the CTA finishing the last chunk of a tile converts its dz rows to bf16, and the
-//       CTA finishing the last run of a chunk sums the chunk's partials in run order -> dB.
+//   reduce_dB_kernel   sums the partials of each chunk in run order -> dB [r, C K] fp32.
+//   dz_to_bf16_kernel  fp32 dz -> bf16 operand for the generator backward.
 //   gen_bwd_kernel     dh = dz A^T (M = 128 tokens, N = 256 of d, K = r) and
 //                      dA += h^T dz (M = 128 of d, N = r, K = 128 tokens) per (256-wide d
-//                      block, token range); the CTA finishing the last token range of a
-//                      d block sums the ranges in order.
+//                      block, token range); reduce_splits_kernel sums the token ranges.
 #include <algorithm>
 #include <cstdio>
 
@@ -58,10 +57,9 @@ constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
 // Backward set-up in one launch: zero the fp32 dz accumulator (float4 stores) and write
 // the tap-major copy Bp[k, j C + c] = B[k, c K + j] (coalesced over the output index).
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat16* __restrict__ Bp, int r, int C,
-                                int K, float4* __restrict__ dz4, int64_t n_dz4, int* __restrict__ cnt, int n_cnt) {
+                                int K, float4* __restrict__ dz4, int64_t n_dz4) {
     pdl_trigger();
     pdl_wait();
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_cnt; i += gridDim.x * blockDim.x) cnt[i] = 0;
     const int64_t n_b = (int64_t)r * C * K;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_dz4 + n_b;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -85,10 +83,6 @@ struct BwdArgs {
     float* dB_part;           // [n_chunks][pieces][64 K][r]
     uint32_t* err;
     int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
-    __nv_bfloat16* dzb;       // [N, r] bf16 copy of dz, written by the last chunk of each tile
-    float* dB;                // [r, C K] fp32 output, written by the last run of each chunk
-    int* cnt_tile;            // [n_tiles] chunks finished per tile (reset by the last)
-    int* cnt_chunk;           // [n_chunks] runs finished per chunk (reset by the last)
 };
 
 template <int K>
@@ -123,7 +117,6 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
     uint8_t* sm = align1024(smem_raw);
     __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dwready, dwfree, dzfull[2], dzempty[2],
         dbfree, dufull, duempty;
-    __shared__ int s_flag;                   // last-arriver flag of the dz / dB reductions (GB warps)
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -422,29 +415,8 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&dzempty[b]);
-            // The CTA that adds the last chunk of this tile converts the tile's dz rows to bf16.
-            __threadfence();
-            named_bar_any<3, 32 * kGbWarps>(false);
-            if (warp == 3 + kGaWarps && lane == 0) {
-                const int old = atomicAdd(a.cnt_tile + tile, 1);
-                s_flag = old == (int)(a.C / 64) - 1;
-                if (s_flag) atomicExch(a.cnt_tile + tile, 0);
-            }
-            named_bar_any<3, 32 * kGbWarps>(false);
-            if (s_flag && n < a.N) {
-                __threadfence();
-                const float* src = a.dz_acc + (int64_t)n * a.r;
-                for (int c = 0; c < a.r; c += 8) {
-                    const float4 v0 = __ldcg(reinterpret_cast<const float4*>(src + c));
-                    const float4 v1 = __ldcg(reinterpret_cast<const float4*>(src + c + 4));
-                    *reinterpret_cast<uint4*>(a.dzb + (int64_t)n * a.r + c) =
-                        make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v0.z, v0.w), pack_bf16(v1.x, v1.y),
-                                   pack_bf16(v1.z, v1.w));
-                }
-            }
             if (last) {                            // the run for this chunk ends: its dB partial
-                const int64_t first_cta = (chunk * a.n_tiles) / a.per_cta;
-                const int64_t piece = (int64_t)blockIdx.x - first_cta;
+                const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
                 float* part = a.dB_part + ((chunk * a.pieces + piece) * (64 * K)) * a.r;
 #pragma unroll
                 for (int bb = 0; bb < NBLK; ++bb) {
@@ -465,28 +437,6 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dbfree);
-                // The CTA that writes the last run's partial of this chunk sums the runs in order.
-                __threadfence();
-                named_bar_any<3, 32 * kGbWarps>(false);
-                const int64_t last_cta = ((chunk + 1) * a.n_tiles - 1) / a.per_cta;
-                if (warp == 3 + kGaWarps && lane == 0) {
-                    const int old = atomicAdd(a.cnt_chunk + chunk, 1);
-                    s_flag = old == (int)(last_cta - first_cta);
-                    if (s_flag) atomicExch(a.cnt_chunk + chunk, 0);
-                }
-                named_bar_any<3, 32 * kGbWarps>(false);
-                if (s_flag) {
-                    __threadfence();
-                    const int np = (int)(last_cta - first_cta) + 1;
-                    const float* base = a.dB_part + (chunk * a.pieces) * (64 * K) * a.r;
-                    for (int e = threadIdx.x - 32 * (3 + kGaWarps); e < 64 * K * a.r; e += 32 * kGbWarps) {
-                        const int m = e / a.r, k = e - m * a.r, j = m >> 6, cl = m & 63;
-                        float acc = 0.f;
-                        for (int pp = 0; pp < np; ++pp) acc += __ldcg(base + (int64_t)pp * (64 * K) * a.r + e);
-                        a.dB[(int64_t)k * a.C * K + (chunk * 64 + cl) * K + j] = acc;
-                    }
-                }
-                named_bar_any<3, 32 * kGbWarps>(false);   // s_flag is rewritten by the next item
             }
         }
     }
@@ -495,6 +445,59 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, 512);
+    }
+}
+
+// dB[k, c K + j] = sum over the runs covering chunk c/64, in run order (one thread per entry).
+template <int K>
+__global__ void reduce_dB_kernel(const float* __restrict__ part, float* __restrict__ dB, int r, int C, int n_tiles,
+                                 int per_cta, int pieces) {
+    pdl_trigger();
+    pdl_wait();
+    const int total = r * C * K;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        const int k = e / (C * K), col = e - k * (C * K), c = col / K, j = col - c * K;
+        const int chunk = c >> 6, m = j * 64 + (c & 63);
+        const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
+        const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
+        const float* src = part + ((int64_t)chunk * pieces * (64 * K) + m) * r + k;
+        float acc = 0.f;
+        for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * (64 * K) * r];
+        dB[e] = acc;
+    }
+}
+
+__global__ void dz_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t count4) {
+    pdl_trigger();
+    pdl_wait();
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = src[i];
+        dst[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    }
+}
+
+// out[i] = sum_s part[s][i] for i < count (count a multiple of 4): one warp per 4 outputs, lane l
+// sums splits l, l + 32, ... in order, then a fixed butterfly combines the lanes (deterministic).
+__global__ void reduce_splits_kernel(const float* __restrict__ part, float* __restrict__ out, int64_t count,
+                                     int n_split) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; w * 4 < count; w += warps) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = lane; s < n_split; s += 32) {
+            const float4 v = *reinterpret_cast<const float4*>(part + s * count + w * 4);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+        }
+        if (lane == 0) *reinterpret_cast<float4*>(out + w * 4) = acc;
     }
 }
 
@@ -517,8 +520,6 @@ struct GenBwdArgs {
     __nv_bfloat16* dh;        // nullable
     float* dP_part;           // [n_split][d][R]
     uint32_t* err;
-    float* dP;                // [d][R] output, summed over the splits by the last split of each d block
-    int* cnt_dblk;            // [n_dblk] splits finished per d block (reset by the last)
 };
 
 template <int XA>
@@ -543,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
     uint8_t* pblk = sm + G::pblk;
     __shared__ uint64_t full[2], empty[2], pfull, hfull, hempty, dpfull;
     __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag, s_last;
+    __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int db = blockIdx.x % a.n_dblk, split = blockIdx.x / a.n_dblk;
     const int64_t t0 = (a.n_tiles * split) / a.n_split, t1 = (a.n_tiles * (split + 1)) / a.n_split;
@@ -674,26 +675,6 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                     }
                 }
             }
-            // The CTA that writes the last split of this d block sums the splits in order.
-            __threadfence();
-            epi_bar_any<kEpiThreads>(false);
-            if (warp == 2 && lane == 0) {
-                const int old = atomicAdd(a.cnt_dblk + db, 1);
-                s_last = old == a.n_split - 1;
-                if (s_last) atomicExch(a.cnt_dblk + db, 0);
-            }
-            epi_bar_any<kEpiThreads>(false);
-            if (s_last) {
-                __threadfence();
-                const int64_t r0 = (int64_t)db * G::DB, r1 = (r0 + G::DB < a.d) ? r0 + G::DB : a.d;
-                const int64_t cnt = (r1 - r0) * a.R, plane = a.d * a.R;
-                for (int64_t e = threadIdx.x - 64; e < cnt; e += kEpiThreads) {
-                    const int64_t idx = r0 * a.R + e;
-                    float acc = 0.f;
-                    for (int sp = 0; sp < a.n_split; ++sp) acc += __ldcg(a.dP_part + sp * plane + idx);
-                    a.dP[idx] = acc;
-                }
-            }
         }
     }
     tc_fence_before();
@@ -732,7 +713,7 @@ int gen_bwd_splits(int64_t N, int64_t d, int R) {
 }
 
 cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
-                            void* dh, float* dP, float* dP_part, int* cnt_dblk, uint32_t* err, cudaStream_t st) {
+                            void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st) {
     const int n_dblk = gen_bwd_dblk(d, R), n_split = gen_bwd_splits(N, d, R);
     const int XA = R <= 64 ? 1 : 2;
     const int DB = XA == 1 ? 256 : 128;
@@ -741,7 +722,7 @@ cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, con
         !make_tmap_bf16(&tp, P, R, d, R, 64, DB))
         return cudaErrorInvalidValue;
     GenBwdArgs ga{N, d, R, (R + 15) / 16 * 16, (R + 15) / 16, hs, n_dblk, n_split, (N + 127) / 128,
-                  static_cast<__nv_bfloat16*>(dh), dP_part, err, dP, cnt_dblk};
+                  static_cast<__nv_bfloat16*>(dh), dP_part, err};
     cudaError_t e;
     const dim3 grid(n_dblk * n_split);
     if (XA == 1) {
@@ -753,12 +734,15 @@ cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, con
         if (e != cudaSuccess) return e;
         DC_LAUNCH(kTcGenBwd, st, e = launch_pdl(gen_bwd_kernel<2>, grid, dim3(kThreads), GbCfg<2>::smem, st, tx, th, tp, ga));
     }
+    if (e != cudaSuccess) return e;
+    DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_splits_kernel, dim3(grid_for(d * R / 4 * 32)), dim3(256), 0, st,
+                                            (const float*)dP_part, dP, d * R, n_split));
     return e;
 }
 
 // Workspace of the tensor-core backward (after the z scratch), byte offsets.
 struct TcBwdLayout {
-    size_t zs, bp, dz, dzb, dbpart, dpart, cnt, total;
+    size_t zs, bp, dz, dzb, dbpart, dpart, total;
     int64_t per_cta, n_items, n_tiles;
     int pieces, grid, n_dblk, n_split;
 };
@@ -783,7 +767,6 @@ TcBwdLayout tc_bwd_layout(const Prob& p) {
     L.dzb = off;     off = al256(off + (size_t)p.N * p.r * 2);                     // dz bf16
     L.dbpart = off;  off = al256(off + (size_t)n_chunks * L.pieces * 64 * p.K * p.r * 4);
     L.dpart = off;   off = al256(off + (size_t)L.n_split * p.d * p.r * 4);
-    L.cnt = off;     off = al256(off + (size_t)(L.n_tiles + n_chunks + L.n_dblk) * 4);
     L.total = off;
     return L;
 }
@@ -804,12 +787,10 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     __nv_bfloat16* dzb = reinterpret_cast<__nv_bfloat16*>(tcws + L.dzb);
     float* dbpart = reinterpret_cast<float*>(tcws + L.dbpart);
     float* dpart = reinterpret_cast<float*>(tcws + L.dpart);
-    int* cnt = reinterpret_cast<int*>(tcws + L.cnt);
-    const int n_cnt = (int)(L.n_tiles + p.C / 64 + L.n_dblk);
     cudaError_t e;
     DC_LAUNCH(kTcPrep, st, e = launch_pdl(bwd_prep_kernel, dim3(grid_for(p.N * p.r / 4 + p.r * p.C * p.K)), dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, reinterpret_cast<float4*>(dz),
-        p.N * p.r / 4, cnt, n_cnt));
+        p.N * p.r / 4));
     if (e != cudaSuccess) return e;
     CUtensorMap tz, tg, tu, tbp, tdu;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
@@ -817,7 +798,7 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128))
         return cudaErrorInvalidValue;
     BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
-               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dzb, dB, cnt, cnt + L.n_tiles};
+               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16)};
     switch (p.K) {
         case 1: e = launch_bwd<1>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
         case 2: e = launch_bwd<2>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
@@ -825,8 +806,26 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         default: e = launch_bwd<4>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
+    switch (p.K) {
+#define DC_REDUCE_DB(KK)                                                                                          \
+    case KK:                                                                                                       \
+        DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_dB_kernel<KK>, dim3(grid_for(p.r * p.C * p.K)), dim3(256), 0, st, \
+                                                (const float*)dbpart, dB, (int)p.r, (int)p.C, (int)L.n_tiles,        \
+                                                (int)L.per_cta, L.pieces));                                          \
+        break;
+        DC_REDUCE_DB(1)
+        DC_REDUCE_DB(2)
+        DC_REDUCE_DB(3)
+        DC_REDUCE_DB(4)
+#undef DC_REDUCE_DB
+    }
+    if (e != cudaSuccess) return e;
+    DC_LAUNCH(kTcReduce, st, e = launch_pdl(dz_to_bf16_kernel, dim3(grid_for(p.N * p.r / 4)), dim3(256), 0, st,
+                                            reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb),
+                                            p.N * p.r / 4));
+    if (e != cudaSuccess) return e;
     // generator backward: dA = h^T dz, dh = dz A^T
-    return tc_gen_backward(dzb, (int)p.r, h, p.hs, A, p.N, p.d, dh, dA, dpart, cnt + L.n_tiles + p.C / 64, err, st);
+    return tc_gen_backward(dzb, (int)p.r, h, p.hs, A, p.N, p.d, dh, dA, dpart, err, st);
 }
 
 }  // namespace dynconv

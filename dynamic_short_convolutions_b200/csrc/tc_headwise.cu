@@ -26,7 +26,7 @@ namespace dynconv {
 cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
                           int64_t out_ld, uint32_t* err, cudaStream_t st);
 cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
-                            void* dh, float* dP, float* dP_part, int* cnt_dblk, uint32_t* err, cudaStream_t st);
+                            void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st);
 int gen_bwd_splits(int64_t N, int64_t d, int R);
 int gen_bwd_dblk(int64_t d, int R);
 
@@ -158,7 +158,7 @@ inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Workspace of the head-wise tensor-core path (inside the tensor-core region).
 struct TcHwLayout {
-    size_t wh, dwh, dpart, cnt, total;
+    size_t wh, dwh, dpart, total;
 };
 
 TcHwLayout tc_hw_layout(const Prob& p) {
@@ -167,7 +167,6 @@ TcHwLayout tc_hw_layout(const Prob& p) {
     L.wh = off;     off = al256(off + (size_t)p.N * p.R * 2);
     L.dwh = off;    off = al256(off + (size_t)p.N * p.R * 2);
     L.dpart = off;  off = al256(off + (size_t)gen_bwd_splits(p.N, p.d, (int)p.R) * p.d * p.R * 4);
-    L.cnt = off;    off = al256(off + (size_t)gen_bwd_dblk(p.d, (int)p.R) * 4);
     L.total = off;
     return L;
 }
@@ -237,7 +236,7 @@ cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, co
     }
     if (e != cudaSuccess) return e;
     return tc_gen_backward(dwh, (int)p.R, h, p.hs, W, p.N, p.d, dh, dW, reinterpret_cast<float*>(tcws + L.dpart),
-                           reinterpret_cast<int*>(tcws + L.cnt), err, st);
+                           err, st);
 }
 
 }  // namespace dynconv

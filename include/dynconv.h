@@ -94,10 +94,10 @@ typedef struct {
 
 /* Workspace needed by dynconv_fwd / dynconv_fwd_varlen / dynconv_bwd for this
  * descriptor (one size serves all three).  Returns 0 for an invalid desc.
- * Zero the whole workspace once before its first use (cudaMemset; torch.zeros):
- * it holds the device error word (cleared by the library when it reports it)
- * and reduction counters that every call leaves at zero again.  One workspace
- * must not be used by two calls that overlap on the device. */
+ * Zero the workspace once before its first use (cudaMemset; torch.zeros): its
+ * first bytes hold the device error word, which the library clears when it
+ * reports it.  One workspace must not be used by two calls that overlap on
+ * the device. */
 DYNCONV_API size_t dynconv_workspace_bytes(const dynconv_desc *desc);
 
 /* Forward, dense batch: y = u + dynamic causal conv(u), filters from h.
