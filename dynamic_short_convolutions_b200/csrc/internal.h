@@ -50,6 +50,18 @@ cudaError_t simt_backward(const Prob& p, const void* g, const void* u, const voi
                           const void* BW, const void* z_saved, void* du, void* dh, float* dA, float* dBW,
                           void* ws, cudaStream_t st);
 
+// Generator GEMM out[N, R] = h[N, d] . P[d, R] on the tensor cores (bf16 in and out).
+// Optionally the same launch also writes the tap-major copy Bp[k, j C + c] = B[k, c K + j]
+// of a low-rank projection (the layout the low-rank conv kernels read), using the
+// epilogue threads before the first accumulator is ready.
+struct BPermute {
+    const void* B = nullptr;
+    void* Bp = nullptr;
+    int r = 0, C = 0, K = 0;
+};
+cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
+                          int64_t out_ld, uint32_t* err, cudaStream_t st, BPermute perm = BPermute{});
+
 // tcgen05 / TMA kernels (bf16 storage, shapes accepted by tc_supported).
 cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW,
                        void* y, void* z_save, void* ws, cudaStream_t st);

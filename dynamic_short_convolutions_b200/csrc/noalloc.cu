@@ -7,7 +7,8 @@
 // pre-partitioned, or in a host process that only receives device pointers
 // from elsewhere).  For them dynconv_fwd_noalloc runs the low-rank tensor-core
 // forward with its scratch in a buffer that is part of this library's device
-// image: the z = h A intermediate (bf16 [N, r]) and the device error word.
+// image: the tap-major copy of B (bf16 [r, K C]), the z = h A intermediate
+// (bf16 [N, r]) unless the caller passes z_save, and the device error word.
 //
 // The buffer is a file-scope device array of kScratchBytes + 256 bytes; every
 // GPU on which the library's kernels are loaded holds it until the process
@@ -15,8 +16,8 @@
 // its device address is looked up with cudaGetSymbolAddress, once per device,
 // by the first call made with that device current (that first call should come
 // before any stream capture).  Every call shares the one buffer and leaves its
-// last contents there: the error word is cleared by each call, z is fully
-// rewritten by each call, and two calls whose work overlaps on the GPU (other
+// last contents there: the error word is cleared by each call, Bp and z are
+// fully rewritten by each call, and two calls whose work overlaps on the GPU (other
 // streams, other host threads) race on it.
 #include <mutex>
 
@@ -28,11 +29,11 @@ namespace dynconv {
 dynconv_status validate_desc(const dynconv_desc* d, Prob* p);
 dynconv_status validate_ptr(const void* ptr, const char* name, bool required);
 cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
-                               void* z, uint32_t* err, cudaStream_t st);
+                               void* z, void* bp, uint32_t* err, cudaStream_t st);
 
 namespace {
 
-constexpr size_t kScratchBytes = size_t(8) << 20;   // room for z: N * r * 2 bytes
+constexpr size_t kScratchBytes = size_t(8) << 20;   // room for Bp (r C K 2 bytes) and z (N r 2 bytes)
 constexpr size_t kErrBytes = 256;                   // the device error word, padded
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kErrBytes + kScratchBytes];
@@ -80,11 +81,13 @@ extern "C" DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc* de
         return DYNCONV_ERR_UNSUPPORTED;
     }
     if (p.N == 0) return DYNCONV_OK;
-    const size_t z_bytes = (size_t)p.N * p.r * 2;
-    if (!z_save && z_bytes > kScratchBytes) {
-        set_error("dynconv_fwd_noalloc needs %zu bytes of scratch for z (N * rank * 2); the built-in buffer holds "
-                  "%zu bytes: pass z_save or use dynconv_fwd with a workspace",
-                  z_bytes, kScratchBytes);
+    const size_t bp_bytes = ((size_t)p.r * p.C * p.K * 2 + 255) / 256 * 256;
+    const size_t z_bytes = z_save ? 0 : (size_t)p.N * p.r * 2;
+    if (bp_bytes + z_bytes > kScratchBytes) {
+        set_error("dynconv_fwd_noalloc needs %zu bytes of scratch (rank * channels * ksize * 2 for the tap-major "
+                  "projection, plus N * rank * 2 for z unless z_save is given); the built-in buffer holds %zu bytes: "
+                  "use dynconv_fwd with a workspace",
+                  bp_bytes + z_bytes, kScratchBytes);
         return DYNCONV_ERR_UNSUPPORTED;
     }
     if ((s = validate_ptr(u, "u", true)) || (s = validate_ptr(h, "h", true)) || (s = validate_ptr(A, "A", true)) ||
@@ -95,9 +98,10 @@ extern "C" DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc* de
     if ((s = scratch_address(&base)) != DYNCONV_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t* err = static_cast<uint32_t*>(base);
-    void* z = z_save ? z_save : static_cast<void*>(static_cast<unsigned char*>(base) + kErrBytes);
+    unsigned char* bp = static_cast<unsigned char*>(base) + kErrBytes;
+    void* z = z_save ? z_save : static_cast<void*>(bp + bp_bytes);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st);
-    if (e == cudaSuccess) e = tc_forward_scratch(p, u, h, A, B, y, z, err, st);
+    if (e == cudaSuccess) e = tc_forward_scratch(p, u, h, A, B, y, z, bp, err, st);
     if (e != cudaSuccess) {
         set_error("dynconv_fwd_noalloc launch: %s", cudaGetErrorString(e));
         return DYNCONV_ERR_CUDA;

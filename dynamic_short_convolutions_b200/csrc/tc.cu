@@ -4,9 +4,10 @@
 // gist.science technical summary: "Parameterization" 1 and the "Fused Low-Rank
 // Kernel" paragraph of "Efficient Training Implementation"):
 //   gen_kernel         z = h A                        (M = 128 tokens, N = r, K = d)
+//                      (the same launch writes Bp, the tap-major copy of B)
 //   lowrank_fwd_kernel per (128-token tile, 64-channel chunk):
-//                      W = z B_chunk  -> TMEM        (M = 128, N = 64 K, K = r)
-//                      y = u + sum_j W[:, c K + j] u[t - j, c]  (epilogue, CUDA cores)
+//                      W = z Bp_chunk -> TMEM        (M = 128, N = 64 K, K = r)
+//                      y = u + sum_j W[:, 64 j + c] u[t - j, c]  (epilogue, CUDA cores)
 //                      the [N, C, K] filter lives only in TMEM and registers.
 //
 // Every kernel here is warp-specialised: warp 0 issues TMA loads, warp 1 issues
@@ -46,6 +47,9 @@ struct GenArgs {
     int stages;
     int64_t out_ld;
     uint32_t* err;
+    const __nv_bfloat16* pB;   // optional side job: Bp[k, j C + c] = B[k, c K + j]
+    __nv_bfloat16* pBp;
+    int pr, pC, pK;
 };
 
 template <typename OutT>
@@ -129,6 +133,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
             }
         }
     } else {
+        if (a.pB) {                              // the side job, before the first accumulator is ready
+            const int CK = a.pC * a.pK;
+            const int64_t total = (int64_t)a.pr * CK, stride = (int64_t)gridDim.x * kEpiThreads;
+            int64_t o = (int64_t)blockIdx.x * kEpiThreads + (threadIdx.x - 64);
+            for (; o + 3 * stride < total; o += 4 * stride) {
+                __nv_bfloat16 v[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int e = (int)(o + x * stride), k = e / CK, rem = e - k * CK, j = rem / a.pC, c = rem - j * a.pC;
+                    v[x] = a.pB[(int64_t)k * CK + c * a.pK + j];
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) a.pBp[o + x * stride] = v[x];
+            }
+            for (; o < total; o += stride) {
+                const int e = (int)o, k = e / CK, rem = e - k * CK, j = rem / a.pC, c = rem - j * a.pC;
+                a.pBp[o] = a.pB[(int64_t)k * CK + c * a.pK + j];
+            }
+        }
         const int q = warp & 3;                  // TMEM lane quarter of this warp
         const int half = (warp - 2) >> 2;        // which columns of the row this warp converts
         const int row = q * 32 + lane;
@@ -178,10 +201,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 // chunk-major runs, one run per CTA, so the chunk's B stays in shared memory.
 //   stage smem (ring of kFwdStages): z tile [128][64] (K-major A) | u tile [136 rows =
 //               m0-8 .. m0+127][64 channels]
-//   resident:   B chunk as K atoms [64 r-rows][64] (MN-major B), reloaded when the chunk changes
-//   TMEM: W[128 tokens][64 K] fp32, column c K + j = w[m0 + row, c0 + c, j]; two buffers.
+//   resident:   the chunk's slice of the tap-major Bp (Bp[k, j C + c] = B[k, c K + j], written by
+//               the generator launch) as K atoms [64 r-rows][64] (MN-major B), reloaded when the
+//               chunk changes
+//   TMEM: W[128 tokens][64 K] fp32, column 64 j + c = w[m0 + row, c0 + c, j]; two buffers.
 //   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3..10 epilogue (a TMEM lane quarter and half of
-//   the channels each): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, c K + j] u[t - j, c]
+//   the channels each): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
 //   -> bf16 staging (128-byte swizzled) -> TMA store by warp 2.
 // =====================================================================================
 struct FwdArgs {
@@ -204,25 +229,25 @@ struct FwdSmem {
     static constexpr uint32_t total = ys + 2 * kYBytes + 1024;
 };
 
-// y for 8 channels of one row from the K filter taps (wv[c K + j] = W[t, (g*8 + c) K + j]).
+// y for 8 channels of one row: wv[j][c] = W_j[t, 8 g + c] (fp32 bits), uj[j] = u[t - j, 8 g .. 8 g + 7].
+// Channel pairs go through the packed fp32 FMA.
 template <int K>
-__device__ __forceinline__ uint4 conv8(const uint32_t* wv, const uint4* uj, int32_t pos) {
+__device__ __forceinline__ uint4 conv8(const uint32_t (*wv)[8], const uint4* uj, int32_t pos) {
     float acc[8];
     const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
 #pragma unroll
-    for (int c = 0; c < 8; c += 2) {
-        acc[c] = bf16_lo(u0[c >> 1]);
-        acc[c + 1] = bf16_hi(u0[c >> 1]);
+    for (int p = 0; p < 4; ++p) {
+        acc[2 * p] = bf16_lo(u0[p]);
+        acc[2 * p + 1] = bf16_hi(u0[p]);
     }
 #pragma unroll
     for (int j = 0; j < K; ++j) {
         if (j <= pos) {
             const uint32_t* uu = reinterpret_cast<const uint32_t*>(&uj[j]);
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) {
-                acc[c] = fmaf(__uint_as_float(wv[c * K + j]), bf16_lo(uu[c >> 1]), acc[c]);
-                acc[c + 1] = fmaf(__uint_as_float(wv[(c + 1) * K + j]), bf16_hi(uu[c >> 1]), acc[c + 1]);
-            }
+            for (int p = 0; p < 4; ++p)
+                ffma2(acc[2 * p], acc[2 * p + 1], __uint_as_float(wv[j][2 * p]), __uint_as_float(wv[j][2 * p + 1]),
+                      bf16_lo(uu[p]), bf16_hi(uu[p]));
         }
     }
     uint4 pk;
@@ -290,7 +315,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
                 if (chunk != prev) {
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * 8192);
-                    for (int j = 0; j < K; ++j) tma_load_2d(sm + S::bres + j * 8192, &tm_b, &bfull, c0 * K + 64 * j, 0);
+                    for (int j = 0; j < K; ++j)
+                        tma_load_2d(sm + S::bres + j * 8192, &tm_b, &bfull, (int32_t)(j * a.C) + c0, 0);
                     ++cc;
                     prev = chunk;
                 }
@@ -363,12 +389,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
 #pragma unroll 1
             for (int gp = 0; gp < 2; ++gp) {            // two groups of 8 channels per batch
                 const int g0 = 4 * half + 2 * gp;
-                uint32_t wv[2][8 * K];
+                uint32_t wv[2][K][8];
 #pragma unroll
                 for (int x = 0; x < 2; ++x)
 #pragma unroll
-                    for (int i = 0; i < K; ++i)
-                        tmem_ld8(taddr + (g0 + x) * 8 * K + 8 * i, *reinterpret_cast<uint32_t(*)[8]>(wv[x] + 8 * i));
+                    for (int j = 0; j < K; ++j) tmem_ld8(taddr + 64 * j + 8 * (g0 + x), wv[x][j]);
                 uint4 uj[2][K];
 #pragma unroll
                 for (int x = 0; x < 2; ++x)
@@ -413,14 +438,15 @@ cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, con
 }  // namespace
 
 cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
-                          int64_t out_ld, uint32_t* err, cudaStream_t st) {
+                          int64_t out_ld, uint32_t* err, cudaStream_t st, BPermute perm) {
     CUtensorMap th, tp;
     if (!make_tmap_bf16(&th, h, d, N, hs, 64, 128) || !make_tmap_bf16(&tp, P, R, d, R, 64, 64))
         return cudaErrorInvalidValue;
     const int NB = (R + 63) / 64;
     const int stage_bytes = 16384 + NB * 8192;
     const int stages = std::max(2, std::min<int>(kGenMaxStages, (int)(kGenSmemBudget / stage_bytes)));
-    GenArgs ga{N, d, R, NB, (R + 15) / 16 * 16, stages, out_ld, err};
+    GenArgs ga{N, d, R, NB, (R + 15) / 16 * 16, stages, out_ld, err, static_cast<const __nv_bfloat16*>(perm.B),
+               static_cast<__nv_bfloat16*>(perm.Bp), perm.r, perm.C, perm.K};
     const int smem = 1024 + stages * stage_bytes;
     cudaError_t e = cudaFuncSetAttribute(gen_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -457,7 +483,7 @@ bool tc_supported(const Prob& p) {
     if (p.r % 8 != 0 || p.r > 64) return false;
     if (p.C % 64 != 0 || p.d % 8 != 0) return false;
     if (p.K < 1 || p.K > 4) return false;
-    if (p.N >= (int64_t(1) << 31)) return false;
+    if (p.N >= (int64_t(1) << 31) || p.r * p.C * p.K >= (int64_t(1) << 31)) return false;
     return tensor_map_encoder() != nullptr;
 }
 
@@ -470,36 +496,29 @@ bool tc_supported_bwd(const Prob& p) {
 
 size_t tc_workspace_bytes(const Prob& p) { return p.kind == 1 ? tc_hw_layout(p).total : tc_bwd_layout(p).total; }
 
+cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
+                               void* z, void* bp, uint32_t* err, cudaStream_t st);
+
 cudaError_t tc_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
                        void* z_save, void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
     if (p.kind == 1) return tc_headwise_forward(p, u, h, BW, y, z_save, static_cast<char*>(ws) + L.tc, err, st);
-    void* z = z_save ? z_save : static_cast<void*>(static_cast<char*>(ws) + L.tc);
-    cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
-    if (e != cudaSuccess) return e;
-    CUtensorMap tz, tb, tu, ty;
-    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
-        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
-        return cudaErrorInvalidValue;
-    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16)};
-    const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
-    switch (p.K) {
-        case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);
-        case 2: return launch_lowrank_fwd<2>(tz, tb, tu, ty, fa, items, st);
-        case 3: return launch_lowrank_fwd<3>(tz, tb, tu, ty, fa, items, st);
-        default: return launch_lowrank_fwd<4>(tz, tb, tu, ty, fa, items, st);
-    }
+    const TcBwdLayout TL = tc_bwd_layout(p);
+    char* tcws = static_cast<char*>(ws) + L.tc;
+    void* z = z_save ? z_save : static_cast<void*>(tcws + TL.zs);
+    return tc_forward_scratch(p, u, h, A, BW, y, z, tcws + TL.bp, err, st);
 }
 
-// Forward on the tensor cores with caller-chosen scratch: z (bf16 [N, r]) and the
-// device error word; used by the entry point that allocates nothing.
+// Low-rank forward on the tensor cores with caller-chosen scratch: z (bf16 [N, r]), Bp
+// (bf16 [r, K C]) and the device error word.
 cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
-                               void* z, uint32_t* err, cudaStream_t st) {
-    cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st);
+                               void* z, void* bp, uint32_t* err, cudaStream_t st) {
+    cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st,
+                                  BPermute{BW, bp, (int)p.r, (int)p.C, (int)p.K});
     if (e != cudaSuccess) return e;
     CUtensorMap tz, tb, tu, ty;
-    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, BW, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
         !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
         return cudaErrorInvalidValue;
     FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16)};

@@ -20,7 +20,8 @@
 //       MMA1  Wd_j[t, c] = sum_k z[t+j, k] Bp[k, j C + c]   (the filter of token t+j:
 //             the z tile is loaded with 8 rows of look-ahead and the A operand starts
 //             j rows into it), so du needs no exchange between threads;
-//       epi A du (-> TMA store) and dw (-> bf16 tile in shared memory, 64 channels per tap);
+//       epi A du (stored from registers) and dw (-> bf16 tile in shared memory, 64 channels
+//             per tap);
 //       MMA2  dz  = dW Bp_chunk^T      (M = 128 tokens, N = r, K = 64 K)
 //       MMA3  dBt += dW^T z            (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
 //       epi B dz -> fp32 atomic add into a [N, r] buffer (reduction over chunks);
@@ -40,9 +41,6 @@
 #include "tmap.h"
 
 namespace dynconv {
-
-cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
-                          int64_t out_ld, uint32_t* err, cudaStream_t st);
 
 namespace {
 
@@ -81,25 +79,33 @@ struct BwdArgs {
     int pieces;               // partial slots per chunk
     float* dz_acc;            // [N, r] fp32, zero on entry
     float* dB_part;           // [n_chunks][pieces][64 K][r]
+    __nv_bfloat16* du;        // [N, C] dense
     uint32_t* err;
     int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
 };
 
+// Shared memory of lowrank_bwd_kernel<K>: NST z | g | u stages (three for K <= 3: a stage
+// lives from its TMA load until the dB MMA has read z, so the loads of two later items must
+// be in flight meanwhile), one dW tile (K tap atoms of 128 tokens x 64 channels) and the
+// chunk's Bp slice.  The dB MMA reads dW in 128-row blocks of two tap atoms; for odd K the
+// last block's second atom lies past the tile (in the Bp region, which is at least one atom
+// long) and only feeds accumulator rows that are never read.
 template <int K>
 struct BwdSmem {
-    static constexpr int NA = 2 * ((K + 1) / 2);            // dW atoms (padded to whole 128-row MMA blocks)
+    static constexpr int NST = K <= 3 ? 3 : 2;
     static constexpr uint32_t stage = 3 * kRowTile;         // z | g | u
-    static constexpr uint32_t bp = 2 * stage;
-    static constexpr uint32_t dw = bp + K * 8192;
-    static constexpr uint32_t dust = dw + NA * kAtom128;
-    static constexpr uint32_t total = dust + kAtom128 + 1024;
+    static constexpr uint32_t dw = NST * stage;
+    static constexpr uint32_t dw_buf = K * kAtom128;
+    static constexpr uint32_t bp = dw + dw_buf;
+    static constexpr uint32_t bp_bytes = K * 8192 > kAtom128 ? K * 8192 : kAtom128;
+    static constexpr uint32_t total = bp + bp_bytes + 1024;
 };
 
-// Warp roles of lowrank_bwd_kernel: 0 TMA loads, 1 MMA issue (and TMEM owner), 2 TMA stores of
-// du, 3..10 the du / dw epilogue (GA: a TMEM lane quarter and half of the channels each),
-// 11..14 the dz / dB readout (GB: one TMEM lane quarter each).
-constexpr int kGaWarps = 8, kGbWarps = 4;
-constexpr int kBwdPipeThreads = 32 * (3 + kGaWarps + kGbWarps);
+// Warp roles of lowrank_bwd_kernel: 0 TMA loads, 1 MMA issue (and TMEM owner), 2..9 the du / dw
+// epilogue (GA: a TMEM lane quarter and half of the channels each), 10..13 the dz / dB readout
+// (GB: one TMEM lane quarter each).
+constexpr int kGaWarps = 8, kGbWarps = 4, kGa0 = 2, kGb0 = kGa0 + kGaWarps;
+constexpr int kBwdPipeThreads = 32 * (kGb0 + kGbWarps);
 
 // TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
 constexpr uint32_t kColDz = 256, kColDb = 384;
@@ -109,55 +115,49 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                                                                          const __grid_constant__ CUtensorMap tm_g,
                                                                          const __grid_constant__ CUtensorMap tm_u,
                                                                          const __grid_constant__ CUtensorMap tm_bp,
-                                                                         const __grid_constant__ CUtensorMap tm_du,
                                                                          BwdArgs a) {
     using S = BwdSmem<K>;
-    constexpr int NBLK = S::NA / 2;
+    constexpr int NBLK = (K + 1) / 2;
+    constexpr int NST = S::NST;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ uint64_t full[2], empty[2], bfull, bempty, wfull, wempty, dwready, dwfree, dzfull[2], dzempty[2],
-        dbfree, dufull, duempty;
+    // dwready / dwfree: per 128-row block (two tap atoms) of the dW tile, so the MMAs of one
+    // block overlap the writing of the next and the next item's first block
+    __shared__ uint64_t full[NST], empty[NST], bfull, bempty, wfull, wempty, dwready[NBLK], dwfree[NBLK], dzfull[2],
+        dzempty[2], dbfree;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t i0 = (int64_t)blockIdx.x * a.per_cta;
     const int64_t i1 = min(i0 + a.per_cta, a.n_items);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + kGaWarps);
-            mbar_init(&dzfull[s], 1);
-            mbar_init(&dzempty[s], kGbWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&dzfull[b], 1);
+            mbar_init(&dzempty[b], kGbWarps);
+        }
+        for (int bb = 0; bb < NBLK; ++bb) {
+            mbar_init(&dwready[bb], kGaWarps);
+            mbar_init(&dwfree[bb], 1);
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
         mbar_init(&wfull, 1);
         mbar_init(&wempty, kGaWarps);
-        mbar_init(&dwready, kGaWarps);
-        mbar_init(&dwfree, 1);
         mbar_init(&dbfree, kGbWarps);
-        mbar_init(&dufull, kGaWarps);
-        mbar_init(&duempty, 1);
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_z);
         tma_prefetch(&tm_g);
         tma_prefetch(&tm_u);
         tma_prefetch(&tm_bp);
-        tma_prefetch(&tm_du);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
-    }
-    if (warp >= 3 && warp < 3 + kGaWarps) {
-        // dW atoms past the last tap stay zero for the whole kernel (they pad the
-        // last 128-row block of the dB MMA).
-        const int row = (warp & 3) * 32 + lane, half = (warp - 3) >> 2;
-        for (int at = K; at < S::NA; ++at)
-            for (int q = 4 * half; q < 4 * half + 4; ++q)
-                *reinterpret_cast<uint4*>(sm + S::dw + at * kAtom128 + sw128_off(row, q)) = make_uint4(0, 0, 0, 0);
-        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                     ++cc;
                     prev = chunk;
                 }
-                const int s = it & 1;
-                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                const int s = it % NST;
+                if (!mbar_wait(&empty[s], ((it / NST) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* st = sm + s * S::stage;
                 const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
                 mbar_arrive_expect_tx(&full[s], S::stage);
@@ -196,14 +196,14 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
             const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
             const uint32_t idesc_db = idesc_bf16(128, a.ndz, true, true);
-            const uint32_t bp0 = smem_u32(sm + S::bp), dw0 = smem_u32(sm + S::dw);
+            const uint32_t bp0 = smem_u32(sm + S::bp);
             const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
             uint32_t cc = 0;          // B loads consumed
             uint32_t m = 0;           // chunks whose dB accumulation has started
             // Filter MMA of item `it`: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows in).
             auto mma1 = [&](uint32_t it) -> bool {
-                const int s = it & 1;
-                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) return false;
+                const int s = it % NST;
+                if (!mbar_wait(&full[s], (it / NST) & 1, &abort_flag, a.err)) return false;
                 tc_fence_after();
                 const uint32_t z0 = smem_u32(sm + s * S::stage);
 #pragma unroll
@@ -224,33 +224,37 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 const bool first = it == 0 || chunk_of(item - 1) != chunk;
                 const bool has_next = it + 1 < nit;
                 const bool next_same = has_next && chunk_of(item + 1) == chunk;
-                const int s = it & 1, b = it & 1;
+                const int s = it % NST, b = it & 1;
                 if (next_same) {          // the next filter MMA as soon as Wd has been read
                     if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
                     if (!mma1(it + 1)) break;
                 }
-                if (!mbar_wait(&dwready, it & 1, &abort_flag, a.err)) break;
                 if (!mbar_wait(&dzempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
                 if (first && m > 0 && !mbar_wait(&dbfree, (m - 1) & 1, &abort_flag, a.err)) break;
-                tc_fence_after();
                 const uint32_t z0 = smem_u32(sm + s * S::stage);
-                // dz = dW . Bp^T  (both K-major, K = (tap, channel))
+                const uint32_t dw0 = smem_u32(sm + S::dw);
+                bool blk_ok = true;
 #pragma unroll
-                for (int j = 0; j < K; ++j)
+                for (int bb = 0; bb < NBLK; ++bb) {
+                    if (!mbar_wait(&dwready[bb], it & 1, &abort_flag, a.err)) { blk_ok = false; break; }
+                    tc_fence_after();
+                    // dz += dW_j . Bp_j^T for the block's taps (both K-major, K = 64 channels)
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_bf16(tbase + kColDz + 64 * b, kmajor_desc(dw0 + j * kAtom128, k),
-                                  kmajor_desc(bp0 + j * 8192, k), idesc_dz, (j | k) != 0);
-                // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
+                    for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j)
 #pragma unroll
-                for (int bb = 0; bb < NBLK; ++bb)
+                        for (int k = 0; k < 4; ++k)
+                            umma_bf16(tbase + kColDz + 64 * b, kmajor_desc(dw0 + j * kAtom128, k),
+                                      kmajor_desc(bp0 + j * 8192, k), idesc_dz, (j | k) != 0);
+                    // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
                         umma_bf16(tbase + kColDb + 64 * bb, mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks),
                                   mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
+                    umma_commit(&dwfree[bb]);
+                }
+                if (!blk_ok) break;
                 if (first) ++m;
                 umma_commit(&dzfull[b]);
-                umma_commit(&dwfree);
                 umma_commit(&empty[s]);
                 if (has_next && !next_same) {      // chunk changes: B is reloaded after these MMAs
                     umma_commit(&bempty);
@@ -261,34 +265,18 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 }
             }
         }
-    } else if (warp == 2) {
-        if (lane == 0) {
-            uint32_t it = 0;
-            for (int64_t item = i0; item < i1; ++item, ++it) {
-                const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
-                if (!mbar_wait(&dufull, it & 1, &abort_flag, a.err)) break;
-                tma_store_2d(&tm_du, sm + S::dust, (int32_t)(chunk * 64), (int32_t)(tile * 128));
-                tma_store_commit();
-                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                mbar_arrive(&duempty);
-            }
-            tma_store_wait_all();
-        }
-    } else if (warp < 3 + kGaWarps) {
-        // ---- GA: du (A1) and dw (A2) of each item
+    } else if (warp < kGb0) {
+        // ---- GA: du (A1, stored straight from registers) and dw (A2) of each item
         const int q = warp & 3;
-        const int half = (warp - 3) >> 2;      // channel groups 4*half .. 4*half+3
+        const int half = (warp - kGa0) >> 2;   // channel groups 4*half .. 4*half+3
         const int row = q * 32 + lane;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
-        uint8_t* dws = sm + S::dw;
-        uint8_t* dus = sm + S::dust;
         uint32_t it = 0;
         for (int64_t item = i0; item < i1; ++item, ++it) {
-            const int64_t tile = item % a.n_tiles;
-            const int s = it & 1;
+            const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
+            const int s = it % NST;
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
-                      mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err) &&
-                      mbar_wait(&duempty, (it & 1) ^ 1, &abort_flag, a.err);
+                      mbar_wait(&full[s], (it / NST) & 1, &abort_flag, a.err);
             if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
             tc_fence_after();
             const int32_t n = (int32_t)(tile * 128) + row;
@@ -301,83 +289,91 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             }
             const uint8_t* gt = sm + s * S::stage + kRowTile;
             const uint8_t* ut = gt + kRowTile;
-            // A1: du[t, c] = g[t, c] + sum_{j <= epos} Wd_j[t, c] g[t + j, c]
-#pragma unroll 1
-            for (int g8 = 4 * half; g8 < 4 * half + 4; ++g8) {
-                uint32_t wv[K][8];
+            __nv_bfloat16* du_row = a.du + (int64_t)n * a.C + chunk * 64;
+            // A1: du[t, c] = g[t, c] + sum_{j <= epos} Wd_j[t, c] g[t + j, c], two 8-channel
+            // groups per TMEM wait, channel pairs on the packed fp32 FMA
 #pragma unroll
-                for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * g8, wv[j]);
-                uint4 gg[K];
+            for (int gp = 0; gp < 2; ++gp) {
+                const int g0 = 4 * half + 2 * gp;
+                uint32_t wv[2][K][8];
 #pragma unroll
-                for (int j = 0; j < K; ++j) gg[j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g8));
+                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                    for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * (g0 + x), wv[x][j]);
+                uint4 gg[2][K];
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                    for (int j = 0; j < K; ++j)
+                        gg[x][j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
                 tmem_wait_ld();
-                float acc[8];
-                const uint32_t* g0 = reinterpret_cast<const uint32_t*>(&gg[0]);
+                uint4 res[2];
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    acc[c] = bf16_lo(g0[c >> 1]);
-                    acc[c + 1] = bf16_hi(g0[c >> 1]);
-                }
+                for (int x = 0; x < 2; ++x) {
+                    float acc[8];
+                    const uint32_t* g0w = reinterpret_cast<const uint32_t*>(&gg[x][0]);
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    if (j <= epos) {
-                        const uint32_t* gj = reinterpret_cast<const uint32_t*>(&gg[j]);
+                    for (int p = 0; p < 4; ++p) {
+                        acc[2 * p] = bf16_lo(g0w[p]);
+                        acc[2 * p + 1] = bf16_hi(g0w[p]);
+                    }
 #pragma unroll
-                        for (int c = 0; c < 8; c += 2) {
-                            acc[c] = fmaf(__uint_as_float(wv[j][c]), bf16_lo(gj[c >> 1]), acc[c]);
-                            acc[c + 1] = fmaf(__uint_as_float(wv[j][c + 1]), bf16_hi(gj[c >> 1]), acc[c + 1]);
+                    for (int j = 0; j < K; ++j) {
+                        if (j <= epos) {
+                            const uint32_t* gj = reinterpret_cast<const uint32_t*>(&gg[x][j]);
+#pragma unroll
+                            for (int p = 0; p < 4; ++p)
+                                ffma2(acc[2 * p], acc[2 * p + 1], __uint_as_float(wv[x][j][2 * p]),
+                                      __uint_as_float(wv[x][j][2 * p + 1]), bf16_lo(gj[p]), bf16_hi(gj[p]));
                         }
                     }
+                    res[x] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                                        pack_bf16(acc[6], acc[7]));
                 }
-                *reinterpret_cast<uint4*>(dus + sw128_off(row, g8)) =
-                    make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                               pack_bf16(acc[6], acc[7]));
+                if (n < a.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(du_row + 8 * g0);
+                    dst[0] = res[0];
+                    dst[1] = res[1];
+                }
             }
             tc_fence_before();
-            fence_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&wempty);
-                mbar_arrive(&dufull);
-            }
-            // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16, one 64-channel atom per tap) once the
-            // dz / dB MMAs of the previous item have finished reading the dW tile
-            ok = mbar_wait(&dwfree, (it & 1) ^ 1, &abort_flag, a.err);
-            if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
-#pragma unroll 1
-            for (int g8 = 4 * half; g8 < 4 * half + 4; ++g8) {
-                uint4 uu[K];
-                const uint4 gv = *reinterpret_cast<const uint4*>(gt + sw128_off(row, g8));
+            if (lane == 0) mbar_arrive(&wempty);
+            // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap), block
+            // by block (taps 2 bb, 2 bb + 1), each once the MMAs that last read it have finished
+            uint4 gv[4];
 #pragma unroll
-                for (int j = 0; j < K; ++j) uu[j] = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
-                const uint32_t* g0 = reinterpret_cast<const uint32_t*>(&gv);
-                float gf[8];
+            for (int i = 0; i < 4; ++i) gv[i] = *reinterpret_cast<const uint4*>(gt + sw128_off(row, 4 * half + i));
+            uint8_t* dws = sm + S::dw;
+            bool quit = false;       // uniform over the GA warps
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    gf[c] = bf16_lo(g0[c >> 1]);
-                    gf[c + 1] = bf16_hi(g0[c >> 1]);
+            for (int bb = 0; bb < NBLK; ++bb) {
+                ok = mbar_wait(&dwfree[bb], (it & 1) ^ 1, &abort_flag, a.err);
+                if (named_bar_any<2, 32 * kGaWarps>(!ok)) {
+                    quit = true;
+                    break;
                 }
 #pragma unroll
-                for (int j = 0; j < K; ++j) {
-                    const bool v = j <= pos;
-                    const uint32_t* uj = reinterpret_cast<const uint32_t*>(&uu[j]);
-                    float d[8];
+                for (int i = 0; i < 4; ++i) {
+                    const int g8 = 4 * half + i;
 #pragma unroll
-                    for (int c = 0; c < 8; c += 2) {
-                        d[c] = v ? gf[c] * bf16_lo(uj[c >> 1]) : 0.f;
-                        d[c + 1] = v ? gf[c + 1] * bf16_hi(uj[c >> 1]) : 0.f;
+                    for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j) {
+                        const uint4 uu = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
+                        const bool v = j <= pos;
+                        uint4 d;
+                        d.x = v ? mul_bf16x2(gv[i].x, uu.x) : 0u;
+                        d.y = v ? mul_bf16x2(gv[i].y, uu.y) : 0u;
+                        d.z = v ? mul_bf16x2(gv[i].z, uu.z) : 0u;
+                        d.w = v ? mul_bf16x2(gv[i].w, uu.w) : 0u;
+                        *reinterpret_cast<uint4*>(dws + j * kAtom128 + sw128_off(row, g8)) = d;
                     }
-                    *reinterpret_cast<uint4*>(dws + j * kAtom128 + sw128_off(row, g8)) =
-                        make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
-                                   pack_bf16(d[6], d[7]));
                 }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dwready[bb]);
             }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&dwready);
-                mbar_arrive(&empty[s]);
-            }
+            if (quit) break;
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     } else {
         // ---- GB: dz readout (fp32 atomic add, reduction over chunks) and dB partials
@@ -692,12 +688,13 @@ inline unsigned grid_for(int64_t n, int threads = 256) {
 
 template <int K>
 cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
-                       const CUtensorMap& tdu, const BwdArgs& ba, unsigned grid, cudaStream_t st) {
+                       const BwdArgs& ba, unsigned grid, cudaStream_t st) {
     constexpr uint32_t smem = BwdSmem<K>::total;
+    static_assert(smem <= 232448, "shared memory of lowrank_bwd_kernel");
     cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K>, dim3(grid), dim3(kBwdPipeThreads), smem, st, tz, tg,
-                                                tu, tbp, tdu, ba));
+                                                tu, tbp, ba));
     return e;
 }
 
@@ -792,18 +789,17 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, reinterpret_cast<float4*>(dz),
         p.N * p.r / 4));
     if (e != cudaSuccess) return e;
-    CUtensorMap tz, tg, tu, tbp, tdu;
+    CUtensorMap tz, tg, tu, tbp;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
-        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
-        !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128))
+        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64))
         return cudaErrorInvalidValue;
     BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
-               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16)};
+               L.per_cta, L.pieces, dz, dbpart, static_cast<__nv_bfloat16*>(du), err, (int)((p.r + 15) / 16)};
     switch (p.K) {
-        case 1: e = launch_bwd<1>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
-        case 2: e = launch_bwd<2>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
-        case 3: e = launch_bwd<3>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
-        default: e = launch_bwd<4>(tz, tg, tu, tbp, tdu, ba, L.grid, st); break;
+        case 1: e = launch_bwd<1>(tz, tg, tu, tbp, ba, L.grid, st); break;
+        case 2: e = launch_bwd<2>(tz, tg, tu, tbp, ba, L.grid, st); break;
+        case 3: e = launch_bwd<3>(tz, tg, tu, tbp, ba, L.grid, st); break;
+        default: e = launch_bwd<4>(tz, tg, tu, tbp, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
     switch (p.K) {

@@ -9,10 +9,8 @@
 //   du[m, c] = g[m, c] + sum_{j < e(m) - m} wh[m+j, (c/hd)*K + j] g[m+j, c]
 //   dwh[n, q*K + j] = sum_{c in head q} [j <= n - s(n)] g[n, c] u[n-j, c]   (warp shuffles)
 //   dW = h^T dwh,  dh = dwh W^T                                        (tensor cores)
-// The conv kernels are memory-bound CUDA-core kernels: a block covers 64 tokens x 256
-// channels, a thread 8 channels of one token per step (16-byte loads and stores along
-// C); the K-1 earlier/later rows a token needs were just read by the block's other
-// warps and come from L1/L2.
+// The conv kernels are memory-bound CUDA-core kernels (16-byte loads and stores along C,
+// packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh).
 #include <algorithm>
 
 #include "common.cuh"
@@ -23,8 +21,6 @@
 
 namespace dynconv {
 
-cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, int64_t d, int R, void* out,
-                          int64_t out_ld, uint32_t* err, cudaStream_t st);
 cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, const void* P, int64_t N, int64_t d,
                             void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st);
 int gen_bwd_splits(int64_t N, int64_t d, int R);
@@ -34,6 +30,10 @@ namespace {
 
 using namespace tc;
 
+// A block covers kTokPerBlock tokens x 256 channels: 8 warps, each lane 8 channels of one
+// token per step (16-byte loads and stores along C), two tokens in flight per step; the K - 1
+// neighbouring rows a token needs were just read by the block's other warps and come from
+// L1 / L2.
 constexpr int kTokPerBlock = 64;
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -49,7 +49,22 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
 }
 
-__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+// acc[0..8) += w * x (8 bf16 in a uint4) on the packed fp32 FMA.
+__device__ __forceinline__ void axpy8(float (&acc)[8], float w, const uint4& x) {
+    const uint32_t* v = reinterpret_cast<const uint32_t*>(&x);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) ffma2(acc[2 * p], acc[2 * p + 1], w, w, bf16_lo(v[p]), bf16_hi(v[p]));
+}
+
+// sum_i a[i] b[i] over 8 values given as bf16 (two fp32 lanes, then their sum).
+__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
+    const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) ffma2(s0, s1, bf16_lo(x[p]), bf16_hi(x[p]), bf16_lo(y[p]), bf16_hi(y[p]));
+    return s0 + s1;
+}
 
 template <int K>
 __device__ __forceinline__ void hw_fwd_token(const __nv_bfloat16* __restrict__ u, int64_t us,
@@ -58,21 +73,25 @@ __device__ __forceinline__ void hw_fwd_token(const __nv_bfloat16* __restrict__ u
                                              int64_t n_docs, __nv_bfloat16* __restrict__ y) {
     const int32_t pos = (int32_t)n - seg_start32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen);
     uint4 uv[K];
-    float w[K];
+    __nv_bfloat16 w[K];
 #pragma unroll
     for (int j = 0; j < K; ++j) {          // issue every load of the token first
         const bool v = j <= pos;
         uv[j] = v ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
-        w[j] = v ? ldbf(wh + n * R + q * K + j) : 0.f;
     }
-    float acc[8], uf[8];
+    const __nv_bfloat16* wp = wh + n * R + q * K;
+    if constexpr (K == 4) {
+        *reinterpret_cast<uint2*>(w) = *reinterpret_cast<const uint2*>(wp);
+    } else if constexpr (K == 2) {
+        *reinterpret_cast<uint32_t*>(w) = *reinterpret_cast<const uint32_t*>(wp);
+    } else {
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = wp[j];
+    }
+    float acc[8];
     unpack8(uv[0], acc);
 #pragma unroll
-    for (int j = 0; j < K; ++j) {
-        unpack8(uv[j], uf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], uf[i], acc[i]);
-    }
+    for (int j = 0; j < K; ++j) axpy8(acc, j <= pos ? __bfloat162float(w[j]) : 0.f, uv[j]);
     *reinterpret_cast<uint4*>(y + n * C + c) = pack8(acc);
 }
 
@@ -93,6 +112,40 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
         hw_fwd_token<K>(u, us, wh, R, q, n, c, C, seqlen, cu, n_docs, y);
         if (n + 8 < n1) hw_fwd_token<K>(u, us, wh, R, q, n + 8, c, C, seqlen, cu, n_docs, y);
     }
+}
+
+// Sums p[0..K) over the L lanes (a power of two) that hold one head and stores dst[j] for
+// j < K, masked to 0 for j > pos.  For K >= 3 and L >= 4 a reduce-scatter: two exchange
+// steps leave each lane one tap, then a butterfly finishes it (log2(L) + 1 shuffles instead
+// of K log2(L)); otherwise a plain butterfly over all K values.
+template <int K>
+__device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int32_t pos,
+                                               __nv_bfloat16* __restrict__ dst) {
+    if constexpr (K >= 3) {
+        if (L >= 4) {
+            const float q3 = K > 3 ? p[K - 1] : 0.f;
+            const int h1 = L >> 1, h2 = L >> 2;
+            const bool b1 = (gl & h1) != 0, b2 = (gl & h2) != 0;
+            const float s0 = b1 ? p[0] : p[2], s1 = b1 ? p[1] : q3;
+            float k0 = b1 ? p[2] : p[0], k1 = b1 ? q3 : p[1];
+            k0 += __shfl_xor_sync(0xffffffffu, s0, h1);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, h1);
+            const float s = b2 ? k0 : k1;
+            float k = b2 ? k1 : k0;
+            k += __shfl_xor_sync(0xffffffffu, s, h2);
+            for (int off = h2 >> 1; off > 0; off >>= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
+            const int tap = (b1 ? 2 : 0) + (b2 ? 1 : 0);
+            if ((gl & (h2 - 1)) == 0 && tap < K) dst[tap] = __float2bfloat16_rn(tap <= pos ? k : 0.f);
+            return;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        for (int off = L >> 1; off > 0; off >>= 1) p[j] += __shfl_xor_sync(0xffffffffu, p[j], off);
+    const int l = gl & (L - 1);
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        if (j % L == l) dst[j] = __float2bfloat16_rn(j <= pos ? p[j] : 0.f);
 }
 
 // L = head_dim / 8 lanes hold one head's channels (a power of two <= 32, aligned in the warp).
@@ -117,38 +170,24 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
         seg_bounds32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb, eb);
         const int32_t pos = (int32_t)n - sb, epos = eb - 1 - (int32_t)n;
         uint4 gv[K], uv[K];
-        float w[K];
+        __nv_bfloat16 w[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {          // issue every load of the token first
             const bool f = j <= epos, p = j <= pos;
             gv[j] = f ? *reinterpret_cast<const uint4*>(g + (n + j) * C + c) : make_uint4(0, 0, 0, 0);
-            w[j] = f ? ldbf(wh + (n + j) * R + q * K + j) : 0.f;     // du: filter of token n+j, tap j
+            w[j] = f ? wh[(n + j) * R + q * K + j] : __float2bfloat16_rn(0.f);   // filter of token n+j, tap j
             uv[j] = p ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
         }
-        float gn[8], acc[8], tmp[8];
-        unpack8(gv[0], gn);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = gn[i];
+        float acc[8];
+        unpack8(gv[0], acc);
         float part[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {
-            unpack8(gv[j], tmp);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], tmp[i], acc[i]);
-            unpack8(uv[j], tmp);                // dwh partial over this thread's 8 channels
-            float pj = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) pj = fmaf(gn[i], tmp[i], pj);
-            part[j] = pj;
+            axpy8(acc, __bfloat162float(w[j]), gv[j]);
+            part[j] = dot8(gv[0], uv[j]);       // dwh partial over this thread's 8 channels
         }
         *reinterpret_cast<uint4*>(du + n * C + c) = pack8(acc);
-        // sum over the head's L lanes (fixed butterfly: deterministic)
-#pragma unroll
-        for (int j = 0; j < K; ++j)
-            for (int off = L >> 1; off > 0; off >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
-        if ((gl & (L - 1)) == 0)
-#pragma unroll
-            for (int j = 0; j < K; ++j) dwh[n * R + q * K + j] = __float2bfloat16_rn(part[j]);
+        head_sum_store<K>(part, L, gl, pos, dwh + n * R + q * K);
     }
 }
 
@@ -186,7 +225,7 @@ static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, v
     DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
         p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
-    (void)e;
+    return e;
 }
 
 template <int K>

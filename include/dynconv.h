@@ -139,19 +139,21 @@ DYNCONV_API dynconv_status dynconv_bwd(const dynconv_desc *desc, const int32_t *
 /* Forward for callers that cannot allocate device memory (no counterpart in
  * the paper: a deployment variant of dynconv_fwd).  Runs the bf16 low-rank
  * tensor-core forward of a dense batch with no workspace argument: its scratch
- * (z = h A, bf16 [N, r], and the device error word) lives in a buffer built
- * into the library, 8 MiB + 256 bytes held on every GPU that loads the library
- * until the process exits.  It calls no cudaMalloc/cudaFree or other
- * allocating routine.
+ * (the tap-major copy of B, bf16 [r, K*C]; z = h A, bf16 [N, r]; the device
+ * error word) lives in a buffer built into the library, 8 MiB + 256 bytes held
+ * on every GPU that loads the library until the process exits.  It calls no
+ * cudaMalloc/cudaFree or other allocating routine.
  *   u, h, A, B, y, z_save: as for dynconv_fwd (z_save nullable; when given, z
- *   is written there and the built-in buffer only holds the error word).
+ *   is written there instead of the built-in buffer).
  *   Returns DYNCONV_ERR_UNSUPPORTED for shapes outside the tensor-core forward
  *   (fp32, head-wise, rank not a multiple of 8 or above 64, channels not a
- *   multiple of 64) and when z_save is NULL and N * rank * 2 exceeds 8 MiB.
+ *   multiple of 64) and when the scratch does not fit 8 MiB: rank * channels *
+ *   ksize * 2 bytes (rounded up to 256) plus, when z_save is NULL,
+ *   N * rank * 2 bytes.
  * The first call with a given device current looks up the buffer's device
  * address (cudaGetSymbolAddress) once for that device; make that first call
  * before any stream capture.  All calls share the buffer, which keeps the last
- * call's contents; each call clears the error word and rewrites z.  Calls
+ * call's contents; each call clears the error word and rewrites Bp and z.  Calls
  * whose work overlaps on the GPU race on the buffer: serialise them. */
 DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc *desc, const void *u, const void *h,
                                                const void *A, const void *B, void *y, void *z_save, void *stream);
