@@ -108,7 +108,7 @@ def kernel_bytes(name, w, layer):
         "tc_lowrank_fwd": N * C * 2 * s + N * R * s + BW * s,
         "tc_lowrank_bwd": N * C * 3 * s + N * R * s + BW * s,
         "tc_gen_bwd": N * d * 2 * s + N * R * s + P * (s + 4),
-        "tc_headwise_fwd": N * C * 2 * s + N * d * s + P * s,
+        "tc_headwise_fwd": N * C * 2 * s + N * R * s,
         "tc_headwise_bwd": N * C * 3 * s + N * R * 4,
     }
     return table.get(name)

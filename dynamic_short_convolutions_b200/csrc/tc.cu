@@ -386,23 +386,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
             const uint8_t* us = sm + s * kFwdStage + kZBytes;
             uint8_t* ys = sm + S::ys + b * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
-#pragma unroll 1
-            for (int gp = 0; gp < 2; ++gp) {            // two groups of 8 channels per batch
-                const int g0 = 4 * half + 2 * gp;
-                uint32_t wv[2][K][8];
+            // NG 8-channel groups per pass (all four of this warp's groups when the registers
+            // allow): every TMEM and shared-memory load first, then one wait, then the arithmetic
+            constexpr int NG = K <= 3 ? 4 : 2;
 #pragma unroll
-                for (int x = 0; x < 2; ++x)
+            for (int pass = 0; pass < 4 / NG; ++pass) {
+                const int g0 = 4 * half + NG * pass;
+                uint32_t wv[NG][K][8];
+#pragma unroll
+                for (int x = 0; x < NG; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j) tmem_ld8(taddr + 64 * j + 8 * (g0 + x), wv[x][j]);
-                uint4 uj[2][K];
+                uint4 uj[NG][K];
 #pragma unroll
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < NG; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j)
                         uj[x][j] = *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g0 + x));
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < NG; ++x)
                     *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = conv8<K>(wv[x], uj[x], pos);
             }
             tc_fence_before();

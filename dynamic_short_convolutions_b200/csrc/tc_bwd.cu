@@ -20,19 +20,21 @@
 //       MMA1  Wd_j[t, c] = sum_k z[t+j, k] Bp[k, j C + c]   (the filter of token t+j:
 //             the z tile is loaded with 8 rows of look-ahead and the A operand starts
 //             j rows into it), so du needs no exchange between threads;
-//       epi A du (stored from registers) and dw (-> bf16 tile in shared memory, 64 channels
-//             per tap);
+//       epi A du (-> staged, TMA store) and dw (-> bf16 tile in shared memory, 64 channels
+//             per tap, handed to the MMAs in blocks of two taps);
 //       MMA2  dz  = dW Bp_chunk^T      (M = 128 tokens, N = r, K = 64 K)
 //       MMA3  dBt += dW^T z            (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
-//       epi B dz -> fp32 atomic add into a [N, r] buffer (reduction over chunks);
+//       epi B dz -> staged fp32 tile, bulk tensor add into a [N, r] buffer (reduction over
+//             chunks; fp32 atomics when the tile does not fit);
 //       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
-//   reduce_dB_kernel   sums the partials of each chunk in run order -> dB [r, C K] fp32.
-//   dz_to_bf16_kernel  fp32 dz -> bf16 operand for the generator backward.
+//   bwd_finish_kernel  sums the dB partials of each chunk in run order -> dB [r, C K] fp32, and
+//                      converts the fp32 dz to the bf16 operand of the generator backward.
 //   gen_bwd_kernel     dh = dz A^T (M = 128 tokens, N = 256 of d, K = r) and
 //                      dA += h^T dz (M = 128 of d, N = r, K = 128 tokens) per (256-wide d
 //                      block, token range); reduce_splits_kernel sums the token ranges.
 #include <algorithm>
 #include <cstdio>
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
@@ -79,26 +81,32 @@ struct BwdArgs {
     int pieces;               // partial slots per chunk
     float* dz_acc;            // [N, r] fp32, zero on entry
     float* dB_part;           // [n_chunks][pieces][64 K][r]
-    __nv_bfloat16* du;        // [N, C] dense
     uint32_t* err;
     int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
+    int dz_tma;               // 1: dz tiles are added with bulk tensor reductions, else fp32 atomics
 };
 
-// Shared memory of lowrank_bwd_kernel<K>: NST z | g | u stages (three for K <= 3: a stage
-// lives from its TMA load until the dB MMA has read z, so the loads of two later items must
-// be in flight meanwhile), one dW tile (K tap atoms of 128 tokens x 64 channels) and the
-// chunk's Bp slice.  The dB MMA reads dW in 128-row blocks of two tap atoms; for odd K the
-// last block's second atom lies past the tile (in the Bp region, which is at least one atom
-// long) and only feeds accumulator rows that are never read.
-template <int K>
+constexpr uint32_t kSmemMax = 232448 - 256;         // dynamic shared memory (static barriers aside)
+
+// Shared memory of lowrank_bwd_kernel<K, R64> (R64: rank above 32).  Two g | u slots (each
+// held from its TMA load until the du / dw epilogue is done with it) and NZ z slots (held
+// until the dB MMA has read z; three when they fit), one dW tile (K tap atoms of 128 tokens x
+// 64 channels, handed to the MMAs in 128-row blocks of two atoms), the du tile staged for its
+// TMA store, the chunk's Bp slice, and (K <= 3) the fp32 dz tile staged for its bulk reduction.
+// The dB MMA reads dW in blocks of two atoms; for odd K the last block's second atom is the du
+// staging tile and only feeds accumulator rows that are never read.
+template <int K, bool R64>
 struct BwdSmem {
-    static constexpr int NST = K <= 3 ? 3 : 2;
-    static constexpr uint32_t stage = 3 * kRowTile;         // z | g | u
-    static constexpr uint32_t dw = NST * stage;
-    static constexpr uint32_t dw_buf = K * kAtom128;
-    static constexpr uint32_t bp = dw + dw_buf;
-    static constexpr uint32_t bp_bytes = K * 8192 > kAtom128 ? K * 8192 : kAtom128;
-    static constexpr uint32_t total = bp + bp_bytes + 1024;
+    static constexpr uint32_t gu = 2 * kRowTile;
+    static constexpr uint32_t dzst_bytes = K <= 3 ? (R64 ? 2 * kAtom128 : kAtom128) : 0;
+    static constexpr uint32_t fixed = K * kAtom128 + kAtom128 + K * 8192 + dzst_bytes;
+    static constexpr int NZ = 2 * gu + 3 * kRowTile + fixed + 1024 <= kSmemMax ? 3 : 2;
+    static constexpr uint32_t z0 = 2 * gu;
+    static constexpr uint32_t dw = z0 + NZ * kRowTile;
+    static constexpr uint32_t dust = dw + K * kAtom128;
+    static constexpr uint32_t bp = dust + kAtom128;
+    static constexpr uint32_t dzst = bp + K * 8192;
+    static constexpr uint32_t total = dzst + dzst_bytes + 1024;
 };
 
 // Warp roles of lowrank_bwd_kernel: 0 TMA loads, 1 MMA issue (and TMEM owner), 2..9 the du / dw
@@ -110,34 +118,38 @@ constexpr int kBwdPipeThreads = 32 * (kGb0 + kGbWarps);
 // TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
 constexpr uint32_t kColDz = 256, kColDb = 384;
 
-template <int K>
+template <int K, bool R64>
 __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                          const __grid_constant__ CUtensorMap tm_g,
                                                                          const __grid_constant__ CUtensorMap tm_u,
                                                                          const __grid_constant__ CUtensorMap tm_bp,
+                                                                         const __grid_constant__ CUtensorMap tm_du,
+                                                                         const __grid_constant__ CUtensorMap tm_dz,
                                                                          BwdArgs a) {
-    using S = BwdSmem<K>;
+    using S = BwdSmem<K, R64>;
     constexpr int NBLK = (K + 1) / 2;
-    constexpr int NST = S::NST;
+    constexpr int NZ = S::NZ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     // dwready / dwfree: per 128-row block (two tap atoms) of the dW tile, so the MMAs of one
     // block overlap the writing of the next and the next item's first block
-    __shared__ uint64_t full[NST], empty[NST], bfull, bempty, wfull, wempty, dwready[NBLK], dwfree[NBLK], dzfull[2],
-        dzempty[2], dbfree;
+    __shared__ uint64_t gufull[2], guempty[2], zfull[NZ], zempty[NZ], bfull, bempty, wfull, wempty, dwready[NBLK],
+        dwfree[NBLK], dzfull[2], dzempty[2], dbfree;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t i0 = (int64_t)blockIdx.x * a.per_cta;
     const int64_t i1 = min(i0 + a.per_cta, a.n_items);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kGaWarps);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&gufull[s], 1);
+            mbar_init(&guempty[s], kGaWarps);
+            mbar_init(&dzfull[s], 1);
+            mbar_init(&dzempty[s], kGbWarps);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&dzfull[b], 1);
-            mbar_init(&dzempty[b], kGbWarps);
+        for (int s = 0; s < NZ; ++s) {
+            mbar_init(&zfull[s], 1);
+            mbar_init(&zempty[s], 1);
         }
         for (int bb = 0; bb < NBLK; ++bb) {
             mbar_init(&dwready[bb], kGaWarps);
@@ -154,6 +166,8 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
         tma_prefetch(&tm_g);
         tma_prefetch(&tm_u);
         tma_prefetch(&tm_bp);
+        tma_prefetch(&tm_du);
+        if (a.dz_tma) tma_prefetch(&tm_dz);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base, 512);
@@ -181,14 +195,16 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                     ++cc;
                     prev = chunk;
                 }
-                const int s = it % NST;
-                if (!mbar_wait(&empty[s], ((it / NST) & 1) ^ 1, &abort_flag, a.err)) break;
-                uint8_t* st = sm + s * S::stage;
                 const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
-                mbar_arrive_expect_tx(&full[s], S::stage);
-                tma_load_2d(st, &tm_z, &full[s], 0, m0);
-                tma_load_2d(st + kRowTile, &tm_g, &full[s], c0, m0);
-                tma_load_2d(st + 2 * kRowTile, &tm_u, &full[s], c0, m0 - 8);
+                const int zs = it % NZ, gs = it & 1;
+                if (!mbar_wait(&zempty[zs], ((it / NZ) & 1) ^ 1, &abort_flag, a.err)) break;
+                mbar_arrive_expect_tx(&zfull[zs], kRowTile);
+                tma_load_2d(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, m0);
+                if (!mbar_wait(&guempty[gs], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                uint8_t* gu = sm + gs * S::gu;
+                mbar_arrive_expect_tx(&gufull[gs], S::gu);
+                tma_load_2d(gu, &tm_g, &gufull[gs], c0, m0);
+                tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], c0, m0 - 8);
             }
         }
     } else if (warp == 1) {
@@ -197,15 +213,16 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
             const uint32_t idesc_db = idesc_bf16(128, a.ndz, true, true);
             const uint32_t bp0 = smem_u32(sm + S::bp);
+            const uint32_t dw0 = smem_u32(sm + S::dw);
             const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
             uint32_t cc = 0;          // B loads consumed
             uint32_t m = 0;           // chunks whose dB accumulation has started
             // Filter MMA of item `it`: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows in).
             auto mma1 = [&](uint32_t it) -> bool {
-                const int s = it % NST;
-                if (!mbar_wait(&full[s], (it / NST) & 1, &abort_flag, a.err)) return false;
+                const int zs = it % NZ;
+                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) return false;
                 tc_fence_after();
-                const uint32_t z0 = smem_u32(sm + s * S::stage);
+                const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
 #pragma unroll
                 for (int j = 0; j < K; ++j)
                     for (int k = 0; k < a.ksteps; ++k)
@@ -224,19 +241,21 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 const bool first = it == 0 || chunk_of(item - 1) != chunk;
                 const bool has_next = it + 1 < nit;
                 const bool next_same = has_next && chunk_of(item + 1) == chunk;
-                const int s = it % NST, b = it & 1;
+                const int zs = it % NZ, b = it & 1;
                 if (next_same) {          // the next filter MMA as soon as Wd has been read
                     if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
                     if (!mma1(it + 1)) break;
                 }
                 if (!mbar_wait(&dzempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
                 if (first && m > 0 && !mbar_wait(&dbfree, (m - 1) & 1, &abort_flag, a.err)) break;
-                const uint32_t z0 = smem_u32(sm + s * S::stage);
-                const uint32_t dw0 = smem_u32(sm + S::dw);
+                const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
                 bool blk_ok = true;
 #pragma unroll
                 for (int bb = 0; bb < NBLK; ++bb) {
-                    if (!mbar_wait(&dwready[bb], it & 1, &abort_flag, a.err)) { blk_ok = false; break; }
+                    if (!mbar_wait(&dwready[bb], it & 1, &abort_flag, a.err)) {
+                        blk_ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     // dz += dW_j . Bp_j^T for the block's taps (both K-major, K = 64 channels)
 #pragma unroll
@@ -255,7 +274,7 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 if (!blk_ok) break;
                 if (first) ++m;
                 umma_commit(&dzfull[b]);
-                umma_commit(&empty[s]);
+                umma_commit(&zempty[zs]);
                 if (has_next && !next_same) {      // chunk changes: B is reloaded after these MMAs
                     umma_commit(&bempty);
                     if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
@@ -266,17 +285,21 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             }
         }
     } else if (warp < kGb0) {
-        // ---- GA: du (A1, stored straight from registers) and dw (A2) of each item
+        // ---- GA: du (A1, staged for a TMA store) and dw (A2) of each item
         const int q = warp & 3;
         const int half = (warp - kGa0) >> 2;   // channel groups 4*half .. 4*half+3
         const int row = q * 32 + lane;
+        const bool leader = warp == kGa0 && lane == 0;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
+        uint8_t* dus = sm + S::dust;
+        uint8_t* dws = sm + S::dw;
         uint32_t it = 0;
         for (int64_t item = i0; item < i1; ++item, ++it) {
             const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
-            const int s = it % NST;
+            const int gs = it & 1;
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
-                      mbar_wait(&full[s], (it / NST) & 1, &abort_flag, a.err);
+                      mbar_wait(&gufull[gs], (it >> 1) & 1, &abort_flag, a.err);
+            if (leader) tma_store_wait_read_all();     // the previous du store has read the staging tile
             if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
             tc_fence_after();
             const int32_t n = (int32_t)(tile * 128) + row;
@@ -287,11 +310,11 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 pos = n - sb;
                 epos = eb - 1 - n;
             }
-            const uint8_t* gt = sm + s * S::stage + kRowTile;
+            const uint8_t* gt = sm + gs * S::gu;
             const uint8_t* ut = gt + kRowTile;
-            __nv_bfloat16* du_row = a.du + (int64_t)n * a.C + chunk * 64;
             // A1: du[t, c] = g[t, c] + sum_{j <= epos} Wd_j[t, c] g[t + j, c], two 8-channel
-            // groups per TMEM wait, channel pairs on the packed fp32 FMA
+            // groups per TMEM wait, channel pairs on the packed fp32 FMA; g[t] is kept for A2
+            uint4 gv[4];
 #pragma unroll
             for (int gp = 0; gp < 2; ++gp) {
                 const int g0 = 4 * half + 2 * gp;
@@ -307,9 +330,9 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                     for (int j = 0; j < K; ++j)
                         gg[x][j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
                 tmem_wait_ld();
-                uint4 res[2];
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
+                    gv[2 * gp + x] = gg[x][0];
                     float acc[8];
                     const uint32_t* g0w = reinterpret_cast<const uint32_t*>(&gg[x][0]);
 #pragma unroll
@@ -327,24 +350,17 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                                       __uint_as_float(wv[x][j][2 * p + 1]), bf16_lo(gj[p]), bf16_hi(gj[p]));
                         }
                     }
-                    res[x] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                                        pack_bf16(acc[6], acc[7]));
-                }
-                if (n < a.N) {
-                    uint4* dst = reinterpret_cast<uint4*>(du_row + 8 * g0);
-                    dst[0] = res[0];
-                    dst[1] = res[1];
+                    *reinterpret_cast<uint4*>(dus + sw128_off(row, g0 + x)) =
+                        make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                                   pack_bf16(acc[6], acc[7]));
                 }
             }
             tc_fence_before();
+            fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty);
             // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap), block
             // by block (taps 2 bb, 2 bb + 1), each once the MMAs that last read it have finished
-            uint4 gv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) gv[i] = *reinterpret_cast<const uint4*>(gt + sw128_off(row, 4 * half + i));
-            uint8_t* dws = sm + S::dw;
             bool quit = false;       // uniform over the GA warps
 #pragma unroll
             for (int bb = 0; bb < NBLK; ++bb) {
@@ -352,6 +368,10 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 if (named_bar_any<2, 32 * kGaWarps>(!ok)) {
                     quit = true;
                     break;
+                }
+                if (bb == 0 && leader) {                 // every GA warp has staged its du rows
+                    tma_store_2d(&tm_du, dus, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                    tma_store_commit();
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -373,19 +393,25 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 if (lane == 0) mbar_arrive(&dwready[bb]);
             }
             if (quit) break;
-            if (lane == 0) mbar_arrive(&empty[s]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&guempty[gs]);
         }
+        if (leader) tma_store_wait_all();
     } else {
-        // ---- GB: dz readout (fp32 atomic add, reduction over chunks) and dB partials
+        // ---- GB: dz readout (added into the [N, r] fp32 buffer: reduction over chunks) and dB partials
         const int q = warp & 3;
         const int row = q * 32 + lane;
+        const bool leader = warp == kGb0 && lane == 0;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
+        uint8_t* dzs = sm + S::dzst;
+        const bool via_tma = S::dzst_bytes > 0 && a.dz_tma;
         uint32_t it = 0;
         for (int64_t item = i0; item < i1; ++item, ++it) {
             const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
             const bool last = (item + 1 == i1) || (chunk_of(item + 1) != chunk);
             const int b = it & 1;
             const bool ok = mbar_wait(&dzfull[b], (it >> 1) & 1, &abort_flag, a.err);
+            if (via_tma && leader) tma_store_wait_read_all();   // the previous reduction has read the tile
             if (named_bar_any<3, 32 * kGbWarps>(!ok)) break;
             tc_fence_after();
             const int32_t n = (int32_t)(tile * 128) + row;
@@ -394,7 +420,21 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 tmem_ld8(lane_base + kColDz + 64 * b + c, v[0]);
                 if (c + 8 < a.r) tmem_ld8(lane_base + kColDz + 64 * b + c + 8, v[1]);
                 tmem_wait_ld();
-                if (n < a.N) {
+                if (via_tma) {
+                    // fp32 tile [128 rows][32 columns] per 128-byte swizzled box
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int cc = c + 8 * h;
+                        if (cc < a.r) {
+                            uint8_t* box = dzs + (cc >> 5) * kAtom128;
+                            const int qq = (cc & 31) >> 2;
+                            *reinterpret_cast<uint4*>(box + sw128_off(row, qq)) =
+                                make_uint4(v[h][0], v[h][1], v[h][2], v[h][3]);
+                            *reinterpret_cast<uint4*>(box + sw128_off(row, qq + 1)) =
+                                make_uint4(v[h][4], v[h][5], v[h][6], v[h][7]);
+                        }
+                    }
+                } else if (n < a.N) {
                     float4* dst = reinterpret_cast<float4*>(a.dz_acc + (int64_t)n * a.r + c);
                     atomicAdd(dst, make_float4(__uint_as_float(v[0][0]), __uint_as_float(v[0][1]),
                                                __uint_as_float(v[0][2]), __uint_as_float(v[0][3])));
@@ -409,20 +449,29 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 }
             }
             tc_fence_before();
+            if (via_tma) fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&dzempty[b]);
+            if (via_tma) {
+                named_bar_any<3, 32 * kGbWarps>(false);     // every GB warp has staged its dz rows
+                if (leader) {
+                    for (int bx = 0; bx * 32 < a.r; ++bx)
+                        tma_reduce_add_2d(&tm_dz, dzs + bx * kAtom128, bx * 32, (int32_t)(tile * 128));
+                    tma_store_commit();
+                }
+            }
             if (last) {                            // the run for this chunk ends: its dB partial
                 const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
                 float* part = a.dB_part + ((chunk * a.pieces + piece) * (64 * K)) * a.r;
 #pragma unroll
                 for (int bb = 0; bb < NBLK; ++bb) {
-                    const int m = bb * 128 + row;     // (tap, channel) row = j * 64 + c
+                    const int mrow = bb * 128 + row;     // (tap, channel) row = j * 64 + c
                     for (int c = 0; c < a.r; c += 8) {
                         uint32_t v[8];
                         tmem_ld8(lane_base + kColDb + 64 * bb + c, v);
                         tmem_wait_ld();
-                        if (m < 64 * K) {
-                            float4* dst = reinterpret_cast<float4*>(part + (int64_t)m * a.r + c);
+                        if (mrow < 64 * K) {
+                            float4* dst = reinterpret_cast<float4*>(part + (int64_t)mrow * a.r + c);
                             dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
                                                  __uint_as_float(v[3]));
                             dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
@@ -435,6 +484,7 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                 if (lane == 0) mbar_arrive(&dbfree);
             }
         }
+        if (via_tma && leader) tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -444,31 +494,33 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
     }
 }
 
-// dB[k, c K + j] = sum over the runs covering chunk c/64, in run order (one thread per entry).
+// After the backward kernel, in one launch: dB[k, c K + j] = the sum of the partials of the runs
+// covering chunk c/64, in run order (one thread per entry), and the fp32 dz accumulator -> bf16
+// operand of the generator backward (four values per thread).
 template <int K>
-__global__ void reduce_dB_kernel(const float* __restrict__ part, float* __restrict__ dB, int r, int C, int n_tiles,
-                                 int per_cta, int pieces) {
+__global__ void bwd_finish_kernel(const float* __restrict__ part, float* __restrict__ dB, int r, int C, int n_tiles,
+                                  int per_cta, int pieces, const float4* __restrict__ dz4, uint2* __restrict__ dzb,
+                                  int64_t count4) {
     pdl_trigger();
     pdl_wait();
-    const int total = r * C * K;
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-        const int k = e / (C * K), col = e - k * (C * K), c = col / K, j = col - c * K;
-        const int chunk = c >> 6, m = j * 64 + (c & 63);
-        const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
-        const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
-        const float* src = part + ((int64_t)chunk * pieces * (64 * K) + m) * r + k;
-        float acc = 0.f;
-        for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * (64 * K) * r];
-        dB[e] = acc;
-    }
-}
-
-__global__ void dz_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t count4) {
-    pdl_trigger();
-    pdl_wait();
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count4; i += (int64_t)gridDim.x * blockDim.x) {
-        const float4 v = src[i];
-        dst[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    const int64_t nb = (int64_t)r * C * K;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nb + count4;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        if (e < nb) {
+            const int ei = (int)e;
+            const int k = ei / (C * K), col = ei - k * (C * K), c = col / K, j = col - c * K;
+            const int chunk = c >> 6, m = j * 64 + (c & 63);
+            const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
+            const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
+            const float* src = part + ((int64_t)chunk * pieces * (64 * K) + m) * r + k;
+            float acc = 0.f;
+            for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * (64 * K) * r];
+            dB[e] = acc;
+        } else {
+            const int64_t i4 = e - nb;
+            const float4 v = dz4[i4];
+            dzb[i4] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+        }
     }
 }
 
@@ -686,15 +738,17 @@ inline unsigned grid_for(int64_t n, int threads = 256) {
     return (unsigned)std::max<int64_t>(1, std::min<int64_t>(b, 148 * 16));
 }
 
-template <int K>
+template <int K, bool R64>
 cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
-                       const BwdArgs& ba, unsigned grid, cudaStream_t st) {
-    constexpr uint32_t smem = BwdSmem<K>::total;
-    static_assert(smem <= 232448, "shared memory of lowrank_bwd_kernel");
-    cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                       const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba, unsigned grid, cudaStream_t st) {
+    using S = BwdSmem<K, R64>;
+    static_assert(S::total <= kSmemMax, "shared memory of lowrank_bwd_kernel");
+    if (S::dzst_bytes == 0) ba.dz_tma = 0;
+    cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K, R64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::total);
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K>, dim3(grid), dim3(kBwdPipeThreads), smem, st, tz, tg,
-                                                tu, tbp, ba));
+    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64>, dim3(grid), dim3(kBwdPipeThreads), S::total,
+                                                st, tz, tg, tu, tbp, tdu, tdz, ba));
     return e;
 }
 
@@ -789,36 +843,43 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
         static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, reinterpret_cast<float4*>(dz),
         p.N * p.r / 4));
     if (e != cudaSuccess) return e;
-    CUtensorMap tz, tg, tu, tbp;
+    CUtensorMap tz, tg, tu, tbp, tdu, tdz;
+    std::memset(&tdz, 0, sizeof(tdz));                 // unused unless dz goes through bulk reductions
+    const bool dz_tma = p.r % 32 == 0;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
-        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64))
+        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+        !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128) ||
+        (dz_tma && !make_tmap_2d(&tdz, dz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.r, p.N, p.r * 4, 32, 128, true)))
         return cudaErrorInvalidValue;
     BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
-               L.per_cta, L.pieces, dz, dbpart, static_cast<__nv_bfloat16*>(du), err, (int)((p.r + 15) / 16)};
-    switch (p.K) {
-        case 1: e = launch_bwd<1>(tz, tg, tu, tbp, ba, L.grid, st); break;
-        case 2: e = launch_bwd<2>(tz, tg, tu, tbp, ba, L.grid, st); break;
-        case 3: e = launch_bwd<3>(tz, tg, tu, tbp, ba, L.grid, st); break;
-        default: e = launch_bwd<4>(tz, tg, tu, tbp, ba, L.grid, st); break;
+               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dz_tma ? 1 : 0};
+    const bool r64 = p.r > 32;
+    switch (p.K * 2 + (r64 ? 1 : 0)) {
+        case 2: e = launch_bwd<1, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 3: e = launch_bwd<1, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 4: e = launch_bwd<2, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 5: e = launch_bwd<2, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 6: e = launch_bwd<3, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 7: e = launch_bwd<3, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 8: e = launch_bwd<4, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        default: e = launch_bwd<4, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
     switch (p.K) {
-#define DC_REDUCE_DB(KK)                                                                                          \
+#define DC_FINISH(KK)                                                                                             \
     case KK:                                                                                                       \
-        DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_dB_kernel<KK>, dim3(grid_for(p.r * p.C * p.K)), dim3(256), 0, st, \
-                                                (const float*)dbpart, dB, (int)p.r, (int)p.C, (int)L.n_tiles,        \
-                                                (int)L.per_cta, L.pieces));                                          \
+        DC_LAUNCH(kTcReduce, st, e = launch_pdl(bwd_finish_kernel<KK>, dim3(grid_for(p.r * p.C * p.K + p.N * p.r / 4)), \
+                                                dim3(256), 0, st, (const float*)dbpart, dB, (int)p.r, (int)p.C,      \
+                                                (int)L.n_tiles, (int)L.per_cta, L.pieces,                            \
+                                                reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb), \
+                                                p.N * p.r / 4));                                                     \
         break;
-        DC_REDUCE_DB(1)
-        DC_REDUCE_DB(2)
-        DC_REDUCE_DB(3)
-        DC_REDUCE_DB(4)
-#undef DC_REDUCE_DB
+        DC_FINISH(1)
+        DC_FINISH(2)
+        DC_FINISH(3)
+        DC_FINISH(4)
+#undef DC_FINISH
     }
-    if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcReduce, st, e = launch_pdl(dz_to_bf16_kernel, dim3(grid_for(p.N * p.r / 4)), dim3(256), 0, st,
-                                            reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb),
-                                            p.N * p.r / 4));
     if (e != cudaSuccess) return e;
     // generator backward: dA = h^T dz, dh = dz A^T
     return tc_gen_backward(dzb, (int)p.r, h, p.hs, A, p.N, p.d, dh, dA, dpart, err, st);
