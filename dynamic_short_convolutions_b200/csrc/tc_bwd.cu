@@ -29,8 +29,8 @@
 //       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
 //   bwd_finish_kernel  sums the dB partials of each chunk in run order -> dB [r, C K] fp32, and
 //                      converts the fp32 dz to the bf16 operand of the generator backward.
-//   gen_bwd_kernel     dh = dz A^T (M = 128 tokens, N = 256 of d, K = r) and
-//                      dA += h^T dz (M = 128 of d, N = r, K = 128 tokens) per (256-wide d
+//   gen_bwd_kernel     dh = dz A^T (M = 128 tokens, N = 128 of d, K = r; staged, TMA store) and
+//                      dA += h^T dz (M = 128 of d, N = r, K = 128 tokens) per (128-wide d
 //                      block, token range); reduce_splits_kernel sums the token ranges.
 #include <algorithm>
 #include <cstdio>
@@ -550,14 +550,15 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, float* __re
 }
 
 // =====================================================================================
-// gen_bwd_kernel<XA>: per (DB-wide block db of d, token range), X = dz (low-rank) or the
+// gen_bwd_kernel<XA>: per (128-wide block db of d, token range), X = dz (low-rank) or the
 // head-wise filter gradient dwh, P = A or W, with R = X's width:
-//   dh[t, db*DB + i] = sum_k X[t, k] P[db*DB + i, k]
-//   dPpart[split][db*DB + i, k] = sum_{t in range} h[t, db*DB + i] X[t, k]
-// XA = 64-wide atoms of X (1: R <= 64, DB = 256; 2: R <= 128, DB = 128).
-// smem: stage = X tile [128 tokens][XA atoms] (K-major A of dh; MN-major B of dP) + h tile
-//       [128 tokens][DB/64 atoms] (MN-major A of dP); P block [DB rows of d][XA atoms] resident
-//       (K-major B of dh).  TMEM: dh [128][DB] at column 0, dP blocks [128 rows of d][R] after it.
+//   dh[t, db*128 + i] = sum_k X[t, k] P[db*128 + i, k]
+//   dPpart[split][db*128 + i, k] = sum_{t in range} h[t, db*128 + i] X[t, k]
+// XA = 64-wide atoms of X (1: R <= 64, 2: R <= 128).
+// smem: NS stages of X tile [128 tokens][XA atoms] (K-major A of dh; MN-major B of dP) + h tile
+//       [128 tokens][2 atoms] (MN-major A of dP); P block [128 rows of d][XA atoms] resident
+//       (K-major B of dh); the bf16 dh tile [128 tokens][2 atoms] staged for its TMA store.
+// TMEM: dh [128][128] at column 0, the dP block [128 rows of d][R] at column 128.
 // =====================================================================================
 struct GenBwdArgs {
     int64_t N, d;
@@ -565,40 +566,43 @@ struct GenBwdArgs {
     int64_t hs;
     int n_dblk, n_split;
     int64_t n_tiles;
-    __nv_bfloat16* dh;        // nullable
+    int want_dh;
     float* dP_part;           // [n_split][d][R]
     uint32_t* err;
 };
 
 template <int XA>
 struct GbCfg {
-    static constexpr int DB = XA == 1 ? 256 : 128;          // d columns per CTA
-    static constexpr int HA = DB / 64;                      // h atoms per stage
-    static constexpr uint32_t stage = (XA + HA) * kAtom128;
-    static constexpr uint32_t pblk = 2 * stage;
-    static constexpr uint32_t smem = pblk + DB * 128 * XA + 1024;
-    static constexpr uint32_t col_dp = DB;                  // TMEM column of the first dP block
-    static constexpr uint32_t dp_stride = XA == 1 ? 64 : 128;
+    static constexpr int DB = 128;                          // d columns per CTA
+    static constexpr int NS = XA == 1 ? 3 : 2;
+    static constexpr uint32_t stage = (XA + 2) * kAtom128;
+    static constexpr uint32_t pblk = NS * stage;
+    static constexpr uint32_t dhst = pblk + DB * 128 * XA;
+    static constexpr uint32_t smem = dhst + 2 * kAtom128 + 1024;
+    static constexpr uint32_t col_dp = DB;                  // TMEM column of the dP block
 };
 
 template <int XA>
 __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_h,
                                                               const __grid_constant__ CUtensorMap tm_p,
+                                                              const __grid_constant__ CUtensorMap tm_dh,
                                                               GenBwdArgs a) {
     using G = GbCfg<XA>;
+    constexpr int NS = G::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint8_t* pblk = sm + G::pblk;
-    __shared__ uint64_t full[2], empty[2], pfull, hfull, hempty, dpfull;
+    uint8_t* dhs = sm + G::dhst;
+    __shared__ uint64_t full[NS], empty[NS], pfull, hfull, hempty, dpfull;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int db = blockIdx.x % a.n_dblk, split = blockIdx.x / a.n_dblk;
     const int64_t t0 = (a.n_tiles * split) / a.n_split, t1 = (a.n_tiles * (split + 1)) / a.n_split;
-    const bool want_dh = a.dh != nullptr;
+    const bool want_dh = a.want_dh != 0;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -611,9 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
         tma_prefetch(&tm_x);
         tma_prefetch(&tm_h);
         tma_prefetch(&tm_p);
+        if (want_dh) tma_prefetch(&tm_dh);
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_base, 512);
+        tmem_alloc(&tmem_base, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -629,12 +634,12 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
             for (int xa = 0; xa < XA; ++xa) tma_load_2d(pblk + xa * G::DB * 128, &tm_p, &pfull, 64 * xa, db * G::DB);
             uint32_t it = 0;
             for (int64_t tile = t0; tile < t1 && !abort_flag; ++tile, ++it) {
-                const int s = it & 1;
-                if (!mbar_wait(&empty[s], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+                const int s = it % NS;
+                if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* st = sm + s * G::stage;
                 mbar_arrive_expect_tx(&full[s], G::stage);
                 for (int xa = 0; xa < XA; ++xa) tma_load_2d(st + xa * kAtom128, &tm_x, &full[s], 64 * xa, (int32_t)(tile * 128));
-                for (int at = 0; at < G::HA; ++at)
+                for (int at = 0; at < 2; ++at)
                     tma_load_2d(st + kAtom128 * (XA + at), &tm_h, &full[s], db * G::DB + 64 * at, (int32_t)(tile * 128));
             }
         }
@@ -646,8 +651,8 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
             bool ok = mbar_wait(&pfull, 0, &abort_flag, a.err);
             uint32_t it = 0;
             for (int64_t tile = t0; ok && tile < t1 && !abort_flag; ++tile, ++it) {
-                const int s = it & 1;
-                if (!mbar_wait(&full[s], (it >> 1) & 1, &abort_flag, a.err)) break;
+                const int s = it % NS;
+                if (!mbar_wait(&full[s], (it / NS) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
                 const uint32_t x0 = smem_u32(sm + s * G::stage), h0 = x0 + XA * kAtom128;
                 if (want_dh) {
@@ -658,69 +663,72 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                                   kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3), idesc_dh, k != 0);
                     umma_commit(&hfull);
                 }
-                for (int b = 0; b < G::DB / 128; ++b)
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tbase + G::col_dp + G::dp_stride * b,
-                                  mnmajor_desc(h0 + 2 * b * kAtom128, kAtom128, 16 * ks),
-                                  mnmajor_desc(x0, kAtom128, 16 * ks), idesc_dp, !(tile == t0 && ks == 0));
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16(tbase + G::col_dp, mnmajor_desc(h0, kAtom128, 16 * ks), mnmajor_desc(x0, kAtom128, 16 * ks),
+                              idesc_dp, !(tile == t0 && ks == 0));
                 umma_commit(&empty[s]);
             }
             umma_commit(&dpfull);     // every dP MMA of this CTA has completed
         }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;      // dh columns half*DB/2 ..; dP columns 8*half + 16 i
+        const int half = (warp - 2) >> 2;      // dh columns 64 half ..; dP columns 8 half + 16 i
         const int row = q * 32 + lane;
+        const bool leader = warp == 2 && lane == 0;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint32_t it = 0;
         bool ok = true;
         if (want_dh) {
             for (int64_t tile = t0; tile < t1; ++tile, ++it) {
                 ok = mbar_wait(&hfull, it & 1, &abort_flag, a.err);
+                if (leader) tma_store_wait_read_all();     // the previous dh store has read the staging tile
                 if (epi_bar_any<kEpiThreads>(!ok)) break;
                 tc_fence_after();
-                const int64_t n = tile * 128 + row;
+                // columns 64 half .. 64 half + 63 of the block = staging atom `half`
 #pragma unroll 1
-                for (int c = (G::DB / 2) * half; c < (G::DB / 2) * (half + 1); c += 32) {
+                for (int c = 0; c < 64; c += 32) {
                     uint32_t v[4][8];
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) tmem_ld8(lane_base + c + 8 * x, v[x]);
+                    for (int x = 0; x < 4; ++x) tmem_ld8(lane_base + 64 * half + c + 8 * x, v[x]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const int64_t col = (int64_t)db * G::DB + c + 8 * x;
-                        if (n < a.N && col < a.d) {
-                            uint4 pk;
-                            pk.x = pack_bf16(__uint_as_float(v[x][0]), __uint_as_float(v[x][1]));
-                            pk.y = pack_bf16(__uint_as_float(v[x][2]), __uint_as_float(v[x][3]));
-                            pk.z = pack_bf16(__uint_as_float(v[x][4]), __uint_as_float(v[x][5]));
-                            pk.w = pack_bf16(__uint_as_float(v[x][6]), __uint_as_float(v[x][7]));
-                            *reinterpret_cast<uint4*>(a.dh + n * a.d + col) = pk;
-                        }
+                        uint4 pk;
+                        pk.x = pack_bf16(__uint_as_float(v[x][0]), __uint_as_float(v[x][1]));
+                        pk.y = pack_bf16(__uint_as_float(v[x][2]), __uint_as_float(v[x][3]));
+                        pk.z = pack_bf16(__uint_as_float(v[x][4]), __uint_as_float(v[x][5]));
+                        pk.w = pack_bf16(__uint_as_float(v[x][6]), __uint_as_float(v[x][7]));
+                        *reinterpret_cast<uint4*>(dhs + half * kAtom128 + sw128_off(row, (c >> 3) + x)) = pk;
                     }
                 }
                 tc_fence_before();
+                fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&hempty);
+                epi_bar_any<kEpiThreads>(false);          // every epilogue warp has staged its rows
+                if (leader) {
+                    for (int at = 0; at < 2; ++at)
+                        tma_store_2d(&tm_dh, dhs + at * kAtom128, db * G::DB + 64 * at, (int32_t)(tile * 128));
+                    tma_store_commit();
+                }
             }
+            if (leader) tma_store_wait_all();
         }
         if (ok && t1 > t0) ok = mbar_wait(&dpfull, 0, &abort_flag, a.err);
         if (!epi_bar_any<kEpiThreads>(!ok) && t1 > t0) {
             tc_fence_after();
             float* part = a.dP_part + (int64_t)split * a.d * a.R;
-            for (int b = 0; b < G::DB / 128; ++b) {
-                const int64_t drow = (int64_t)db * G::DB + b * 128 + row;
-                for (int c = 8 * half; c < a.R; c += 16) {
-                    uint32_t v[8];
-                    tmem_ld8(lane_base + G::col_dp + G::dp_stride * b + c, v);
-                    tmem_wait_ld();
-                    if (drow < a.d) {
-                        float4* dst = reinterpret_cast<float4*>(part + drow * a.R + c);
-                        dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
-                                             __uint_as_float(v[3]));
-                        dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
-                                             __uint_as_float(v[7]));
-                    }
+            const int64_t drow = (int64_t)db * G::DB + row;
+            for (int c = 8 * half; c < a.R; c += 16) {
+                uint32_t v[8];
+                tmem_ld8(lane_base + G::col_dp + c, v);
+                tmem_wait_ld();
+                if (drow < a.d) {
+                    float4* dst = reinterpret_cast<float4*>(part + drow * a.R + c);
+                    dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                         __uint_as_float(v[3]));
+                    dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                         __uint_as_float(v[7]));
                 }
             }
         }
@@ -729,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, 512);
+        tmem_dealloc(tbase, 256);
     }
 }
 
@@ -757,7 +765,7 @@ cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUten
 // Generator backward on the tensor cores: dP = h^T X (fp32, overwritten) and, when dh is
 // non-null, dh = X P^T (bf16), for X [N, R] bf16 (R <= 128, multiple of 8), P [d, R] bf16.
 // dP_part must hold n_split * d * R floats (gen_bwd_splits()).
-int gen_bwd_dblk(int64_t d, int R) { return (int)((d + (R <= 64 ? 256 : 128) - 1) / (R <= 64 ? 256 : 128)); }
+int gen_bwd_dblk(int64_t d, int R) { return (int)((d + 127) / 128); }
 int gen_bwd_splits(int64_t N, int64_t d, int R) {
     const int64_t n_tiles = (N + 127) / 128;
     return (int)std::max<int64_t>(1, std::min<int64_t>(148 / std::max(1, gen_bwd_dblk(d, R)), n_tiles));
@@ -767,23 +775,25 @@ cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, con
                             void* dh, float* dP, float* dP_part, uint32_t* err, cudaStream_t st) {
     const int n_dblk = gen_bwd_dblk(d, R), n_split = gen_bwd_splits(N, d, R);
     const int XA = R <= 64 ? 1 : 2;
-    const int DB = XA == 1 ? 256 : 128;
-    CUtensorMap tx, th, tp;
+    CUtensorMap tx, th, tp, tdh;
+    std::memset(&tdh, 0, sizeof(tdh));                 // unused when dh is not requested
     if (!make_tmap_bf16(&tx, X, R, N, R, 64, 128) || !make_tmap_bf16(&th, h, d, N, hs, 64, 128) ||
-        !make_tmap_bf16(&tp, P, R, d, R, 64, DB))
+        !make_tmap_bf16(&tp, P, R, d, R, 64, 128) || (dh && !make_tmap_bf16(&tdh, dh, d, N, d, 64, 128)))
         return cudaErrorInvalidValue;
-    GenBwdArgs ga{N, d, R, (R + 15) / 16 * 16, (R + 15) / 16, hs, n_dblk, n_split, (N + 127) / 128,
-                  static_cast<__nv_bfloat16*>(dh), dP_part, err};
+    GenBwdArgs ga{N, d, R, (R + 15) / 16 * 16, (R + 15) / 16, hs, n_dblk, n_split, (N + 127) / 128, dh ? 1 : 0,
+                  dP_part, err};
     cudaError_t e;
     const dim3 grid(n_dblk * n_split);
     if (XA == 1) {
         e = cudaFuncSetAttribute(gen_bwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, GbCfg<1>::smem);
         if (e != cudaSuccess) return e;
-        DC_LAUNCH(kTcGenBwd, st, e = launch_pdl(gen_bwd_kernel<1>, grid, dim3(kThreads), GbCfg<1>::smem, st, tx, th, tp, ga));
+        DC_LAUNCH(kTcGenBwd, st, e = launch_pdl(gen_bwd_kernel<1>, grid, dim3(kThreads), GbCfg<1>::smem, st, tx, th, tp,
+                                                tdh, ga));
     } else {
         e = cudaFuncSetAttribute(gen_bwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, GbCfg<2>::smem);
         if (e != cudaSuccess) return e;
-        DC_LAUNCH(kTcGenBwd, st, e = launch_pdl(gen_bwd_kernel<2>, grid, dim3(kThreads), GbCfg<2>::smem, st, tx, th, tp, ga));
+        DC_LAUNCH(kTcGenBwd, st, e = launch_pdl(gen_bwd_kernel<2>, grid, dim3(kThreads), GbCfg<2>::smem, st, tx, th, tp,
+                                                tdh, ga));
     }
     if (e != cudaSuccess) return e;
     DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_splits_kernel, dim3(grid_for(d * R / 4 * 32)), dim3(256), 0, st,
