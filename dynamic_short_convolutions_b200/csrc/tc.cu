@@ -11,8 +11,8 @@
 //                      the [N, C, K] filter lives only in TMEM and registers.
 //
 // Every kernel here is warp-specialised: warp 0 issues TMA loads, warp 1 issues
-// tcgen05.mma (one elected thread) and owns the tensor memory, warps 2-5 are the
-// epilogue (thread = token row = TMEM lane).  Shared-memory stages and TMEM
+// tcgen05.mma (one elected thread) and owns the tensor memory, the remaining warps
+// are the epilogue (thread = token row = TMEM lane).  Shared-memory stages and TMEM
 // accumulators are handed over with mbarriers; every wait is bounded.
 #include <algorithm>
 #include <cstdio>
@@ -205,8 +205,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 //               the generator launch) as K atoms [64 r-rows][64] (MN-major B), reloaded when the
 //               chunk changes
 //   TMEM: W[128 tokens][64 K] fp32, column 64 j + c = w[m0 + row, c0 + c, j]; two buffers.
-//   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3..10 epilogue (a TMEM lane quarter and half of
-//   the channels each): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
+//   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3.. epilogue (FwdEpi<K>::warps; each a TMEM lane
+//   quarter and a share of the channels): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
 //   -> bf16 staging (128-byte swizzled) -> TMA store by warp 2.
 // =====================================================================================
 struct FwdArgs {
@@ -220,7 +220,15 @@ struct FwdArgs {
 constexpr int kFwdStages = 4;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
 constexpr uint32_t kFwdStage = kZBytes + kUBytes;
-constexpr int kFwdThreads = 96 + kEpiThreads;      // producer, MMA, store warps + epilogue
+// Epilogue warps of lowrank_fwd_kernel<K>: 16 (two 8-channel groups each) for K <= 3, where the
+// extra warps hide more latency; 8 (four groups each) for K = 4, whose larger per-group state
+// would not fit the registers of 16 warps.
+template <int K>
+struct FwdEpi {
+    static constexpr int warps = K <= 3 ? 16 : 8;
+    static constexpr int groups = 32 / warps;        // 8-channel groups per warp
+    static constexpr int threads = 96 + 32 * warps;  // producer, MMA, store warps + epilogue
+};
 
 template <int K>
 struct FwdSmem {
@@ -259,13 +267,14 @@ __device__ __forceinline__ uint4 conv8(const uint32_t (*wv)[8], const uint4* uj,
 }
 
 template <int K>
-__global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+__global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                      const __grid_constant__ CUtensorMap tm_b,
                                                                      const __grid_constant__ CUtensorMap tm_u,
                                                                      const __grid_constant__ CUtensorMap tm_y,
                                                                      FwdArgs a) {
     using S = FwdSmem<K>;
     constexpr int NMMA = 64 * K;
+    constexpr int kFwdEpiWarps = FwdEpi<K>::warps, kFwdGroups = FwdEpi<K>::groups;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ uint64_t full[kFwdStages], empty[kFwdStages], bfull, bempty, tfull[2], tempty[2], yfull[2], yempty[2];
@@ -277,14 +286,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFwdStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kEpiWarps);
+            mbar_init(&empty[s], 1 + kFwdEpiWarps);
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
-            mbar_init(&yfull[b], kEpiWarps);
+            mbar_init(&tempty[b], kFwdEpiWarps);
+            mbar_init(&yfull[b], kFwdEpiWarps);
             mbar_init(&yempty[b], 1);
         }
         abort_flag = 0;
@@ -370,16 +379,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
         }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 3) >> 2;      // channel groups 4*half .. 4*half+3
+        const int half = (warp - 3) >> 2;      // channel groups kFwdGroups*half ..
         const int row = q * 32 + lane;
         uint32_t it = 0;
         for (int64_t item = i0; item < i1; ++item, ++it) {
             const int64_t tile = item % n_tiles;
             const int s = it % kFwdStages, b = it & 1;
+            // each warp goes at its own pace (no barrier among the epilogue warps): a failed
+            // wait sets the abort flag, and every other wait then gives up too
             const bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, &abort_flag, a.err) &&
                             mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err) &&
                             mbar_wait(&yempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err);
-            if (epi_bar_any<kEpiThreads>(!ok)) break;
+            if (!ok) break;
             tc_fence_after();
             const int32_t n = (int32_t)(tile * 128) + row;
             const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
@@ -388,10 +399,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) lowrank_fwd_kernel(const __gri
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
             // NG 8-channel groups per pass (all four of this warp's groups when the registers
             // allow): every TMEM and shared-memory load first, then one wait, then the arithmetic
-            constexpr int NG = K <= 3 ? 4 : 2;
+            constexpr int NG = kFwdGroups < 4 ? kFwdGroups : (K <= 3 ? 4 : 2);
 #pragma unroll
-            for (int pass = 0; pass < 4 / NG; ++pass) {
-                const int g0 = 4 * half + NG * pass;
+            for (int pass = 0; pass < kFwdGroups / NG; ++pass) {
+                const int g0 = kFwdGroups * half + NG * pass;
                 uint32_t wv[NG][K][8];
 #pragma unroll
                 for (int x = 0; x < NG; ++x)
@@ -434,7 +445,8 @@ cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, con
     if (e != cudaSuccess) return e;
     fa.per_cta = (items + num_sms() - 1) / num_sms();
     const unsigned grid = (unsigned)((items + fa.per_cta - 1) / fa.per_cta);
-    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K>, dim3(grid), dim3(kFwdThreads), smem, st, tz, tb, tu, ty, fa));
+    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K>, dim3(grid), dim3(FwdEpi<K>::threads), smem, st, tz,
+                                                tb, tu, ty, fa));
     return e;
 }
 

@@ -109,17 +109,25 @@ struct BwdSmem {
     static constexpr uint32_t total = dzst + dzst_bytes + 1024;
 };
 
-// Warp roles of lowrank_bwd_kernel: 0 TMA loads, 1 MMA issue (and TMEM owner), 2..9 the du / dw
-// epilogue (GA: a TMEM lane quarter and half of the channels each), 10..13 the dz / dB readout
-// (GB: one TMEM lane quarter each).
-constexpr int kGaWarps = 8, kGbWarps = 4, kGa0 = 2, kGb0 = kGa0 + kGaWarps;
-constexpr int kBwdPipeThreads = 32 * (kGb0 + kGbWarps);
+// Warp roles of lowrank_bwd_kernel<K>: 0 TMA loads, 1 MMA issue (and TMEM owner), then the
+// du / dw epilogue (GA: BwdEpi<K>::ga warps, each a TMEM lane quarter and a share of the
+// channels), then 4 warps of dz / dB readout (GB: one TMEM lane quarter each).  GA has 8 warps
+// for K <= 3 and 16 for K = 4, where the per-item epilogue work is largest (measured).
+template <int K>
+struct BwdEpi {
+    static constexpr int ga = K <= 3 ? 8 : 16;
+    static constexpr int groups = 32 / ga;             // 8-channel groups per GA warp
+    static constexpr int per_wait = ga <= 8 ? 2 : 1;   // groups per TMEM wait in A1
+    static constexpr int gb0 = 2 + ga;
+    static constexpr int threads = 32 * (gb0 + 4);
+};
+constexpr int kGbWarps = 4, kGa0 = 2;
 
 // TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
 constexpr uint32_t kColDz = 256, kColDb = 384;
 
 template <int K, bool R64>
-__global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
+__global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                          const __grid_constant__ CUtensorMap tm_g,
                                                                          const __grid_constant__ CUtensorMap tm_u,
                                                                          const __grid_constant__ CUtensorMap tm_bp,
@@ -128,6 +136,8 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                                                                          BwdArgs a) {
     using S = BwdSmem<K, R64>;
     constexpr int NBLK = (K + 1) / 2;
+    constexpr int kGaWarps = BwdEpi<K>::ga, kGaGroups = BwdEpi<K>::groups, kGaPerWait = BwdEpi<K>::per_wait;
+    constexpr int kGb0 = BwdEpi<K>::gb0;
     constexpr int NZ = S::NZ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
     } else if (warp < kGb0) {
         // ---- GA: du (A1, staged for a TMA store) and dw (A2) of each item
         const int q = warp & 3;
-        const int half = (warp - kGa0) >> 2;   // channel groups 4*half .. 4*half+3
+        const int half = (warp - kGa0) >> 2;   // channel groups kGaGroups*half ..
         const int row = q * 32 + lane;
         const bool leader = warp == kGa0 && lane == 0;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
@@ -314,25 +324,25 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
             const uint8_t* ut = gt + kRowTile;
             // A1: du[t, c] = g[t, c] + sum_{j <= epos} Wd_j[t, c] g[t + j, c], two 8-channel
             // groups per TMEM wait, channel pairs on the packed fp32 FMA; g[t] is kept for A2
-            uint4 gv[4];
+            uint4 gv[kGaGroups];
 #pragma unroll
-            for (int gp = 0; gp < 2; ++gp) {
-                const int g0 = 4 * half + 2 * gp;
-                uint32_t wv[2][K][8];
+            for (int gp = 0; gp < kGaGroups / kGaPerWait; ++gp) {
+                const int g0 = kGaGroups * half + kGaPerWait * gp;
+                uint32_t wv[kGaPerWait][K][8];
 #pragma unroll
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < kGaPerWait; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j) tmem_ld8(lane_base + 64 * j + 8 * (g0 + x), wv[x][j]);
-                uint4 gg[2][K];
+                uint4 gg[kGaPerWait][K];
 #pragma unroll
-                for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < kGaPerWait; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j)
                         gg[x][j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    gv[2 * gp + x] = gg[x][0];
+                for (int x = 0; x < kGaPerWait; ++x) {
+                    gv[kGaPerWait * gp + x] = gg[x][0];
                     float acc[8];
                     const uint32_t* g0w = reinterpret_cast<const uint32_t*>(&gg[x][0]);
 #pragma unroll
@@ -374,8 +384,8 @@ __global__ void __launch_bounds__(kBwdPipeThreads, 1) lowrank_bwd_kernel(const _
                     tma_store_commit();
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int g8 = 4 * half + i;
+                for (int i = 0; i < kGaGroups; ++i) {
+                    const int g8 = kGaGroups * half + i;
 #pragma unroll
                     for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j) {
                         const uint4 uu = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
@@ -755,7 +765,7 @@ cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUten
     cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K, R64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::total);
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64>, dim3(grid), dim3(kBwdPipeThreads), S::total,
+    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64>, dim3(grid), dim3(BwdEpi<K>::threads), S::total,
                                                 st, tz, tg, tu, tbp, tdu, tdz, ba));
     return e;
 }
