@@ -80,7 +80,7 @@ struct BwdArgs {
     int64_t n_tiles, n_items, per_cta;
     int pieces;               // partial slots per chunk
     float* dz_acc;            // [N, r] fp32, zero on entry
-    float* dB_part;           // [n_chunks][pieces][64 K][r]
+    float* dB_part;           // [n_chunks][pieces][r][64 K]
     uint32_t* err;
     int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
     int dz_tma;               // 1: dz tiles are added with bulk tensor reductions, else fp32 atomics
@@ -471,8 +471,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 }
             }
             if (last) {                            // the run for this chunk ends: its dB partial
+                // partial [k][m] (m = j * 64 + c): a warp writes 32 consecutive m per k
                 const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
-                float* part = a.dB_part + ((chunk * a.pieces + piece) * (64 * K)) * a.r;
+                float* part = a.dB_part + ((chunk * a.pieces + piece) * a.r) * (64 * K);
 #pragma unroll
                 for (int bb = 0; bb < NBLK; ++bb) {
                     const int mrow = bb * 128 + row;     // (tap, channel) row = j * 64 + c
@@ -481,11 +482,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                         tmem_ld8(lane_base + kColDb + 64 * bb + c, v);
                         tmem_wait_ld();
                         if (mrow < 64 * K) {
-                            float4* dst = reinterpret_cast<float4*>(part + (int64_t)mrow * a.r + c);
-                            dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
-                                                 __uint_as_float(v[3]));
-                            dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
-                                                 __uint_as_float(v[7]));
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                part[(int64_t)(c + i) * (64 * K) + mrow] = __uint_as_float(v[i]);
                         }
                     }
                 }
@@ -517,15 +516,16 @@ __global__ void bwd_finish_kernel(const float* __restrict__ part, float* __restr
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nb + count4;
          e += (int64_t)gridDim.x * blockDim.x) {
         if (e < nb) {
+            // e runs over (k, chunk, m = j * 64 + c) so that the partial reads are coalesced
             const int ei = (int)e;
-            const int k = ei / (C * K), col = ei - k * (C * K), c = col / K, j = col - c * K;
-            const int chunk = c >> 6, m = j * 64 + (c & 63);
+            const int k = ei / (C * K), rem = ei - k * (C * K), chunk = rem / (64 * K), m = rem - chunk * (64 * K);
+            const int j = m >> 6, c = chunk * 64 + (m & 63);
             const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
             const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
-            const float* src = part + ((int64_t)chunk * pieces * (64 * K) + m) * r + k;
+            const float* src = part + ((int64_t)chunk * pieces * r + k) * (64 * K) + m;
             float acc = 0.f;
-            for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * (64 * K) * r];
-            dB[e] = acc;
+            for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * r * (64 * K)];
+            dB[(int64_t)k * (C * K) + c * K + j] = acc;
         } else {
             const int64_t i4 = e - nb;
             const float4 v = dz4[i4];
