@@ -235,6 +235,162 @@ def oracle_sample_rate(w, budget_s: float):
     return smp.tokens / secs, f"{seqs} sequence(s) x {T} tokens", secs
 
 
+# ----------------------------------------------------------------------------- decode mode
+DECODE_METRIC = "dyn-conv decode-step tokens/s at 1 B200 (one new token per sequence, rolling K-1 state)"
+
+
+def decode_bytes(w, layer, batch):
+    """Algorithmic HBM bytes of one decode step of one layer call: u, h read, y written,
+    the state read and rewritten, the generator parameters read once."""
+    s = 2 if w.dtype == "bf16" else 4
+    d, C, K = layer.d_model, layer.channels, w.ksize
+    per_seq = s * (2 * C + d + 2 * (K - 1) * C)
+    if w.kind == "lowrank":
+        params = s * (d * w.rank + w.rank * C * K)
+    else:
+        params = s * d * (C // w.head_dim) * K
+    return batch * per_seq + params
+
+
+def run_decode(args, rank, world, local_rank):
+    """Decode steps of every layer of the workload for a batch of sequences: one call of
+    dynconv_decode_step per layer per step, L2 flushed between timed steps."""
+    import numpy as np
+    import torch
+
+    from dynamic_short_convolutions_b200 import _lib as L, workloads as W
+
+    L.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.CONFIGS[args.config]
+    Bd = args.decode_batch
+    dt = W.storage_dtype(w)
+    kind = L.LOWRANK if w.kind == W.LOWRANK else L.HEADWISE
+    seed = w.seed + 7919 * rank
+    calls = []
+    for li, layer in enumerate(w.layers):
+        d, C, K = layer.d_model, layer.channels, w.ksize
+        rnd = lambda tag, n, std=1.0: W.normal_torch(seed, f"dec{li}{tag}", n, std, device=dev).to(dt)
+        if kind == L.LOWRANK:
+            A = rnd("A", d * w.rank, 1 / np.sqrt(d)).view(d, w.rank)
+            BW = rnd("B", w.rank * C * K, 1 / np.sqrt(w.rank)).view(w.rank, C * K)
+        else:
+            A = None
+            BW = rnd("W", d * (C // w.head_dim) * K, 1 / np.sqrt(d)).view(d, (C // w.head_dim) * K)
+        u, h = rnd("u", Bd * C).view(Bd, C), rnd("h", Bd * d).view(Bd, d)
+        desc = L.make_desc(kind, L.BF16 if dt == torch.bfloat16 else L.F32, Bd, 1, d, C, K, w.rank, w.head_dim)
+        ws = torch.zeros(L.dynconv_workspace_bytes(desc), dtype=torch.uint8, device=dev)
+        state = torch.zeros((Bd, K - 1, C), dtype=dt, device=dev) if K > 1 else None
+        y = torch.empty((Bd, C), dtype=dt, device=dev)
+        calls.append((layer, desc, u, h, A, BW, state, y, ws))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for layer, desc, u, h, A, BW, state, y, ws in calls:
+            L.dynconv_decode_step(desc, u, h, A, BW, state, y, ws)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for *_, ws in calls:
+        assert L.dynconv_device_status(ws) == 0, L.dynconv_last_error()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    total_ms = float(sum(a.elapsed_time(b) for a, b in ev))
+    L.dynconv_profile_read(reset=True)
+    L.dynconv_profile_enable(True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    L.dynconv_profile_enable(False)
+    prof = L.dynconv_profile_read(reset=True)
+    # end to end: the step's inputs copied in from pinned host memory, outputs copied back
+    host = [(u.cpu().pin_memory(), h.cpu().pin_memory(), torch.empty_like(y, device="cpu").pin_memory())
+            for _, _, u, h, _, _, _, y, _ in calls]
+    h2d = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b, _ in host)
+    d2h = sum(c.numel() * c.element_size() for _, _, c in host)
+
+    def e2e_step():
+        for (layer, desc, u, h, A, BW, state, y, ws), (hu, hh, hy) in zip(calls, host):
+            u.copy_(hu, non_blocking=True)
+            h.copy_(hh, non_blocking=True)
+            L.dynconv_decode_step(desc, u, h, A, BW, state, y, ws)
+            hy.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    pk, pk_src = peaks()
+    ms_step = total_ms / args.steps
+    step_bytes = sum(decode_bytes(w, c[0], Bd) for c in calls)
+    achieved = step_bytes / (ms_step / 1e3) / 1e9
+    kernels = {n: {"launches": nl, "ms_total": round(ms, 4), "us_per_launch": round(1e3 * ms / nl, 2)}
+               for n, (nl, ms) in prof.items()}
+    line = {"metric": DECODE_METRIC, "mode": "decode", "value": round(Bd * args.steps / (total_ms / 1e3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "decode_batch": Bd, "ksize": w.ksize, "rank": w.rank,
+                       "head_dim": w.head_dim, "layers": [[l.name, l.d_model, l.channels] for l in w.layers],
+                       "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None, "peak_source": pk_src,
+                         "algorithmic_bytes_per_step": int(step_bytes)},
+            "kernels": kernels,
+            "e2e": {"value": round(Bd * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": int(sum(v[0] for v in prof.values())), "clocks": clk.summary()}
+    return line
+
+
+def oracle_decode_rate(w, batch, budget_s):
+    """tokens/s of the fp64 oracle's decode step on the workload's layers (batch sequences)."""
+    import numpy as np
+
+    from dynamic_short_convolutions_b200 import workloads as W
+    from oracle import oracle as O
+
+    O.build()
+    calls = []
+    for li, layer in enumerate(w.layers):
+        d, C, K = layer.d_model, layer.channels, w.ksize
+        rnd = lambda tag, n, std=1.0: W.round_to_storage(W.normal(w.seed, f"odec{li}{tag}", n, std), w.dtype)
+        if w.kind == W.LOWRANK:
+            A, BW = rnd("A", d * w.rank).reshape(d, w.rank), rnd("B", w.rank * C * K).reshape(w.rank, C * K)
+        else:
+            A, BW = None, rnd("W", d * (C // w.head_dim) * K).reshape(d, (C // w.head_dim) * K)
+        p = O.Problem(O.LOWRANK if w.kind == W.LOWRANK else O.HEADWISE, batch, d, C, K, [0, batch], rank=w.rank,
+                      head_dim=w.head_dim)
+        calls.append((p, rnd("u", batch * C).reshape(batch, C), rnd("h", batch * d).reshape(batch, d), A, BW,
+                      np.zeros((batch, K - 1, C))))
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        for i, (p, u, h, A, BW, st) in enumerate(calls):
+            _, st = O.decode_step(p, u, h, A, BW, st)
+            calls[i] = (p, u, h, A, BW, st)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    secs = time.perf_counter() - t0
+    return batch * steps / secs, f"{steps} decode step(s) of {batch} sequences, every layer", secs
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -414,6 +570,9 @@ def main():
     ap.add_argument("--algo", type=int, default=0, help="0 auto, 1 CUDA-core kernels, 2 tensor-core kernels")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="train", choices=["train", "decode"],
+                    help="train: forward + backward step (default); decode: one decode step per layer")
+    ap.add_argument("--decode-batch", type=int, default=64, help="sequences per decode step")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -421,6 +580,23 @@ def main():
     from dynamic_short_convolutions_b200 import workloads as W
 
     w = W.CONFIGS[args.config]
+    if args.impl == "reference" and args.mode == "decode":
+        if rank != 0:
+            return 0
+        # the reference arm of the decode mode: the oracle's decode step as it stands
+        rates = [oracle_decode_rate(w, args.decode_batch, 1.0) for _ in range(args.warmup + args.steps)]
+        rates = rates[args.warmup:]
+        value = sum(r for r, _, _ in rates) / len(rates)
+        line = {"metric": DECODE_METRIC, "mode": "decode", "value": round(value, 2), "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * args.decode_batch / value, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": w.name, "decode_batch": args.decode_batch},
+                "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+                                 "sample": rates[0][1]},
+                "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     if args.impl == "reference":
         if rank != 0:
             return 0
@@ -454,10 +630,17 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_decode if args.mode == "decode" else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
+    if rank == 0 and args.mode == "decode":
+        if world == 1 and not args.no_cpu_baseline:
+            rate, desc, secs = oracle_decode_rate(w, args.decode_batch, min(args.cpu_budget, 5.0))
+            line["cpu_baseline"] = {"value": round(rate, 2), "unit": "tokens/s", "cores": cores_used(),
+                                    "kind": "oracle", "sample": f"fp64 oracle: {desc} ({secs:.1f} s)"}
+        print(json.dumps(line), flush=True)
+        return 0
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             rate, desc, secs = oracle_sample_rate(w, args.cpu_budget)

@@ -27,7 +27,8 @@ ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 # Every entry point the header declares (checked against the library's exports by the tests).
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
-           "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc")
+           "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc",
+           "dynconv_decode_step")
 
 
 class DynConvError(RuntimeError):
@@ -71,7 +72,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_device_status.argtypes = [vp, sz, vp]
     lib.dynconv_fwd_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp]
     lib.dynconv_fwd_noalloc.restype = ctypes.c_int
-    for f in (lib.dynconv_fwd, lib.dynconv_fwd_varlen, lib.dynconv_bwd, lib.dynconv_device_status):
+    lib.dynconv_decode_step.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    for f in (lib.dynconv_fwd, lib.dynconv_fwd_varlen, lib.dynconv_bwd, lib.dynconv_device_status,
+              lib.dynconv_decode_step):
         f.restype = ctypes.c_int
     lib.dynconv_last_error.restype = ctypes.c_char_p
     lib.dynconv_status_string.argtypes = [ctypes.c_int]
@@ -138,6 +141,11 @@ def dynconv_fwd_noalloc(desc, u, h, A, B, y, z_save=None, stream=None):
     """Forward with no workspace argument (scratch built into the library); see include/dynconv.h."""
     _check(load().dynconv_fwd_noalloc(ctypes.byref(desc), _ptr(u), _ptr(h), _ptr(A), _ptr(B), _ptr(y), _ptr(z_save),
                                       _stream(stream, u)))
+
+
+def dynconv_decode_step(desc, u, h, A, B_or_W, state, y, ws, stream=None):
+    _check(load().dynconv_decode_step(ctypes.byref(desc), _ptr(u), _ptr(h), _ptr(A), _ptr(B_or_W), _ptr(state),
+                                      _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream, u)))
 
 
 def dynconv_device_status(ws, stream=None) -> int:

@@ -154,6 +154,8 @@ WsLayout ws_layout(const Prob& p) {
     L.tc = off;
     L.tc_bytes = tc_supported(p) ? tc_workspace_bytes(p) : 0;
     off = align_up(off + L.tc_bytes, 256);
+    L.dec = off;
+    if (p.seqlen == 1) off = align_up(off + decode_partial_bytes(p), 256);
     L.total = off;
     return L;
 }
@@ -223,6 +225,27 @@ dynconv_status dynconv_bwd(const dynconv_desc* desc, const int32_t* cu_seqlens, 
                         ? tc_backward(p, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or_dW, ws, st)
                         : simt_backward(p, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or_dW, ws, st);
     return cuda_status(e, "backward launch");
+}
+
+dynconv_status dynconv_decode_step(const dynconv_desc* desc, const void* u, const void* h, const void* A,
+                                   const void* B_or_W, void* state, void* y, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    g_err[0] = 0;
+    Prob p;
+    dynconv_status s = make_prob(desc, &p);
+    if (s != DYNCONV_OK) return s;
+    if (p.seqlen != 1) {
+        set_error("dynconv_decode_step takes one new token per sequence: seqlen must be 1");
+        return DYNCONV_ERR_INVALID;
+    }
+    if (p.N == 0) return DYNCONV_OK;
+    if ((s = check_ptr(u, "u", true)) || (s = check_ptr(h, "h", true)) || (s = check_ptr(A, "A", p.kind == 0)) ||
+        (s = check_ptr(B_or_W, p.kind == 0 ? "B" : "W", true)) || (s = check_ptr(state, "state", p.K > 1)) ||
+        (s = check_ptr(y, "y", true)))
+        return s;
+    if ((s = workspace_ok(p, ws, ws_bytes)) != DYNCONV_OK) return s;
+    return cuda_status(decode_step(p, u, h, A, B_or_W, state, y, ws, static_cast<cudaStream_t>(stream)),
+                       "decode launch");
 }
 
 dynconv_status dynconv_device_status(void* ws, size_t ws_bytes, void* stream) {

@@ -35,6 +35,7 @@ struct WsLayout {
     size_t dgen;        // fp32 [N, R]: dz or dwh
     size_t tc;          // start of the tensor-core path's private region
     size_t tc_bytes;
+    size_t dec;         // decode step (seqlen == 1): split-d partial generator rows
     size_t total;
 };
 
@@ -69,6 +70,11 @@ cudaError_t tc_backward(const Prob& p, const void* g, const void* u, const void*
                         const void* BW, const void* z_saved, void* du, void* dh, float* dA, float* dBW,
                         void* ws, cudaStream_t st);
 
+// Bytes of the decode step's partial generator rows (split-d), for ws_layout.
+size_t decode_partial_bytes(const Prob& p);
+// One decode step for p.batch sequences (p.seqlen == 1), CUDA-core kernels.
+cudaError_t decode_step(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* state,
+                        void* y, void* ws, cudaStream_t st);
 cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st);
 
 // Text for the thread-local error message.

@@ -158,6 +158,31 @@ DYNCONV_API dynconv_status dynconv_bwd(const dynconv_desc *desc, const int32_t *
 DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc *desc, const void *u, const void *h,
                                                const void *A, const void *B, void *y, void *z_save, void *stream);
 
+/* One decode step: the newest token of each of desc->batch sequences (desc->seqlen
+ * must be 1), with the K-1 previous conv inputs of every sequence carried in a
+ * rolling state.  The operation is the Mechanism formula of "Dynamic Short
+ * Convolutions Improve Transformers" (gist.science technical summary, "Dynamic
+ * Short Convolutions") at the last position, with the filter generated from h as
+ * in dynconv_fwd and the residual added once:
+ *   y[b,c] = u[b,c] + sum_{j<K} w[b,c,j] x_j[b,c],  x_0 = u[b,c], x_j = state[b,j-1,c]
+ * after which the state rolls by one token: state[b,j,c] <- x_j[b,c], j = 0..K-2.
+ * The pages leave inference unoptimised (atlas.scime.ai summary, "Limitations");
+ * this is the step a generation loop calls.  Feeding a sequence token by token
+ * from a zero state reproduces dynconv_fwd on that sequence.
+ *   u      [batch, C] (row stride desc->u_row_stride): the new token's conv input
+ *   h      [batch, d] (row stride desc->h_row_stride): its generator input
+ *   A, B_or_W: as for dynconv_fwd
+ *   state  [batch, K-1, C] in the storage dtype, read and rewritten in place;
+ *          zero it when a sequence starts (taps before the start read zero);
+ *          may be NULL when K = 1
+ *   y      [batch, C] output, dense
+ *   ws     workspace of dynconv_workspace_bytes(desc), zeroed once
+ * Always runs the CUDA-core kernels (fp32 accumulation) whatever desc->algo says.
+ * Errors: as dynconv_fwd, and DYNCONV_ERR_INVALID when seqlen != 1. */
+DYNCONV_API dynconv_status dynconv_decode_step(const dynconv_desc *desc, const void *u, const void *h,
+                                               const void *A, const void *B_or_W, void *state, void *y,
+                                               void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream` and reports device-side check failures raised by the
  * calls that used this workspace since the last query (then clears them):
  * DYNCONV_ERR_DEVICE_CHECK for a malformed cu_seqlens or a pipeline wait that

@@ -363,3 +363,44 @@ int orc_param_grad_entries(const orc_problem *p, const double *g, const double *
     free(st);
     return ORC_OK;
 }
+
+/*
+ * One decode step for a batch of sequences (the Mechanism formula at the newest
+ * token of each sequence; the K-1 previous conv inputs come from a rolling state):
+ *   y[b,c] = u[b,c] + sum_{j<K} w[b,c,j] x_j[b,c],   x_0 = u[b,c],  x_j = state[b, j-1, c]
+ * with w[b,:,:] the filter generated from h[b,:]; then state[b,j,c] <- x_j[b,c]
+ * for j = 0 .. K-2.  p->n_tokens is the batch (one token per sequence); the
+ * segment table is not used.  state is [batch, K-1, C], updated in place.
+ */
+int orc_decode_step(const orc_problem *p, const double *u, const double *h, const double *A, const double *BW,
+                    double *state, double *y)
+{
+    if (p->n_tokens < 0 || p->d_model < 1 || p->channels < 1 || p->ksize < 1) return ORC_BAD;
+    if (p->kind == 0 && p->rank < 1) return ORC_BAD;
+    if (p->kind == 1 && (p->head_dim < 1 || p->channels % p->head_dim != 0)) return ORC_BAD;
+    const int64_t C = p->channels, K = p->ksize;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t b = 0; b < p->n_tokens; ++b) {
+        double *w = (double *)malloc(sizeof(double) * (size_t)(C * K));
+        double *z = (double *)malloc(sizeof(double) * (size_t)(zdim(p)));
+        double *x = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!w || !z || !x) {
+            bad = 1;
+        } else {
+            filter_row(p, h, A, BW, b, z, w);
+            for (int64_t c = 0; c < C; ++c) {
+                x[0] = u[b * C + c];
+                for (int64_t j = 1; j < K; ++j) x[j] = state[(b * (K - 1) + (j - 1)) * C + c];
+                double acc = x[0];
+                for (int64_t j = 0; j < K; ++j) acc += w[c * K + j] * x[j];
+                y[b * C + c] = acc;
+                for (int64_t j = 0; j + 1 < K; ++j) state[(b * (K - 1) + j) * C + c] = x[j];
+            }
+        }
+        free(w);
+        free(z);
+        free(x);
+    }
+    return bad ? ORC_BAD : ORC_OK;
+}

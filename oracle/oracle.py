@@ -58,7 +58,9 @@ def _load():
             lib.orc_param_grads.argtypes = [P, dp, dp, dp, dp, dp, dp, dp]
             lib.orc_param_grad_entries.argtypes = [P, dp, dp, dp, dp, dp, ctypes.c_int64, ctypes.c_int64,
                                                    ip, ip, dp]
-            for f in (lib.orc_forward, lib.orc_backward_rows, lib.orc_param_grads, lib.orc_param_grad_entries):
+            lib.orc_decode_step.argtypes = [P, dp, dp, dp, dp, dp, dp]
+            for f in (lib.orc_forward, lib.orc_backward_rows, lib.orc_param_grads, lib.orc_param_grad_entries,
+                      lib.orc_decode_step):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -178,3 +180,20 @@ def param_grad_entries(p: Problem, g, u, h, A, BW, which: str, idx0, idx1):
     if rc != 0:
         raise ValueError("oracle rejected the request")
     return out
+
+
+def decode_step(p: Problem, u, h, A, BW, state):
+    """One decode step: p.n_tokens sequences, one new token each (u [B, C], h [B, d]),
+    state [B, K-1, C] = the previous K-1 conv inputs (zero before a sequence start).
+    Returns (y [B, C], new state); the argument is not modified."""
+    lib = _load()
+    u, h, A, BW = _f64(u), _f64(h), _f64(A), _f64(BW)
+    st = np.array(state, dtype=np.float64, copy=True).reshape(p.n_tokens, max(p.ksize - 1, 0), p.channels)
+    st = np.ascontiguousarray(st)
+    y = np.zeros((p.n_tokens, p.channels))
+    s, cu = p._c()
+    rc = lib.orc_decode_step(ctypes.byref(s), _d(u), _d(h), _d(A) if A is not None else None, _d(BW),
+                             st.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if st.size else None, _d(y))
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return y, st
