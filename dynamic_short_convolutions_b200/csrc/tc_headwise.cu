@@ -148,7 +148,29 @@ __device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int
         if (j % L == l) dst[j] = __float2bfloat16_rn(j <= pos ? p[j] : 0.f);
 }
 
+// The K taps of one head's filter for one token, as floats (8- or 4-byte loads when aligned,
+// which holds for K = 4 and K = 2 since R = H K).
+template <int K>
+__device__ __forceinline__ void load_taps(const __nv_bfloat16* __restrict__ p, float (&w)[K]) {
+    if constexpr (K == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = bf16_lo(v.x);
+        w[1] = bf16_hi(v.x);
+        w[2] = bf16_lo(v.y);
+        w[3] = bf16_hi(v.y);
+    } else if constexpr (K == 2) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+        w[0] = bf16_lo(v);
+        w[1] = bf16_hi(v);
+    } else {
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = __bfloat162float(p[j]);
+    }
+}
+
 // L = head_dim / 8 lanes hold one head's channels (a power of two <= 32, aligned in the warp).
+// A thread takes two consecutive tokens n, n + 1, which share K of their K + 1 rows of g, of u
+// and of the filter: each row is loaded once for both.
 template <int K>
 __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* __restrict__ g,
                                                           const __nv_bfloat16* __restrict__ u, int64_t us,
@@ -165,29 +187,41 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
     const int L = hd >> 3;
     const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
     const int64_t n1 = min(N, n0 + kTokPerBlock);
-    for (int64_t n = n0 + tl; n < n1; n += 8) {
-        int32_t sb, eb;
-        seg_bounds32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb, eb);
-        const int32_t pos = (int32_t)n - sb, epos = eb - 1 - (int32_t)n;
-        uint4 gv[K], uv[K];
-        __nv_bfloat16 w[K];
+    for (int64_t n = n0 + 2 * tl; n < n1; n += 16) {
+        const bool two = n + 1 < n1;                     // uniform over the warp
+        int32_t sb[2], eb[2];
+        seg_bounds32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb[0], eb[0]);
+        if (two) seg_bounds32((int32_t)n + 1, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb[1], eb[1]);
+        else { sb[1] = sb[0]; eb[1] = eb[0]; }
+        // rows n .. n + K of g and of the filter, rows n - K + 1 .. n + 1 of u (zero outside [0, N))
+        uint4 gr[K + 1], ur[K + 1];
+        float wr[K + 1][K];
 #pragma unroll
-        for (int j = 0; j < K; ++j) {          // issue every load of the token first
-            const bool f = j <= epos, p = j <= pos;
-            gv[j] = f ? *reinterpret_cast<const uint4*>(g + (n + j) * C + c) : make_uint4(0, 0, 0, 0);
-            w[j] = f ? wh[(n + j) * R + q * K + j] : __float2bfloat16_rn(0.f);   // filter of token n+j, tap j
-            uv[j] = p ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
-        }
-        float acc[8];
-        unpack8(gv[0], acc);
-        float part[K];
+        for (int i = 0; i <= K; ++i) {                   // every load of the pair first
+            const int64_t mg = n + i, mu = n - K + 1 + i;
+            gr[i] = mg < N ? *reinterpret_cast<const uint4*>(g + mg * C + c) : make_uint4(0, 0, 0, 0);
+            ur[i] = (mu >= 0 && mu < N) ? *reinterpret_cast<const uint4*>(u + mu * us + c) : make_uint4(0, 0, 0, 0);
+            if (mg < N) load_taps<K>(wh + mg * R + q * K, wr[i]);
+            else
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-            axpy8(acc, __bfloat162float(w[j]), gv[j]);
-            part[j] = dot8(gv[0], uv[j]);       // dwh partial over this thread's 8 channels
+                for (int j = 0; j < K; ++j) wr[i][j] = 0.f;
         }
-        *reinterpret_cast<uint4*>(du + n * C + c) = pack8(acc);
-        head_sum_store<K>(part, L, gl, pos, dwh + n * R + q * K);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (t == 1 && !two) break;
+            const int32_t m = (int32_t)n + t;
+            const int32_t pos = m - sb[t], epos = eb[t] - 1 - m;
+            float acc[8];
+            unpack8(gr[t], acc);
+            float part[K];
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                axpy8(acc, j <= epos ? wr[t + j][j] : 0.f, gr[t + j]);   // filter of token m+j, tap j
+                part[j] = dot8(gr[t], ur[K - 1 + t - j]);                 // g[m] . u[m-j] over 8 channels
+            }
+            *reinterpret_cast<uint4*>(du + (int64_t)m * C + c) = pack8(acc);
+            head_sum_store<K>(part, L, gl, pos, dwh + (int64_t)m * R + q * K);
+        }
     }
 }
 
