@@ -66,35 +66,27 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
     return s0 + s1;
 }
 
+// The K taps of one head's filter for one token, as floats (8- or 4-byte loads when aligned,
+// which holds for K = 4 and K = 2 since R = H K).
 template <int K>
-__device__ __forceinline__ void hw_fwd_token(const __nv_bfloat16* __restrict__ u, int64_t us,
-                                             const __nv_bfloat16* __restrict__ wh, int R, int q, int64_t n,
-                                             int64_t c, int64_t C, int64_t seqlen, const int32_t* __restrict__ cu,
-                                             int64_t n_docs, __nv_bfloat16* __restrict__ y) {
-    const int32_t pos = (int32_t)n - seg_start32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen);
-    uint4 uv[K];
-    __nv_bfloat16 w[K];
-#pragma unroll
-    for (int j = 0; j < K; ++j) {          // issue every load of the token first
-        const bool v = j <= pos;
-        uv[j] = v ? *reinterpret_cast<const uint4*>(u + (n - j) * us + c) : make_uint4(0, 0, 0, 0);
-    }
-    const __nv_bfloat16* wp = wh + n * R + q * K;
+__device__ __forceinline__ void load_taps(const __nv_bfloat16* __restrict__ p, float (&w)[K]) {
     if constexpr (K == 4) {
-        *reinterpret_cast<uint2*>(w) = *reinterpret_cast<const uint2*>(wp);
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = bf16_lo(v.x);
+        w[1] = bf16_hi(v.x);
+        w[2] = bf16_lo(v.y);
+        w[3] = bf16_hi(v.y);
     } else if constexpr (K == 2) {
-        *reinterpret_cast<uint32_t*>(w) = *reinterpret_cast<const uint32_t*>(wp);
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+        w[0] = bf16_lo(v);
+        w[1] = bf16_hi(v);
     } else {
 #pragma unroll
-        for (int j = 0; j < K; ++j) w[j] = wp[j];
+        for (int j = 0; j < K; ++j) w[j] = __bfloat162float(p[j]);
     }
-    float acc[8];
-    unpack8(uv[0], acc);
-#pragma unroll
-    for (int j = 0; j < K; ++j) axpy8(acc, j <= pos ? __bfloat162float(w[j]) : 0.f, uv[j]);
-    *reinterpret_cast<uint4*>(y + n * C + c) = pack8(acc);
 }
 
+// A thread takes two consecutive tokens n, n + 1, which share K of their K + 1 rows of u.
 template <int K>
 __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
                                                           const __nv_bfloat16* __restrict__ wh, int R, int hd,
@@ -108,9 +100,29 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
     const int q = (int)(c / hd);
     const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
     const int64_t n1 = min(N, n0 + kTokPerBlock);
-    for (int64_t n = n0 + tl; n < n1; n += 16) {       // two tokens per step: more loads in flight
-        hw_fwd_token<K>(u, us, wh, R, q, n, c, C, seqlen, cu, n_docs, y);
-        if (n + 8 < n1) hw_fwd_token<K>(u, us, wh, R, q, n + 8, c, C, seqlen, cu, n_docs, y);
+    for (int64_t n = n0 + 2 * tl; n < n1; n += 16) {
+        const bool two = n + 1 < n1;                     // uniform over the warp
+        // rows n - K + 1 .. n + 1 of u (zero outside [0, N)); the filters of n and n + 1
+        uint4 ur[K + 1];
+        float w[2][K];
+#pragma unroll
+        for (int i = 0; i <= K; ++i) {
+            const int64_t m = n - K + 1 + i;
+            ur[i] = (m >= 0 && m < N) ? *reinterpret_cast<const uint4*>(u + m * us + c) : make_uint4(0, 0, 0, 0);
+        }
+        load_taps<K>(wh + n * R + q * K, w[0]);
+        if (two) load_taps<K>(wh + (n + 1) * R + q * K, w[1]);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (t == 1 && !two) break;
+            const int32_t m = (int32_t)n + t;
+            const int32_t pos = m - seg_start32(m, cu, (int32_t)n_docs, (int32_t)seqlen);
+            float acc[8];
+            unpack8(ur[K - 1 + t], acc);
+#pragma unroll
+            for (int j = 0; j < K; ++j) axpy8(acc, j <= pos ? w[t][j] : 0.f, ur[K - 1 + t - j]);
+            *reinterpret_cast<uint4*>(y + (int64_t)m * C + c) = pack8(acc);
+        }
     }
 }
 
@@ -146,26 +158,6 @@ __device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int
 #pragma unroll
     for (int j = 0; j < K; ++j)
         if (j % L == l) dst[j] = __float2bfloat16_rn(j <= pos ? p[j] : 0.f);
-}
-
-// The K taps of one head's filter for one token, as floats (8- or 4-byte loads when aligned,
-// which holds for K = 4 and K = 2 since R = H K).
-template <int K>
-__device__ __forceinline__ void load_taps(const __nv_bfloat16* __restrict__ p, float (&w)[K]) {
-    if constexpr (K == 4) {
-        const uint2 v = *reinterpret_cast<const uint2*>(p);
-        w[0] = bf16_lo(v.x);
-        w[1] = bf16_hi(v.x);
-        w[2] = bf16_lo(v.y);
-        w[3] = bf16_hi(v.y);
-    } else if constexpr (K == 2) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-        w[0] = bf16_lo(v);
-        w[1] = bf16_hi(v);
-    } else {
-#pragma unroll
-        for (int j = 0; j < K; ++j) w[j] = __bfloat162float(p[j]);
-    }
 }
 
 // L = head_dim / 8 lanes hold one head's channels (a power of two <= 32, aligned in the warp).
