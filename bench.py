@@ -84,6 +84,12 @@ def layer_flops(w, layer):
     return N * 6 * d * H * K
 
 
+# DRAM bytes (read + write) per launch of a workload's dominant kernel, from one ncu capture of
+# the kernel as it is built now (profiles/<kernel>_<workload>.md); absent where none was taken.
+NCU_TRAFFIC = {("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): 204585728,
+               ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): 280690432}
+
+
 def kernel_bytes(name, w, layer):
     """Algorithmic bytes of ONE launch of a library kernel on one layer call
     (inputs read once, outputs written once, at the kernel's interface)."""
@@ -530,7 +536,8 @@ def run_ours(args, rank, world, local_rank):
         avg_s = ms / n_l / 1e3
         achieved = per_launch_bytes / avg_s / 1e9
         roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                "traffic": NCU_TRAFFIC.get((name, w.name)),
                 "peak_source": pk_src, "avg_launch_us": round(avg_s * 1e6, 2),
                 "algorithmic_bytes_per_launch": int(per_launch_bytes)}
     step_bytes = sum(layer_bytes(w, layer) for layer in w.layers)
