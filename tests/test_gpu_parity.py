@@ -32,6 +32,7 @@ SMALL = [
     (_case("c2_qkv_150m_lowrank", 1, 1, "single_token"), 0),
     (_case("c2_qkv_150m_lowrank", 2, 129, "k1_r16", ksize=1, rank=16), 0),
     (_case("c2_qkv_150m_lowrank", 2, 257, "k2_r64", ksize=2, rank=64), 0),
+    (_case("c2_qkv_150m_lowrank", 1, 140, "k1_r64", ksize=1, rank=64), 0),
     (_case("c2_qkv_150m_lowrank", 1, 200, "k4_r8", ksize=4, rank=8), 0),
     (_case("c2_qkv_150m_lowrank", 1, 130, "odd_channels", layers=(W.Layer("x", 40, 72),)), 0),
     (_case("c3_qkv_2b_headwise_gqa", 1, 150, "hw_k2_hd64", ksize=2, head_dim=64,
