@@ -220,13 +220,14 @@ struct FwdArgs {
 constexpr int kFwdStages = 4;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
 constexpr uint32_t kFwdStage = kZBytes + kUBytes;
-// Epilogue warps of lowrank_fwd_kernel<K>: 16 (two 8-channel groups each) for K <= 3, where the
-// extra warps hide more latency; 8 (four groups each) for K = 4, whose larger per-group state
-// would not fit the registers of 16 warps.
+// Epilogue of lowrank_fwd_kernel<K>: 16 warps, two 8-channel groups each (four warps per TMEM
+// lane quarter: more warps hide more of the TMEM / shared-memory latency than fewer, larger
+// ones, measured); K = 4 takes one group per TMEM wait to stay within the registers of 16 warps.
 template <int K>
 struct FwdEpi {
-    static constexpr int warps = K <= 3 ? 16 : 8;
+    static constexpr int warps = 16;
     static constexpr int groups = 32 / warps;        // 8-channel groups per warp
+    static constexpr int per_pass = K <= 3 ? 2 : 1;  // groups per TMEM wait
     static constexpr int threads = 96 + 32 * warps;  // producer, MMA, store warps + epilogue
 };
 
@@ -397,9 +398,9 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             const uint8_t* us = sm + s * kFwdStage + kZBytes;
             uint8_t* ys = sm + S::ys + b * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
-            // NG 8-channel groups per pass (all four of this warp's groups when the registers
-            // allow): every TMEM and shared-memory load first, then one wait, then the arithmetic
-            constexpr int NG = kFwdGroups < 4 ? kFwdGroups : (K <= 3 ? 4 : 2);
+            // NG 8-channel groups per pass: every TMEM and shared-memory load first, then one wait,
+            // then the arithmetic
+            constexpr int NG = FwdEpi<K>::per_pass;
 #pragma unroll
             for (int pass = 0; pass < kFwdGroups / NG; ++pass) {
                 const int g0 = kFwdGroups * half + NG * pass;
