@@ -13,7 +13,8 @@
 // where s(t) / e(t) are the first / one-past-last token of t's sequence or document.
 //
 // Kernels
-//   permute_b_kernel   B [r, C K] -> Bp [r, K C] tap-major (Bp[k, j C + c] = B[k, c K + j]).
+//   bwd_prep_kernel    zeroes the dz accumulator and writes Bp [r, K C], the tap-major copy of B
+//                      (Bp[k, j C + c] = B[k, c K + j]).
 //   lowrank_bwd_kernel one CTA per contiguous run of (64-channel chunk, 128-token tile)
 //                      work items, chunk-major, so the chunk's Bp stays in shared memory
 //                      and dB for the chunk accumulates in TMEM across the run:

@@ -30,10 +30,9 @@ namespace {
 
 using namespace tc;
 
-// A block covers kTokPerBlock tokens x 256 channels: 8 warps, each lane 8 channels of one
-// token per step (16-byte loads and stores along C), two tokens in flight per step; the K - 1
-// neighbouring rows a token needs were just read by the block's other warps and come from
-// L1 / L2.
+// A block covers kTokPerBlock tokens x 256 channels: 8 warps, each lane 8 channels (16-byte
+// loads and stores along C) of two consecutive tokens per step; the rows beyond the pair were
+// just read by the block's other warps and come from L1 / L2.
 constexpr int kTokPerBlock = 64;
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {

@@ -60,6 +60,34 @@ class DynConvPlan:
         return out
 
 
+class DynConvDecoder:
+    """Decode steps for `batch` sequences (one new token each per step) with the K-1
+    previous conv inputs of every sequence kept on the device (``self.state``,
+    ``[batch, K-1, C]``, zero = sequence start; call :meth:`reset` to start over)."""
+
+    def __init__(self, kind: int, dtype: torch.dtype, batch: int, d_model: int, channels: int, ksize: int,
+                 rank: int = 0, head_dim: int = 0, u_row_stride: int = 0, h_row_stride: int = 0, device=None):
+        self.desc = L.make_desc(kind, L.BF16 if dtype == torch.bfloat16 else L.F32, batch, 1, d_model, channels,
+                                ksize, rank, head_dim, u_row_stride, h_row_stride, 0, L.ALGO_AUTO)
+        nbytes = L.dynconv_workspace_bytes(self.desc)
+        if nbytes == 0:
+            raise L.DynConvError(1, "invalid descriptor")
+        dev = device or "cuda"
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.state = torch.zeros((batch, ksize - 1, channels), dtype=dtype, device=dev) if ksize > 1 else None
+        self.dtype, self.batch, self.C = dtype, batch, channels
+
+    def reset(self):
+        if self.state is not None:
+            self.state.zero_()
+
+    def step(self, u, h, A, B_or_W, y=None, stream=None):
+        if y is None:
+            y = torch.empty((self.batch, self.C), dtype=self.dtype, device=u.device)
+        L.dynconv_decode_step(self.desc, u, h, A, B_or_W, self.state, y, self.ws, stream)
+        return y
+
+
 class DynamicShortConv(torch.autograd.Function):
     """y = u + dynamic causal depthwise conv(u) with filters generated from h.
 
