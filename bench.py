@@ -273,7 +273,7 @@ def run_decode(args, rank, world, local_rank):
     Bd = args.decode_batch
     dt = W.storage_dtype(w)
     kind = L.LOWRANK if w.kind == W.LOWRANK else L.HEADWISE
-    seed = w.seed + 7919 * rank
+    seed = shard_seed(w.seed, rank)
     calls = []
     for li, layer in enumerate(w.layers):
         d, C, K = layer.d_model, layer.channels, w.ksize
@@ -303,6 +303,11 @@ def run_decode(args, rank, world, local_rank):
     for *_, ws in calls:
         assert L.dynconv_device_status(ws) == 0, L.dynconv_last_error()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
@@ -310,7 +315,9 @@ def run_decode(args, rank, world, local_rank):
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    total_ms = float(sum(a.elapsed_time(b) for a, b in ev))
+    if world > 1:
+        dist.barrier()
+    total_ms = max_over_ranks(float(sum(a.elapsed_time(b) for a, b in ev)), world, dev)
     L.dynconv_profile_read(reset=True)
     L.dynconv_profile_enable(True)
     for i in range(args.steps):
@@ -341,14 +348,14 @@ def run_decode(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     pk, pk_src = peaks()
     ms_step = total_ms / args.steps
     step_bytes = sum(decode_bytes(w, c[0], Bd) for c in calls)
     achieved = step_bytes / (ms_step / 1e3) / 1e9
     kernels = {n: {"launches": nl, "ms_total": round(ms, 4), "us_per_launch": round(1e3 * ms / nl, 2)}
                for n, (nl, ms) in prof.items()}
-    line = {"metric": DECODE_METRIC, "mode": "decode", "value": round(Bd * args.steps / (total_ms / 1e3), 1),
+    line = {"metric": DECODE_METRIC, "mode": "decode", "value": round(job_throughput(Bd, world, args.steps, total_ms), 1),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
@@ -359,7 +366,7 @@ def run_decode(args, rank, world, local_rank):
                          "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None, "peak_source": pk_src,
                          "algorithmic_bytes_per_step": int(step_bytes)},
             "kernels": kernels,
-            "e2e": {"value": round(Bd * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+            "e2e": {"value": round(job_throughput(Bd, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": int(sum(v[0] for v in prof.values())), "clocks": clk.summary()}
     return line
@@ -397,6 +404,31 @@ def oracle_decode_rate(w, batch, budget_s):
     return batch * steps / secs, f"{steps} decode step(s) of {batch} sequences, every layer", secs
 
 
+# ----------------------------------------------------------------------------- ranks
+def shard_seed(seed: int, rank: int) -> int:
+    """Seed of rank `rank`'s shard of a workload: each rank draws its own tokens (weak
+    scaling, replicas with no exchange in the hot path)."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """The maximum of `value` over the ranks (device time of the slowest rank); the value
+    itself with one rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: the tokens every rank processed over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (max_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -410,7 +442,7 @@ def run_ours(args, rank, world, local_rank):
     w = W.CONFIGS[args.config]
     if rank:
         import dataclasses
-        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)   # each rank: its own shard
+        w = dataclasses.replace(w, seed=shard_seed(w.seed, rank))   # each rank: its own shard
     kind = L.LOWRANK if w.kind == W.LOWRANK else L.HEADWISE
     dt = W.storage_dtype(w)
     layers = []
@@ -471,13 +503,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     L.dynconv_profile_enable(False)
     prof = L.dynconv_profile_read(reset=True)
-    total_ms = float(sum(step_ms))
-    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax.item())
-    tokens_all = w.tokens * world * args.steps
-    value = tokens_all / (total_ms / 1e3)
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
+    value = job_throughput(w.tokens, world, args.steps, total_ms)
 
     # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
     host = []
@@ -516,10 +543,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = w.tokens * world * e2e_steps / (float(e2e_ms.item()) / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(w.tokens, world, e2e_steps, e2e_ms)
 
     # ---- roofline of the dominant kernel (live CUDA-event timing from the library's tracer)
     pk, pk_src = peaks()
