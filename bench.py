@@ -449,15 +449,21 @@ def run_ours(args, rank, world, local_rank):
     for li, layer in enumerate(w.layers):
         t = W.make_inputs(w, layer, li, device=dev)
         batch, seqlen = (1, w.tokens) if w.varlen else (w.batch, w.seqlen)
+        cf = args.layout == "channel_first"
         plan = ops.DynConvPlan(kind, dt, batch, seqlen, layer.d_model, layer.channels, w.ksize, w.rank,
-                               w.head_dim, algo=args.algo, device=dev)
+                               w.head_dim, algo=args.algo, device=dev,
+                               layout=L.CHANNEL_FIRST if cf else L.TOKEN_MAJOR)
         A = t.get("A")
         BW = t["B"] if kind == L.LOWRANK else t["W"]
         N = w.tokens
-        bufs = dict(y=torch.empty((N, layer.channels), dtype=dt, device=dev),
+        conv_shape = (batch, layer.channels, seqlen) if cf else (N, layer.channels)
+        if cf:      # u and g stored [batch, C, seqlen] (converted once, outside the timed region)
+            for k in ("u", "g"):
+                t[k] = t[k].reshape(batch, seqlen, layer.channels).transpose(1, 2).contiguous()
+        bufs = dict(y=torch.empty(conv_shape, dtype=dt, device=dev),
                     z=torch.empty((N, w.rank if kind == L.LOWRANK else (layer.channels // w.head_dim) * w.ksize),
                                   dtype=dt, device=dev),
-                    out={"du": torch.empty((N, layer.channels), dtype=dt, device=dev),
+                    out={"du": torch.empty(conv_shape, dtype=dt, device=dev),
                          "dh": torch.empty((N, layer.d_model), dtype=dt, device=dev),
                          "dA": torch.empty(tuple(A.shape), dtype=torch.float32, device=dev) if A is not None else None,
                          "dBW": torch.empty(tuple(BW.shape), dtype=torch.float32, device=dev)})
@@ -562,7 +568,7 @@ def run_ours(args, rank, world, local_rank):
         achieved = per_launch_bytes / avg_s / 1e9
         roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                "traffic": NCU_TRAFFIC.get((name, w.name)),
+                "traffic": NCU_TRAFFIC.get((name, w.name)) if args.layout == "token_major" else None,
                 "peak_source": pk_src, "avg_launch_us": round(avg_s * 1e6, 2),
                 "algorithmic_bytes_per_launch": int(per_launch_bytes)}
     step_bytes = sum(layer_bytes(w, layer) for layer in w.layers)
@@ -584,7 +590,7 @@ def run_ours(args, rank, world, local_rank):
                        "layers": [[l.name, l.d_model, l.channels] for l in w.layers],
                        "varlen": w.varlen, "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (256 MiB write, outside the step events)",
-                       "algo": {0: "auto", 1: "simt", 2: "tc"}[args.algo]},
+                       "algo": {0: "auto", 1: "simt", 2: "tc"}[args.algo], "layout": args.layout},
             "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
@@ -605,6 +611,8 @@ def main():
     ap.add_argument("--mode", default="train", choices=["train", "decode"],
                     help="train: forward + backward step (default); decode: one decode step per layer")
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences per decode step")
+    ap.add_argument("--layout", default="token_major", choices=["token_major", "channel_first"],
+                    help="memory layout of u, y, g, du: [N, C] or [batch, C, seqlen]")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

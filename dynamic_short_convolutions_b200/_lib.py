@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "DYNCONV_OK", 1: "DYNCONV_ERR_INVALID", 2: "DYNCONV_ERR_UNSUP
 LOWRANK, HEADWISE = 0, 1
 F32, BF16 = 0, 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
+TOKEN_MAJOR, CHANNEL_FIRST = 0, 1
 
 # Every entry point the header declares (checked against the library's exports by the tests).
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
@@ -46,7 +47,7 @@ class dynconv_desc(ctypes.Structure):
                 ("seqlen", ctypes.c_int64), ("d_model", ctypes.c_int64), ("channels", ctypes.c_int64),
                 ("ksize", ctypes.c_int64), ("rank", ctypes.c_int64), ("head_dim", ctypes.c_int64),
                 ("u_row_stride", ctypes.c_int64), ("h_row_stride", ctypes.c_int64),
-                ("deterministic", ctypes.c_int32), ("algo", ctypes.c_int32)]
+                ("deterministic", ctypes.c_int32), ("algo", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
 
 _lib = None
@@ -110,9 +111,9 @@ def _check(status: int):
 
 def make_desc(kind: int, dtype: int, batch: int, seqlen: int, d_model: int, channels: int, ksize: int,
               rank: int = 0, head_dim: int = 0, u_row_stride: int = 0, h_row_stride: int = 0,
-              deterministic: int = 0, algo: int = ALGO_AUTO) -> dynconv_desc:
+              deterministic: int = 0, algo: int = ALGO_AUTO, layout: int = TOKEN_MAJOR) -> dynconv_desc:
     return dynconv_desc(kind, dtype, batch, seqlen, d_model, channels, ksize, rank, head_dim, u_row_stride,
-                        h_row_stride, deterministic, algo)
+                        h_row_stride, deterministic, algo, layout)
 
 
 def dynconv_workspace_bytes(desc: dynconv_desc) -> int:

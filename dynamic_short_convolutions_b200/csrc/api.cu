@@ -56,11 +56,24 @@ dynconv_status make_prob(const dynconv_desc* d, Prob* p) {
     p->d = d->d_model;
     p->C = d->channels;
     p->K = d->ksize;
-    p->us = d->u_row_stride ? d->u_row_stride : d->channels;
+    if (d->layout != DYNCONV_TOKEN_MAJOR && d->layout != DYNCONV_CHANNEL_FIRST) {
+        set_error("bad layout %d", d->layout);
+        return DYNCONV_ERR_INVALID;
+    }
+    p->layout = d->layout;
     p->hs = d->h_row_stride ? d->h_row_stride : d->d_model;
-    if (p->us < p->C || p->hs < p->d) { set_error("row stride below row width"); return DYNCONV_ERR_INVALID; }
     const int64_t vec = d->dtype == DYNCONV_BF16 ? 8 : 4;
-    if (p->us % vec || p->hs % vec) { set_error("row strides must be multiples of 16 bytes"); return DYNCONV_ERR_INVALID; }
+    if (p->layout == DYNCONV_TOKEN_MAJOR) {
+        p->us = d->u_row_stride ? d->u_row_stride : d->channels;
+        if (p->us < p->C) { set_error("u row stride below the channel count"); return DYNCONV_ERR_INVALID; }
+        if (p->us % vec) { set_error("u row stride must be a multiple of 16 bytes"); return DYNCONV_ERR_INVALID; }
+    } else {
+        // channel-first: any channel stride >= seqlen (the vectorised kernels check their own alignment)
+        p->us = d->u_row_stride ? d->u_row_stride : d->seqlen;
+        if (p->us < p->seqlen) { set_error("u channel stride below seqlen"); return DYNCONV_ERR_INVALID; }
+    }
+    if (p->hs < p->d) { set_error("h row stride below d_model"); return DYNCONV_ERR_INVALID; }
+    if (p->hs % vec) { set_error("h row stride must be a multiple of 16 bytes"); return DYNCONV_ERR_INVALID; }
     if (d->kind == DYNCONV_LOWRANK) {
         if (d->rank < 1) { set_error("low-rank needs rank >= 1"); return DYNCONV_ERR_INVALID; }
         if (d->rank > 128) { set_error("rank %lld > 128 is not supported", (long long)d->rank); return DYNCONV_ERR_UNSUPPORTED; }
@@ -238,6 +251,15 @@ dynconv_status dynconv_decode_step(const dynconv_desc* desc, const void* u, cons
         set_error("dynconv_decode_step takes one new token per sequence: seqlen must be 1");
         return DYNCONV_ERR_INVALID;
     }
+    if (p.layout == DYNCONV_CHANNEL_FIRST) {
+        // [batch, C, 1] with unit channel stride is the token-major [batch, C]
+        if (p.us != 1) {
+            set_error("channel-first decode needs u_row_stride 0 or 1");
+            return DYNCONV_ERR_UNSUPPORTED;
+        }
+        p.layout = DYNCONV_TOKEN_MAJOR;
+        p.us = p.C;
+    }
     if (p.N == 0) return DYNCONV_OK;
     if ((s = check_ptr(u, "u", true)) || (s = check_ptr(h, "h", true)) || (s = check_ptr(A, "A", p.kind == 0)) ||
         (s = check_ptr(B_or_W, p.kind == 0 ? "B" : "W", true)) || (s = check_ptr(state, "state", p.K > 1)) ||
@@ -280,6 +302,6 @@ const char* dynconv_status_string(dynconv_status status) {
     return "unknown status";
 }
 
-int dynconv_version(void) { return 100; }
+int dynconv_version(void) { return 110; }
 
 }  // extern "C"

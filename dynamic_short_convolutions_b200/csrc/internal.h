@@ -22,7 +22,8 @@ struct Prob {
     int64_t r;          // low-rank rank
     int64_t hd, H;      // head-wise head_dim and head count
     int64_t R;          // generator width: r (low-rank) or H*K (head-wise)
-    int64_t us, hs;     // row strides of u and h, in elements
+    int64_t us, hs;     // u: token-major row stride / channel-first channel stride; h: row stride
+    int layout;         // 0 token-major [N, C]; 1 channel-first [batch, C, seqlen] (u, y, g, du)
     const int32_t* cu;  // device cu_seqlens or nullptr (dense batch)
     int64_t n_docs;
     int deterministic;
@@ -38,6 +39,13 @@ struct WsLayout {
     size_t dec;         // decode step (seqlen == 1): split-d partial generator rows
     size_t total;
 };
+
+// Channel-first problems the tiled kernels take: seqlen and u's channel stride multiples of 8
+// elements (16-byte TMA rows and vector loads), TMA coordinates within int32.
+inline bool cf_tiles_ok(const Prob& p) {
+    return p.seqlen % 8 == 0 && p.us % 8 == 0 && p.batch * p.C < (int64_t(1) << 31) &&
+           p.seqlen < (int64_t(1) << 31);
+}
 
 WsLayout ws_layout(const Prob& p);
 size_t tc_workspace_bytes(const Prob& p);

@@ -23,6 +23,27 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// Element (token n, channel c) of a conv-side tensor (u, y, g, du) in either layout:
+//   token-major   n * ts + c
+//   channel-first (n / T) * bs + (n % T) + c * cs    (T = seqlen; sequences bs apart, channels cs apart)
+struct Ax {
+    int64_t T, bs, ts, cs;
+    int cf;
+    __device__ __forceinline__ int64_t operator()(int64_t n, int64_t c) const {
+        return cf ? (n / T) * bs + (n % T) + c * cs : n * ts + c;
+    }
+};
+
+// u (strided) and the dense conv-side tensors of a problem.
+inline Ax ax_u(const Prob& p) {
+    const int64_t T = p.seqlen > 0 ? p.seqlen : 1;
+    return p.layout ? Ax{T, p.C * p.us, 1, p.us, 1} : Ax{T, 0, p.us, 1, 0};
+}
+inline Ax ax_dense(const Prob& p) {
+    const int64_t T = p.seqlen > 0 ? p.seqlen : 1;
+    return p.layout ? Ax{T, p.C * T, 1, T, 1} : Ax{T, 0, p.C, 1, 0};
+}
+
 // X[n, k] = sum_i h[n, i] P[i, k]   (z = h A or head-wise filters h W), fp32 out;
 // optionally also stored to zsave in the storage type.
 template <typename T>
@@ -60,19 +81,19 @@ __device__ __forceinline__ float filter_tap(const float* xs, const T* __restrict
 
 template <typename T, int KIND>
 __global__ void __launch_bounds__(kThreads) conv_fwd_kernel(
-    const T* __restrict__ u, int64_t us, const float* __restrict__ X, int64_t R, const T* __restrict__ B,
+    const T* __restrict__ u, Ax au, const float* __restrict__ X, int64_t R, const T* __restrict__ B,
     int64_t C, int64_t K, int64_t hd, const int32_t* __restrict__ cu, int64_t n_docs, int64_t seqlen,
-    T* __restrict__ y) {
+    T* __restrict__ y, Ax ay) {
     extern __shared__ float xs[];
     const int64_t n = blockIdx.x;
     for (int64_t k = threadIdx.x; k < R; k += blockDim.x) xs[k] = X[n * R + k];
     __syncthreads();
     const int64_t s = seg_start(n, cu, n_docs, seqlen);
     for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-        float acc = to_f32(u[n * us + c]);
+        float acc = to_f32(u[au(n, c)]);
         for (int64_t j = 0; j < K; ++j)
-            if (n - j >= s) acc = fmaf(filter_tap<T, KIND>(xs, B, R, C, K, hd, c, j), to_f32(u[(n - j) * us + c]), acc);
-        y[n * C + c] = from_f32<T>(acc);
+            if (n - j >= s) acc = fmaf(filter_tap<T, KIND>(xs, B, R, C, K, hd, c, j), to_f32(u[au(n - j, c)]), acc);
+        y[ay(n, c)] = from_f32<T>(acc);
     }
 }
 
@@ -82,7 +103,7 @@ __global__ void __launch_bounds__(kThreads) conv_fwd_kernel(
 // with dw[m,c,j] = g[m,c] u[m-j,c] for m-j >= s(m).
 template <typename T, int KIND>
 __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(
-    const T* __restrict__ g, const T* __restrict__ u, int64_t us, const float* __restrict__ X, int64_t R,
+    const T* __restrict__ g, const T* __restrict__ u, Ax au, Ax ad, const float* __restrict__ X, int64_t R,
     const T* __restrict__ B, int64_t N, int64_t C, int64_t K, int64_t hd, const int32_t* __restrict__ cu,
     int64_t n_docs, int64_t seqlen, T* __restrict__ du, float* __restrict__ dgen) {
     extern __shared__ float sm[];
@@ -101,10 +122,10 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(
     }
     __syncthreads();
     for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-        float acc = to_f32(g[m * C + c]);
+        float acc = to_f32(g[ad(m, c)]);
         for (int64_t j = 0; j < K; ++j)
-            if (valid[j]) acc = fmaf(filter_tap<T, KIND>(xs + j * R, B, R, C, K, hd, c, j), to_f32(g[(m + j) * C + c]), acc);
-        du[m * C + c] = from_f32<T>(acc);
+            if (valid[j]) acc = fmaf(filter_tap<T, KIND>(xs + j * R, B, R, C, K, hd, c, j), to_f32(g[ad(m + j, c)]), acc);
+        du[ad(m, c)] = from_f32<T>(acc);
     }
     if (KIND == 0) {
         // dz[m, k] for every k: block reduction over channels in a fixed order.
@@ -112,9 +133,9 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(
         for (int64_t k = 0; k < R; ++k) {
             float part = 0.f;
             for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-                const float gm = to_f32(g[m * C + c]);
+                const float gm = to_f32(g[ad(m, c)]);
                 for (int64_t j = 0; j < K; ++j)
-                    if (m - j >= sm_) part = fmaf(gm * to_f32(u[(m - j) * us + c]), to_f32(B[k * C * K + c * K + j]), part);
+                    if (m - j >= sm_) part = fmaf(gm * to_f32(u[au(m - j, c)]), to_f32(B[k * C * K + c * K + j]), part);
             }
             for (int off = 16; off > 0; off >>= 1) part += __shfl_down_sync(0xffffffffu, part, off);
             if (lane == 0) red[warp] = part;
@@ -132,7 +153,7 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(
             const int64_t q = e / K, j = e % K;
             float t = 0.f;
             if (m - j >= sm_)
-                for (int64_t c = q * hd; c < (q + 1) * hd; ++c) t = fmaf(to_f32(g[m * C + c]), to_f32(u[(m - j) * us + c]), t);
+                for (int64_t c = q * hd; c < (q + 1) * hd; ++c) t = fmaf(to_f32(g[ad(m, c)]), to_f32(u[au(m - j, c)]), t);
             dgen[m * R + e] = t;
         }
     }
@@ -141,7 +162,7 @@ __global__ void __launch_bounds__(kThreads) conv_bwd_kernel(
 // dB[k, c*K+j] = sum_n z[n,k] g[n,c] u[n-j,c]  (n-j >= s(n)), one thread per entry.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) dB_kernel(
-    const float* __restrict__ Z, int64_t r, const T* __restrict__ g, const T* __restrict__ u, int64_t us,
+    const float* __restrict__ Z, int64_t r, const T* __restrict__ g, const T* __restrict__ u, Ax au, Ax ad,
     int64_t N, int64_t C, int64_t K, const int32_t* __restrict__ cu, int64_t n_docs, int64_t seqlen,
     float* __restrict__ dB) {
     const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -150,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) dB_kernel(
     float acc = 0.f;
     for (int64_t n = j; n < N; ++n)
         if (n - j >= seg_start(n, cu, n_docs, seqlen))
-            acc = fmaf(Z[n * r + k], to_f32(g[n * C + c]) * to_f32(u[(n - j) * us + c]), acc);
+            acc = fmaf(Z[n * r + k], to_f32(g[ad(n, c)]) * to_f32(u[au(n - j, c)]), acc);
     dB[e] = acc;
 }
 
@@ -200,12 +221,12 @@ cudaError_t forward_t(const Prob& p, const void* u, const void* h, const void* A
     const size_t smem = sizeof(float) * (size_t)p.R;
     if (p.kind == 0)
         DC_LAUNCH(kSimtConvFwd, st, conv_fwd_kernel<T, 0><<<(unsigned)p.N, kThreads, smem, st>>>(
-            static_cast<const T*>(u), p.us, X, p.R, static_cast<const T*>(BW), p.C, p.K, 1, p.cu, p.n_docs,
-            p.seqlen, static_cast<T*>(y)));
+            static_cast<const T*>(u), ax_u(p), X, p.R, static_cast<const T*>(BW), p.C, p.K, 1, p.cu, p.n_docs,
+            p.seqlen, static_cast<T*>(y), ax_dense(p)));
     else
         DC_LAUNCH(kSimtConvFwd, st, conv_fwd_kernel<T, 1><<<(unsigned)p.N, kThreads, smem, st>>>(
-            static_cast<const T*>(u), p.us, X, p.R, nullptr, p.C, p.K, p.hd, p.cu, p.n_docs, p.seqlen,
-            static_cast<T*>(y)));
+            static_cast<const T*>(u), ax_u(p), X, p.R, nullptr, p.C, p.K, p.hd, p.cu, p.n_docs, p.seqlen,
+            static_cast<T*>(y), ax_dense(p)));
     return cudaGetLastError();
 }
 
@@ -228,16 +249,16 @@ cudaError_t backward_t(const Prob& p, const void* g, const void* u, const void* 
     const size_t smem = sizeof(float) * (size_t)(p.K * p.R + kThreads / 32);
     if (p.kind == 0)
         DC_LAUNCH(kSimtConvBwd, st, conv_bwd_kernel<T, 0><<<(unsigned)p.N, kThreads, smem, st>>>(
-            static_cast<const T*>(g), static_cast<const T*>(u), p.us, X, p.R, static_cast<const T*>(BW), p.N,
-            p.C, p.K, 1, p.cu, p.n_docs, p.seqlen, static_cast<T*>(du), DG));
+            static_cast<const T*>(g), static_cast<const T*>(u), ax_u(p), ax_dense(p), X, p.R,
+            static_cast<const T*>(BW), p.N, p.C, p.K, 1, p.cu, p.n_docs, p.seqlen, static_cast<T*>(du), DG));
     else
         DC_LAUNCH(kSimtConvBwd, st, conv_bwd_kernel<T, 1><<<(unsigned)p.N, kThreads, smem, st>>>(
-            static_cast<const T*>(g), static_cast<const T*>(u), p.us, X, p.R, nullptr, p.N, p.C, p.K, p.hd,
-            p.cu, p.n_docs, p.seqlen, static_cast<T*>(du), DG));
+            static_cast<const T*>(g), static_cast<const T*>(u), ax_u(p), ax_dense(p), X, p.R, nullptr, p.N, p.C,
+            p.K, p.hd, p.cu, p.n_docs, p.seqlen, static_cast<T*>(du), DG));
     if (p.kind == 0) {
         DC_LAUNCH(kSimtDB, st, dB_kernel<T><<<blocks_for(p.r * p.C * p.K), kThreads, 0, st>>>(
-            X, p.r, static_cast<const T*>(g), static_cast<const T*>(u), p.us, p.N, p.C, p.K, p.cu, p.n_docs,
-            p.seqlen, dBW));
+            X, p.r, static_cast<const T*>(g), static_cast<const T*>(u), ax_u(p), ax_dense(p), p.N, p.C, p.K, p.cu,
+            p.n_docs, p.seqlen, dBW));
         DC_LAUNCH(kSimtHTX, st, hTX_kernel<T><<<blocks_for(p.d * p.R), kThreads, 0, st>>>(
             static_cast<const T*>(h), p.hs, DG, p.N, p.d, p.R, dA));
     } else {

@@ -208,6 +208,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 //   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3.. epilogue (FwdEpi<K>::warps; each a TMEM lane
 //   quarter and a share of the channels): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
 //   -> bf16 staging (128-byte swizzled) -> TMA store by warp 2.
+// CF (channel-first u and y, [batch * C, seqlen]): the u tile is a [64 channels][136 tokens]
+// box (272-byte rows, no swizzle), y is staged [64 channels][128 tokens]; token tiles stay
+// inside one sequence (tps tiles per sequence), the z tile starts at the tile's first token.
 // =====================================================================================
 struct FwdArgs {
     int64_t N, C, seqlen, n_docs;
@@ -215,11 +218,13 @@ struct FwdArgs {
     uint32_t* err;
     int64_t per_cta;         // work items per CTA (contiguous run)
     int ksteps;              // 16-wide K steps of the filter MMA: r / 16 rounded up
+    int64_t n_tiles, tps;    // token tiles; tiles per sequence (channel-first)
 };
 
 constexpr int kFwdStages = 4;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
 constexpr uint32_t kFwdStage = kZBytes + kUBytes;
+constexpr uint32_t kCfUPitch = 136 * 2, kCfYPitch = 128 * 2;   // channel-first tile rows (bytes)
 // Epilogue of lowrank_fwd_kernel<K>: 16 warps, two 8-channel groups each (four warps per TMEM
 // lane quarter: more warps hide more of the TMEM / shared-memory latency than fewer, larger
 // ones, measured); K = 4 takes one group per TMEM wait to stay within the registers of 16 warps.
@@ -267,7 +272,7 @@ __device__ __forceinline__ uint4 conv8(const uint32_t (*wv)[8], const uint4* uj,
     return pk;
 }
 
-template <int K>
+template <int K, bool CF>
 __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                      const __grid_constant__ CUtensorMap tm_b,
                                                                      const __grid_constant__ CUtensorMap tm_u,
@@ -282,7 +287,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n_tiles = (a.N + 127) / 128, n_items = n_tiles * (a.C / 64);
+    const int64_t n_tiles = a.n_tiles, n_items = n_tiles * (a.C / 64);
     const int64_t i0 = (int64_t)blockIdx.x * a.per_cta, i1 = min(i0 + a.per_cta, n_items);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFwdStages; ++s) {
@@ -321,7 +326,8 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             uint32_t cc = 0, it = 0;
             for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
                 const int64_t chunk = item / n_tiles, tile = item % n_tiles;
-                const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
+                const int32_t c0 = (int32_t)(chunk * 64);
+                const TileAt ta = tile_at<CF>(tile, c0, a.tps, a.seqlen, a.C);
                 if (chunk != prev) {
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * 8192);
@@ -334,8 +340,9 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 if (!mbar_wait(&empty[s], ((it / kFwdStages) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* st = sm + s * kFwdStage;
                 mbar_arrive_expect_tx(&full[s], kFwdStage);
-                tma_load_2d(st, &tm_z, &full[s], 0, m0);
-                tma_load_2d(st + kZBytes, &tm_u, &full[s], c0, m0 - 8);
+                tma_load_2d(st, &tm_z, &full[s], 0, ta.m0);
+                if (CF) tma_load_2d(st + kZBytes, &tm_u, &full[s], ta.x - 8, ta.y);
+                else tma_load_2d(st + kZBytes, &tm_u, &full[s], ta.x, ta.y - 8);
             }
         }
     } else if (warp == 1) {
@@ -371,7 +378,8 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 const int64_t chunk = item / n_tiles, tile = item % n_tiles;
                 const int b = it & 1;
                 if (!mbar_wait(&yfull[b], (it >> 1) & 1, &abort_flag, a.err)) break;
-                tma_store_2d(&tm_y, sm + S::ys + b * kYBytes, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
+                tma_store_2d(&tm_y, sm + S::ys + b * kYBytes, ta.x, ta.y);
                 tma_store_commit();
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                 mbar_arrive(&yempty[b]);
@@ -393,14 +401,14 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                             mbar_wait(&yempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err);
             if (!ok) break;
             tc_fence_after();
-            const int32_t n = (int32_t)(tile * 128) + row;
+            const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
             const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
             const uint8_t* us = sm + s * kFwdStage + kZBytes;
             uint8_t* ys = sm + S::ys + b * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
             // NG 8-channel groups per pass: every TMEM and shared-memory load first, then one wait,
-            // then the arithmetic
-            constexpr int NG = FwdEpi<K>::per_pass;
+            // then the arithmetic (channel-first: one group, its 8 K column loads are enough in flight)
+            constexpr int NG = CF ? 1 : FwdEpi<K>::per_pass;
 #pragma unroll
             for (int pass = 0; pass < kFwdGroups / NG; ++pass) {
                 const int g0 = kFwdGroups * half + NG * pass;
@@ -414,11 +422,15 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 for (int x = 0; x < NG; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j)
-                        uj[x][j] = *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g0 + x));
+                        uj[x][j] = CF ? cf_gather8(us, kCfUPitch, g0 + x, row + 8 - j)
+                                      : *reinterpret_cast<const uint4*>(us + sw128_off(row + 8 - j, g0 + x));
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < NG; ++x)
-                    *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = conv8<K>(wv[x], uj[x], pos);
+                for (int x = 0; x < NG; ++x) {
+                    const uint4 yv = conv8<K>(wv[x], uj[x], pos);
+                    if (CF) cf_scatter8(ys, kCfYPitch, g0 + x, row, yv);
+                    else *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = yv;
+                }
             }
             tc_fence_before();
             fence_async_smem();
@@ -438,17 +450,25 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     }
 }
 
-template <int K>
+template <int K, bool CF>
 cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
                                const CUtensorMap& ty, FwdArgs fa, int64_t items, cudaStream_t st) {
     constexpr uint32_t smem = FwdSmem<K>::total;
-    cudaError_t e = cudaFuncSetAttribute(lowrank_fwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(lowrank_fwd_kernel<K, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     fa.per_cta = (items + num_sms() - 1) / num_sms();
     const unsigned grid = (unsigned)((items + fa.per_cta - 1) / fa.per_cta);
-    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K>, dim3(grid), dim3(FwdEpi<K>::threads), smem, st, tz,
-                                                tb, tu, ty, fa));
+    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K, CF>, dim3(grid), dim3(FwdEpi<K>::threads), smem,
+                                                st, tz, tb, tu, ty, fa));
     return e;
+}
+
+template <int K>
+cudaError_t launch_lowrank_fwd_l(bool cf, const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
+                                 const CUtensorMap& ty, FwdArgs fa, int64_t items, cudaStream_t st) {
+    return cf ? launch_lowrank_fwd<K, true>(tz, tb, tu, ty, fa, items, st)
+              : launch_lowrank_fwd<K, false>(tz, tb, tu, ty, fa, items, st);
 }
 
 }  // namespace
@@ -500,6 +520,7 @@ bool tc_supported(const Prob& p) {
     if (p.C % 64 != 0 || p.d % 8 != 0) return false;
     if (p.K < 1 || p.K > 4) return false;
     if (p.N >= (int64_t(1) << 31) || p.r * p.C * p.K >= (int64_t(1) << 31)) return false;
+    if (p.layout == 1 && !cf_tiles_ok(p)) return false;
     return tensor_map_encoder() != nullptr;
 }
 
@@ -533,17 +554,24 @@ cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, cons
     cudaError_t e = tc_gen_launch(h, p.hs, A, p.N, p.d, (int)p.r, z, p.r, err, st,
                                   BPermute{BW, bp, (int)p.r, (int)p.C, (int)p.K});
     if (e != cudaSuccess) return e;
+    const bool cf = p.layout == 1;
     CUtensorMap tz, tb, tu, ty;
-    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
-        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128))
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 128) || !make_tmap_bf16(&tb, bp, p.C * p.K, p.r, p.C * p.K, 64, 64))
         return cudaErrorInvalidValue;
-    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16)};
-    const int64_t items = ((p.N + 127) / 128) * (p.C / 64);
+    if (cf ? !(make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, 136, 64, false) &&
+               make_tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.seqlen * 2, 128, 64,
+                            false))
+           : !(make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) && make_tmap_bf16(&ty, y, p.C, p.N, p.C, 64, 128)))
+        return cudaErrorInvalidValue;
+    const int64_t tps = (p.seqlen + 127) / 128;
+    const int64_t n_tiles = cf ? p.batch * tps : (p.N + 127) / 128;
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16), n_tiles, tps};
+    const int64_t items = n_tiles * (p.C / 64);
     switch (p.K) {
-        case 1: return launch_lowrank_fwd<1>(tz, tb, tu, ty, fa, items, st);
-        case 2: return launch_lowrank_fwd<2>(tz, tb, tu, ty, fa, items, st);
-        case 3: return launch_lowrank_fwd<3>(tz, tb, tu, ty, fa, items, st);
-        default: return launch_lowrank_fwd<4>(tz, tb, tu, ty, fa, items, st);
+        case 1: return launch_lowrank_fwd_l<1>(cf, tz, tb, tu, ty, fa, items, st);
+        case 2: return launch_lowrank_fwd_l<2>(cf, tz, tb, tu, ty, fa, items, st);
+        case 3: return launch_lowrank_fwd_l<3>(cf, tz, tb, tu, ty, fa, items, st);
+        default: return launch_lowrank_fwd_l<4>(cf, tz, tb, tu, ty, fa, items, st);
     }
 }
 

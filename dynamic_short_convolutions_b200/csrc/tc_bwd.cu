@@ -76,6 +76,7 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat
 
 struct BwdArgs {
     int64_t N, C, seqlen, n_docs;
+    int64_t tps;              // token tiles per sequence (channel-first)
     const int32_t* cu;
     int r, ndz;               // rank, MMA N for dz / dB (r rounded up to 16)
     int64_t n_tiles, n_items, per_cta;
@@ -127,7 +128,9 @@ constexpr int kGbWarps = 4, kGa0 = 2;
 // TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
 constexpr uint32_t kColDz = 256, kColDb = 384;
 
-template <int K, bool R64>
+constexpr uint32_t kCfPitch = 136 * 2, kCfStPitch = 128 * 2;   // channel-first tile rows (bytes)
+
+template <int K, bool R64, bool CF>
 __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                          const __grid_constant__ CUtensorMap tm_g,
                                                                          const __grid_constant__ CUtensorMap tm_u,
@@ -206,16 +209,17 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     ++cc;
                     prev = chunk;
                 }
-                const int32_t m0 = (int32_t)(tile * 128), c0 = (int32_t)(chunk * 64);
+                const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
                 const int zs = it % NZ, gs = it & 1;
                 if (!mbar_wait(&zempty[zs], ((it / NZ) & 1) ^ 1, &abort_flag, a.err)) break;
                 mbar_arrive_expect_tx(&zfull[zs], kRowTile);
-                tma_load_2d(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, m0);
+                tma_load_2d(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, ta.m0);
                 if (!mbar_wait(&guempty[gs], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* gu = sm + gs * S::gu;
                 mbar_arrive_expect_tx(&gufull[gs], S::gu);
-                tma_load_2d(gu, &tm_g, &gufull[gs], c0, m0);
-                tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], c0, m0 - 8);
+                tma_load_2d(gu, &tm_g, &gufull[gs], ta.x, ta.y);
+                if (CF) tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], ta.x - 8, ta.y);
+                else tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], ta.x, ta.y - 8);
             }
         }
     } else if (warp == 1) {
@@ -313,7 +317,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             if (leader) tma_store_wait_read_all();     // the previous du store has read the staging tile
             if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
             tc_fence_after();
-            const int32_t n = (int32_t)(tile * 128) + row;
+            const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
+            const int32_t n = ta.m0 + row;
             int32_t pos = -1, epos = -1;             // valid past / future taps of this row
             if (n < a.N) {
                 int32_t sb, eb;
@@ -339,7 +344,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 for (int x = 0; x < kGaPerWait; ++x)
 #pragma unroll
                     for (int j = 0; j < K; ++j)
-                        gg[x][j] = *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
+                        gg[x][j] = CF ? cf_gather8(gt, kCfPitch, g0 + x, row + j)
+                                      : *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < kGaPerWait; ++x) {
@@ -361,9 +367,10 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                                       __uint_as_float(wv[x][j][2 * p + 1]), bf16_lo(gj[p]), bf16_hi(gj[p]));
                         }
                     }
-                    *reinterpret_cast<uint4*>(dus + sw128_off(row, g0 + x)) =
-                        make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                                   pack_bf16(acc[6], acc[7]));
+                    const uint4 dv = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                                                pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+                    if (CF) cf_scatter8(dus, kCfStPitch, g0 + x, row, dv);
+                    else *reinterpret_cast<uint4*>(dus + sw128_off(row, g0 + x)) = dv;
                 }
             }
             tc_fence_before();
@@ -381,7 +388,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     break;
                 }
                 if (bb == 0 && leader) {                 // every GA warp has staged its du rows
-                    tma_store_2d(&tm_du, dus, (int32_t)(chunk * 64), (int32_t)(tile * 128));
+                    tma_store_2d(&tm_du, dus, ta.x, ta.y);
                     tma_store_commit();
                 }
 #pragma unroll
@@ -389,7 +396,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     const int g8 = kGaGroups * half + i;
 #pragma unroll
                     for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j) {
-                        const uint4 uu = *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
+                        const uint4 uu = CF ? cf_gather8(ut, kCfPitch, g8, row + 8 - j)
+                                            : *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
                         const bool v = j <= pos;
                         uint4 d;
                         d.x = v ? mul_bf16x2(gv[i].x, uu.x) : 0u;
@@ -425,7 +433,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             if (via_tma && leader) tma_store_wait_read_all();   // the previous reduction has read the tile
             if (named_bar_any<3, 32 * kGbWarps>(!ok)) break;
             tc_fence_after();
-            const int32_t n = (int32_t)(tile * 128) + row;
+            const int32_t m0 = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0;
+            const int32_t n = m0 + row;
             for (int c = 0; c < a.r; c += 16) {
                 uint32_t v[2][8];
                 tmem_ld8(lane_base + kColDz + 64 * b + c, v[0]);
@@ -467,7 +476,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 named_bar_any<3, 32 * kGbWarps>(false);     // every GB warp has staged its dz rows
                 if (leader) {
                     for (int bx = 0; bx * 32 < a.r; ++bx)
-                        tma_reduce_add_2d(&tm_dz, dzs + bx * kAtom128, bx * 32, (int32_t)(tile * 128));
+                        tma_reduce_add_2d(&tm_dz, dzs + bx * kAtom128, bx * 32, m0);
                     tma_store_commit();
                 }
             }
@@ -757,18 +766,26 @@ inline unsigned grid_for(int64_t n, int threads = 256) {
     return (unsigned)std::max<int64_t>(1, std::min<int64_t>(b, 148 * 16));
 }
 
-template <int K, bool R64>
-cudaError_t launch_bwd(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
-                       const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba, unsigned grid, cudaStream_t st) {
+template <int K, bool R64, bool CF>
+cudaError_t launch_bwd_l(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
+                         const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba, unsigned grid, cudaStream_t st) {
     using S = BwdSmem<K, R64>;
     static_assert(S::total <= kSmemMax, "shared memory of lowrank_bwd_kernel");
     if (S::dzst_bytes == 0) ba.dz_tma = 0;
-    cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K, R64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K, R64, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::total);
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64>, dim3(grid), dim3(BwdEpi<K>::threads), S::total,
-                                                st, tz, tg, tu, tbp, tdu, tdz, ba));
+    DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64, CF>, dim3(grid), dim3(BwdEpi<K>::threads),
+                                                S::total, st, tz, tg, tu, tbp, tdu, tdz, ba));
     return e;
+}
+
+template <int K, bool R64>
+cudaError_t launch_bwd(bool cf, const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu,
+                       const CUtensorMap& tbp, const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba,
+                       unsigned grid, cudaStream_t st) {
+    return cf ? launch_bwd_l<K, R64, true>(tz, tg, tu, tbp, tdu, tdz, ba, grid, st)
+              : launch_bwd_l<K, R64, false>(tz, tg, tu, tbp, tdu, tdz, ba, grid, st);
 }
 
 }  // namespace
@@ -824,7 +841,7 @@ static inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 TcBwdLayout tc_bwd_layout(const Prob& p) {
     TcBwdLayout L{};
     const int sms = 148;   // sizing only; the launch uses at most this many CTAs
-    L.n_tiles = (p.N + 127) / 128;
+    L.n_tiles = p.layout == 1 ? p.batch * ((p.seqlen + 127) / 128) : (p.N + 127) / 128;
     const int64_t n_chunks = p.C / 64;
     L.n_items = L.n_tiles * n_chunks;
     L.per_cta = std::max<int64_t>(1, (L.n_items + sms - 1) / sms);
@@ -867,23 +884,29 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     CUtensorMap tz, tg, tu, tbp, tdu, tdz;
     std::memset(&tdz, 0, sizeof(tdz));                 // unused unless dz goes through bulk reductions
     const bool dz_tma = p.r % 32 == 0;
-    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) ||
-        !make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
-        !make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128) ||
+    const bool cf = p.layout == 1;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
         (dz_tma && !make_tmap_2d(&tdz, dz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.r, p.N, p.r * 4, 32, 128, true)))
         return cudaErrorInvalidValue;
-    BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16), L.n_tiles, L.n_items,
-               L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dz_tma ? 1 : 0};
+    if (cf ? !(make_tmap_2d(&tg, g, BF, p.seqlen, p.batch * p.C, p.seqlen * 2, 136, 64, false) &&
+               make_tmap_2d(&tu, u, BF, p.seqlen, p.batch * p.C, p.us * 2, 136, 64, false) &&
+               make_tmap_2d(&tdu, du, BF, p.seqlen, p.batch * p.C, p.seqlen * 2, 128, 64, false))
+           : !(make_tmap_bf16(&tg, g, p.C, p.N, p.C, 64, 136) && make_tmap_bf16(&tu, u, p.C, p.N, p.us, 64, 136) &&
+               make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128)))
+        return cudaErrorInvalidValue;
+    BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, (p.seqlen + 127) / 128, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16),
+               L.n_tiles, L.n_items, L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dz_tma ? 1 : 0};
     const bool r64 = p.r > 32;
     switch (p.K * 2 + (r64 ? 1 : 0)) {
-        case 2: e = launch_bwd<1, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 3: e = launch_bwd<1, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 4: e = launch_bwd<2, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 5: e = launch_bwd<2, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 6: e = launch_bwd<3, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 7: e = launch_bwd<3, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 8: e = launch_bwd<4, false>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        default: e = launch_bwd<4, true>(tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 2: e = launch_bwd<1, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 3: e = launch_bwd<1, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 4: e = launch_bwd<2, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 5: e = launch_bwd<2, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 6: e = launch_bwd<3, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 7: e = launch_bwd<3, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 8: e = launch_bwd<4, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        default: e = launch_bwd<4, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
     switch (p.K) {

@@ -186,6 +186,43 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Byte offset of 16-byte chunk q of row r inside a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
 
+// Channel-first tiles (TMA boxes of a [batch * C, seqlen] tensor, no swizzle): one row of
+// `pitch` bytes per channel, tokens contiguous.  cf_gather8 reads token column i of channels
+// 8 c8 .. 8 c8 + 7 and packs them like a 16-byte segment of a token-major row; cf_scatter8
+// writes such a segment back as a column.  A warp's lanes take consecutive tokens, so each
+// 2-byte access of a warp covers 64 contiguous bytes (no bank conflict).
+__device__ __forceinline__ uint4 cf_gather8(const uint8_t* tile, uint32_t pitch, int c8, int i) {
+    const uint8_t* p = tile + (uint32_t)(8 * c8) * pitch + 2u * (uint32_t)i;
+    uint32_t v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const uint16_t*>(p + e * pitch);
+    return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
+}
+__device__ __forceinline__ void cf_scatter8(uint8_t* tile, uint32_t pitch, int c8, int i, uint4 v) {
+    uint8_t* p = tile + (uint32_t)(8 * c8) * pitch + 2u * (uint32_t)i;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        *reinterpret_cast<uint16_t*>(p + (2 * e) * pitch) = (uint16_t)(w[e] & 0xFFFFu);
+        *reinterpret_cast<uint16_t*>(p + (2 * e + 1) * pitch) = (uint16_t)(w[e] >> 16);
+    }
+}
+
+// Token tile `tile` (128 tokens) and 64-channel chunk c0 of a conv-side tensor (u, g, y, du):
+// m0 = its first token (the row of z / dz), (x, y) = the TMA coordinates of the tile.
+//   token-major   [N, C]:                 x = c0, y = m0
+//   channel-first [batch * C, seqlen]:    x = t0 (first token within the sequence), y = b C + c0,
+//                 with tps = tiles per sequence, so a tile never spans two sequences
+struct TileAt {
+    int32_t m0, x, y;
+};
+template <bool CF>
+__device__ __forceinline__ TileAt tile_at(int64_t tile, int32_t c0, int64_t tps, int64_t seqlen, int64_t C) {
+    if (!CF) return TileAt{(int32_t)(tile * 128), c0, (int32_t)(tile * 128)};
+    const int64_t b = tile / tps, t0 = (tile - b * tps) * 128;
+    return TileAt{(int32_t)(b * seqlen + t0), (int32_t)t0, (int32_t)(b * C + c0)};
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);

@@ -216,6 +216,217 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
     }
 }
 
+// ---- channel-first layout: u, y, g, du are [batch * C, seqlen] rows (tokens contiguous) ----
+// A block is 8 warps on one sequence b, tokens t0 .. t0 + 32 V - 1 (V consecutive tokens per
+// lane, one 8- or 16-byte load per row), and one head q; warp w takes channels w, w + 8, ... of
+// the head, so a lane's filter taps stay in registers across the head's channels.  The K - 1
+// tokens before a lane's first come from the previous lane by shuffle (lane 0 loads them), the
+// K - 1 after its last from the next lane (lane 31 loads them).  seqlen is a multiple of 8, so a
+// lane's V tokens are all inside the sequence or all past its end.
+
+// V bf16 values of one row, as V / 2 packed pairs.
+template <int V>
+__device__ __forceinline__ void ldrow(const __nv_bfloat16* __restrict__ p, uint32_t (&w)[V / 2]) {
+    if constexpr (V == 8) {
+        const uint4 t = *reinterpret_cast<const uint4*>(p);
+        w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    } else {
+        const uint2 t = *reinterpret_cast<const uint2*>(p);
+        w[0] = t.x; w[1] = t.y;
+    }
+}
+template <int V>
+__device__ __forceinline__ void strow(__nv_bfloat16* __restrict__ p, const float (&f)[V]) {
+    if constexpr (V == 8) {
+        *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                                  pack_bf16(f[6], f[7]));
+    } else {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+    }
+}
+// Element i (0 <= i < 2 P) of P packed bf16 pairs.
+template <int P>
+__device__ __forceinline__ float elem(const uint32_t (&w)[P], int i) {
+    return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+}
+
+// Row values of tokens t - 4 .. t + V - 1 (prev = the 4 before the lane's first) and, for the
+// backward, t + V .. t + V + 3 (next), for a lane whose V tokens start at t.
+template <int V>
+__device__ __forceinline__ void row_halo_prev(const __nv_bfloat16* __restrict__ row, const uint32_t (&cur)[V / 2],
+                                              int lane, int64_t t, bool live, uint32_t (&prev)[2]) {
+    prev[0] = __shfl_up_sync(0xffffffffu, cur[V / 2 - 2], 1);
+    prev[1] = __shfl_up_sync(0xffffffffu, cur[V / 2 - 1], 1);
+    if (lane == 0) {
+        if (live && t >= 4) {
+            const uint2 v = *reinterpret_cast<const uint2*>(row + t - 4);
+            prev[0] = v.x;
+            prev[1] = v.y;
+        } else {
+            prev[0] = prev[1] = 0u;
+        }
+    }
+}
+template <int V>
+__device__ __forceinline__ void row_halo_next(const __nv_bfloat16* __restrict__ row, const uint32_t (&cur)[V / 2],
+                                              int lane, int64_t t, int64_t T, uint32_t (&next)[2]) {
+    next[0] = __shfl_down_sync(0xffffffffu, cur[0], 1);
+    next[1] = __shfl_down_sync(0xffffffffu, cur[1], 1);
+    if (lane == 31) {
+        if (t + V < T) {
+            const uint2 v = *reinterpret_cast<const uint2*>(row + t + V);
+            next[0] = v.x;
+            next[1] = v.y;
+        } else {
+            next[0] = next[1] = 0u;
+        }
+    }
+}
+
+// y[c, t] = u[c, t] + sum_{j <= t - s(t)} wh[t, q K + j] u[c, t - j]  (the same FMA order as the
+// token-major kernel, so both layouts give the same bits).
+template <int K, int V>
+__global__ void __launch_bounds__(256) hw_conv_fwd_cf_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
+                                                             const __nv_bfloat16* __restrict__ wh, int R, int hd,
+                                                             int64_t N, int64_t C, int64_t T, int64_t tps,
+                                                             const int32_t* __restrict__ cu, int64_t n_docs,
+                                                             __nv_bfloat16* __restrict__ y) {
+    pdl_trigger();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t b = blockIdx.x / tps;
+    const int64_t t = (blockIdx.x - b * tps) * (32 * V) + lane * V;
+    const int q = blockIdx.y;
+    const bool live = t < T;
+    const int64_t n0 = b * T + t;
+    float w[V][K];
+    int32_t pos[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        if (live) {
+            load_taps<K>(wh + (n0 + i) * R + q * K, w[i]);
+            pos[i] = (int32_t)(n0 + i - seg_start(n0 + i, cu, n_docs, T));
+        } else {
+#pragma unroll
+            for (int j = 0; j < K; ++j) w[i][j] = 0.f;
+            pos[i] = 0;
+        }
+    }
+    for (int c = q * hd + warp; c < (q + 1) * hd; c += 8) {
+        const __nv_bfloat16* urow = u + (b * C + c) * us;
+        uint32_t cur[V / 2], prev[2];
+        if (live) ldrow<V>(urow + t, cur);
+        else
+#pragma unroll
+            for (int k = 0; k < V / 2; ++k) cur[k] = 0u;
+        row_halo_prev<V>(urow, cur, lane, t, live, prev);
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            acc[i] = elem(cur, i);
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const float x = i - j >= 0 ? elem(cur, i - j) : elem(prev, 4 + i - j);
+                acc[i] = fmaf(j <= pos[i] ? w[i][j] : 0.f, x, acc[i]);
+            }
+        }
+        if (live) strow<V>(y + (b * C + c) * T + t, acc);
+    }
+}
+
+// du[c, t] = g[c, t] + sum_{j < e(t) - t} wh[t + j, q K + j] g[c, t + j]; dwh[t, q K + j] =
+// sum_{c in q} [j <= t - s(t)] g[c, t] u[c, t - j]: each warp sums its channels in order, then
+// the block sums the 8 warps' partials in order (no atomics).
+template <int K, int V>
+__global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __nv_bfloat16* __restrict__ g,
+                                                             const __nv_bfloat16* __restrict__ u, int64_t us,
+                                                             const __nv_bfloat16* __restrict__ wh, int R, int hd,
+                                                             int64_t N, int64_t C, int64_t T, int64_t tps,
+                                                             const int32_t* __restrict__ cu, int64_t n_docs,
+                                                             __nv_bfloat16* __restrict__ du,
+                                                             __nv_bfloat16* __restrict__ dwh) {
+    __shared__ float red[8][32 * V][K];
+    pdl_trigger();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t b = blockIdx.x / tps;
+    const int64_t tb = (blockIdx.x - b * tps) * (32 * V);
+    const int64_t t = tb + lane * V;
+    const int q = blockIdx.y;
+    const bool live = t < T;
+    const int64_t n0 = b * T + t;
+    // wf[i][j]: tap j of the filter of token t + i (i < V + K - 1), zero past the sequence end
+    float wf[V + K - 1][K];
+    int32_t pos[V], epos[V];
+#pragma unroll
+    for (int i = 0; i < V + K - 1; ++i) {
+        if (live && t + i < T) load_taps<K>(wh + (n0 + i) * R + q * K, wf[i]);
+        else
+#pragma unroll
+            for (int j = 0; j < K; ++j) wf[i][j] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        if (live) {
+            int64_t sb, eb;
+            seg_bounds(n0 + i, cu, n_docs, T, N, sb, eb);
+            pos[i] = (int32_t)(n0 + i - sb);
+            epos[i] = (int32_t)(eb - 1 - (n0 + i));
+        } else {
+            pos[i] = epos[i] = -1;
+        }
+    }
+    float dacc[V][K];
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+#pragma unroll
+        for (int j = 0; j < K; ++j) dacc[i][j] = 0.f;
+    for (int c = q * hd + warp; c < (q + 1) * hd; c += 8) {
+        const __nv_bfloat16* grow = g + (b * C + c) * T;
+        const __nv_bfloat16* urow = u + (b * C + c) * us;
+        uint32_t gc[V / 2], uc[V / 2], gn[2], up[2];
+        if (live) {
+            ldrow<V>(grow + t, gc);
+            ldrow<V>(urow + t, uc);
+        } else {
+#pragma unroll
+            for (int k = 0; k < V / 2; ++k) gc[k] = uc[k] = 0u;
+        }
+        row_halo_next<V>(grow, gc, lane, t, T, gn);
+        row_halo_prev<V>(urow, uc, lane, t, live, up);
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const float gi = elem(gc, i);
+            acc[i] = gi;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                const float gx = i + j < V ? elem(gc, i + j) : elem(gn, i + j - V);
+                acc[i] = fmaf(j <= epos[i] ? wf[i + j][j] : 0.f, gx, acc[i]);
+                const float ux = i - j >= 0 ? elem(uc, i - j) : elem(up, 4 + i - j);
+                dacc[i][j] = fmaf(gi, ux, dacc[i][j]);
+            }
+        }
+        if (live) strow<V>(du + (b * C + c) * T + t, acc);
+    }
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+#pragma unroll
+        for (int j = 0; j < K; ++j) red[warp][lane * V + i][j] = dacc[i][j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * V * K; e += 256) {
+        const int k = e / K, j = e - k * K;
+        const int64_t tt = tb + k;
+        if (tt >= T) continue;
+        float sum = 0.f;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][k][j];
+        const int64_t n = b * T + tt;
+        const int32_t ps = (int32_t)(n - seg_start(n, cu, n_docs, T));
+        dwh[n * R + q * K + j] = __float2bfloat16_rn(j <= ps ? sum : 0.f);
+    }
+}
+
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
@@ -237,16 +448,29 @@ TcHwLayout tc_hw_layout(const Prob& p) {
 
 bool tc_headwise_supported(const Prob& p) {
     if (p.dtype != 1 || p.kind != 1) return false;
-    if (p.R > 128 || p.R % 8 != 0) return false;
+    if (p.R > 128 || p.R % 8 != 0 || p.d % 8 != 0) return false;
+    if (p.K < 1 || p.K > 4) return false;
+    if (p.layout == 1) return cf_tiles_ok(p) && p.H < 65536;
     if (p.hd < 8 || p.hd > 256 || (p.hd & (p.hd - 1)) != 0) return false;
-    if (p.C % 256 != 0 || p.d % 8 != 0) return false;
-    return p.K >= 1 && p.K <= 4;
+    return p.C % 256 == 0;
 }
+
+// Channel-first: 8 tokens per lane in the forward, 4 in the backward (fewer registers for
+// the look-ahead filters and the dwh partials).
+constexpr int kCfFwdV = 8, kCfBwdV = 4;
 
 template <int K>
 static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, cudaStream_t st) {
-    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
     cudaError_t e;
+    if (p.layout == 1) {
+        const int64_t tps = (p.seqlen + 32 * kCfFwdV - 1) / (32 * kCfFwdV);
+        const dim3 grid((unsigned)(p.batch * tps), (unsigned)p.H);
+        DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_cf_kernel<K, kCfFwdV>, grid, dim3(256), 0, st,
+            static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
+            p.N, p.C, p.seqlen, tps, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
+        return e;
+    }
+    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
     DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
         p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
@@ -256,8 +480,17 @@ static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, v
 template <int K>
 static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
                           cudaStream_t st) {
-    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
     cudaError_t e;
+    if (p.layout == 1) {
+        const int64_t tps = (p.seqlen + 32 * kCfBwdV - 1) / (32 * kCfBwdV);
+        const dim3 grid((unsigned)(p.batch * tps), (unsigned)p.H);
+        DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_cf_kernel<K, kCfBwdV>, grid, dim3(256), 0, st,
+            static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
+            static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, tps, p.cu, p.n_docs,
+            static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
+        return e;
+    }
+    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
     DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
         static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, p.cu, p.n_docs,

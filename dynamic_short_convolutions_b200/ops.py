@@ -21,27 +21,33 @@ def _dtype_code(t: torch.Tensor) -> int:
 class DynConvPlan:
     """Descriptor + workspace for one problem shape.
 
-    u: [N, C] (rows may be strided, channels contiguous), h: [N, d] likewise.
-    For packed documents pass ``cu_seqlens`` (int32 device tensor [docs+1]) and
-    batch = 1, seqlen = N.
+    Token-major (default): u [N, C] (rows may be strided, channels contiguous),
+    y, g, du [N, C].  Channel-first (``layout=L.CHANNEL_FIRST``): u, y, g, du
+    [batch, C, seqlen] (u's channel rows ``u_row_stride`` apart, 0 = seqlen).
+    h is [N, d] in both.  For packed documents pass ``cu_seqlens`` (int32 device
+    tensor [docs+1]) and batch = 1, seqlen = N.
     """
 
     def __init__(self, kind: int, dtype: torch.dtype, batch: int, seqlen: int, d_model: int, channels: int,
                  ksize: int, rank: int = 0, head_dim: int = 0, u_row_stride: int = 0, h_row_stride: int = 0,
-                 deterministic: bool = False, algo: int = L.ALGO_AUTO, device=None):
+                 deterministic: bool = False, algo: int = L.ALGO_AUTO, device=None, layout: int = L.TOKEN_MAJOR):
         self.desc = L.make_desc(kind, L.BF16 if dtype == torch.bfloat16 else L.F32, batch, seqlen, d_model,
                                 channels, ksize, rank, head_dim, u_row_stride, h_row_stride, int(deterministic),
-                                algo)
+                                algo, layout)
         nbytes = L.dynconv_workspace_bytes(self.desc)
         if nbytes == 0:
             raise L.DynConvError(1, "invalid descriptor")
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
-        self.kind, self.dtype = kind, dtype
+        self.kind, self.dtype, self.layout = kind, dtype, layout
         self.N, self.d, self.C, self.K, self.r = batch * seqlen, d_model, channels, ksize, rank
+        self.batch, self.seqlen = batch, seqlen
+
+    def _conv_shape(self):
+        return (self.batch, self.C, self.seqlen) if self.layout == L.CHANNEL_FIRST else (self.N, self.C)
 
     def forward(self, u, h, A, B_or_W, cu_seqlens=None, y=None, z_save=None, stream=None):
         if y is None:
-            y = torch.empty((self.N, self.C), dtype=self.dtype, device=u.device)
+            y = torch.empty(self._conv_shape(), dtype=self.dtype, device=u.device)
         if cu_seqlens is None:
             L.dynconv_fwd(self.desc, u, h, A, B_or_W, y, z_save, self.ws, stream)
         else:
@@ -51,7 +57,7 @@ class DynConvPlan:
     def backward(self, g, u, h, A, B_or_W, cu_seqlens=None, z_saved=None, want_dh=True, out=None, stream=None):
         dev = g.device
         if out is None:
-            out = {"du": torch.empty((self.N, self.C), dtype=self.dtype, device=dev),
+            out = {"du": torch.empty(self._conv_shape(), dtype=self.dtype, device=dev),
                    "dh": torch.empty((self.N, self.d), dtype=self.dtype, device=dev) if want_dh else None,
                    "dA": torch.empty(tuple(A.shape), dtype=torch.float32, device=dev) if A is not None else None,
                    "dBW": torch.empty(tuple(B_or_W.shape), dtype=torch.float32, device=dev)}
@@ -97,13 +103,19 @@ class DynamicShortConv(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, u, h, A, B_or_W, ksize: int, head_dim: int, batch: int, cu_seqlens, algo: int):
-        N, C = u.shape
         d = h.shape[1]
         kind = L.LOWRANK if A is not None else L.HEADWISE
         rank = A.shape[1] if A is not None else 0
-        seqlen = N // batch
-        plan = DynConvPlan(kind, u.dtype, batch, seqlen, d, C, ksize, rank, head_dim, u.stride(0), h.stride(0),
-                           algo=algo, device=u.device)
+        if u.dim() == 3:        # channel-first [batch, C, seqlen]
+            batch, C, seqlen = u.shape
+            if u.stride(2) != 1 or u.stride(0) != C * u.stride(1):
+                u = u.contiguous()
+            N, layout, us = batch * seqlen, L.CHANNEL_FIRST, u.stride(1)
+        else:
+            N, C = u.shape
+            seqlen, layout, us = N // batch, L.TOKEN_MAJOR, u.stride(0)
+        plan = DynConvPlan(kind, u.dtype, batch, seqlen, d, C, ksize, rank, head_dim, us, h.stride(0),
+                           algo=algo, device=u.device, layout=layout)
         R = rank if A is not None else (C // head_dim) * ksize
         z = torch.empty((N, R), dtype=u.dtype, device=u.device)    # generator output, reused by backward
         y = plan.forward(u, h, A, B_or_W, cu_seqlens, z_save=z)
@@ -122,5 +134,6 @@ class DynamicShortConv(torch.autograd.Function):
 def dynamic_short_conv(u: torch.Tensor, h: torch.Tensor, A: Optional[torch.Tensor], B_or_W: torch.Tensor,
                        ksize: int, head_dim: int = 0, batch: int = 1,
                        cu_seqlens: Optional[torch.Tensor] = None, algo: int = L.ALGO_AUTO) -> torch.Tensor:
-    """Functional form with autograd (u, h: [N, C], [N, d]; N = batch * seqlen)."""
+    """Functional form with autograd: u [N, C] token-major (N = batch * seqlen) or
+    [batch, C, seqlen] channel-first; h [N, d]."""
     return DynamicShortConv.apply(u, h, A, B_or_W, ksize, head_dim, batch, cu_seqlens, algo)

@@ -23,20 +23,35 @@
  * w [N,C,K] is never written to memory by the tensor-core path.
  *
  * Conventions shared by every entry point
- *   - Layout: token-major, channels contiguous.  u is [N, C] with row stride
+ *   - Layout (default, desc->layout = DYNCONV_TOKEN_MAJOR): token-major,
+ *     channels contiguous.  u is [N, C] with row stride
  *     desc->u_row_stride elements (0 means C), so u may be a column slice of
  *     a fused QKV output; h is [N, d] with row stride desc->h_row_stride
  *     (0 means d).  y, g, du are dense [N, C]; dh is dense [N, d]; A is
  *     [d, r]; B is [r, C*K] (column c*K + j); W is [d, H*K] (column q*K + j).
  *     N = batch * seqlen tokens.
+ *   - Channel-first layout (desc->layout = DYNCONV_CHANNEL_FIRST), the layout
+ *     of the depthwise causal convolutions in linear-RNN blocks (Mamba-2,
+ *     Gated DeltaNet), whose static conv the dynamic one replaces (gist.science
+ *     technical summary, "Language Modeling", linear RNNs; atlas.scime.ai
+ *     summary, "Surprising findings"):
+ *     u, y, g and du are [batch, C, seqlen], tokens contiguous; u's channel
+ *     rows are desc->u_row_stride elements apart (0 means seqlen) and its
+ *     sequences C * u_row_stride apart; y, g, du are dense.  Packed documents
+ *     (batch 1) are [C, N].  h, dh and z stay token-major [N, d] / [N, R]: the
+ *     generator input is the token's hidden state.  The tensor-core and
+ *     vectorised kernels take channel-first problems whose seqlen and
+ *     u_row_stride are multiples of 8 elements; other shapes run the generic
+ *     kernels (any seqlen, any u_row_stride >= seqlen).
  *   - Storage dtype desc->dtype (fp32 or bf16) for u, h, A, B/W, y, z, g, du,
  *     dh; accumulation is always fp32; parameter gradients dA, dB/dW are fp32
  *     and OVERWRITTEN (not accumulated).
  *   - Ownership: the caller allocates every buffer, including the workspace
  *     (size from dynconv_workspace_bytes).  All pointers are device pointers
  *     (a host pointer is rejected with DYNCONV_ERR_INVALID: there is no CPU
- *     path).  Pointers must be 16-byte aligned and row strides multiples of
- *     8 elements for bf16 / 4 for fp32.  The library allocates nothing.
+ *     path).  Pointers must be 16-byte aligned and token-major row strides
+ *     (u_row_stride, h_row_stride) multiples of 8 elements for bf16 / 4 for
+ *     fp32.  The library allocates nothing.
  *   - Stream: `stream` is a cudaStream_t (NULL = legacy default stream).  All
  *     work is enqueued asynchronously on it; nothing synchronises.
  *   - Errors: arguments are validated before any launch; a failed launch
@@ -76,6 +91,9 @@ typedef enum { DYNCONV_LOWRANK = 0, DYNCONV_HEADWISE = 1 } dynconv_kind;
  * fp32, which must not be rounded to a tensor-core input type). */
 typedef enum { DYNCONV_ALGO_AUTO = 0, DYNCONV_ALGO_SIMT = 1, DYNCONV_ALGO_TC = 2 } dynconv_algo;
 
+/* Memory layout of u, y, g, du (see "Conventions" above). */
+typedef enum { DYNCONV_TOKEN_MAJOR = 0, DYNCONV_CHANNEL_FIRST = 1 } dynconv_layout;
+
 typedef struct {
     int32_t kind;           /* dynconv_kind */
     int32_t dtype;          /* dynconv_dtype */
@@ -86,10 +104,12 @@ typedef struct {
     int64_t ksize;          /* K: taps, 1..4 */
     int64_t rank;           /* low-rank r (1..128); head-wise: 0 */
     int64_t head_dim;       /* head-wise channels per head (C % head_dim == 0); low-rank: 0 */
-    int64_t u_row_stride;   /* elements between tokens of u; 0 = channels */
+    int64_t u_row_stride;   /* token-major: elements between tokens of u (0 = channels);
+                               channel-first: elements between channels of u (0 = seqlen) */
     int64_t h_row_stride;   /* elements between tokens of h; 0 = d_model */
     int32_t deterministic;  /* 1: every reduction in a fixed order, no float atomics */
     int32_t algo;           /* dynconv_algo */
+    int32_t layout;         /* dynconv_layout of u, y, g, du */
 } dynconv_desc;
 
 /* Workspace needed by dynconv_fwd / dynconv_fwd_varlen / dynconv_bwd for this
@@ -101,7 +121,8 @@ typedef struct {
 DYNCONV_API size_t dynconv_workspace_bytes(const dynconv_desc *desc);
 
 /* Forward, dense batch: y = u + dynamic causal conv(u), filters from h.
- *   u      [N, C] (u_row_stride), h [N, d] (h_row_stride)
+ *   u      [N, C] (u_row_stride), h [N, d] (h_row_stride); channel-first:
+ *          u and y are [batch, C, seqlen]
  *   A      [d, r] (low-rank) or NULL (head-wise)
  *   B_or_W [r, C*K] (low-rank) or [d, H*K] (head-wise)
  *   y      [N, C] output, dense
@@ -124,6 +145,7 @@ DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const in
                                   void *y, void *z_save, void *ws, size_t ws_bytes, void *stream);
 
 /* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch).
+ * Channel-first: g, u and du are [batch, C, seqlen] ([C, N] for packed documents).
  *   g        [N, C] upstream gradient dL/dy, dense
  *   z_saved  nullable: the generator output saved by the forward ([N, r] or
  *            [N, H*K]); NULL recomputes it
@@ -178,6 +200,8 @@ DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc *desc, const v
  *   y      [batch, C] output, dense
  *   ws     workspace of dynconv_workspace_bytes(desc), zeroed once
  * Always runs the CUDA-core kernels (fp32 accumulation) whatever desc->algo says.
+ * desc->layout may be channel-first only with u_row_stride 0 or 1 (u [batch, C, 1]
+ * is then the same memory as [batch, C]).
  * Errors: as dynconv_fwd, and DYNCONV_ERR_INVALID when seqlen != 1. */
 DYNCONV_API dynconv_status dynconv_decode_step(const dynconv_desc *desc, const void *u, const void *h,
                                                const void *A, const void *B_or_W, void *state, void *y,

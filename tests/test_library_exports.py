@@ -50,3 +50,43 @@ def test_pure_host_entry_points_without_gpu():
     assert L.dynconv_workspace_bytes(d) > 0
     assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 0, 32)) == 0
     assert L.dynconv_workspace_bytes(L.make_desc(L.HEADWISE, L.BF16, 1, 10, 8, 12, 3, 0, 5)) == 0
+
+
+def test_descriptor_layout_matches_header(tmp_path):
+    """The ctypes descriptor has the C struct's size and field offsets (gcc on the header)."""
+    import shutil
+    import subprocess
+
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in L.dynconv_desc._fields_]
+    src = tmp_path / "probe.c"
+    body = "\n".join(f'    printf("{f} %zu\\n", offsetof(dynconv_desc, {f}));' for f in fields)
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "dynconv.h"\nint main(void) {\n'
+                   f'    printf("size %zu\\n", sizeof(dynconv_desc));\n{body}\n    return 0;\n}}\n')
+    exe = tmp_path / "probe"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                       check=True).stdout.splitlines())
+    assert int(out["size"]) == ctypes.sizeof(L.dynconv_desc)
+    for f in fields:
+        assert int(out[f]) == getattr(L.dynconv_desc, f).offset, f
+
+
+def test_channel_first_descriptor_validation():
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    if not os.path.exists(LIB):
+        pytest.skip("library not built")
+    cf = dict(layout=L.CHANNEL_FIRST)
+    ok = L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 3, 32, **cf)
+    assert L.dynconv_workspace_bytes(ok) > 0
+    # any channel stride >= seqlen (odd ones take the generic kernels); below seqlen is invalid
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 13, 64, 64, 3, 8, u_row_stride=15, **cf)) > 0
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 16, 64, 64, 3, 8, u_row_stride=15, **cf)) == 0
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 16, 64, 64, 3, 8, layout=2)) == 0
+    # token-major keeps its 16-byte row-stride rule
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 16, 64, 64, 3, 8, u_row_stride=65)) == 0
