@@ -24,7 +24,8 @@
 //       epi A du (-> staged, TMA store) and dw (-> bf16 tile in shared memory, 64 channels
 //             per tap, handed to the MMAs in blocks of two taps);
 //       MMA2  dz  = dW Bp_chunk^T      (M = 128 tokens, N = r, K = 64 K)
-//       MMA3  dBt += dW^T z            (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
+//       MMA3  K <= 3: dB += z^T dW     (M = 128 (r rows used), N = 64 K, K = 128 tokens)
+//             K = 4:  dBt += dW^T z    (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
 //       epi B dz -> staged fp32 tile, bulk tensor add into a [N, r] buffer (reduction over
 //             chunks; fp32 atomics when the tile does not fit);
 //       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
@@ -94,20 +95,22 @@ constexpr uint32_t kSmemMax = 232448 - 256;         // dynamic shared memory (st
 // held from its TMA load until the du / dw epilogue is done with it) and NZ z slots (held
 // until the dB MMA has read z; three when they fit), one dW tile (K tap atoms of 128 tokens x
 // 64 channels, handed to the MMAs in 128-row blocks of two atoms), the du tile staged for its
-// TMA store, the chunk's Bp slice, and (K <= 3) the fp32 dz tile staged for its bulk reduction.
+// TMA store, the chunk's Bp slice (rank rounded up to 16 rows per tap), and (K <= 3) the fp32 dz
+// tile staged for its bulk reduction.
 // The dB MMA reads dW in blocks of two atoms; for odd K the last block's second atom is the du
 // staging tile and only feeds accumulator rows that are never read.
 template <int K, bool R64>
 struct BwdSmem {
     static constexpr uint32_t gu = 2 * kRowTile;
     static constexpr uint32_t dzst_bytes = K <= 3 ? (R64 ? 2 * kAtom128 : kAtom128) : 0;
-    static constexpr uint32_t fixed = K * kAtom128 + kAtom128 + K * 8192 + dzst_bytes;
+    static constexpr uint32_t bp_tap = R64 ? 8192 : 4096;
+    static constexpr uint32_t fixed = K * kAtom128 + kAtom128 + K * bp_tap + dzst_bytes;
     static constexpr int NZ = 2 * gu + 3 * kRowTile + fixed + 1024 <= kSmemMax ? 3 : 2;
     static constexpr uint32_t z0 = 2 * gu;
     static constexpr uint32_t dw = z0 + NZ * kRowTile;
     static constexpr uint32_t dust = dw + K * kAtom128;
     static constexpr uint32_t bp = dust + kAtom128;
-    static constexpr uint32_t dzst = bp + K * 8192;
+    static constexpr uint32_t dzst = bp + K * bp_tap;
     static constexpr uint32_t total = dzst + dzst_bytes + 1024;
 };
 
@@ -125,8 +128,18 @@ struct BwdEpi {
 };
 constexpr int kGbWarps = 4, kGa0 = 2;
 
-// TMEM columns: Wd taps at 0 (64 K <= 256), dz double buffer at 256 / 320, dB^T blocks at 384 / 448.
-constexpr uint32_t kColDz = 256, kColDb = 384;
+// dB orientation.  A tcgen05.mma of M = 128, K = 16 costs about the same for every N up to 128
+// (measured on the B200: ~60 ns, N = 256 ~71 ns), so the instruction count sets the tensor time.
+// K <= 3: dB[r][(j, c)] += z^T dW, one chain of 8 MMAs (N = 64 K, K = 128 tokens; A = z^T with the
+// r index on the TMEM lanes, rows r .. 127 unused).  K = 4: dB^T[(j, c)][r] += dW^T z in 128-row
+// blocks of two taps, 16 MMAs (N = 64 K = 256 would not leave TMEM for dz).
+template <int K>
+struct BwdCols {
+    static constexpr bool dbt = K <= 3;
+    // TMEM columns: Wd taps at 0 (64 K); dB; dz double buffer
+    static constexpr uint32_t db = dbt ? 192 : 384;    // dbt: 64 K columns; else two blocks of 64
+    static constexpr uint32_t dz = dbt ? 384 : 256;    // two buffers of 64
+};
 
 constexpr uint32_t kCfPitch = 136 * 2, kCfStPitch = 128 * 2;   // channel-first tile rows (bytes)
 
@@ -140,6 +153,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                                                                          BwdArgs a) {
     using S = BwdSmem<K, R64>;
     constexpr int NBLK = (K + 1) / 2;
+    constexpr bool kDbt = BwdCols<K>::dbt;
+    constexpr uint32_t kColDz = BwdCols<K>::dz, kColDb = BwdCols<K>::db;
     constexpr int kGaWarps = BwdEpi<K>::ga, kGaGroups = BwdEpi<K>::groups, kGaPerWait = BwdEpi<K>::per_wait;
     constexpr int kGb0 = BwdEpi<K>::gb0;
     constexpr int NZ = S::NZ;
@@ -203,9 +218,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
                 if (chunk != prev) {
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
-                    mbar_arrive_expect_tx(&bfull, K * 8192);
+                    mbar_arrive_expect_tx(&bfull, K * a.ndz * 128);
                     for (int j = 0; j < K; ++j)
-                        tma_load_2d(sm + S::bp + j * 8192, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0);
+                        tma_load_2d(sm + S::bp + j * S::bp_tap, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0);
                     ++cc;
                     prev = chunk;
                 }
@@ -226,7 +241,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         if (lane == 0) {
             const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
             const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
-            const uint32_t idesc_db = idesc_bf16(128, a.ndz, true, true);
+            const uint32_t idesc_db = kDbt ? idesc_bf16(128, 64 * K, true, true) : idesc_bf16(128, a.ndz, true, true);
             const uint32_t bp0 = smem_u32(sm + S::bp);
             const uint32_t dw0 = smem_u32(sm + S::dw);
             const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
@@ -241,8 +256,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
 #pragma unroll
                 for (int j = 0; j < K; ++j)
                     for (int k = 0; k < a.ksteps; ++k)
-                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k), mnmajor_desc(bp0 + j * 8192, 8192, 16 * k),
-                                  idesc_w, k != 0);
+                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k),
+                                  mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k), idesc_w, k != 0);
                 umma_commit(&wfull);
                 return true;
             };
@@ -278,15 +293,28 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             umma_bf16(tbase + kColDz + 64 * b, kmajor_desc(dw0 + j * kAtom128, k),
-                                      kmajor_desc(bp0 + j * 8192, k), idesc_dz, (j | k) != 0);
-                    // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
+                                      kmajor_desc(bp0 + j * S::bp_tap, k), idesc_dz, (j | k) != 0);
+                    if constexpr (!kDbt) {
+                        // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tbase + kColDb + 64 * bb, mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks),
-                                  mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
-                    umma_commit(&dwfree[bb]);
+                        for (int ks = 0; ks < 8; ++ks)
+                            umma_bf16(tbase + kColDb + 64 * bb,
+                                      mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks),
+                                      mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
+                        umma_commit(&dwfree[bb]);
+                    }
                 }
                 if (!blk_ok) break;
+                if constexpr (kDbt) {
+                    // dB += z^T . dW over every tap at once (A: z tile, MN-major, its second 64-row
+                    // M atom is the next tile and only feeds unused rows; B: the K dW atoms, MN-major)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tbase + kColDb, mnmajor_desc(z0, kRowTile, 16 * ks),
+                                  mnmajor_desc(dw0, kAtom128, 16 * ks), idesc_db, !(first && ks == 0));
+#pragma unroll
+                    for (int bb = 0; bb < NBLK; ++bb) umma_commit(&dwfree[bb]);
+                }
                 if (first) ++m;
                 umma_commit(&dzfull[b]);
                 umma_commit(&zempty[zs]);
@@ -484,17 +512,37 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 // partial [k][m] (m = j * 64 + c): a warp writes 32 consecutive m per k
                 const int64_t piece = (int64_t)blockIdx.x - (chunk * a.n_tiles) / a.per_cta;
                 float* part = a.dB_part + ((chunk * a.pieces + piece) * a.r) * (64 * K);
+                if constexpr (kDbt) {
+                    // lane = k (rows below r), columns j * 64 + c: 32 contiguous bytes per load
+                    if (q * 32 < a.r) {
+                        float* dst = part + (int64_t)row * (64 * K);
+                        for (int c = 0; c < 64 * K; c += 8) {
+                            uint32_t v[8];
+                            tmem_ld8(lane_base + kColDb + c, v);
+                            tmem_wait_ld();
+                            if (row < a.r) {
+                                *reinterpret_cast<float4*>(dst + c) =
+                                    make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                                __uint_as_float(v[3]));
+                                *reinterpret_cast<float4*>(dst + c + 4) =
+                                    make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                                __uint_as_float(v[7]));
+                            }
+                        }
+                    }
+                } else {
 #pragma unroll
-                for (int bb = 0; bb < NBLK; ++bb) {
-                    const int mrow = bb * 128 + row;     // (tap, channel) row = j * 64 + c
-                    for (int c = 0; c < a.r; c += 8) {
-                        uint32_t v[8];
-                        tmem_ld8(lane_base + kColDb + 64 * bb + c, v);
-                        tmem_wait_ld();
-                        if (mrow < 64 * K) {
+                    for (int bb = 0; bb < NBLK; ++bb) {
+                        const int mrow = bb * 128 + row;     // (tap, channel) row = j * 64 + c
+                        for (int c = 0; c < a.r; c += 8) {
+                            uint32_t v[8];
+                            tmem_ld8(lane_base + kColDb + 64 * bb + c, v);
+                            tmem_wait_ld();
+                            if (mrow < 64 * K) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                part[(int64_t)(c + i) * (64 * K) + mrow] = __uint_as_float(v[i]);
+                                for (int i = 0; i < 8; ++i)
+                                    part[(int64_t)(c + i) * (64 * K) + mrow] = __uint_as_float(v[i]);
+                            }
                         }
                     }
                 }
@@ -886,7 +934,7 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     const bool dz_tma = p.r % 32 == 0;
     const bool cf = p.layout == 1;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, 64) ||
+    if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, (uint32_t)((p.r + 15) / 16 * 16)) ||
         (dz_tma && !make_tmap_2d(&tdz, dz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.r, p.N, p.r * 4, 32, 128, true)))
         return cudaErrorInvalidValue;
     if (cf ? !(make_tmap_2d(&tg, g, BF, p.seqlen, p.batch * p.C, p.seqlen * 2, 136, 64, false) &&
