@@ -5,7 +5,9 @@
 // tensor-core operand type) and the path for bf16 shapes outside the
 // tensor-core kernels' coverage.  One thread block per token for the per-token
 // steps; one thread per output entry for the token reductions, each summed in
-// token order (deterministic).
+// token order (deterministic).  u, y, g and du are addressed through their
+// strides, so the same kernels serve the token-major [N, C] and the
+// channel-first [batch, C, seqlen] layouts, any seqlen and channel stride.
 //
 // Operation ("Dynamic Short Convolutions Improve Transformers", gist.science
 // technical summary, "Dynamic Short Convolutions": Mechanism, Parameterization,

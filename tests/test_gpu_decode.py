@@ -103,3 +103,35 @@ def test_decode_argument_errors():
     desc1 = L.make_desc(L.LOWRANK, L.BF16, 2, 1, 8, 8, 1, 8, 0)               # K = 1: no state needed
     L.dynconv_decode_step(desc1, t, t, t, t, None, t, ws)
     torch.cuda.synchronize()
+
+
+def test_decode_channel_first_descriptor():
+    """A channel-first [batch, C, 1] token is the same memory as [batch, C]: a channel-first
+    descriptor decodes bitwise like the token-major one; other channel strides are refused."""
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    Bs, d, C, K, r = 3, 64, 128, 3, 16
+    x = _tensors("lowrank", "bf16", Bs, 2, d, C, K, r, 0, seed=5)
+    dev = lambda a: torch.tensor(a, dtype=torch.float64).to(torch.bfloat16).cuda().contiguous()
+    A, B = dev(x["A"]), dev(x["BW"])
+    outs = []
+    for layout in (L.TOKEN_MAJOR, L.CHANNEL_FIRST):
+        desc = L.make_desc(L.LOWRANK, L.BF16, Bs, 1, d, C, K, r, 0, layout=layout)
+        ws = torch.zeros(L.dynconv_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+        state = torch.zeros((Bs, K - 1, C), dtype=torch.bfloat16, device="cuda")
+        ys = []
+        for t in range(2):
+            y = torch.empty((Bs, C), dtype=torch.bfloat16, device="cuda")
+            L.dynconv_decode_step(desc, dev(x["u"][t]), dev(x["h"][t]), A, B, state, y, ws)
+            ys.append(y)
+        torch.cuda.synchronize()
+        outs.append((torch.stack(ys), state.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    desc = L.make_desc(L.LOWRANK, L.BF16, Bs, 1, d, C, K, r, 0, u_row_stride=2, layout=L.CHANNEL_FIRST)
+    ws = torch.zeros(L.dynconv_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    t = torch.zeros((Bs, 2 * C), dtype=torch.bfloat16, device="cuda")
+    state = torch.zeros((Bs, K - 1, C), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(L.DynConvError) as e:
+        L.dynconv_decode_step(desc, t, dev(x["h"][0]), A, B, state, torch.empty((Bs, C), dtype=torch.bfloat16,
+                                                                                  device="cuda"), ws)
+    assert e.value.status == 2
