@@ -71,6 +71,11 @@ dynconv_status make_prob(const dynconv_desc* d, Prob* p) {
         // channel-first: any channel stride >= seqlen (the vectorised kernels check their own alignment)
         p->us = d->u_row_stride ? d->u_row_stride : d->seqlen;
         if (p->us < p->seqlen) { set_error("u channel stride below seqlen"); return DYNCONV_ERR_INVALID; }
+        // one token per sequence with unit channel stride: [batch, C, 1] is the memory of [batch, C]
+        if (p->seqlen == 1 && p->us == 1 && p->C % vec == 0) {
+            p->layout = DYNCONV_TOKEN_MAJOR;
+            p->us = p->C;
+        }
     }
     if (p->hs < p->d) { set_error("h row stride below d_model"); return DYNCONV_ERR_INVALID; }
     if (p->hs % vec) { set_error("h row stride must be a multiple of 16 bytes"); return DYNCONV_ERR_INVALID; }
@@ -252,13 +257,9 @@ dynconv_status dynconv_decode_step(const dynconv_desc* desc, const void* u, cons
         return DYNCONV_ERR_INVALID;
     }
     if (p.layout == DYNCONV_CHANNEL_FIRST) {
-        // [batch, C, 1] with unit channel stride is the token-major [batch, C]
-        if (p.us != 1) {
-            set_error("channel-first decode needs u_row_stride 0 or 1");
-            return DYNCONV_ERR_UNSUPPORTED;
-        }
-        p.layout = DYNCONV_TOKEN_MAJOR;
-        p.us = p.C;
+        // validation already turned [batch, C, 1] with unit channel stride and 16-byte rows into [batch, C]
+        set_error("channel-first decode needs u_row_stride 0 or 1 and channels a multiple of 16 bytes");
+        return DYNCONV_ERR_UNSUPPORTED;
     }
     if (p.N == 0) return DYNCONV_OK;
     if ((s = check_ptr(u, "u", true)) || (s = check_ptr(h, "h", true)) || (s = check_ptr(A, "A", p.kind == 0)) ||

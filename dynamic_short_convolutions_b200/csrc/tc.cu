@@ -205,8 +205,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 //               the generator launch) as K atoms [64 r-rows][64] (MN-major B), reloaded when the
 //               chunk changes
 //   TMEM: W[128 tokens][64 K] fp32, column 64 j + c = w[m0 + row, c0 + c, j]; two buffers.
-//   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3.. epilogue (FwdEpi<K>::warps; each a TMEM lane
-//   quarter and a share of the channels): y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
+//   warps: 0 TMA loads, 1 MMA, 2 TMA stores, 3.. epilogue (FwdEpi<K>::warps in two teams taking
+//   alternate items; each warp a TMEM lane quarter and a share of the channels):
+//   y[t, c] = u[t, c] + sum_{j <= t - s(t)} W[t, 64 j + c] u[t - j, c]
 //   -> bf16 staging (128-byte swizzled) -> TMA store by warp 2.
 // CF (channel-first u and y, [batch * C, seqlen]): the u tile is a [64 channels][136 tokens]
 // box (272-byte rows, no swizzle), y is staged [64 channels][128 tokens]; token tiles stay
@@ -225,15 +226,19 @@ constexpr int kFwdStages = 4;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
 constexpr uint32_t kFwdStage = kZBytes + kUBytes;
 constexpr uint32_t kCfUPitch = 136 * 2, kCfYPitch = 128 * 2;   // channel-first tile rows (bytes)
-// Epilogue of lowrank_fwd_kernel<K>: 16 warps, two 8-channel groups each (four warps per TMEM
-// lane quarter: more warps hide more of the TMEM / shared-memory latency than fewer, larger
-// ones, measured); K = 4 takes one group per TMEM wait to stay within the registers of 16 warps.
+// Epilogue of lowrank_fwd_kernel<K>: 16 warps in two teams of 8 that take alternate items
+// (ping-pong: one team's arithmetic overlaps the other's TMEM and shared-memory loads; measured
+// 46 -> 42 us at the 150M QKV layer, 343 -> 279 us at the packed workload, against all 16 warps on
+// every item); in a team, two warps per TMEM lane quarter, four 8-channel groups each; K = 4
+// takes one group per TMEM wait to stay within the registers of 16 warps.
 template <int K>
 struct FwdEpi {
     static constexpr int warps = 16;
-    static constexpr int groups = 32 / warps;        // 8-channel groups per warp
-    static constexpr int per_pass = K <= 3 ? 2 : 1;  // groups per TMEM wait
-    static constexpr int threads = 96 + 32 * warps;  // producer, MMA, store warps + epilogue
+    static constexpr int teams = 2;
+    static constexpr int team_warps = warps / teams;
+    static constexpr int groups = 8 / (team_warps / 4);   // 8-channel groups per warp and item
+    static constexpr int per_pass = K <= 3 ? 2 : 1;       // groups per TMEM wait
+    static constexpr int threads = 96 + 32 * warps;       // producer, MMA, store warps + epilogue
 };
 
 template <int K>
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                                                                      FwdArgs a) {
     using S = FwdSmem<K>;
     constexpr int NMMA = 64 * K;
-    constexpr int kFwdEpiWarps = FwdEpi<K>::warps, kFwdGroups = FwdEpi<K>::groups;
+    constexpr int kFwdGroups = FwdEpi<K>::groups;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ uint64_t full[kFwdStages], empty[kFwdStages], bfull, bempty, tfull[2], tempty[2], yfull[2], yempty[2];
@@ -292,14 +297,14 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFwdStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kFwdEpiWarps);
+            mbar_init(&empty[s], 1 + FwdEpi<K>::team_warps);
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kFwdEpiWarps);
-            mbar_init(&yfull[b], kFwdEpiWarps);
+            mbar_init(&tempty[b], FwdEpi<K>::team_warps);
+            mbar_init(&yfull[b], FwdEpi<K>::team_warps);
             mbar_init(&yempty[b], 1);
         }
         abort_flag = 0;
@@ -387,11 +392,13 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             tma_store_wait_all();
         }
     } else {
+        // team t takes items t, t + 2, ... of the run, so it always uses TMEM buffer and y buffer t
         const int q = warp & 3;
-        const int half = (warp - 3) >> 2;      // channel groups kFwdGroups*half ..
+        const int team = (warp - 3) / FwdEpi<K>::team_warps;
+        const int half = ((warp - 3) % FwdEpi<K>::team_warps) >> 2;   // channel groups kFwdGroups*half ..
         const int row = q * 32 + lane;
-        uint32_t it = 0;
-        for (int64_t item = i0; item < i1; ++item, ++it) {
+        uint32_t it = team;
+        for (int64_t item = i0 + team; item < i1; item += FwdEpi<K>::teams, it += FwdEpi<K>::teams) {
             const int64_t tile = item % n_tiles;
             const int s = it % kFwdStages, b = it & 1;
             // each warp goes at its own pace (no barrier among the epilogue warps): a failed

@@ -200,8 +200,9 @@ DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc *desc, const v
  *   y      [batch, C] output, dense
  *   ws     workspace of dynconv_workspace_bytes(desc), zeroed once
  * Always runs the CUDA-core kernels (fp32 accumulation) whatever desc->algo says.
- * desc->layout may be channel-first only with u_row_stride 0 or 1 (u [batch, C, 1]
- * is then the same memory as [batch, C]).
+ * desc->layout may be channel-first only with u_row_stride 0 or 1 and channels a
+ * multiple of 8 (bf16) / 4 (fp32): u [batch, C, 1] is then the same memory as
+ * [batch, C] (every entry point treats such a descriptor as token-major).
  * Errors: as dynconv_fwd, and DYNCONV_ERR_INVALID when seqlen != 1. */
 DYNCONV_API dynconv_status dynconv_decode_step(const dynconv_desc *desc, const void *u, const void *h,
                                                const void *A, const void *B_or_W, void *state, void *y,
