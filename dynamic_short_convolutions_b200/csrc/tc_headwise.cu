@@ -9,8 +9,10 @@
 //   du[m, c] = g[m, c] + sum_{j < e(m) - m} wh[m+j, (c/hd)*K + j] g[m+j, c]
 //   dwh[n, q*K + j] = sum_{c in head q} [j <= n - s(n)] g[n, c] u[n-j, c]   (warp shuffles)
 //   dW = h^T dwh,  dh = dwh W^T                                        (tensor cores)
-// The conv kernels are memory-bound CUDA-core kernels (16-byte loads and stores along C,
-// packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh).
+// The conv kernels are memory-bound CUDA-core kernels: token-major (16-byte loads and stores
+// along C, packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh) and channel-first
+// (loads along the token rows of [batch * C, seqlen], a lane's filter taps held across the
+// head's channels, dwh summed per warp and then over the block's warps in order).
 #include <algorithm>
 
 #include "common.cuh"
