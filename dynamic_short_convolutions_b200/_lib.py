@@ -29,7 +29,7 @@ TOKEN_MAJOR, CHANNEL_FIRST = 0, 1
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
            "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc",
-           "dynconv_decode_step")
+           "dynconv_decode_step", "dynconv_noalloc_status")
 
 
 class DynConvError(RuntimeError):
@@ -73,6 +73,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_device_status.argtypes = [vp, sz, vp]
     lib.dynconv_fwd_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp]
     lib.dynconv_fwd_noalloc.restype = ctypes.c_int
+    lib.dynconv_noalloc_status.argtypes = [vp]
+    lib.dynconv_noalloc_status.restype = ctypes.c_int
     lib.dynconv_decode_step.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for f in (lib.dynconv_fwd, lib.dynconv_fwd_varlen, lib.dynconv_bwd, lib.dynconv_device_status,
               lib.dynconv_decode_step):
@@ -142,6 +144,13 @@ def dynconv_fwd_noalloc(desc, u, h, A, B, y, z_save=None, stream=None):
     """Forward with no workspace argument (scratch built into the library); see include/dynconv.h."""
     _check(load().dynconv_fwd_noalloc(ctypes.byref(desc), _ptr(u), _ptr(h), _ptr(A), _ptr(B), _ptr(y), _ptr(z_save),
                                       _stream(stream, u)))
+
+
+def dynconv_noalloc_status(stream=None) -> int:
+    """Synchronises the stream; returns the status of the no-workspace forward calls (does not raise)."""
+    st = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)) \
+        if stream is not None else ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return int(load().dynconv_noalloc_status(st))
 
 
 def dynconv_decode_step(desc, u, h, A, B_or_W, state, y, ws, stream=None):

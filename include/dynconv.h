@@ -173,12 +173,24 @@ DYNCONV_API dynconv_status dynconv_bwd(const dynconv_desc *desc, const int32_t *
  *   ksize * 2 bytes (rounded up to 256) plus, when z_save is NULL,
  *   N * rank * 2 bytes.
  * The first call with a given device current looks up the buffer's device
- * address (cudaGetSymbolAddress) once for that device; make that first call
- * before any stream capture.  All calls share the buffer, which keeps the last
- * call's contents; each call clears the error word and rewrites Bp and z.  Calls
- * whose work overlaps on the GPU race on the buffer: serialise them. */
+ * address (cudaGetSymbolAddress) once for that device and context, and zeroes
+ * the error word on `stream`; make that first call before any stream capture.
+ * A call that finds another context current than the one of the lookup (after
+ * cudaDeviceReset) looks the address up again.  All calls share the buffer,
+ * which keeps the last call's contents: each call rewrites Bp and z, and the
+ * error word collects the device-side failures (a pipeline wait that ran out
+ * of its time limit) of every call until dynconv_noalloc_status reads it.
+ * Calls whose work overlaps on the GPU race on the buffer: serialise them. */
 DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc *desc, const void *u, const void *h,
                                                const void *A, const void *B, void *y, void *z_save, void *stream);
+
+/* Device-side status of the dynconv_fwd_noalloc calls on the current device
+ * (no counterpart in the paper).  Synchronises `stream`, reads the error word
+ * of the built-in buffer and clears it: DYNCONV_ERR_DEVICE_CHECK if a call
+ * since the last query had a pipeline wait run out of its time limit (its y is
+ * then not valid), else DYNCONV_OK; DYNCONV_ERR_CUDA if the read failed.
+ * Allocates nothing (a copy of 4 bytes into host stack memory). */
+DYNCONV_API dynconv_status dynconv_noalloc_status(void *stream);
 
 /* One decode step: the newest token of each of desc->batch sequences (desc->seqlen
  * must be 1), with the K-1 previous conv inputs of every sequence carried in a

@@ -5,18 +5,33 @@ import numpy as np
 
 from dynamic_short_convolutions_b200 import workloads as W
 
-# Tolerances: fp32 storage rel-L2 <= 1e-5; bf16 storage rel-L2 <= 2e-2 and
-# max-abs <= 5e-2, the max-abs read on the scale of the tensor: max|err| /
-# max(1, max|ref|) (literal for tensors bounded by 1; relative above that,
-# since the bf16 rounding of one stored value of magnitude v is already up to
-# 2^-9 v, i.e. above 5e-2 for |v| > 25).
+# Tolerances (the fp32 and bf16 bounds the hot path is held to):
+#   fp32 storage: rel-L2 <= 1e-5.
+#   bf16 storage, per-token outputs (y, du, dh, z): rel-L2 <= 2e-2 and, element
+#     by element, |a - ref| <= 5e-2 + 2^-8 |ref|.  The second term is the
+#     output's own rounding: storing a value of magnitude v in bf16 moves it by
+#     up to 2^-9 v (half a unit in the last place), and 2^-8 v leaves room for
+#     the rounding of the bf16 operands it was computed from; it only matters
+#     for elements above ~6, whose stored value alone cannot be held to 5e-2.
+#   bf16 storage, parameter gradients (dA, dB, dW; fp32 outputs): rel-L2 <=
+#     2e-2 and max|a - ref| <= 5e-2 * max(1, max|ref|).  Each entry is a sum
+#     over every token of products of bf16-rounded operands, so its rounding
+#     error grows with the sum's size, not with the entry's own value: the
+#     bound is read on the scale of the tensor.
 TOL = {"f32": dict(rel_l2=1e-5, max_abs=None), "bf16": dict(rel_l2=2e-2, max_abs=5e-2)}
+ELEM_REL = 2.0 ** -8
+PARAM_GRADS = ("dA", "dB", "dW", "dBW")
 
 
 def rel_l2(a, ref):
     a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
     den = np.linalg.norm(ref)
     return float(np.linalg.norm(a - ref) / (den if den > 0 else 1.0))
+
+
+def max_abs(a, ref):
+    a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
+    return float(np.max(np.abs(a - ref))) if a.size else 0.0
 
 
 def scaled_max_abs(a, ref):
@@ -26,13 +41,41 @@ def scaled_max_abs(a, ref):
     return float(np.max(np.abs(a - ref)) / max(1.0, float(np.max(np.abs(ref)))))
 
 
-def assert_close(name, a, ref, dtype):
+def elem_excess(a, ref, bound):
+    """max over elements of |a - ref| - (bound + 2^-8 |ref|) (<= 0 when every element passes)."""
+    a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
+    if a.size == 0:
+        return -bound
+    return float(np.max(np.abs(a - ref) - (bound + ELEM_REL * np.abs(ref))))
+
+
+def is_param_grad(name):
+    return name.rsplit(":", 1)[-1] in PARAM_GRADS
+
+
+def check_close(name, a, ref, dtype):
+    """(ok, message) of the comparison; the message gives the observed figures."""
     t = TOL[dtype]
     e = rel_l2(a, ref)
-    assert e <= t["rel_l2"], f"{name}: rel-L2 {e:.3e} > {t['rel_l2']}"
+    msg = f"{name}: rel-L2 {e:.3e} (<= {t['rel_l2']})"
+    ok = e <= t["rel_l2"]
     if t["max_abs"] is not None:
-        m = scaled_max_abs(a, ref)
-        assert m <= t["max_abs"], f"{name}: scaled max-abs {m:.3e} > {t['max_abs']}"
+        m = max_abs(a, ref)
+        if is_param_grad(name):
+            sm = scaled_max_abs(a, ref)
+            msg += f", max-abs {m:.3e}, scaled max-abs {sm:.3e} (<= {t['max_abs']})"
+            ok = ok and sm <= t["max_abs"]
+        else:
+            x = elem_excess(a, ref, t["max_abs"])
+            msg += f", max-abs {m:.3e}, worst element over 5e-2 + 2^-8|ref| by {x:.3e} (<= 0)"
+            ok = ok and x <= 0.0
+    return ok, msg
+
+
+def assert_close(name, a, ref, dtype):
+    ok, msg = check_close(name, a, ref, dtype)
+    assert ok, msg
+    return msg
 
 
 def oracle_problem(w: W.Workload, layer: W.Layer, cu):

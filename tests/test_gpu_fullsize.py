@@ -88,3 +88,30 @@ def test_full_size_sampled(name):
             assert_close(tag + ":dW", W.to_f64(out["dBW"])[ia, cols], dW_ref, w.dtype)
         del t, x, y, z, out
         torch.cuda.empty_cache()
+
+
+def test_c2_every_element():
+    """The 150M QKV layer at its benchmark size, in the bench's launch configuration,
+    compared with the oracle on EVERY element of every output: y, z, du, dh and the
+    full parameter gradients dA [768, 32] and dB [32, 6912] -- the cross-CTA
+    reductions (bulk-tensor dz add-reduce, per-run dB partials, split-token dA
+    partials) included."""
+    from oracle import oracle as O
+
+    w = W.CONFIGS["c2_qkv_150m_lowrank"]
+    layer = w.layers[0]
+    t, y, z, out = _run_layer(w, layer, 0)
+    x = {k: W.to_f64(v) for k, v in t.items() if k != "cu_seqlens"}
+    cu = np.arange(0, w.tokens + 1, w.seqlen)
+    p = oracle_problem(w, layer, cu)
+    yr, zr, _ = O.forward(p, x["u"], x["h"], x["A"], x["B"])
+    assert_close("c2:y", W.to_f64(y), yr, w.dtype)
+    assert_close("c2:z", W.to_f64(z), zr, w.dtype)
+    del yr, zr
+    dur, _, dhr = O.backward_rows(p, x["g"], x["u"], x["h"], x["A"], x["B"])
+    assert_close("c2:du", W.to_f64(out["du"]), dur, w.dtype)
+    assert_close("c2:dh", W.to_f64(out["dh"]), dhr, w.dtype)
+    del dur, dhr
+    dAr, dBr = O.param_grads(p, x["g"], x["u"], x["h"], x["A"], x["B"])
+    assert_close("c2:dA", W.to_f64(out["dA"]), dAr, w.dtype)
+    assert_close("c2:dB", W.to_f64(out["dBW"]), dBr, w.dtype)
