@@ -4,8 +4,9 @@
 One step = one forward and one backward pass of every layer of the workload
 (the hot path: filter generation, causal conv + residual, du, dz/dwh, dA/dB or
 dW, dh) over one batch of seeded synthetic inputs already resident in HBM.
-The default workload is the 150M-scale QKV placement (B=8, T=2048, d=768,
-C=2304, K=3, low-rank r=32, bf16).
+The default workload is the 2B-scale all-linear block (B=4, T=4096, K=3,
+low-rank r=64, bf16; one dynamic conv after each of the QKV (d 2048, C 3072),
+O (2048, 2048), gate+up (2048, 11264) and down (5632, 2048) linears).
 
 Prints ONE JSON line (rank 0).  Under torchrun each rank runs its own replica
 on its own seeded shard (weak scaling, no data-path collective); the timing
@@ -30,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "dyn-conv fwd+bwd tokens/s at 1 B200; achieved HBM GB/s vs ~8 TB/s roofline"
-DEFAULT_CONFIG = "c2_qkv_150m_lowrank"
+DEFAULT_CONFIG = "c4_all_linear_2b_block"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -84,10 +85,52 @@ def layer_flops(w, layer):
     return N * 6 * d * H * K
 
 
-# DRAM bytes (read + write) per launch of a workload's dominant kernel, from one ncu capture of
-# the kernel as it is built now (profiles/<kernel>_<workload>.md); absent where none was taken.
-NCU_TRAFFIC = {("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): 205220608,
-               ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): 280690432}
+# DRAM bytes (read + write) per launch of a workload's dominant kernel, averaged over the launches
+# of one step, from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum, keyed by
+# (kernel, workload) and stored with the SHA-256 of the kernel's source files at capture time: a
+# figure is reported only while those files are unchanged (else traffic is null).
+NCU_TRAFFIC = {}
+KERNEL_SOURCES = {
+    "tc_lowrank_bwd": ("tc_bwd.cu", "tc_common.cuh", "common.cuh"),
+    "tc_lowrank_fwd": ("tc.cu", "tc_common.cuh", "common.cuh"),
+    "tc_headwise_bwd": ("tc_headwise.cu", "tc_common.cuh", "common.cuh"),
+    "tc_headwise_fwd": ("tc_headwise.cu", "tc_common.cuh", "common.cuh"),
+}
+
+
+def kernel_source_sha(name):
+    """SHA-256 (first 16 hex digits) over the source files of a kernel family, or None."""
+    import hashlib
+
+    files = KERNEL_SOURCES.get(name)
+    if not files:
+        return None
+    hsh = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "dynamic_short_convolutions_b200", "csrc", f), "rb") as fh:
+            hsh.update(fh.read())
+    return hsh.hexdigest()[:16]
+
+
+def ncu_traffic(name, workload):
+    rec = NCU_TRAFFIC.get((name, workload))
+    if rec is None:
+        return None
+    nbytes, sha = rec
+    return nbytes if sha == kernel_source_sha(name) else None
+
+
+def kernel_flops(name, w, layer):
+    """Tensor-core FLOPs of ONE launch of a library kernel on one layer call (0 for CUDA-core kernels)."""
+    N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
+    if w.kind == "lowrank":
+        R = w.rank
+        conv = {"tc_lowrank_fwd": 2 * N * R * C * K, "tc_lowrank_bwd": 6 * N * R * C * K}
+    else:
+        R = (C // w.head_dim) * K
+        conv = {}
+    table = {"tc_gen": 2 * N * d * R, "tc_gen_bwd": 4 * N * d * R, **conv}
+    return table.get(name, 0)
 
 
 def kernel_bytes(name, w, layer):
@@ -558,9 +601,22 @@ def run_ours(args, rank, world, local_rank):
     dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
     roof = None
     kernels = {}
+    prof_total = sum(ms for _, ms in prof.values())
     for name, (n_l, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
-        kernels[name] = {"launches": n_l, "ms_total": round(ms, 4), "us_per_launch": round(1e3 * ms / n_l, 2),
-                         "share": round(ms / max(total_ms, 1e-9), 4)}
+        k = {"launches": n_l, "ms_total": round(ms, 4), "us_per_launch": round(1e3 * ms / n_l, 2),
+             "share": round(ms / max(prof_total, 1e-9), 4)}
+        kb = [kernel_bytes(name, w, layer) for layer in w.layers]
+        per_call = len(w.layers) * args.steps / n_l     # launches of this kernel per layer call
+        if all(b is not None for b in kb) and per_call == 1:
+            gbs = sum(kb) * args.steps / (ms / 1e3) / 1e9
+            k["hbm_gbs"] = round(gbs, 1)
+            k["hbm_frac"] = round(gbs / pk["hbm_gbs"], 4)
+        kf = sum(kernel_flops(name, w, layer) for layer in w.layers)
+        if kf and per_call == 1:
+            tf = kf * args.steps / (ms / 1e3) / 1e12
+            k["tensor_tflops"] = round(tf, 1)
+            k["tensor_frac"] = round(tf / pk["bf16_tflops_sustained"], 4)
+        kernels[name] = k
     if dom is not None:
         name, (n_l, ms) = dom
         per_launch_bytes = sum(kernel_bytes(name, w, layer) or 0 for layer in w.layers) / len(w.layers)
@@ -568,8 +624,11 @@ def run_ours(args, rank, world, local_rank):
         achieved = per_launch_bytes / avg_s / 1e9
         roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                "traffic": NCU_TRAFFIC.get((name, w.name)) if args.layout == "token_major" else None,
+                "traffic": ncu_traffic(name, w.name) if args.layout == "token_major" else None,
+                "kernel_source_sha": kernel_source_sha(name),
                 "peak_source": pk_src, "avg_launch_us": round(avg_s * 1e6, 2),
+                "timing": "CUDA events on the launch stream around each launch (this tracer serialises "
+                          "launches, so kernel times sum above the step time, which is taken with it off)",
                 "algorithmic_bytes_per_launch": int(per_launch_bytes)}
     step_bytes = sum(layer_bytes(w, layer) for layer in w.layers)
     step_flops = sum(layer_flops(w, layer) for layer in w.layers)
