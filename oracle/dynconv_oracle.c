@@ -46,6 +46,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <math.h>
 
 typedef struct {
     int64_t kind;        /* 0 = low-rank, 1 = head-wise */
@@ -402,5 +403,54 @@ int orc_decode_step(const orc_problem *p, const double *u, const double *h, cons
         free(z);
         free(x);
     }
+    return bad ? ORC_BAD : ORC_OK;
+}
+
+/*
+ * Rotary position embedding applied to the conv output of the Q and K
+ * channels ("Placement": the conv is applied to Q, K and V before RoPE; the
+ * rotation fused after it).  The pages name RoPE without fixing a variant;
+ * this is the rotation as Su et al. define it ("RoFormer: Enhanced
+ * Transformer with Rotary Position Embedding", section 3.4.2): the
+ * consecutive channel pairs (2i, 2i+1) of each head of hd channels turn by
+ * the angle p * theta_i with theta_i = base^(-2i/hd), p being the token's
+ * position in its sequence or packed document (n - s(n)).  Channels
+ * c >= n_rot are left as they are.
+ *   inverse = 0: (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos)
+ *   inverse = 1: (x0, x1) -> (x0 cos + x1 sin, -x0 sin + x1 cos)   (the adjoint)
+ * x is [nrows, C] for the listed tokens (rows == NULL: every token), rotated
+ * in place; angles and their cosines are computed here in fp64.
+ */
+int orc_rope(const orc_problem *p, int64_t n_rot, int64_t hd, double base, int64_t inverse, int64_t nrows,
+             const int64_t *rows, double *x)
+{
+    if (check(p) != ORC_OK) return ORC_BAD;
+    const int64_t C = p->channels;
+    if (hd < 2 || hd % 2 != 0 || n_rot < 0 || n_rot > C || n_rot % hd != 0 || !(base > 0.0)) return ORC_BAD;
+    int64_t *st = segment_starts(p);
+    int bad = 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t ri = 0; ri < nrows; ++ri) {
+        const int64_t n = rows ? rows[ri] : ri;
+        if (n < 0 || n >= p->n_tokens) {
+            bad = 1;
+            continue;
+        }
+        const double pos = (double)(n - st[n]);
+        for (int64_t c = 0; c < n_rot; c += 2) {
+            const int64_t i = (c % hd) / 2;
+            const double ang = pos * pow(base, -2.0 * (double)i / (double)hd);
+            const double cs = cos(ang), sn = sin(ang);
+            const double x0 = x[ri * C + c], x1 = x[ri * C + c + 1];
+            if (!inverse) {
+                x[ri * C + c] = x0 * cs - x1 * sn;
+                x[ri * C + c + 1] = x0 * sn + x1 * cs;
+            } else {
+                x[ri * C + c] = x0 * cs + x1 * sn;
+                x[ri * C + c + 1] = -x0 * sn + x1 * cs;
+            }
+        }
+    }
+    free(st);
     return bad ? ORC_BAD : ORC_OK;
 }

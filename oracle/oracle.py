@@ -33,7 +33,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp",
-                               "-ffp-contract=off", "-fno-fast-math", _SRC, "-o", tmp])
+                               "-ffp-contract=off", "-fno-fast-math", _SRC, "-o", tmp, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -59,8 +59,10 @@ def _load():
             lib.orc_param_grad_entries.argtypes = [P, dp, dp, dp, dp, dp, ctypes.c_int64, ctypes.c_int64,
                                                    ip, ip, dp]
             lib.orc_decode_step.argtypes = [P, dp, dp, dp, dp, dp, dp]
+            lib.orc_rope.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int64,
+                                     ctypes.c_int64, ip, dp]
             for f in (lib.orc_forward, lib.orc_backward_rows, lib.orc_param_grads, lib.orc_param_grad_entries,
-                      lib.orc_decode_step):
+                      lib.orc_decode_step, lib.orc_rope):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -197,3 +199,19 @@ def decode_step(p: Problem, u, h, A, BW, state):
     if rc != 0:
         raise ValueError("oracle rejected the problem")
     return y, st
+
+
+def rope(p: Problem, x, n_rot: int, head_dim: int, base: float = 10000.0, inverse: bool = False, rows=None):
+    """Rotary position embedding (RoFormer's pairwise rotation) of the listed tokens' rows of x
+    [rows, C]: pairs (2i, 2i+1) of each head_dim-channel head among the first n_rot channels
+    turn by position * base^(-2i/head_dim); inverse=True applies the adjoint.  Returns a copy."""
+    lib = _load()
+    x = np.array(x, dtype=np.float64, copy=True, order="C")
+    rr, rp = _rows(rows)
+    n = p.n_tokens if rr is None else len(rr)
+    assert x.shape == (n, p.channels)
+    s, cu = p._c()
+    rc = lib.orc_rope(ctypes.byref(s), n_rot, head_dim, float(base), int(bool(inverse)), n, rp, _d(x))
+    if rc != 0:
+        raise ValueError("oracle rejected the rotation")
+    return x
