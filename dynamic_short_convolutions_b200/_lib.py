@@ -29,7 +29,7 @@ TOKEN_MAJOR, CHANNEL_FIRST = 0, 1
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
            "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc",
-           "dynconv_decode_step", "dynconv_noalloc_status")
+           "dynconv_decode_step", "dynconv_noalloc_status", "dynconv_query_family")
 
 
 class DynConvError(RuntimeError):
@@ -47,7 +47,9 @@ class dynconv_desc(ctypes.Structure):
                 ("seqlen", ctypes.c_int64), ("d_model", ctypes.c_int64), ("channels", ctypes.c_int64),
                 ("ksize", ctypes.c_int64), ("rank", ctypes.c_int64), ("head_dim", ctypes.c_int64),
                 ("u_row_stride", ctypes.c_int64), ("h_row_stride", ctypes.c_int64),
-                ("deterministic", ctypes.c_int32), ("algo", ctypes.c_int32), ("layout", ctypes.c_int32)]
+                ("deterministic", ctypes.c_int32), ("algo", ctypes.c_int32), ("layout", ctypes.c_int32),
+                ("rope_channels", ctypes.c_int64), ("rope_head_dim", ctypes.c_int64), ("rope_max_pos", ctypes.c_int64),
+                ("rope_cos_sin", ctypes.c_void_p)]
 
 
 _lib = None
@@ -73,6 +75,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_device_status.argtypes = [vp, sz, vp]
     lib.dynconv_fwd_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp]
     lib.dynconv_fwd_noalloc.restype = ctypes.c_int
+    lib.dynconv_query_family.argtypes = [D, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
+    lib.dynconv_query_family.restype = ctypes.c_int
     lib.dynconv_noalloc_status.argtypes = [vp]
     lib.dynconv_noalloc_status.restype = ctypes.c_int
     lib.dynconv_decode_step.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -113,9 +117,13 @@ def _check(status: int):
 
 def make_desc(kind: int, dtype: int, batch: int, seqlen: int, d_model: int, channels: int, ksize: int,
               rank: int = 0, head_dim: int = 0, u_row_stride: int = 0, h_row_stride: int = 0,
-              deterministic: int = 0, algo: int = ALGO_AUTO, layout: int = TOKEN_MAJOR) -> dynconv_desc:
+              deterministic: int = 0, algo: int = ALGO_AUTO, layout: int = TOKEN_MAJOR, rope_channels: int = 0,
+              rope_head_dim: int = 0, rope_table: Optional[torch.Tensor] = None) -> dynconv_desc:
+    """rope_table: device fp32 [max_pos, rope_head_dim] (cos, sin pairs), kept alive by the caller."""
+    rope_max = int(rope_table.shape[0]) if rope_table is not None else 0
+    rope_ptr = ctypes.c_void_p(rope_table.data_ptr()) if rope_table is not None else None
     return dynconv_desc(kind, dtype, batch, seqlen, d_model, channels, ksize, rank, head_dim, u_row_stride,
-                        h_row_stride, deterministic, algo, layout)
+                        h_row_stride, deterministic, algo, layout, rope_channels, rope_head_dim, rope_max, rope_ptr)
 
 
 def dynconv_workspace_bytes(desc: dynconv_desc) -> int:
@@ -161,6 +169,17 @@ def dynconv_decode_step(desc, u, h, A, B_or_W, state, y, ws, stream=None):
 def dynconv_device_status(ws, stream=None) -> int:
     """Synchronises the stream; returns the status (does not raise)."""
     return int(load().dynconv_device_status(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream, ws)))
+
+
+FAMILY_TENSOR_CORE, FAMILY_CUDA_CORE = 1, 2
+FAMILY_NAMES = {FAMILY_TENSOR_CORE: "tensor_core", FAMILY_CUDA_CORE: "cuda_core"}
+
+
+def dynconv_query_family(desc):
+    """(forward family, backward family, reason) for a descriptor; host-only."""
+    f, b = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load().dynconv_query_family(ctypes.byref(desc), ctypes.byref(f), ctypes.byref(b)))
+    return FAMILY_NAMES[f.value], FAMILY_NAMES[b.value], dynconv_last_error()
 
 
 def dynconv_last_error() -> str:

@@ -90,7 +90,31 @@ dynconv_status make_prob(const dynconv_desc* d, Prob* p) {
     p->cu = nullptr;
     p->n_docs = 0;
     p->deterministic = d->deterministic;
+    p->algo = d->algo;
+    p->rope_n = d->rope_channels;
+    p->rope_hd = d->rope_head_dim;
+    p->rope_max = d->rope_max_pos;
+    p->rope_cs = d->rope_cos_sin;
+    if (p->rope_n < 0) { set_error("rope_channels must be >= 0"); return DYNCONV_ERR_INVALID; }
+    if (p->rope_n > 0) {
+        if (p->rope_hd < 2 || p->rope_hd % 2) { set_error("rope_head_dim must be even and >= 2"); return DYNCONV_ERR_INVALID; }
+        if (p->rope_n > p->C || p->rope_n % p->rope_hd) {
+            set_error("rope_channels must be a multiple of rope_head_dim and at most channels");
+            return DYNCONV_ERR_INVALID;
+        }
+        if (p->rope_max < 1) { set_error("rope_max_pos must be >= 1"); return DYNCONV_ERR_INVALID; }
+        if (p->N > 0 && p->batch > 1 && p->seqlen > p->rope_max) {
+            set_error("seqlen %lld exceeds rope_max_pos %lld", (long long)p->seqlen, (long long)p->rope_max);
+            return DYNCONV_ERR_INVALID;
+        }
+    }
     return DYNCONV_OK;
+}
+
+// The RoPE table: a device pointer, 16-byte aligned.
+dynconv_status check_rope(const Prob& p) {
+    if (p.rope_n == 0) return DYNCONV_OK;
+    return check_ptr(p.rope_cs, "rope_cos_sin", true);
 }
 
 bool use_tc(const Prob& p, int algo) {
@@ -132,15 +156,20 @@ dynconv_status forward_common(const dynconv_desc* desc, const int32_t* cu, int64
         return DYNCONV_ERR_UNSUPPORTED;
     }
     if (p.N == 0) return DYNCONV_OK;
+    if (!varlen && p.rope_n > 0 && p.seqlen > p.rope_max) {
+        set_error("seqlen %lld exceeds rope_max_pos %lld", (long long)p.seqlen, (long long)p.rope_max);
+        return DYNCONV_ERR_INVALID;
+    }
     if ((s = check_ptr(u, "u", true)) || (s = check_ptr(h, "h", true)) ||
         (s = check_ptr(A, "A", p.kind == 0)) || (s = check_ptr(BW, p.kind == 0 ? "B" : "W", true)) ||
-        (s = check_ptr(y, "y", true)) || (s = check_ptr(z_save, "z_save", false)))
+        (s = check_ptr(y, "y", true)) || (s = check_ptr(z_save, "z_save", false)) || (s = check_rope(p)))
         return s;
     if ((s = workspace_ok(p, ws, ws_bytes)) != DYNCONV_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
-    if (varlen && (s = cuda_status(launch_check_seqlens(cu, n_docs, p.N, err, st), "cu_seqlens check")))
+    if (varlen && (s = cuda_status(launch_check_seqlens(cu, n_docs, p.N, err, st, p.rope_n > 0 ? p.rope_max : 0),
+                                   "cu_seqlens check")))
         return s;
     cudaError_t e = use_tc(p, desc->algo) ? tc_forward(p, u, h, A, BW, y, z_save, ws, st)
                                           : simt_forward(p, u, h, A, BW, y, z_save, ws, st);
@@ -174,6 +203,9 @@ WsLayout ws_layout(const Prob& p) {
     off = align_up(off + L.tc_bytes, 256);
     L.dec = off;
     if (p.seqlen == 1) off = align_up(off + decode_partial_bytes(p), 256);
+    L.rope = off;      // R^T g for a backward on the CUDA-core kernels (chosen, or forced by desc->algo)
+    if (p.rope_n > 0 && (p.algo == DYNCONV_ALGO_SIMT || !tc_supported_bwd(p)))
+        off = align_up(off + (size_t)p.N * p.C * (p.dtype == 0 ? 4 : 2), 256);
     L.total = off;
     return L;
 }
@@ -229,15 +261,21 @@ dynconv_status dynconv_bwd(const dynconv_desc* desc, const int32_t* cu_seqlens, 
         const size_t nbw = p.kind == 0 ? (size_t)(p.r * p.C * p.K) : (size_t)(p.d * p.R);
         return cuda_status(cudaMemsetAsync(dB_or_dW, 0, sizeof(float) * nbw, st), "memset");
     }
+    if (!cu_seqlens && p.rope_n > 0 && p.seqlen > p.rope_max) {
+        set_error("seqlen %lld exceeds rope_max_pos %lld", (long long)p.seqlen, (long long)p.rope_max);
+        return DYNCONV_ERR_INVALID;
+    }
     if ((s = check_ptr(g, "g", true)) || (s = check_ptr(u, "u", true)) || (s = check_ptr(h, "h", true)) ||
         (s = check_ptr(A, "A", p.kind == 0)) || (s = check_ptr(B_or_W, p.kind == 0 ? "B" : "W", true)) ||
         (s = check_ptr(z_saved, "z_saved", false)) || (s = check_ptr(du, "du", true)) ||
-        (s = check_ptr(dh, "dh", false)))
+        (s = check_ptr(dh, "dh", false)) || (s = check_rope(p)))
         return s;
     if ((s = workspace_ok(p, ws, ws_bytes)) != DYNCONV_OK) return s;
     const WsLayout L = ws_layout(p);
     uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.err);
-    if (cu_seqlens && (s = cuda_status(launch_check_seqlens(cu_seqlens, n_docs, p.N, err, st), "cu_seqlens check")))
+    if (cu_seqlens && (s = cuda_status(launch_check_seqlens(cu_seqlens, n_docs, p.N, err, st,
+                                                            p.rope_n > 0 ? p.rope_max : 0),
+                                       "cu_seqlens check")))
         return s;
     cudaError_t e = (desc->algo != DYNCONV_ALGO_SIMT && tc_supported_bwd(p))
                         ? tc_backward(p, g, u, h, A, B_or_W, z_saved, du, dh, dA, dB_or_dW, ws, st)
@@ -255,6 +293,10 @@ dynconv_status dynconv_decode_step(const dynconv_desc* desc, const void* u, cons
     if (p.seqlen != 1) {
         set_error("dynconv_decode_step takes one new token per sequence: seqlen must be 1");
         return DYNCONV_ERR_INVALID;
+    }
+    if (p.rope_n > 0) {
+        set_error("dynconv_decode_step does not apply RoPE (rope_channels must be 0)");
+        return DYNCONV_ERR_UNSUPPORTED;
     }
     if (p.layout == DYNCONV_CHANNEL_FIRST) {
         // validation already turned [batch, C, 1] with unit channel stride and 16-byte rows into [batch, C]
@@ -284,9 +326,26 @@ dynconv_status dynconv_device_status(void* ws, size_t ws_bytes, void* stream) {
     if (word == 0) return DYNCONV_OK;
     if ((s = cuda_status(cudaMemsetAsync(ws, 0, sizeof(word), st), "clear error word"))) return s;
     if ((s = cuda_status(cudaStreamSynchronize(st), "stream synchronize"))) return s;
-    set_error("device check failed:%s%s", (word & kErrBadSeqlens) ? " malformed cu_seqlens" : "",
-              (word & kErrWaitTimeout) ? " pipeline wait timed out" : "");
+    set_error("device check failed:%s%s%s", (word & kErrBadSeqlens) ? " malformed cu_seqlens" : "",
+              (word & kErrWaitTimeout) ? " pipeline wait timed out" : "",
+              (word & kErrRopePos) ? " a packed document is longer than rope_max_pos" : "");
     return DYNCONV_ERR_DEVICE_CHECK;
+}
+
+dynconv_status dynconv_query_family(const dynconv_desc* desc, int32_t* fwd_family, int32_t* bwd_family) {
+    g_err[0] = 0;
+    Prob p;
+    dynconv_status s = make_prob(desc, &p);
+    if (s != DYNCONV_OK) return s;
+    const char* rf = tc_unsupported_reason(p, false);
+    const char* rb = tc_unsupported_reason(p, true);
+    const bool simt = desc->algo == DYNCONV_ALGO_SIMT;
+    if (fwd_family) *fwd_family = (!simt && !rf) ? DYNCONV_FAMILY_TENSOR_CORE : DYNCONV_FAMILY_CUDA_CORE;
+    if (bwd_family) *bwd_family = (!simt && !rb) ? DYNCONV_FAMILY_TENSOR_CORE : DYNCONV_FAMILY_CUDA_CORE;
+    if (simt) set_error("desc->algo asks for the CUDA-core kernels");
+    else if (rf) set_error("forward and backward on the CUDA-core kernels: %s", rf);
+    else if (rb) set_error("backward on the CUDA-core kernels: %s", rb);
+    return DYNCONV_OK;
 }
 
 const char* dynconv_last_error(void) { return g_err; }
@@ -303,6 +362,6 @@ const char* dynconv_status_string(dynconv_status status) {
     return "unknown status";
 }
 
-int dynconv_version(void) { return 110; }
+int dynconv_version(void) { return 200; }
 
 }  // extern "C"

@@ -97,4 +97,70 @@ __device__ __forceinline__ void seg_bounds(int64_t n, const int32_t* __restrict_
     e = e <= n ? n + 1 : (e > N ? N : e);
 }
 
+// Rotary position embedding of 8 consecutive channels (4 interleaved pairs) of one token, with
+// cs the fp32 table row of its position at the pairs' head-local offset (cos and sin of each pair):
+//   inverse = false: (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos)
+//   inverse = true:  (x0, x1) -> (x0 cos + x1 sin, x1 cos - x0 sin)   (the transpose)
+__device__ __forceinline__ void rope_pairs8(float (&x)[8], const float* __restrict__ cs, bool inverse) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(cs));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(cs) + 1);
+    const float co[4] = {a.x, a.z, b.x, b.z};
+    const float si[4] = {inverse ? -a.y : a.y, inverse ? -a.w : a.w, inverse ? -b.y : b.y, inverse ? -b.w : b.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float x0 = x[2 * q], x1 = x[2 * q + 1];
+        x[2 * q] = fmaf(x0, co[q], -x1 * si[q]);
+        x[2 * q + 1] = fmaf(x0, si[q], x1 * co[q]);
+    }
+}
+
+// The same with the table slice already in registers: a = (cos, sin) of pairs 0, 1; b = of pairs 2, 3.
+__device__ __forceinline__ void rope_pairs8v(float (&x)[8], const float4& a, const float4& b, bool inverse) {
+    const float co[4] = {a.x, a.z, b.x, b.z};
+    const float si[4] = {inverse ? -a.y : a.y, inverse ? -a.w : a.w, inverse ? -b.y : b.y, inverse ? -b.w : b.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float x0 = x[2 * q], x1 = x[2 * q + 1];
+        x[2 * q] = fmaf(x0, co[q], -x1 * si[q]);
+        x[2 * q + 1] = fmaf(x0, si[q], x1 * co[q]);
+    }
+}
+
+// The same on 8 bf16 values packed in a uint4 (rotated in fp32, rounded once back to bf16).
+__device__ __forceinline__ uint4 rope_bf16x8(const uint4& v, const float* __restrict__ cs, bool inverse) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        x[2 * q] = __uint_as_float(w[q] << 16);
+        x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+    rope_pairs8(x, cs, inverse);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        o[q] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// out[n, c] = (R^T or R) x[n, c] for the rotated channels c < rope_n of tokens n = first, first + step, ...
+// (bf16, token-major, 8 channels per thread and step; out has row stride rope_n): the block's threads
+// stride over a token's 8-channel groups.  Positions are clamped below rope_max.
+__device__ __forceinline__ void rope_rows_bf16(const __nv_bfloat16* __restrict__ x, int64_t x_stride,
+                                               __nv_bfloat16* __restrict__ out, int64_t N, int64_t first,
+                                               int64_t step, int rope_n, int rope_hd, int rope_max,
+                                               const float* __restrict__ cs, const int32_t* __restrict__ cu,
+                                               int64_t n_docs, int64_t seqlen, bool inverse) {
+    for (int64_t n = first; n < N; n += step) {
+        int64_t pos = n - seg_start(n, cu, n_docs, seqlen);
+        pos = pos < rope_max ? pos : rope_max - 1;
+        for (int c = 8 * (int)threadIdx.x; c < rope_n; c += 8 * (int)blockDim.x) {
+            const uint4 v = *reinterpret_cast<const uint4*>(x + n * x_stride + c);
+            *reinterpret_cast<uint4*>(out + n * rope_n + c) = rope_bf16x8(v, cs + pos * rope_hd + c % rope_hd, inverse);
+        }
+    }
+}
+
 }  // namespace dynconv

@@ -11,6 +11,7 @@ namespace dynconv {
 enum : uint32_t {
     kErrBadSeqlens = 1u,   // cu_seqlens not 0 ... N, non-decreasing
     kErrWaitTimeout = 2u,  // an mbarrier wait ran out of its iteration limit
+    kErrRopePos = 4u,      // a packed document longer than the RoPE table
 };
 
 // A validated problem: all sizes resolved, strides filled in.
@@ -27,6 +28,10 @@ struct Prob {
     const int32_t* cu;  // device cu_seqlens or nullptr (dense batch)
     int64_t n_docs;
     int deterministic;
+    int algo;           // requested kernel family (dynconv_algo: 0 auto, 1 CUDA cores, 2 tensor cores)
+    // rotary position embedding after the conv (rope_n == 0: none)
+    int64_t rope_n, rope_hd, rope_max;
+    const float* rope_cs;
 };
 
 // Workspace carve-up (byte offsets; every region 256-byte aligned).
@@ -37,6 +42,7 @@ struct WsLayout {
     size_t tc;          // start of the tensor-core path's private region
     size_t tc_bytes;
     size_t dec;         // decode step (seqlen == 1): split-d partial generator rows
+    size_t rope;        // CUDA-core backward with RoPE: R^T g in the storage dtype [N, C]
     size_t total;
 };
 
@@ -47,10 +53,24 @@ inline bool cf_tiles_ok(const Prob& p) {
            p.seqlen < (int64_t(1) << 31);
 }
 
+// Workspace of the low-rank tensor-core path (inside the tensor-core region), byte offsets.
+struct TcBwdLayout {
+    size_t zs, bp, dz, dzb, dbpart, dpart, gr, total;
+    int64_t per_cta, n_items, n_tiles;
+    int pieces, grid, n_dblk, n_split;
+};
+TcBwdLayout tc_bwd_layout(const Prob& p);
+// Workspace of the head-wise tensor-core path (inside the tensor-core region), byte offsets.
+struct TcHwLayout {
+    size_t wh, dwh, dpart, gr, total;
+};
+TcHwLayout tc_hw_layout(const Prob& p);
+
 WsLayout ws_layout(const Prob& p);
 size_t tc_workspace_bytes(const Prob& p);
 bool tc_supported(const Prob& p);      // forward
 bool tc_supported_bwd(const Prob& p);  // backward
+const char* tc_unsupported_reason(const Prob& p, bool bwd);   // nullptr when the tensor cores take it
 
 // Generic CUDA-core kernels (any shape, fp32 or bf16 storage).
 cudaError_t simt_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW,
@@ -83,7 +103,10 @@ size_t decode_partial_bytes(const Prob& p);
 // One decode step for p.batch sequences (p.seqlen == 1), CUDA-core kernels.
 cudaError_t decode_step(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* state,
                         void* y, void* ws, cudaStream_t st);
-cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st);
+cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st,
+                                 int64_t max_doc_len = 0);
+// RoPE on the CUDA-core path: y rotated in place (forward), or out = R^T g (backward), any layout.
+cudaError_t simt_rope(const Prob& p, const void* x, void* out, bool inverse, cudaStream_t st);
 
 // Text for the thread-local error message.
 void set_error(const char* fmt, ...);

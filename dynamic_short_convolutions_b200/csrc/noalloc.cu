@@ -114,6 +114,10 @@ extern "C" DYNCONV_API dynconv_status dynconv_fwd_noalloc(const dynconv_desc* de
     Prob p;
     dynconv_status s = validate_desc(desc, &p);
     if (s != DYNCONV_OK) return s;
+    if (p.rope_n > 0) {
+        set_error("dynconv_fwd_noalloc does not apply RoPE (rope_channels must be 0)");
+        return DYNCONV_ERR_UNSUPPORTED;
+    }
     if (p.kind != 0 || !tc_supported(p)) {
         set_error("dynconv_fwd_noalloc covers the bf16 low-rank tensor-core forward only "
                   "(rank a multiple of 8 up to 64, channels a multiple of 64, d_model a multiple of 8)");

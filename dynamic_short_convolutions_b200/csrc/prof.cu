@@ -30,7 +30,7 @@ int64_t g_launches[kKernelCount];
 const char* kNames[kKernelCount] = {
     "simt_gen", "simt_widen", "simt_conv_fwd", "simt_conv_bwd", "simt_dB", "simt_hTX", "simt_dh",
     "check_seqlens", "tc_gen", "tc_lowrank_fwd", "tc_lowrank_bwd", "tc_gen_bwd", "tc_reduce",
-    "tc_headwise_fwd", "tc_headwise_bwd", "tc_prep", "decode_gen", "decode_conv",
+    "tc_headwise_fwd", "tc_headwise_bwd", "tc_prep", "decode_gen", "decode_conv", "simt_rope",
 };
 
 cudaEvent_t take_event() {

@@ -8,7 +8,7 @@ namespace dynconv {
 enum KernelId {
     kSimtGen = 0, kSimtWiden, kSimtConvFwd, kSimtConvBwd, kSimtDB, kSimtHTX, kSimtDh,
     kCheckSeqlens, kTcGen, kTcLowrankFwd, kTcLowrankBwd, kTcGenBwd, kTcReduce,
-    kTcHeadwiseFwd, kTcHeadwiseBwd, kTcPrep, kDecodeGen, kDecodeConv,
+    kTcHeadwiseFwd, kTcHeadwiseBwd, kTcPrep, kDecodeGen, kDecodeConv, kSimtRope,
     kKernelCount
 };
 

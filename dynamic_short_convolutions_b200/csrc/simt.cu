@@ -203,11 +203,40 @@ __global__ void __launch_bounds__(kThreads) dh_kernel(const float* __restrict__ 
 }
 
 __global__ void check_seqlens_kernel(const int32_t* __restrict__ cu, int64_t n_docs, int64_t N,
-                                     uint32_t* __restrict__ err) {
-    bool bad = false;
-    for (int64_t i = threadIdx.x; i < n_docs; i += blockDim.x) bad |= cu[i + 1] < cu[i];
+                                     uint32_t* __restrict__ err, int64_t max_doc_len) {
+    bool bad = false, longdoc = false;
+    for (int64_t i = threadIdx.x; i < n_docs; i += blockDim.x) {
+        bad |= cu[i + 1] < cu[i];
+        longdoc |= max_doc_len > 0 && (int64_t)cu[i + 1] - (int64_t)cu[i] > max_doc_len;
+    }
     if (threadIdx.x == 0) bad |= (cu[0] != 0) || ((int64_t)cu[n_docs] != N);
     if (bad) atomicOr(err, kErrBadSeqlens);
+    if (longdoc) atomicOr(err, kErrRopePos);
+}
+
+// x -> R x (forward) or R^T x (inverse) on the rotated channels of every token, one block per token:
+// pairs (2i, 2i+1) of each rope_hd-channel head below rope_n turn by the table's angle at the token's
+// position in its sequence / document; the other channels are copied (nothing to do in place).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) rope_kernel(const T* __restrict__ x, Ax ax, T* __restrict__ out, Ax ao,
+                                                         int64_t C, int64_t rope_n, int64_t rope_hd, int64_t rope_max,
+                                                         const float* __restrict__ cs, const int32_t* __restrict__ cu,
+                                                         int64_t n_docs, int64_t seqlen, int inverse, int copy_rest) {
+    const int64_t n = blockIdx.x;
+    int64_t pos = n - seg_start(n, cu, n_docs, seqlen);
+    pos = pos < rope_max ? pos : rope_max - 1;            // in bounds even when the device check fails
+    for (int64_t c = 2 * (int64_t)threadIdx.x; c < C; c += 2 * blockDim.x) {
+        if (c < rope_n) {
+            const float x0 = to_f32(x[ax(n, c)]), x1 = to_f32(x[ax(n, c + 1)]);
+            const float co = cs[pos * rope_hd + (c % rope_hd)];
+            const float si = inverse ? -cs[pos * rope_hd + (c % rope_hd) + 1] : cs[pos * rope_hd + (c % rope_hd) + 1];
+            out[ao(n, c)] = from_f32<T>(fmaf(x0, co, -x1 * si));
+            out[ao(n, c + 1)] = from_f32<T>(fmaf(x0, si, x1 * co));
+        } else if (copy_rest) {
+            out[ao(n, c)] = x[ax(n, c)];
+            if (c + 1 < C) out[ao(n, c + 1)] = x[ax(n, c + 1)];
+        }
+    }
 }
 
 inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
@@ -277,19 +306,42 @@ cudaError_t backward_t(const Prob& p, const void* g, const void* u, const void* 
 
 cudaError_t simt_forward(const Prob& p, const void* u, const void* h, const void* A, const void* BW, void* y,
                          void* z_save, void* ws, cudaStream_t st) {
-    return p.dtype == 0 ? forward_t<float>(p, u, h, A, BW, y, z_save, ws, st)
-                        : forward_t<__nv_bfloat16>(p, u, h, A, BW, y, z_save, ws, st);
+    cudaError_t e = p.dtype == 0 ? forward_t<float>(p, u, h, A, BW, y, z_save, ws, st)
+                                 : forward_t<__nv_bfloat16>(p, u, h, A, BW, y, z_save, ws, st);
+    if (e != cudaSuccess || p.rope_n == 0) return e;
+    return simt_rope(p, y, y, false, st);             // y <- R y, in place
 }
 
 cudaError_t simt_backward(const Prob& p, const void* g, const void* u, const void* h, const void* A,
                           const void* BW, const void* z_saved, void* du, void* dh, float* dA, float* dBW,
                           void* ws, cudaStream_t st) {
+    if (p.rope_n > 0) {                                // the conv backward is fed with R^T g
+        void* gt = static_cast<char*>(ws) + ws_layout(p).rope;
+        cudaError_t e = simt_rope(p, g, gt, true, st);
+        if (e != cudaSuccess) return e;
+        g = gt;
+    }
     return p.dtype == 0 ? backward_t<float>(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, ws, st)
                         : backward_t<__nv_bfloat16>(p, g, u, h, A, BW, z_saved, du, dh, dA, dBW, ws, st);
 }
 
-cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st) {
-    DC_LAUNCH(kCheckSeqlens, st, check_seqlens_kernel<<<1, kThreads, 0, st>>>(cu, n_docs, N, err));
+cudaError_t launch_check_seqlens(const int32_t* cu, int64_t n_docs, int64_t N, uint32_t* err, cudaStream_t st,
+                                 int64_t max_doc_len) {
+    DC_LAUNCH(kCheckSeqlens, st, check_seqlens_kernel<<<1, kThreads, 0, st>>>(cu, n_docs, N, err, max_doc_len));
+    return cudaGetLastError();
+}
+
+cudaError_t simt_rope(const Prob& p, const void* x, void* out, bool inverse, cudaStream_t st) {
+    if (p.N == 0) return cudaSuccess;
+    const bool in_place = x == out;
+    if (p.dtype == 0)
+        DC_LAUNCH(kSimtRope, st, rope_kernel<float><<<(unsigned)p.N, kThreads, 0, st>>>(
+            static_cast<const float*>(x), ax_dense(p), static_cast<float*>(out), ax_dense(p), p.C, p.rope_n,
+            p.rope_hd, p.rope_max, p.rope_cs, p.cu, p.n_docs, p.seqlen, inverse ? 1 : 0, in_place ? 0 : 1));
+    else
+        DC_LAUNCH(kSimtRope, st, rope_kernel<__nv_bfloat16><<<(unsigned)p.N, kThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), ax_dense(p), static_cast<__nv_bfloat16*>(out), ax_dense(p), p.C,
+            p.rope_n, p.rope_hd, p.rope_max, p.rope_cs, p.cu, p.n_docs, p.seqlen, inverse ? 1 : 0, in_place ? 0 : 1));
     return cudaGetLastError();
 }
 

@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             uint32_t it = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
                 for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -102,8 +103,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
                     if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, a.err)) break;
                     uint8_t* st = sm + s * stage_bytes;
                     mbar_arrive_expect_tx(&full[s], stage_bytes);
-                    tma_load_2d(st, &tm_h, &full[s], 64 * kb, (int32_t)(tile * 128));
-                    for (int b = 0; b < a.NB; ++b) tma_load_2d(st + 16384 + b * 8192, &tm_p, &full[s], 64 * b, 64 * kb);
+                    tma_load_2d_hint(st, &tm_h, &full[s], 64 * kb, (int32_t)(tile * 128), stream);
+                    for (int b = 0; b < a.NB; ++b)
+                        tma_load_2d_hint(st + 16384 + b * 8192, &tm_p, &full[s], 64 * b, 64 * kb, keep);
                 }
             }
         }
@@ -220,6 +222,9 @@ struct FwdArgs {
     int64_t per_cta;         // work items per CTA (contiguous run)
     int ksteps;              // 16-wide K steps of the filter MMA: r / 16 rounded up
     int64_t n_tiles, tps;    // token tiles; tiles per sequence (channel-first)
+    const float* rope_cs;    // RoPE table [rope_max][rope_hd] (cos, sin pairs) or nullptr
+    int rope_n, rope_hd;     // rotated channels [0, rope_n), channels per rotary head
+    int rope_max;            // table rows (positions are clamped below it)
 };
 
 constexpr int kFwdStages = 4;
@@ -249,7 +254,31 @@ struct FwdSmem {
 };
 
 // y for 8 channels of one row: wv[j][c] = W_j[t, 8 g + c] (fp32 bits), uj[j] = u[t - j, 8 g .. 8 g + 7].
-// Channel pairs go through the packed fp32 FMA.
+// Channel pairs go through the packed fp32 FMA (conv8f: the fp32 values, before the bf16 rounding).
+template <int K>
+__device__ __forceinline__ void conv8f(const uint32_t (*wv)[8], const uint4* uj, int32_t pos, float (&acc)[8]) {
+    const uint32_t* u0 = reinterpret_cast<const uint32_t*>(&uj[0]);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        acc[2 * p] = bf16_lo(u0[p]);
+        acc[2 * p + 1] = bf16_hi(u0[p]);
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if (j <= pos) {
+            const uint32_t* uu = reinterpret_cast<const uint32_t*>(&uj[j]);
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                ffma2(acc[2 * p], acc[2 * p + 1], __uint_as_float(wv[j][2 * p]), __uint_as_float(wv[j][2 * p + 1]),
+                      bf16_lo(uu[p]), bf16_hi(uu[p]));
+        }
+    }
+}
+__device__ __forceinline__ uint4 pack8f(const float (&acc)[8]) {
+    return make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                      pack_bf16(acc[6], acc[7]));
+}
+
 template <int K>
 __device__ __forceinline__ uint4 conv8(const uint32_t (*wv)[8], const uint4* uj, int32_t pos) {
     float acc[8];
@@ -277,7 +306,7 @@ __device__ __forceinline__ uint4 conv8(const uint32_t (*wv)[8], const uint4* uj,
     return pk;
 }
 
-template <int K, bool CF>
+template <int K, bool CF, bool ROPE>
 __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(const __grid_constant__ CUtensorMap tm_z,
                                                                      const __grid_constant__ CUtensorMap tm_b,
                                                                      const __grid_constant__ CUtensorMap tm_u,
@@ -327,6 +356,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
             for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
@@ -337,7 +367,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * 8192);
                     for (int j = 0; j < K; ++j)
-                        tma_load_2d(sm + S::bres + j * 8192, &tm_b, &bfull, (int32_t)(j * a.C) + c0, 0);
+                        tma_load_2d_hint(sm + S::bres + j * 8192, &tm_b, &bfull, (int32_t)(j * a.C) + c0, 0, keep);
                     ++cc;
                     prev = chunk;
                 }
@@ -345,9 +375,9 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 if (!mbar_wait(&empty[s], ((it / kFwdStages) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* st = sm + s * kFwdStage;
                 mbar_arrive_expect_tx(&full[s], kFwdStage);
-                tma_load_2d(st, &tm_z, &full[s], 0, ta.m0);
-                if (CF) tma_load_2d(st + kZBytes, &tm_u, &full[s], ta.x - 8, ta.y);
-                else tma_load_2d(st + kZBytes, &tm_u, &full[s], ta.x, ta.y - 8);
+                tma_load_2d_hint(st, &tm_z, &full[s], 0, ta.m0, keep);
+                if (CF) tma_load_2d_hint(st + kZBytes, &tm_u, &full[s], ta.x - 8, ta.y, stream);
+                else tma_load_2d_hint(st + kZBytes, &tm_u, &full[s], ta.x, ta.y - 8, stream);
             }
         }
     } else if (warp == 1) {
@@ -384,7 +414,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 const int b = it & 1;
                 if (!mbar_wait(&yfull[b], (it >> 1) & 1, &abort_flag, a.err)) break;
                 const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
-                tma_store_2d(&tm_y, sm + S::ys + b * kYBytes, ta.x, ta.y);
+                tma_store_2d_hint(&tm_y, sm + S::ys + b * kYBytes, ta.x, ta.y, l2_evict_first());
                 tma_store_commit();
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                 mbar_arrive(&yempty[b]);
@@ -401,6 +431,26 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
         for (int64_t item = i0 + team; item < i1; item += FwdEpi<K>::teams, it += FwdEpi<K>::teams) {
             const int64_t tile = item % n_tiles;
             const int s = it % kFwdStages, b = it & 1;
+            const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
+            const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
+            // RoPE: this row's table entries for the thread's channel groups, fetched before the waits
+            // below so that their latency overlaps them (one 32-byte table slice per group)
+            constexpr int kRopeG = ROPE ? kFwdGroups : 1;
+            float4 rcs[kRopeG][2];
+            bool rot = false;
+            if constexpr (ROPE) {
+                const int c0 = (int)(item / n_tiles) * 64 + 8 * kFwdGroups * half;
+                rot = c0 < a.rope_n;         // a chunk lies wholly inside or outside the rotated channels
+                if (rot) {
+                    const float4* t4 = reinterpret_cast<const float4*>(
+                        a.rope_cs + (int64_t)min(pos, a.rope_max - 1) * a.rope_hd + c0 % a.rope_hd);
+#pragma unroll
+                    for (int x = 0; x < kRopeG; ++x) {
+                        rcs[x][0] = __ldg(t4 + 2 * x);
+                        rcs[x][1] = __ldg(t4 + 2 * x + 1);
+                    }
+                }
+            }
             // each warp goes at its own pace (no barrier among the epilogue warps): a failed
             // wait sets the abort flag, and every other wait then gives up too
             const bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, &abort_flag, a.err) &&
@@ -408,14 +458,12 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                             mbar_wait(&yempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err);
             if (!ok) break;
             tc_fence_after();
-            const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
-            const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
             const uint8_t* us = sm + s * kFwdStage + kZBytes;
             uint8_t* ys = sm + S::ys + b * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
             // NG 8-channel groups per pass: every TMEM and shared-memory load first, then one wait,
             // then the arithmetic (channel-first: one group, its 8 K column loads are enough in flight)
-            constexpr int NG = CF ? 1 : FwdEpi<K>::per_pass;
+            constexpr int NG = (CF || ROPE) ? 1 : FwdEpi<K>::per_pass;
 #pragma unroll
             for (int pass = 0; pass < kFwdGroups / NG; ++pass) {
                 const int g0 = kFwdGroups * half + NG * pass;
@@ -434,7 +482,15 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < NG; ++x) {
-                    const uint4 yv = conv8<K>(wv[x], uj[x], pos);
+                    uint4 yv;
+                    if constexpr (ROPE) {
+                        float acc[8];
+                        conv8f<K>(wv[x], uj[x], pos, acc);
+                        if (rot) rope_pairs8v(acc, rcs[NG * pass + x][0], rcs[NG * pass + x][1], false);
+                        yv = pack8f(acc);
+                    } else {
+                        yv = conv8<K>(wv[x], uj[x], pos);
+                    }
                     if (CF) cf_scatter8(ys, kCfYPitch, g0 + x, row, yv);
                     else *reinterpret_cast<uint4*>(ys + sw128_off(row, g0 + x)) = yv;
                 }
@@ -457,25 +513,26 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     }
 }
 
-template <int K, bool CF>
+template <int K, bool CF, bool ROPE>
 cudaError_t launch_lowrank_fwd(const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
                                const CUtensorMap& ty, FwdArgs fa, int64_t items, cudaStream_t st) {
     constexpr uint32_t smem = FwdSmem<K>::total;
     cudaError_t e =
-        cudaFuncSetAttribute(lowrank_fwd_kernel<K, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaFuncSetAttribute(lowrank_fwd_kernel<K, CF, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     fa.per_cta = (items + num_sms() - 1) / num_sms();
     const unsigned grid = (unsigned)((items + fa.per_cta - 1) / fa.per_cta);
-    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K, CF>, dim3(grid), dim3(FwdEpi<K>::threads), smem,
-                                                st, tz, tb, tu, ty, fa));
+    DC_LAUNCH(kTcLowrankFwd, st, e = launch_pdl(lowrank_fwd_kernel<K, CF, ROPE>, dim3(grid), dim3(FwdEpi<K>::threads),
+                                                smem, st, tz, tb, tu, ty, fa));
     return e;
 }
 
 template <int K>
 cudaError_t launch_lowrank_fwd_l(bool cf, const CUtensorMap& tz, const CUtensorMap& tb, const CUtensorMap& tu,
                                  const CUtensorMap& ty, FwdArgs fa, int64_t items, cudaStream_t st) {
-    return cf ? launch_lowrank_fwd<K, true>(tz, tb, tu, ty, fa, items, st)
-              : launch_lowrank_fwd<K, false>(tz, tb, tu, ty, fa, items, st);
+    if (cf) return launch_lowrank_fwd<K, true, false>(tz, tb, tu, ty, fa, items, st);   // RoPE: token-major only
+    return fa.rope_cs ? launch_lowrank_fwd<K, false, true>(tz, tb, tu, ty, fa, items, st)
+                      : launch_lowrank_fwd<K, false, false>(tz, tb, tu, ty, fa, items, st);
 }
 
 }  // namespace
@@ -500,16 +557,7 @@ cudaError_t tc_gen_launch(const void* h, int64_t hs, const void* P, int64_t N, i
     return e;
 }
 
-struct TcBwdLayout {
-    size_t zs, bp, dz, dzb, dbpart, dpart, total;
-    int64_t per_cta, n_items, n_tiles;
-    int pieces, grid, n_dblk, n_split;
-};
-TcBwdLayout tc_bwd_layout(const Prob& p);
-struct TcHwLayout {
-    size_t wh, dwh, dpart, total;
-};
-TcHwLayout tc_hw_layout(const Prob& p);
+
 bool tc_headwise_supported(const Prob& p);
 cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, const void* W, void* y, void* z_save,
                                 char* tcws, uint32_t* err, cudaStream_t st);
@@ -520,23 +568,38 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
                                 const void* B, const void* z_saved, void* du, void* dh, float* dA, float* dB,
                                 char* tcws, uint32_t* err, cudaStream_t st);
 
-bool tc_supported(const Prob& p) {
-    if (p.kind == 1) return tc_headwise_supported(p) && tensor_map_encoder() != nullptr;
-    if (p.dtype != 1 || p.kind != 0) return false;
-    if (p.r % 8 != 0 || p.r > 64) return false;
-    if (p.C % 64 != 0 || p.d % 8 != 0) return false;
-    if (p.K < 1 || p.K > 4) return false;
-    if (p.N >= (int64_t(1) << 31) || p.r * p.C * p.K >= (int64_t(1) << 31)) return false;
-    if (p.layout == 1 && !cf_tiles_ok(p)) return false;
-    return tensor_map_encoder() != nullptr;
+// Why the tensor-core kernels do not take a problem (nullptr: they do).
+const char* tc_unsupported_reason(const Prob& p, bool bwd) {
+    if (p.dtype != 1) return "fp32 storage runs the CUDA-core kernels (no tensor-core rounding of fp32 inputs)";
+    if (tensor_map_encoder() == nullptr) return "the driver entry point cuTensorMapEncodeTiled is unavailable";
+    if (p.kind == 1) {
+        if (p.rope_n > 0 && (p.layout == 1 || p.rope_hd % 8 != 0))
+            return "head-wise RoPE on the tensor cores needs the token-major layout and rope_head_dim % 8 == 0";
+        if (!tc_headwise_supported(p))
+            return "head-wise tensor-core kernels need H*K a multiple of 8 up to 128, d a multiple of 8, and "
+                   "(token-major) head_dim a power of two in [8, 256] with channels a multiple of 256, or "
+                   "(channel-first) seqlen and u_row_stride multiples of 8";
+        return nullptr;
+    }
+    if (p.r % 8 != 0 || p.r > 64) return "low-rank tensor-core kernels need the rank a multiple of 8 up to 64";
+    if (p.C % 64 != 0 || p.d % 8 != 0) return "low-rank tensor-core kernels need channels % 64 == 0 and d % 8 == 0";
+    if (p.K < 1 || p.K > 4) return "ksize outside 1..4";
+    if (p.N >= (int64_t(1) << 31) || p.r * p.C * p.K >= (int64_t(1) << 31)) return "sizes beyond 32-bit indexing";
+    if (p.layout == 1 && !cf_tiles_ok(p))
+        return "channel-first tensor-core kernels need seqlen and u_row_stride multiples of 8";
+    if (p.rope_n > 0 && p.layout == 1) return "RoPE with the channel-first layout runs the CUDA-core kernels";
+    if (p.rope_n > 0 && (p.rope_hd % 8 != 0 || p.rope_n % 64 != 0))
+        return "RoPE on the low-rank tensor-core kernels needs rope_head_dim % 8 == 0 and rope_channels % 64 == 0";
+    // The low-rank backward adds dz over channel chunks with bulk fp32 reductions (order not
+    // fixed), so its deterministic mode runs the CUDA-core kernels; the head-wise backward has
+    // no float atomics (warp-shuffle and fixed-order split reductions).
+    if (bwd && p.deterministic) return "the deterministic low-rank backward runs the CUDA-core kernels";
+    return nullptr;
 }
 
-bool tc_supported_bwd(const Prob& p) {
-    // The low-rank backward reduces dz over channel chunks with fp32 atomics, so its
-    // deterministic mode takes the generic kernels; the head-wise backward has no
-    // atomics (warp-shuffle and fixed-order split reductions).
-    return tc_supported(p) && (p.kind == 1 || !p.deterministic);
-}
+bool tc_supported(const Prob& p) { return tc_unsupported_reason(p, false) == nullptr; }
+
+bool tc_supported_bwd(const Prob& p) { return tc_unsupported_reason(p, true) == nullptr; }
 
 size_t tc_workspace_bytes(const Prob& p) { return p.kind == 1 ? tc_hw_layout(p).total : tc_bwd_layout(p).total; }
 
@@ -572,7 +635,9 @@ cudaError_t tc_forward_scratch(const Prob& p, const void* u, const void* h, cons
         return cudaErrorInvalidValue;
     const int64_t tps = (p.seqlen + 127) / 128;
     const int64_t n_tiles = cf ? p.batch * tps : (p.N + 127) / 128;
-    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16), n_tiles, tps};
+    FwdArgs fa{p.N, p.C, p.seqlen, p.n_docs, p.cu, err, 0, (int)((p.r + 15) / 16), n_tiles, tps,
+               p.rope_n > 0 ? p.rope_cs : nullptr, (int)p.rope_n, p.rope_n > 0 ? (int)p.rope_hd : 1,
+               (int)std::max<int64_t>(1, std::min<int64_t>(p.rope_max, INT32_MAX))};
     const int64_t items = n_tiles * (p.C / 64);
     switch (p.K) {
         case 1: return launch_lowrank_fwd_l<1>(cf, tz, tb, tu, ty, fa, items, st);

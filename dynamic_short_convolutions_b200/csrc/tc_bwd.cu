@@ -56,23 +56,51 @@ constexpr int kThreads = 64 + kEpiThreads;         // warp 0 TMA, warp 1 MMA, wa
 constexpr uint32_t kRowTile = 136 * 128;     // 136-row, 64-column bf16 tile
 constexpr uint32_t kAtom128 = 128 * 128;     // 128-row, 64-column bf16 tile
 
-// Backward set-up in one launch: zero the fp32 dz accumulator (float4 stores) and write
-// the tap-major copy Bp[k, j C + c] = B[k, c K + j] (coalesced over the output index).
+// Backward set-up in one launch.  Blocks [0, r K cb): the tap-major copy Bp[k, j C + c] = B[k, c K + j],
+// block (k K + j) cb + x writing channels 8 (256 x + t) .. + 7 of row (k, j) as one 16-byte store;
+// the remaining blocks zero the fp32 dz accumulator (float4 stores).
+constexpr int kPrepThreads = 256;
+// With RoPE, the last nb_rot blocks also write R^T g of the rotated channels (gr [N, rope_n], bf16),
+// which the backward kernel reads in place of g for those channels.
+struct PrepRope {
+    const __nv_bfloat16* g;
+    __nv_bfloat16* gr;
+    int64_t N, seqlen, n_docs;
+    const int32_t* cu;
+    const float* cs;
+    int rope_n, rope_hd, rope_max, nb_rot;
+};
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat16* __restrict__ Bp, int r, int C,
-                                int K, float4* __restrict__ dz4, int64_t n_dz4) {
+                                int K, int cb, float4* __restrict__ dz4, int64_t n_dz4, PrepRope rp) {
     pdl_trigger();
     pdl_wait();
-    const int64_t n_b = (int64_t)r * C * K;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_dz4 + n_b;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        if (e < n_dz4) {
-            dz4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-            const int o = (int)(e - n_dz4);
-            const int k = o / (C * K), rem = o - k * (C * K), j = rem / C, c = rem - j * C;
-            Bp[o] = B[(int64_t)k * C * K + (int64_t)c * K + j];
-        }
+    if ((int)blockIdx.x >= (int)gridDim.x - rp.nb_rot) {
+        const int b = blockIdx.x - (gridDim.x - rp.nb_rot);
+        rope_rows_bf16(rp.g, C, rp.gr, rp.N, b, rp.nb_rot, rp.rope_n, rp.rope_hd, rp.rope_max, rp.cs, rp.cu,
+                       rp.n_docs, rp.seqlen, true);
+        return;
     }
+    const int nb_bp = r * K * cb;
+    if ((int)blockIdx.x < nb_bp) {
+        const int row = blockIdx.x / cb, x = blockIdx.x - row * cb;
+        const int k = row / K, j = row - k * K;
+        const int c0 = 8 * (kPrepThreads * x + (int)threadIdx.x);
+        if (c0 < C) {
+            const __nv_bfloat16* src = B + (int64_t)k * C * K + (int64_t)c0 * K + j;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t lo = *reinterpret_cast<const uint16_t*>(src + (2 * e) * K);
+                const uint32_t hi = *reinterpret_cast<const uint16_t*>(src + (2 * e + 1) * K);
+                w[e] = lo | (hi << 16);
+            }
+            *reinterpret_cast<uint4*>(Bp + (int64_t)k * C * K + (int64_t)j * C + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        return;
+    }
+    const int64_t nthr = (int64_t)(gridDim.x - rp.nb_rot - nb_bp) * kPrepThreads;
+    for (int64_t e = (int64_t)(blockIdx.x - nb_bp) * kPrepThreads + threadIdx.x; e < n_dz4; e += nthr)
+        dz4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 struct BwdArgs {
@@ -87,25 +115,26 @@ struct BwdArgs {
     uint32_t* err;
     int ksteps;               // 16-wide K steps of the filter MMA: r / 16 rounded up
     int dz_tma;               // 1: dz tiles are added with bulk tensor reductions, else fp32 atomics
+    int rope_chunks;          // channel chunks whose g is read from R^T g (tm_gr): RoPE's rotated channels / 64
 };
 
-constexpr uint32_t kSmemMax = 232448 - 256;         // dynamic shared memory (static barriers aside)
+constexpr uint32_t kSmemTotal = 232448;              // shared memory per CTA (dynamic + static)
 
-// Shared memory of lowrank_bwd_kernel<K, R64> (R64: rank above 32).  Two g | u slots (each
-// held from its TMA load until the du / dw epilogue is done with it) and NZ z slots (held
-// until the dB MMA has read z; three when they fit), one dW tile (K tap atoms of 128 tokens x
-// 64 channels, handed to the MMAs in 128-row blocks of two atoms), the du tile staged for its
-// TMA store, the chunk's Bp slice (rank rounded up to 16 rows per tap), and (K <= 3) the fp32 dz
-// tile staged for its bulk reduction.
-// The dB MMA reads dW in blocks of two atoms; for odd K the last block's second atom is the du
-// staging tile and only feeds accumulator rows that are never read.
+// Shared memory of lowrank_bwd_kernel<K, R64> (R64: rank above 32).  Two g | u slots (each held
+// from its TMA load until the du / dw epilogue is done with it) and NZ z slots (held until the dB
+// MMA has read z; three when they fit), one dW tile (K tap atoms of 128 tokens x 64 channels,
+// handed to the MMAs in 128-row blocks of two atoms), the du tile staged for its TMA store, the
+// chunk's Bp slice (rank rounded up to 16 rows per tap), and one fp32 dz box [128 rows][32 ranks]
+// staged for its bulk reduction (rank 64: the two boxes in turn), when it fits (else dz goes
+// through fp32 atomics).
 template <int K, bool R64>
 struct BwdSmem {
     static constexpr uint32_t gu = 2 * kRowTile;
-    static constexpr uint32_t dzst_bytes = K <= 3 ? (R64 ? 2 * kAtom128 : kAtom128) : 0;
     static constexpr uint32_t bp_tap = R64 ? 8192 : 4096;
-    static constexpr uint32_t fixed = K * kAtom128 + kAtom128 + K * bp_tap + dzst_bytes;
-    static constexpr int NZ = 2 * gu + 3 * kRowTile + fixed + 1024 <= kSmemMax ? 3 : 2;
+    static constexpr uint32_t stat = 512;                                     // static shared memory
+    static constexpr uint32_t base2 = 2 * gu + 2 * kRowTile + K * kAtom128 + kAtom128 + K * bp_tap + 1024 + stat;
+    static constexpr uint32_t dzst_bytes = base2 + kAtom128 <= kSmemTotal ? kAtom128 : 0;
+    static constexpr int NZ = base2 + kRowTile + dzst_bytes <= kSmemTotal ? 3 : 2;
     static constexpr uint32_t z0 = 2 * gu;
     static constexpr uint32_t dw = z0 + NZ * kRowTile;
     static constexpr uint32_t dust = dw + K * kAtom128;
@@ -115,12 +144,13 @@ struct BwdSmem {
 };
 
 // Warp roles of lowrank_bwd_kernel<K>: 0 TMA loads, 1 MMA issue (and TMEM owner), then the
-// du / dw epilogue (GA: BwdEpi<K>::ga warps, each a TMEM lane quarter and a share of the
-// channels), then 4 warps of dz / dB readout (GB: one TMEM lane quarter each).  GA has 8 warps
-// for K <= 3 and 16 for K = 4, where the per-item epilogue work is largest (measured).
+// du / dw epilogue (GA: 16 warps, four per TMEM lane quarter, each a quarter of the channels),
+// then 4 warps of dz / dB readout (GB: one TMEM lane quarter each).  The epilogue is latency-bound
+// (two warps per scheduler leave its TMEM / shared-memory round trips exposed), so it takes 16
+// warps for every K (measured: 3-5 % faster than 8 at the 150M QKV and 2B all-linear shapes).
 template <int K>
 struct BwdEpi {
-    static constexpr int ga = K <= 3 ? 8 : 16;
+    static constexpr int ga = 16;
     static constexpr int groups = 32 / ga;             // 8-channel groups per GA warp
     static constexpr int per_wait = ga <= 8 ? 2 : 1;   // groups per TMEM wait in A1
     static constexpr int gb0 = 2 + ga;
@@ -150,6 +180,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                                                                          const __grid_constant__ CUtensorMap tm_bp,
                                                                          const __grid_constant__ CUtensorMap tm_du,
                                                                          const __grid_constant__ CUtensorMap tm_dz,
+                                                                         const __grid_constant__ CUtensorMap tm_gr,
                                                                          BwdArgs a) {
     using S = BwdSmem<K, R64>;
     constexpr int NBLK = (K + 1) / 2;
@@ -197,6 +228,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         tma_prefetch(&tm_bp);
         tma_prefetch(&tm_du);
         if (a.dz_tma) tma_prefetch(&tm_dz);
+        if (a.rope_chunks) tma_prefetch(&tm_gr);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_base, 512);
@@ -212,6 +244,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
             for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
@@ -220,7 +253,8 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * a.ndz * 128);
                     for (int j = 0; j < K; ++j)
-                        tma_load_2d(sm + S::bp + j * S::bp_tap, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0);
+                        tma_load_2d_hint(sm + S::bp + j * S::bp_tap, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0,
+                                         keep);
                     ++cc;
                     prev = chunk;
                 }
@@ -228,13 +262,14 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 const int zs = it % NZ, gs = it & 1;
                 if (!mbar_wait(&zempty[zs], ((it / NZ) & 1) ^ 1, &abort_flag, a.err)) break;
                 mbar_arrive_expect_tx(&zfull[zs], kRowTile);
-                tma_load_2d(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, ta.m0);
+                tma_load_2d_hint(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, ta.m0, keep);
                 if (!mbar_wait(&guempty[gs], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* gu = sm + gs * S::gu;
                 mbar_arrive_expect_tx(&gufull[gs], S::gu);
-                tma_load_2d(gu, &tm_g, &gufull[gs], ta.x, ta.y);
-                if (CF) tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], ta.x - 8, ta.y);
-                else tma_load_2d(gu + kRowTile, &tm_u, &gufull[gs], ta.x, ta.y - 8);
+                // RoPE: the conv backward of a rotated chunk reads R^T g, written by the set-up kernel
+                tma_load_2d_hint(gu, chunk < a.rope_chunks ? &tm_gr : &tm_g, &gufull[gs], ta.x, ta.y, stream);
+                if (CF) tma_load_2d_hint(gu + kRowTile, &tm_u, &gufull[gs], ta.x - 8, ta.y, stream);
+                else tma_load_2d_hint(gu + kRowTile, &tm_u, &gufull[gs], ta.x, ta.y - 8, stream);
             }
         }
     } else if (warp == 1) {
@@ -416,7 +451,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     break;
                 }
                 if (bb == 0 && leader) {                 // every GA warp has staged its du rows
-                    tma_store_2d(&tm_du, dus, ta.x, ta.y);
+                    tma_store_2d_hint(&tm_du, dus, ta.x, ta.y, l2_evict_first());
                     tma_store_commit();
                 }
 #pragma unroll
@@ -463,50 +498,64 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             tc_fence_after();
             const int32_t m0 = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0;
             const int32_t n = m0 + row;
-            for (int c = 0; c < a.r; c += 16) {
-                uint32_t v[2][8];
-                tmem_ld8(lane_base + kColDz + 64 * b + c, v[0]);
-                if (c + 8 < a.r) tmem_ld8(lane_base + kColDz + 64 * b + c + 8, v[1]);
-                tmem_wait_ld();
-                if (via_tma) {
-                    // fp32 tile [128 rows][32 columns] per 128-byte swizzled box
+            if (via_tma) {
+                // one fp32 box [128 rows][32 ranks] at a time through the staging tile, each added into
+                // the [N, r] buffer by one bulk tensor reduction
+                for (int bx = 0; bx * 32 < a.r; ++bx) {
+                    if (bx > 0) {                       // the previous box's reduction has read the tile
+                        if (leader) tma_store_wait_read_all();
+                        named_bar_any<3, 32 * kGbWarps>(false);
+                    }
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int cc = c + 8 * h;
-                        if (cc < a.r) {
-                            uint8_t* box = dzs + (cc >> 5) * kAtom128;
-                            const int qq = (cc & 31) >> 2;
-                            *reinterpret_cast<uint4*>(box + sw128_off(row, qq)) =
+                    for (int c = 0; c < 32; c += 16) {
+                        uint32_t v[2][8];
+                        tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c, v[0]);
+                        tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c + 8, v[1]);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int qq = (c + 8 * h) >> 2;
+                            *reinterpret_cast<uint4*>(dzs + sw128_off(row, qq)) =
                                 make_uint4(v[h][0], v[h][1], v[h][2], v[h][3]);
-                            *reinterpret_cast<uint4*>(box + sw128_off(row, qq + 1)) =
+                            *reinterpret_cast<uint4*>(dzs + sw128_off(row, qq + 1)) =
                                 make_uint4(v[h][4], v[h][5], v[h][6], v[h][7]);
                         }
                     }
-                } else if (n < a.N) {
-                    float4* dst = reinterpret_cast<float4*>(a.dz_acc + (int64_t)n * a.r + c);
-                    atomicAdd(dst, make_float4(__uint_as_float(v[0][0]), __uint_as_float(v[0][1]),
-                                               __uint_as_float(v[0][2]), __uint_as_float(v[0][3])));
-                    atomicAdd(dst + 1, make_float4(__uint_as_float(v[0][4]), __uint_as_float(v[0][5]),
-                                                   __uint_as_float(v[0][6]), __uint_as_float(v[0][7])));
-                    if (c + 8 < a.r) {
-                        atomicAdd(dst + 2, make_float4(__uint_as_float(v[1][0]), __uint_as_float(v[1][1]),
-                                                       __uint_as_float(v[1][2]), __uint_as_float(v[1][3])));
-                        atomicAdd(dst + 3, make_float4(__uint_as_float(v[1][4]), __uint_as_float(v[1][5]),
-                                                       __uint_as_float(v[1][6]), __uint_as_float(v[1][7])));
+                    if ((bx + 1) * 32 >= a.r) {         // every dz column of this buffer has been read
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&dzempty[b]);
+                    }
+                    fence_async_smem();
+                    named_bar_any<3, 32 * kGbWarps>(false);     // every GB warp has staged its dz rows
+                    if (leader) {
+                        tma_reduce_add_2d_hint(&tm_dz, dzs, bx * 32, m0, l2_evict_last());
+                        tma_store_commit();
                     }
                 }
-            }
-            tc_fence_before();
-            if (via_tma) fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&dzempty[b]);
-            if (via_tma) {
-                named_bar_any<3, 32 * kGbWarps>(false);     // every GB warp has staged its dz rows
-                if (leader) {
-                    for (int bx = 0; bx * 32 < a.r; ++bx)
-                        tma_reduce_add_2d(&tm_dz, dzs + bx * kAtom128, bx * 32, m0);
-                    tma_store_commit();
+            } else {
+                for (int c = 0; c < a.r; c += 16) {
+                    uint32_t v[2][8];
+                    tmem_ld8(lane_base + kColDz + 64 * b + c, v[0]);
+                    if (c + 8 < a.r) tmem_ld8(lane_base + kColDz + 64 * b + c + 8, v[1]);
+                    tmem_wait_ld();
+                    if (n < a.N) {
+                        float4* dst = reinterpret_cast<float4*>(a.dz_acc + (int64_t)n * a.r + c);
+                        atomicAdd(dst, make_float4(__uint_as_float(v[0][0]), __uint_as_float(v[0][1]),
+                                                   __uint_as_float(v[0][2]), __uint_as_float(v[0][3])));
+                        atomicAdd(dst + 1, make_float4(__uint_as_float(v[0][4]), __uint_as_float(v[0][5]),
+                                                       __uint_as_float(v[0][6]), __uint_as_float(v[0][7])));
+                        if (c + 8 < a.r) {
+                            atomicAdd(dst + 2, make_float4(__uint_as_float(v[1][0]), __uint_as_float(v[1][1]),
+                                                           __uint_as_float(v[1][2]), __uint_as_float(v[1][3])));
+                            atomicAdd(dst + 3, make_float4(__uint_as_float(v[1][4]), __uint_as_float(v[1][5]),
+                                                           __uint_as_float(v[1][6]), __uint_as_float(v[1][7])));
+                        }
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dzempty[b]);
             }
             if (last) {                            // the run for this chunk ends: its dB partial
                 // partial [k][m] (m = j * 64 + c): a warp writes 32 consecutive m per k
@@ -561,60 +610,53 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
     }
 }
 
-// After the backward kernel, in one launch: dB[k, c K + j] = the sum of the partials of the runs
-// covering chunk c/64, in run order (one thread per entry), and the fp32 dz accumulator -> bf16
+// After the backward kernel, in one launch.  Blocks [0, n_chunks r): block chunk r + k sums, for
+// each m = j 64 + c (one thread each), the partials of the runs covering the chunk in run order
+// -> dB[k, (64 chunk + c) K + j]; the remaining blocks convert the fp32 dz accumulator to the bf16
 // operand of the generator backward (four values per thread).
 template <int K>
-__global__ void bwd_finish_kernel(const float* __restrict__ part, float* __restrict__ dB, int r, int C, int n_tiles,
-                                  int per_cta, int pieces, const float4* __restrict__ dz4, uint2* __restrict__ dzb,
-                                  int64_t count4) {
+__global__ void __launch_bounds__(64 * K) bwd_finish_kernel(const float* __restrict__ part, float* __restrict__ dB,
+                                                            int r, int C, int n_tiles, int per_cta, int pieces,
+                                                            const float4* __restrict__ dz4, uint2* __restrict__ dzb,
+                                                            int64_t count4) {
     pdl_trigger();
     pdl_wait();
-    const int64_t nb = (int64_t)r * C * K;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nb + count4;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        if (e < nb) {
-            // e runs over (k, chunk, m = j * 64 + c) so that the partial reads are coalesced
-            const int ei = (int)e;
-            const int k = ei / (C * K), rem = ei - k * (C * K), chunk = rem / (64 * K), m = rem - chunk * (64 * K);
-            const int j = m >> 6, c = chunk * 64 + (m & 63);
-            const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
-            const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
-            const float* src = part + ((int64_t)chunk * pieces * r + k) * (64 * K) + m;
-            float acc = 0.f;
-            for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * r * (64 * K)];
-            dB[(int64_t)k * (C * K) + c * K + j] = acc;
-        } else {
-            const int64_t i4 = e - nb;
-            const float4 v = dz4[i4];
-            dzb[i4] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-        }
+    const int n_chunks = C / 64;
+    const int nb = n_chunks * r;
+    if ((int)blockIdx.x < nb) {
+        const int chunk = blockIdx.x / r, k = blockIdx.x - chunk * r;
+        const int m = threadIdx.x, j = m >> 6, c = chunk * 64 + (m & 63);
+        const int first = (int)(((int64_t)chunk * n_tiles) / per_cta);
+        const int lastc = (int)(((int64_t)(chunk + 1) * n_tiles - 1) / per_cta);
+        const float* src = part + ((int64_t)chunk * pieces * r + k) * (64 * K) + m;
+        float acc = 0.f;
+        for (int p = 0; p <= lastc - first; ++p) acc += src[(int64_t)p * r * (64 * K)];
+        dB[(int64_t)k * (C * K) + (int64_t)c * K + j] = acc;
+        return;
+    }
+    const int64_t nthr = (int64_t)(gridDim.x - nb) * blockDim.x;
+    for (int64_t i4 = (int64_t)(blockIdx.x - nb) * blockDim.x + threadIdx.x; i4 < count4; i4 += nthr) {
+        const float4 v = dz4[i4];
+        dzb[i4] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
     }
 }
 
-// out[i] = sum_s part[s][i] for i < count (count a multiple of 4): one warp per 4 outputs, lane l
-// sums splits l, l + 32, ... in order, then a fixed butterfly combines the lanes (deterministic).
+// out[i] = sum_s part[s][i] for i < count (count a multiple of 4): one thread per 4 outputs, summing
+// the splits in order (deterministic).
 __global__ void reduce_splits_kernel(const float* __restrict__ part, float* __restrict__ out, int64_t count,
                                      int n_split) {
     pdl_trigger();
     pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; w * 4 < count; w += warps) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = lane; s < n_split; s += 32) {
-            const float4 v = *reinterpret_cast<const float4*>(part + s * count + w * 4);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-        }
-        if (lane == 0) *reinterpret_cast<float4*>(out + w * 4) = acc;
+    const int64_t i4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i4 * 4 >= count) return;
+    const float4* p = reinterpret_cast<const float4*>(part) + i4;
+    const int64_t stride = count / 4;
+    float4 acc = p[0];
+    for (int s = 1; s < n_split; ++s) {
+        const float4 v = p[s * stride];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    reinterpret_cast<float4*>(out)[i4] = acc;
 }
 
 // =====================================================================================
@@ -698,17 +740,21 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             mbar_arrive_expect_tx(&pfull, G::DB * 128 * XA);
-            for (int xa = 0; xa < XA; ++xa) tma_load_2d(pblk + xa * G::DB * 128, &tm_p, &pfull, 64 * xa, db * G::DB);
+            for (int xa = 0; xa < XA; ++xa)
+                tma_load_2d_hint(pblk + xa * G::DB * 128, &tm_p, &pfull, 64 * xa, db * G::DB, keep);
             uint32_t it = 0;
             for (int64_t tile = t0; tile < t1 && !abort_flag; ++tile, ++it) {
                 const int s = it % NS;
                 if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, &abort_flag, a.err)) break;
                 uint8_t* st = sm + s * G::stage;
                 mbar_arrive_expect_tx(&full[s], G::stage);
-                for (int xa = 0; xa < XA; ++xa) tma_load_2d(st + xa * kAtom128, &tm_x, &full[s], 64 * xa, (int32_t)(tile * 128));
+                for (int xa = 0; xa < XA; ++xa)
+                    tma_load_2d_hint(st + xa * kAtom128, &tm_x, &full[s], 64 * xa, (int32_t)(tile * 128), keep);
                 for (int at = 0; at < 2; ++at)
-                    tma_load_2d(st + kAtom128 * (XA + at), &tm_h, &full[s], db * G::DB + 64 * at, (int32_t)(tile * 128));
+                    tma_load_2d_hint(st + kAtom128 * (XA + at), &tm_h, &full[s], db * G::DB + 64 * at,
+                                     (int32_t)(tile * 128), stream);
             }
         }
     } else if (warp == 1) {
@@ -776,7 +822,8 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                 epi_bar_any<kEpiThreads>(false);          // every epilogue warp has staged its rows
                 if (leader) {
                     for (int at = 0; at < 2; ++at)
-                        tma_store_2d(&tm_dh, dhs + at * kAtom128, db * G::DB + 64 * at, (int32_t)(tile * 128));
+                        tma_store_2d_hint(&tm_dh, dhs + at * kAtom128, db * G::DB + 64 * at, (int32_t)(tile * 128),
+                                          l2_evict_first());
                     tma_store_commit();
                 }
             }
@@ -809,31 +856,27 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
     }
 }
 
-inline unsigned grid_for(int64_t n, int threads = 256) {
-    const int64_t b = (n + threads - 1) / threads;
-    return (unsigned)std::max<int64_t>(1, std::min<int64_t>(b, 148 * 16));
-}
-
 template <int K, bool R64, bool CF>
 cudaError_t launch_bwd_l(const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu, const CUtensorMap& tbp,
-                         const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba, unsigned grid, cudaStream_t st) {
+                         const CUtensorMap& tdu, const CUtensorMap& tdz, const CUtensorMap& tgr, BwdArgs ba,
+                         unsigned grid, cudaStream_t st) {
     using S = BwdSmem<K, R64>;
-    static_assert(S::total <= kSmemMax, "shared memory of lowrank_bwd_kernel");
+    static_assert(S::total + S::stat <= kSmemTotal, "shared memory of lowrank_bwd_kernel");
     if (S::dzst_bytes == 0) ba.dz_tma = 0;
     cudaError_t e = cudaFuncSetAttribute(lowrank_bwd_kernel<K, R64, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::total);
     if (e != cudaSuccess) return e;
     DC_LAUNCH(kTcLowrankBwd, st, e = launch_pdl(lowrank_bwd_kernel<K, R64, CF>, dim3(grid), dim3(BwdEpi<K>::threads),
-                                                S::total, st, tz, tg, tu, tbp, tdu, tdz, ba));
+                                                S::total, st, tz, tg, tu, tbp, tdu, tdz, tgr, ba));
     return e;
 }
 
 template <int K, bool R64>
 cudaError_t launch_bwd(bool cf, const CUtensorMap& tz, const CUtensorMap& tg, const CUtensorMap& tu,
-                       const CUtensorMap& tbp, const CUtensorMap& tdu, const CUtensorMap& tdz, BwdArgs ba,
-                       unsigned grid, cudaStream_t st) {
-    return cf ? launch_bwd_l<K, R64, true>(tz, tg, tu, tbp, tdu, tdz, ba, grid, st)
-              : launch_bwd_l<K, R64, false>(tz, tg, tu, tbp, tdu, tdz, ba, grid, st);
+                       const CUtensorMap& tbp, const CUtensorMap& tdu, const CUtensorMap& tdz, const CUtensorMap& tgr,
+                       BwdArgs ba, unsigned grid, cudaStream_t st) {
+    return cf ? launch_bwd_l<K, R64, true>(tz, tg, tu, tbp, tdu, tdz, tgr, ba, grid, st)
+              : launch_bwd_l<K, R64, false>(tz, tg, tu, tbp, tdu, tdz, tgr, ba, grid, st);
 }
 
 }  // namespace
@@ -872,17 +915,11 @@ cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, con
                                                 tdh, ga));
     }
     if (e != cudaSuccess) return e;
-    DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_splits_kernel, dim3(grid_for(d * R / 4 * 32)), dim3(256), 0, st,
+    DC_LAUNCH(kTcReduce, st, e = launch_pdl(reduce_splits_kernel, dim3((unsigned)((d * R / 4 + 255) / 256)), dim3(256), 0, st,
                                             (const float*)dP_part, dP, d * R, n_split));
     return e;
 }
 
-// Workspace of the tensor-core backward (after the z scratch), byte offsets.
-struct TcBwdLayout {
-    size_t zs, bp, dz, dzb, dbpart, dpart, total;
-    int64_t per_cta, n_items, n_tiles;
-    int pieces, grid, n_dblk, n_split;
-};
 
 static inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -904,6 +941,7 @@ TcBwdLayout tc_bwd_layout(const Prob& p) {
     L.dzb = off;     off = al256(off + (size_t)p.N * p.r * 2);                     // dz bf16
     L.dbpart = off;  off = al256(off + (size_t)n_chunks * L.pieces * 64 * p.K * p.r * 4);
     L.dpart = off;   off = al256(off + (size_t)L.n_split * p.d * p.r * 4);
+    L.gr = off;      off = al256(off + (size_t)p.N * p.rope_n * 2);                // RoPE: R^T g of the rotated channels
     L.total = off;
     return L;
 }
@@ -925,12 +963,22 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     float* dbpart = reinterpret_cast<float*>(tcws + L.dbpart);
     float* dpart = reinterpret_cast<float*>(tcws + L.dpart);
     cudaError_t e;
-    DC_LAUNCH(kTcPrep, st, e = launch_pdl(bwd_prep_kernel, dim3(grid_for(p.N * p.r / 4 + p.r * p.C * p.K)), dim3(256), 0, st,
-        static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, reinterpret_cast<float4*>(dz),
-        p.N * p.r / 4));
+    const int cb = (int)((p.C / 8 + kPrepThreads - 1) / kPrepThreads);     // channel blocks per Bp row
+    __nv_bfloat16* gr = reinterpret_cast<__nv_bfloat16*>(tcws + L.gr);
+    const PrepRope rp{static_cast<const __nv_bfloat16*>(g), gr, p.N, p.seqlen, p.n_docs, p.cu, p.rope_cs,
+                      (int)p.rope_n, p.rope_n > 0 ? (int)p.rope_hd : 1,
+                      (int)std::max<int64_t>(1, std::min<int64_t>(p.rope_max, INT32_MAX)),
+                      p.rope_n > 0 ? (int)std::min<int64_t>(p.N, 148 * 8) : 0};
+    const unsigned prep_grid = (unsigned)(p.r * p.K * cb + std::min<int64_t>((p.N * p.r / 4 + 1023) / 1024, 1024) +
+                                          rp.nb_rot);
+    DC_LAUNCH(kTcPrep, st, e = launch_pdl(bwd_prep_kernel, dim3(prep_grid), dim3(kPrepThreads), 0, st,
+        static_cast<const __nv_bfloat16*>(B), bp, (int)p.r, (int)p.C, (int)p.K, cb, reinterpret_cast<float4*>(dz),
+        p.N * p.r / 4, rp));
     if (e != cudaSuccess) return e;
-    CUtensorMap tz, tg, tu, tbp, tdu, tdz;
+    CUtensorMap tz, tg, tu, tbp, tdu, tdz, tgr;
     std::memset(&tdz, 0, sizeof(tdz));                 // unused unless dz goes through bulk reductions
+    std::memset(&tgr, 0, sizeof(tgr));                 // unused without RoPE
+    if (p.rope_n > 0 && !make_tmap_bf16(&tgr, gr, p.rope_n, p.N, p.rope_n, 64, 136)) return cudaErrorInvalidValue;
     const bool dz_tma = p.r % 32 == 0;
     const bool cf = p.layout == 1;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -944,24 +992,26 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
                make_tmap_bf16(&tdu, du, p.C, p.N, p.C, 64, 128)))
         return cudaErrorInvalidValue;
     BwdArgs ba{p.N, p.C, p.seqlen, p.n_docs, (p.seqlen + 127) / 128, p.cu, (int)p.r, (int)((p.r + 15) / 16 * 16),
-               L.n_tiles, L.n_items, L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dz_tma ? 1 : 0};
+               L.n_tiles, L.n_items, L.per_cta, L.pieces, dz, dbpart, err, (int)((p.r + 15) / 16), dz_tma ? 1 : 0,
+               (int)(p.rope_n / 64)};
     const bool r64 = p.r > 32;
     switch (p.K * 2 + (r64 ? 1 : 0)) {
-        case 2: e = launch_bwd<1, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 3: e = launch_bwd<1, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 4: e = launch_bwd<2, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 5: e = launch_bwd<2, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 6: e = launch_bwd<3, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 7: e = launch_bwd<3, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        case 8: e = launch_bwd<4, false>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
-        default: e = launch_bwd<4, true>(cf, tz, tg, tu, tbp, tdu, tdz, ba, L.grid, st); break;
+        case 2: e = launch_bwd<1, false>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 3: e = launch_bwd<1, true>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 4: e = launch_bwd<2, false>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 5: e = launch_bwd<2, true>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 6: e = launch_bwd<3, false>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 7: e = launch_bwd<3, true>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        case 8: e = launch_bwd<4, false>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
+        default: e = launch_bwd<4, true>(cf, tz, tg, tu, tbp, tdu, tdz, tgr, ba, L.grid, st); break;
     }
     if (e != cudaSuccess) return e;
     switch (p.K) {
 #define DC_FINISH(KK)                                                                                             \
     case KK:                                                                                                       \
-        DC_LAUNCH(kTcReduce, st, e = launch_pdl(bwd_finish_kernel<KK>, dim3(grid_for(p.r * p.C * p.K + p.N * p.r / 4)), \
-                                                dim3(256), 0, st, (const float*)dbpart, dB, (int)p.r, (int)p.C,      \
+        DC_LAUNCH(kTcReduce, st, e = launch_pdl(bwd_finish_kernel<KK>,                                              \
+                                                dim3((unsigned)(p.C / 64 * p.r + std::min<int64_t>((p.N * p.r / 4 + 64 * KK * 4 - 1) / (64 * KK * 4), 1024))), \
+                                                dim3(64 * KK), 0, st, (const float*)dbpart, dB, (int)p.r, (int)p.C,  \
                                                 (int)L.n_tiles, (int)L.per_cta, L.pieces,                            \
                                                 reinterpret_cast<const float4*>(dz), reinterpret_cast<uint2*>(dzb), \
                                                 p.N * p.r / 4));                                                     \

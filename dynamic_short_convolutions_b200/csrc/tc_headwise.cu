@@ -93,7 +93,9 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
                                                           const __nv_bfloat16* __restrict__ wh, int R, int hd,
                                                           int64_t N, int64_t C, int64_t seqlen,
                                                           const int32_t* __restrict__ cu, int64_t n_docs,
-                                                          __nv_bfloat16* __restrict__ y) {
+                                                          __nv_bfloat16* __restrict__ y,
+                                                          const float* __restrict__ rope_cs, int rope_n, int rope_hd,
+                                                          int rope_max) {
     pdl_trigger();
     pdl_wait();
     const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
@@ -113,15 +115,33 @@ __global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* _
         }
         load_taps<K>(wh + n * R + q * K, w[0]);
         if (two) load_taps<K>(wh + (n + 1) * R + q * K, w[1]);
+        int32_t pos[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int32_t m = (int32_t)n + (two ? t : 0);
+            pos[t] = m - seg_start32(m, cu, (int32_t)n_docs, (int32_t)seqlen);
+        }
+        // RoPE: the two tokens' table slices, loaded with the rows above
+        const bool rot = rope_cs && c < rope_n;
+        float4 rc[2][2];
+        if (rot) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const float4* t4 = reinterpret_cast<const float4*>(
+                    rope_cs + (int64_t)min(pos[t], rope_max - 1) * rope_hd + c % rope_hd);
+                rc[t][0] = __ldg(t4);
+                rc[t][1] = __ldg(t4 + 1);
+            }
+        }
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (t == 1 && !two) break;
             const int32_t m = (int32_t)n + t;
-            const int32_t pos = m - seg_start32(m, cu, (int32_t)n_docs, (int32_t)seqlen);
             float acc[8];
             unpack8(ur[K - 1 + t], acc);
 #pragma unroll
-            for (int j = 0; j < K; ++j) axpy8(acc, j <= pos ? w[t][j] : 0.f, ur[K - 1 + t - j]);
+            for (int j = 0; j < K; ++j) axpy8(acc, j <= pos[t] ? w[t][j] : 0.f, ur[K - 1 + t - j]);
+            if (rot) rope_pairs8v(acc, rc[t][0], rc[t][1], false);
             *reinterpret_cast<uint4*>(y + (int64_t)m * C + c) = pack8(acc);
         }
     }
@@ -171,7 +191,8 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
                                                           int64_t N, int64_t C, int64_t seqlen,
                                                           const int32_t* __restrict__ cu, int64_t n_docs,
                                                           __nv_bfloat16* __restrict__ du,
-                                                          __nv_bfloat16* __restrict__ dwh) {
+                                                          __nv_bfloat16* __restrict__ dwh,
+                                                          const __nv_bfloat16* __restrict__ gr, int rope_n) {
     pdl_trigger();
     pdl_wait();
     const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
@@ -180,6 +201,10 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
     const int L = hd >> 3;
     const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
     const int64_t n1 = min(N, n0 + kTokPerBlock);
+    // RoPE: the rotated channels' rows of g come from R^T g (gr [N, rope_n]), written beforehand
+    const bool rot = gr != nullptr && c < rope_n;
+    const __nv_bfloat16* gsrc = rot ? gr : g;
+    const int64_t gstride = rot ? rope_n : C;
     for (int64_t n = n0 + 2 * tl; n < n1; n += 16) {
         const bool two = n + 1 < n1;                     // uniform over the warp
         int32_t sb[2], eb[2];
@@ -192,7 +217,7 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* _
 #pragma unroll
         for (int i = 0; i <= K; ++i) {                   // every load of the pair first
             const int64_t mg = n + i, mu = n - K + 1 + i;
-            gr[i] = mg < N ? *reinterpret_cast<const uint4*>(g + mg * C + c) : make_uint4(0, 0, 0, 0);
+            gr[i] = mg < N ? *reinterpret_cast<const uint4*>(gsrc + mg * gstride + c) : make_uint4(0, 0, 0, 0);
             ur[i] = (mu >= 0 && mu < N) ? *reinterpret_cast<const uint4*>(u + mu * us + c) : make_uint4(0, 0, 0, 0);
             if (mg < N) load_taps<K>(wh + mg * R + q * K, wr[i]);
             else
@@ -429,14 +454,24 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __nv_bfloat16
     }
 }
 
+// gr[n, c] = (R^T g)[n, c] for the rotated channels c < rope_n (bf16, token-major), blocks striding over tokens.
+__global__ void __launch_bounds__(128) rope_rows_kernel(const __nv_bfloat16* __restrict__ g, int64_t C,
+                                                        __nv_bfloat16* __restrict__ gr, int64_t N, int rope_n,
+                                                        int rope_hd, int rope_max, const float* __restrict__ cs,
+                                                        const int32_t* __restrict__ cu, int64_t n_docs,
+                                                        int64_t seqlen) {
+    pdl_trigger();
+    pdl_wait();
+    rope_rows_bf16(g, C, gr, N, blockIdx.x, gridDim.x, rope_n, rope_hd, rope_max, cs, cu, n_docs, seqlen, true);
+}
+
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Rows of the RoPE table as an int (at least 1; positions are clamped below it).
+inline int rope_rows(const Prob& p) { return (int)std::max<int64_t>(1, std::min<int64_t>(p.rope_max, INT32_MAX)); }
 
 }  // namespace
 
-// Workspace of the head-wise tensor-core path (inside the tensor-core region).
-struct TcHwLayout {
-    size_t wh, dwh, dpart, total;
-};
 
 TcHwLayout tc_hw_layout(const Prob& p) {
     TcHwLayout L{};
@@ -444,6 +479,7 @@ TcHwLayout tc_hw_layout(const Prob& p) {
     L.wh = off;     off = al256(off + (size_t)p.N * p.R * 2);
     L.dwh = off;    off = al256(off + (size_t)p.N * p.R * 2);
     L.dpart = off;  off = al256(off + (size_t)gen_bwd_splits(p.N, p.d, (int)p.R) * p.d * p.R * 4);
+    L.gr = off;     off = al256(off + (size_t)p.N * p.rope_n * 2);                  // RoPE: R^T g, rotated channels
     L.total = off;
     return L;
 }
@@ -454,7 +490,8 @@ bool tc_headwise_supported(const Prob& p) {
     if (p.K < 1 || p.K > 4) return false;
     if (p.layout == 1) return cf_tiles_ok(p) && p.H < 65536;
     if (p.hd < 8 || p.hd > 256 || (p.hd & (p.hd - 1)) != 0) return false;
-    return p.C % 256 == 0;
+    // one grid row per kTokPerBlock tokens (grid y up to 65535), 32-bit token indices
+    return p.C % 256 == 0 && p.N < int64_t(kTokPerBlock) * 65535;
 }
 
 // Channel-first: 8 tokens per lane in the forward, 4 in the backward (fewer registers for
@@ -475,13 +512,14 @@ static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, v
     const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
     DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
-        p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
+        p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y), p.rope_n > 0 ? p.rope_cs : nullptr,
+        (int)p.rope_n, p.rope_n > 0 ? (int)p.rope_hd : 1, rope_rows(p)));
     return e;
 }
 
 template <int K>
 static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
-                          cudaStream_t st) {
+                                 const void* gr, cudaStream_t st) {
     cudaError_t e;
     if (p.layout == 1) {
         const int64_t tps = (p.seqlen + 32 * kCfBwdV - 1) / (32 * kCfBwdV);
@@ -496,7 +534,8 @@ static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, co
     DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_kernel<K>, grid, dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
         static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, p.cu, p.n_docs,
-        static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
+        static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh), static_cast<const __nv_bfloat16*>(gr),
+        (int)p.rope_n));
     return e;
 }
 
@@ -527,11 +566,20 @@ cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, co
     }
     void* dwh = tcws + L.dwh;
     cudaError_t e;
+    void* gr = nullptr;
+    if (p.rope_n > 0) {                    // R^T g of the rotated channels, read by the conv backward
+        gr = tcws + L.gr;
+        DC_LAUNCH(kTcPrep, st, e = launch_pdl(rope_rows_kernel, dim3((unsigned)std::min<int64_t>(p.N, 148 * 8)),
+                                              dim3(128), 0, st, static_cast<const __nv_bfloat16*>(g), p.C,
+                                              static_cast<__nv_bfloat16*>(gr), p.N, (int)p.rope_n, (int)p.rope_hd,
+                                              rope_rows(p), p.rope_cs, p.cu, p.n_docs, p.seqlen));
+        if (e != cudaSuccess) return e;
+    }
     switch (p.K) {
-        case 1: e = launch_hw_bwd<1>(p, g, u, wh, du, dwh, st); break;
-        case 2: e = launch_hw_bwd<2>(p, g, u, wh, du, dwh, st); break;
-        case 3: e = launch_hw_bwd<3>(p, g, u, wh, du, dwh, st); break;
-        default: e = launch_hw_bwd<4>(p, g, u, wh, du, dwh, st); break;
+        case 1: e = launch_hw_bwd<1>(p, g, u, wh, du, dwh, gr, st); break;
+        case 2: e = launch_hw_bwd<2>(p, g, u, wh, du, dwh, gr, st); break;
+        case 3: e = launch_hw_bwd<3>(p, g, u, wh, du, dwh, gr, st); break;
+        default: e = launch_hw_bwd<4>(p, g, u, wh, du, dwh, gr, st); break;
     }
     if (e != cudaSuccess) return e;
     return tc_gen_backward(dwh, (int)p.R, h, p.hs, W, p.N, p.d, dh, dW, reinterpret_cast<float*>(tcws + L.dpart),

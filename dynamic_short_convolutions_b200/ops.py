@@ -18,6 +18,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"storage dtype must be bf16 or fp32, got {t.dtype}")
 
 
+def rope_table(max_pos: int, head_dim: int, base: float = 10000.0, device=None) -> torch.Tensor:
+    """The RoPE table the C ABI reads: fp32 [max_pos, head_dim] with entries 2i, 2i+1 of row p
+    the cosine and sine of p * base^(-2i/head_dim) (RoFormer's angles), computed once in fp64."""
+    p = torch.arange(max_pos, dtype=torch.float64).unsqueeze(1)
+    theta = base ** (-torch.arange(0, head_dim, 2, dtype=torch.float64) / head_dim)
+    ang = p * theta
+    return torch.stack((ang.cos(), ang.sin()), dim=-1).reshape(max_pos, head_dim).float().to(device or "cuda")
+
+
 class DynConvPlan:
     """Descriptor + workspace for one problem shape.
 
@@ -30,10 +39,12 @@ class DynConvPlan:
 
     def __init__(self, kind: int, dtype: torch.dtype, batch: int, seqlen: int, d_model: int, channels: int,
                  ksize: int, rank: int = 0, head_dim: int = 0, u_row_stride: int = 0, h_row_stride: int = 0,
-                 deterministic: bool = False, algo: int = L.ALGO_AUTO, device=None, layout: int = L.TOKEN_MAJOR):
+                 deterministic: bool = False, algo: int = L.ALGO_AUTO, device=None, layout: int = L.TOKEN_MAJOR,
+                 rope_channels: int = 0, rope_head_dim: int = 0, rope_table: Optional[torch.Tensor] = None):
+        self.rope_table = rope_table            # kept alive: the descriptor holds its address
         self.desc = L.make_desc(kind, L.BF16 if dtype == torch.bfloat16 else L.F32, batch, seqlen, d_model,
                                 channels, ksize, rank, head_dim, u_row_stride, h_row_stride, int(deterministic),
-                                algo, layout)
+                                algo, layout, rope_channels, rope_head_dim, rope_table)
         nbytes = L.dynconv_workspace_bytes(self.desc)
         if nbytes == 0:
             raise L.DynConvError(1, "invalid descriptor")

@@ -110,7 +110,35 @@ typedef struct {
     int32_t deterministic;  /* 1: every reduction in a fixed order, no float atomics */
     int32_t algo;           /* dynconv_algo */
     int32_t layout;         /* dynconv_layout of u, y, g, du */
+    /* Rotary position embedding fused after the conv (0 channels = none): see "RoPE" below. */
+    int64_t rope_channels;  /* channels [0, rope_channels) of y are rotated (Q and K of a fused QKV) */
+    int64_t rope_head_dim;  /* channels per rotary head: even, divides rope_channels */
+    int64_t rope_max_pos;   /* rows of rope_cos_sin; every position must be below it */
+    const float *rope_cos_sin; /* DEVICE fp32 [rope_max_pos, rope_head_dim]: entries 2i, 2i+1 of row p
+                                  are cos and sin of pair i's angle at position p */
 } dynconv_desc;
+
+/* RoPE.  The pages apply the conv to Q, K and V "before RoPE"; with
+ * rope_channels > 0 the library fuses that rotation into the conv, so that
+ *   dynconv_fwd returns y_rot = R(y), y = u + dynamic causal conv(u), and
+ *   dynconv_bwd takes g = dL/dy_rot and returns the gradients of L through R:
+ *   the conv backward is fed with R^T g.
+ * R rotates the consecutive channel pairs (2i, 2i+1) of each head of
+ * rope_head_dim channels among the first rope_channels, at the token's
+ * position p = n - s(n) in its sequence or packed document, as Su et al.
+ * define the rotation (RoFormer, section 3.4.2):
+ *   (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos),
+ * cos and sin read from rope_cos_sin[p, 2i] and [p, 2i + 1] (the caller's
+ * table; RoFormer's angle p * base^(-2i/rope_head_dim) with base 10000 is the
+ * usual choice, e.g. dynamic_short_convolutions_b200.ops.rope_table).  Channels
+ * from rope_channels on pass unrotated.  Positions are checked against
+ * rope_max_pos: a dense batch needs seqlen <= rope_max_pos
+ * (DYNCONV_ERR_INVALID otherwise); a packed document longer than that raises
+ * the device check (DYNCONV_ERR_DEVICE_CHECK from dynconv_device_status).
+ * The tensor-core kernels take RoPE on the token-major layout with
+ * rope_head_dim a multiple of 8; other shapes run the CUDA-core kernels.
+ * dynconv_decode_step and dynconv_fwd_noalloc reject rope_channels > 0
+ * (DYNCONV_ERR_UNSUPPORTED). */
 
 /* Workspace needed by dynconv_fwd / dynconv_fwd_varlen / dynconv_bwd for this
  * descriptor (one size serves all three).  Returns 0 for an invalid desc.
@@ -225,6 +253,23 @@ DYNCONV_API dynconv_status dynconv_decode_step(const dynconv_desc *desc, const v
  * DYNCONV_ERR_DEVICE_CHECK for a malformed cu_seqlens or a pipeline wait that
  * ran out of its iteration limit, else DYNCONV_OK. */
 DYNCONV_API dynconv_status dynconv_device_status(void *ws, size_t ws_bytes, void *stream);
+
+/* Kernel families (see dynconv_query_family). */
+typedef enum { DYNCONV_FAMILY_TENSOR_CORE = 1, DYNCONV_FAMILY_CUDA_CORE = 2 } dynconv_family;
+
+/* Which kernel family dynconv_fwd / dynconv_fwd_varlen (*fwd_family) and
+ * dynconv_bwd (*bwd_family) run for this descriptor (either pointer may be
+ * NULL): DYNCONV_FAMILY_TENSOR_CORE (tcgen05/TMA kernels) or
+ * DYNCONV_FAMILY_CUDA_CORE (the generic kernels).  With DYNCONV_ALGO_AUTO a
+ * descriptor falls to the CUDA-core kernels for fp32 storage, shapes outside
+ * the tensor-core kernels' coverage (low-rank rank above 64 or not a multiple
+ * of 8, channels not a multiple of 64, ...) and, backward only, the
+ * deterministic low-rank mode; dynconv_last_error() then names the reason
+ * (else it is "").  Host-only: no device work, no allocation.
+ * Returns DYNCONV_ERR_INVALID / _UNSUPPORTED for a descriptor that the entry
+ * points would reject. */
+DYNCONV_API dynconv_status dynconv_query_family(const dynconv_desc *desc, int32_t *fwd_family,
+                                                int32_t *bwd_family);
 
 /* Thread-local text of the last failure in this thread ("" if none). */
 DYNCONV_API const char *dynconv_last_error(void);

@@ -215,3 +215,20 @@ def test_argument_errors():
     cu2 = torch.tensor([0, 40, 63], dtype=torch.int32, device="cuda")   # does not end at N
     L.dynconv_fwd_varlen(vdesc, cu2, u, h, A, B, y, None, ws)
     assert L.dynconv_device_status(ws) == 5
+
+
+def test_query_family_names_the_fallbacks():
+    """On the GPU the tensor-core kernels take the workload shapes; the deterministic
+    low-rank backward, ranks above 64 and fp32 storage are reported as CUDA-core runs."""
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    q = L.dynconv_query_family
+    assert q(L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 3, 32))[:2] == ("tensor_core", "tensor_core")
+    assert q(L.make_desc(L.HEADWISE, L.BF16, 4, 4096, 2048, 3072, 4, head_dim=128))[:2] == \
+        ("tensor_core", "tensor_core")
+    f, b, why = q(L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 3, 32, deterministic=1))
+    assert (f, b) == ("tensor_core", "cuda_core") and "deterministic" in why
+    f, b, why = q(L.make_desc(L.LOWRANK, L.BF16, 1, 256, 256, 256, 3, 128))
+    assert (f, b) == ("cuda_core", "cuda_core") and "rank" in why
+    f, b, why = q(L.make_desc(L.LOWRANK, L.F32, 2, 128, 64, 64, 3, 4))
+    assert (f, b) == ("cuda_core", "cuda_core") and "fp32" in why

@@ -90,3 +90,22 @@ def test_channel_first_descriptor_validation():
     assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 16, 64, 64, 3, 8, layout=2)) == 0
     # token-major keeps its 16-byte row-stride rule
     assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 2, 16, 64, 64, 3, 8, u_row_stride=65)) == 0
+
+
+def test_query_family_host_only():
+    """dynconv_query_family answers without device work: a valid descriptor gets a family
+    for each pass, an invalid one its validation status."""
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    if not os.path.exists(LIB):
+        pytest.skip("library not built")
+    fwd, bwd, _ = L.dynconv_query_family(L.make_desc(L.LOWRANK, L.BF16, 8, 2048, 768, 2304, 3, 32))
+    assert fwd in ("tensor_core", "cuda_core") and bwd in ("tensor_core", "cuda_core")
+    fwd, bwd, why = L.dynconv_query_family(L.make_desc(L.LOWRANK, L.F32, 2, 128, 64, 64, 3, 4))
+    assert (fwd, bwd) == ("cuda_core", "cuda_core") and why
+    fwd, bwd, why = L.dynconv_query_family(L.make_desc(L.LOWRANK, L.BF16, 1, 64, 64, 64, 3, 16,
+                                                       algo=L.ALGO_SIMT))
+    assert (fwd, bwd) == ("cuda_core", "cuda_core") and "CUDA-core" in why
+    with pytest.raises(L.DynConvError) as e:
+        L.dynconv_query_family(L.make_desc(L.LOWRANK, L.BF16, 1, 64, 64, 64, 5, 16))
+    assert e.value.status == 2
