@@ -120,12 +120,6 @@ def ncu_traffic(name, workload):
     return nbytes if sha == kernel_source_sha(name) else None
 
 
-# RoPE fused after the conv on the QKV placement: (rotated channels = Q and K, rotary head dim).
-# 150M: 12 heads of 64 for each of Q, K, V; 2B GQA: Q 16 heads, K 4 and V 4 heads of 128.
-ROPE_QKV = {"c2_qkv_150m_lowrank": (1536, 64), "c3_qkv_2b_headwise_gqa": (2560, 128),
-            "c4_all_linear_2b_block": (2560, 128)}
-
-
 def kernel_flops(name, w, layer):
     """Tensor-core FLOPs of ONE launch of a library kernel on one layer call (0 for CUDA-core kernels)."""
     N, d, C, K = w.tokens, layer.d_model, layer.channels, w.ksize
@@ -499,7 +493,7 @@ def run_ours(args, rank, world, local_rank):
         t = W.make_inputs(w, layer, li, device=dev)
         batch, seqlen = (1, w.tokens) if w.varlen else (w.batch, w.seqlen)
         cf = args.layout == "channel_first"
-        rope = ROPE_QKV.get(w.name) if args.rope and layer.name == "qkv" else None
+        rope = W.ROPE_QKV.get(w.name) if args.rope and layer.name == "qkv" else None
         table = ops.rope_table(max(seqlen, 1), rope[1], device=dev) if rope else None
         plan = ops.DynConvPlan(kind, dt, batch, seqlen, layer.d_model, layer.channels, w.ksize, w.rank,
                                w.head_dim, algo=args.algo, device=dev,
@@ -661,8 +655,8 @@ def run_ours(args, rank, world, local_rank):
                        "varlen": w.varlen, "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (256 MiB write, outside the step events)",
                        "algo": {0: "auto", 1: "simt", 2: "tc"}[args.algo], "layout": args.layout,
-                       "rope": ({"channels": ROPE_QKV[w.name][0], "head_dim": ROPE_QKV[w.name][1], "layers": ["qkv"]}
-                                if args.rope and w.name in ROPE_QKV else None),
+                       "rope": ({"channels": W.ROPE_QKV[w.name][0], "head_dim": W.ROPE_QKV[w.name][1],
+                                 "layers": ["qkv"]} if args.rope and w.name in W.ROPE_QKV else None),
                        "kernel_family": {"fwd": fam[0], "bwd": fam[1], "note": fam[2]}},
             "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),

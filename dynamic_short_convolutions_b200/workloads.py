@@ -175,6 +175,11 @@ def _cfg() -> Dict[str, Workload]:
 
 
 CONFIGS: Dict[str, Workload] = _cfg()
+
+# RoPE fused after the conv of the QKV placement: (rotated channels = Q and K, rotary head dim).
+# 150M: 12 heads of 64 for each of Q, K, V; 2B GQA: Q 16 heads, K 4 and V 4 heads of 128.
+ROPE_QKV = {"c2_qkv_150m_lowrank": (1536, 64), "c3_qkv_2b_headwise_gqa": (2560, 128),
+            "c4_all_linear_2b_block": (2560, 128)}
 CONFIG_ORDER = list(CONFIGS)
 
 
