@@ -89,7 +89,12 @@ def layer_flops(w, layer):
 # of one step, from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum, keyed by
 # (kernel, workload) and stored with the SHA-256 of the kernel's source files at capture time: a
 # figure is reported only while those files are unchanged (else traffic is null).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("tc_lowrank_bwd", "c4_all_linear_2b_block"): (550702773, "c703e0499eb26495"),
+    ("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): (196987392, "c703e0499eb26495"),
+    ("tc_lowrank_bwd", "c5_varlen_packed"): (2186995669, "c703e0499eb26495"),
+    ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): (277365077, "7dbc4f07b10b5f1e"),
+}
 KERNEL_SOURCES = {
     "tc_lowrank_bwd": ("tc_bwd.cu", "tc_common.cuh", "common.cuh"),
     "tc_lowrank_fwd": ("tc.cu", "tc_common.cuh", "common.cuh"),
