@@ -399,8 +399,10 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                 if (!mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(sm + s * kFwdStage);
-                for (int k = 0; k < a.ksteps; ++k)
-                    umma_bf16(tbase + b * 256, kmajor_desc(st, k), mnmajor_desc(b0, 8192, 16 * k), idesc, k != 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)      // ksteps = r / 16 rounded up, at most 4
+                    if (k < a.ksteps)
+                        umma_bf16(tbase + b * 256, kmajor_desc(st, k), mnmajor_desc(b0, 8192, 16 * k), idesc, k != 0);
                 umma_commit(&tfull[b]);
                 umma_commit(&empty[s]);
                 if (last) umma_commit(&bempty);

@@ -37,6 +37,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -158,10 +159,10 @@ struct BwdEpi {
 };
 constexpr int kGbWarps = 4, kGa0 = 2;
 
-// dB orientation.  A tcgen05.mma of M = 128, K = 16 costs about the same for every N up to 128
-// (measured on the B200: ~60 ns, N = 256 ~71 ns), so the instruction count sets the tensor time.
-// K <= 3: dB[r][(j, c)] += z^T dW, one chain of 8 MMAs (N = 64 K, K = 128 tokens; A = z^T with the
-// r index on the TMEM lanes, rows r .. 127 unused).  K = 4: dB^T[(j, c)][r] += dW^T z in 128-row
+// dB orientation.  A tcgen05.mma of M = 128, K = 16 issued back to back takes ~28 ns at N = 64,
+// ~36 ns at N = 128, ~52 ns at N = 192 and ~70 ns at N = 256 on the B200 (M = 64 costs the same
+// as M = 128), so fewer, wider MMAs are cheaper.  K <= 3: dB[r][(j, c)] += z^T dW, one chain of
+// 8 MMAs (N = 64 K, K = 128 tokens; A = z^T with the r index on the TMEM lanes, rows r .. 127 unused).  K = 4: dB^T[(j, c)][r] += dW^T z in 128-row
 // blocks of two taps, 16 MMAs (N = 64 K = 256 would not leave TMEM for dz).
 template <int K>
 struct BwdCols {
@@ -282,17 +283,32 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
             uint32_t cc = 0;          // B loads consumed
             uint32_t m = 0;           // chunks whose dB accumulation has started
-            // Filter MMA of item `it`: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows in).
+            // Filter MMAs: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows into the z slot),
+            // KS 16-wide steps over the rank, unrolled: this thread shares its scheduler with busy
+            // epilogue warps, and a loop with a run-time trip count per tap cost ~2.5x the issue
+            // time of the unrolled form.
+            auto filter_mmas = [&](auto ks, uint32_t z0) {
+                constexpr int KS = decltype(ks)::value;
+#pragma unroll
+                for (int j = 0; j < K; ++j)
+#pragma unroll
+                    for (int k = 0; k < KS; ++k)
+                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k),
+                                  mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k), idesc_w, k != 0);
+            };
             auto mma1 = [&](uint32_t it) -> bool {
                 const int zs = it % NZ;
                 if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) return false;
                 tc_fence_after();
                 const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
-#pragma unroll
-                for (int j = 0; j < K; ++j)
-                    for (int k = 0; k < a.ksteps; ++k)
-                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k),
-                                  mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k), idesc_w, k != 0);
+                // ksteps = ceil(r / 16): 3 or 4 when r > 32, else 1 or 2
+                if constexpr (R64) {
+                    if (a.ksteps == 4) filter_mmas(std::integral_constant<int, 4>{}, z0);
+                    else filter_mmas(std::integral_constant<int, 3>{}, z0);
+                } else {
+                    if (a.ksteps == 2) filter_mmas(std::integral_constant<int, 2>{}, z0);
+                    else filter_mmas(std::integral_constant<int, 1>{}, z0);
+                }
                 umma_commit(&wfull);
                 return true;
             };
@@ -772,11 +788,15 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
                 if (want_dh) {
                     if (!mbar_wait(&hempty, (it & 1) ^ 1, &abort_flag, a.err)) break;
                     tc_fence_after();
-                    for (int k = 0; k < a.ksteps; ++k)
-                        umma_bf16(tbase, kmajor_desc(x0 + (k >> 2) * kAtom128, k & 3),
-                                  kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3), idesc_dh, k != 0);
+                    // dh = X . P^T: ksteps (R / 16 rounded up, at most 8) 16-wide steps over R, unrolled
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        if (k < a.ksteps)
+                            umma_bf16(tbase, kmajor_desc(x0 + (k >> 2) * kAtom128, k & 3),
+                                      kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3), idesc_dh, k != 0);
                     umma_commit(&hfull);
                 }
+#pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     umma_bf16(tbase + G::col_dp, mnmajor_desc(h0, kAtom128, 16 * ks), mnmajor_desc(x0, kAtom128, 16 * ks),
                               idesc_dp, !(tile == t0 && ks == 0));
