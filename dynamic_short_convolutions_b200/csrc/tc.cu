@@ -359,8 +359,9 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
-                const int64_t chunk = item / n_tiles, tile = item % n_tiles;
+            ItemPos ipos(i0, n_tiles);
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it, ipos.next()) {
+                const int64_t chunk = ipos.chunk, tile = ipos.tile;
                 const int32_t c0 = (int32_t)(chunk * 64);
                 const TileAt ta = tile_at<CF>(tile, c0, a.tps, a.seqlen, a.C);
                 if (chunk != prev) {
@@ -386,9 +387,10 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             const uint32_t b0 = smem_u32(sm + S::bres);
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
-                const int64_t chunk = item / n_tiles;
-                const bool last = (item + 1 == i1) || ((item + 1) / n_tiles != chunk);
+            ItemPos ipos(i0, n_tiles);
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it, ipos.next()) {
+                const int64_t chunk = ipos.chunk;
+                const bool last = (item + 1 == i1) || ipos.last_of_chunk();
                 if (chunk != prev) {
                     if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
                     ++cc;
@@ -411,8 +413,9 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     } else if (warp == 2) {
         if (lane == 0) {
             uint32_t it = 0;
-            for (int64_t item = i0; item < i1; ++item, ++it) {
-                const int64_t chunk = item / n_tiles, tile = item % n_tiles;
+            ItemPos ipos(i0, n_tiles);
+            for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
+                const int64_t chunk = ipos.chunk, tile = ipos.tile;
                 const int b = it & 1;
                 if (!mbar_wait(&yfull[b], (it >> 1) & 1, &abort_flag, a.err)) break;
                 const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
@@ -429,9 +432,12 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
         const int team = (warp - 3) / FwdEpi<K>::team_warps;
         const int half = ((warp - 3) % FwdEpi<K>::team_warps) >> 2;   // channel groups kFwdGroups*half ..
         const int row = q * 32 + lane;
+        static_assert(FwdEpi<K>::teams == 2, "each team steps its item position twice per item");
         uint32_t it = team;
-        for (int64_t item = i0 + team; item < i1; item += FwdEpi<K>::teams, it += FwdEpi<K>::teams) {
-            const int64_t tile = item % n_tiles;
+        ItemPos ipos(i0 + team, n_tiles);
+        for (int64_t item = i0 + team; item < i1;
+             item += FwdEpi<K>::teams, it += FwdEpi<K>::teams, ipos.next(), ipos.next()) {
+            const int64_t tile = ipos.tile;
             const int s = it % kFwdStages, b = it & 1;
             const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
             const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
@@ -441,7 +447,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             float4 rcs[kRopeG][2];
             bool rot = false;
             if constexpr (ROPE) {
-                const int c0 = (int)(item / n_tiles) * 64 + 8 * kFwdGroups * half;
+                const int c0 = (int)ipos.chunk * 64 + 8 * kFwdGroups * half;
                 rot = c0 < a.rope_n;         // a chunk lies wholly inside or outside the rotated channels
                 if (rot) {
                     const float4* t4 = reinterpret_cast<const float4*>(

@@ -241,15 +241,15 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
     const uint32_t tbase = tmem_base;
     pdl_trigger();
     pdl_wait();
-    auto chunk_of = [&](int64_t item) { return item / a.n_tiles; };
 
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             int64_t prev = -1;
             uint32_t cc = 0, it = 0;
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it) {
-                const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
+            ItemPos ipos(i0, a.n_tiles);
+            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it, ipos.next()) {
+                const int64_t chunk = ipos.chunk, tile = ipos.tile;
                 if (chunk != prev) {
                     if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
                     mbar_arrive_expect_tx(&bfull, K * a.ndz * 128);
@@ -317,11 +317,11 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 cc = 1;
                 ok = mma1(0);
             }
-            for (uint32_t it = 0; ok && it < nit && !abort_flag; ++it) {
-                const int64_t item = i0 + it, chunk = chunk_of(item);
-                const bool first = it == 0 || chunk_of(item - 1) != chunk;
+            ItemPos ipos(i0, a.n_tiles);
+            for (uint32_t it = 0; ok && it < nit && !abort_flag; ++it, ipos.next()) {
+                const bool first = it == 0 || ipos.tile == 0;
                 const bool has_next = it + 1 < nit;
-                const bool next_same = has_next && chunk_of(item + 1) == chunk;
+                const bool next_same = has_next && !ipos.last_of_chunk();
                 const int zs = it % NZ, b = it & 1;
                 if (next_same) {          // the next filter MMA as soon as Wd has been read
                     if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
@@ -388,8 +388,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         uint8_t* dus = sm + S::dust;
         uint8_t* dws = sm + S::dw;
         uint32_t it = 0;
-        for (int64_t item = i0; item < i1; ++item, ++it) {
-            const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
+        ItemPos ipos(i0, a.n_tiles);
+        for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
+            const int64_t chunk = ipos.chunk, tile = ipos.tile;
             const int gs = it & 1;
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
                       mbar_wait(&gufull[gs], (it >> 1) & 1, &abort_flag, a.err);
@@ -456,17 +457,24 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty);
-            // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap), block
-            // by block (taps 2 bb, 2 bb + 1), each once the MMAs that last read it have finished
+            // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap).  K <= 3:
+            // every tap in one pass (the dB MMA reads every tap, so the blocks are freed together, and
+            // each pass costs a barrier and an async-proxy fence); K = 4: block by block (taps 2 bb,
+            // 2 bb + 1), each once the MMAs that last read it have finished.
+            constexpr int kPasses = kDbt ? 1 : NBLK;
             bool quit = false;       // uniform over the GA warps
 #pragma unroll
-            for (int bb = 0; bb < NBLK; ++bb) {
-                ok = mbar_wait(&dwfree[bb], (it & 1) ^ 1, &abort_flag, a.err);
+            for (int ps = 0; ps < kPasses; ++ps) {
+                const int blk0 = kDbt ? 0 : ps, blk1 = kDbt ? NBLK : ps + 1;
+                ok = true;
+#pragma unroll
+                for (int bb = blk0; bb < blk1; ++bb)
+                    ok = ok && mbar_wait(&dwfree[bb], (it & 1) ^ 1, &abort_flag, a.err);
                 if (named_bar_any<2, 32 * kGaWarps>(!ok)) {
                     quit = true;
                     break;
                 }
-                if (bb == 0 && leader) {                 // every GA warp has staged its du rows
+                if (ps == 0 && leader) {                 // every GA warp has staged its du rows
                     tma_store_2d_hint(&tm_du, dus, ta.x, ta.y, l2_evict_first());
                     tma_store_commit();
                 }
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 for (int i = 0; i < kGaGroups; ++i) {
                     const int g8 = kGaGroups * half + i;
 #pragma unroll
-                    for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j) {
+                    for (int j = 2 * blk0; j < 2 * blk1 && j < K; ++j) {
                         const uint4 uu = CF ? cf_gather8(ut, kCfPitch, g8, row + 8 - j)
                                             : *reinterpret_cast<const uint4*>(ut + sw128_off(row + 8 - j, g8));
                         const bool v = j <= pos;
@@ -488,7 +496,10 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 }
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dwready[bb]);
+                if (lane == 0) {
+#pragma unroll
+                    for (int bb = blk0; bb < blk1; ++bb) mbar_arrive(&dwready[bb]);
+                }
             }
             if (quit) break;
             __syncwarp();
@@ -504,9 +515,10 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         uint8_t* dzs = sm + S::dzst;
         const bool via_tma = S::dzst_bytes > 0 && a.dz_tma;
         uint32_t it = 0;
-        for (int64_t item = i0; item < i1; ++item, ++it) {
-            const int64_t chunk = chunk_of(item), tile = item % a.n_tiles;
-            const bool last = (item + 1 == i1) || (chunk_of(item + 1) != chunk);
+        ItemPos ipos(i0, a.n_tiles);
+        for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
+            const int64_t chunk = ipos.chunk, tile = ipos.tile;
+            const bool last = (item + 1 == i1) || ipos.last_of_chunk();
             const int b = it & 1;
             const bool ok = mbar_wait(&dzfull[b], (it >> 1) & 1, &abort_flag, a.err);
             if (via_tma && leader) tma_store_wait_read_all();   // the previous reduction has read the tile

@@ -246,6 +246,20 @@ __device__ __forceinline__ void cf_scatter8(uint8_t* tile, uint32_t pitch, int c
 //   token-major   [N, C]:                 x = c0, y = m0
 //   channel-first [batch * C, seqlen]:    x = t0 (first token within the sequence), y = b C + c0,
 //                 with tps = tiles per sequence, so a tile never spans two sequences
+// Position (channel chunk, token tile) of a work item in a CTA's contiguous, chunk-major run,
+// stepped item by item (no 64-bit division per item).
+struct ItemPos {
+    int64_t chunk, tile, n_tiles;
+    __device__ __forceinline__ ItemPos(int64_t item, int64_t nt) : chunk(item / nt), tile(item - (item / nt) * nt), n_tiles(nt) {}
+    __device__ __forceinline__ void next() {
+        if (++tile == n_tiles) {
+            tile = 0;
+            ++chunk;
+        }
+    }
+    __device__ __forceinline__ bool last_of_chunk() const { return tile + 1 == n_tiles; }
+};
+
 struct TileAt {
     int32_t m0, x, y;
 };
