@@ -144,9 +144,9 @@ struct BwdSmem {
     static constexpr uint32_t total = dzst + dzst_bytes + 1024;
 };
 
-// Warp roles of lowrank_bwd_kernel<K>: 0 TMA loads, 1 MMA issue (and TMEM owner), then the
+// Warp roles of lowrank_bwd_kernel<K>: 0 TMA loads, 1 filter MMA issue (and TMEM owner), then the
 // du / dw epilogue (GA: 16 warps, four per TMEM lane quarter, each a quarter of the channels),
-// then 4 warps of dz / dB readout (GB: one TMEM lane quarter each).  The epilogue is latency-bound
+// then 4 warps of dz / dB readout (GB: one TMEM lane quarter each), then the dz / dB MMA issue.  The epilogue is latency-bound
 // (two warps per scheduler leave its TMEM / shared-memory round trips exposed), so it takes 16
 // warps for every K (measured: 3-5 % faster than 8 at the 150M QKV and 2B all-linear shapes).
 template <int K>
@@ -155,7 +155,9 @@ struct BwdEpi {
     static constexpr int groups = 32 / ga;             // 8-channel groups per GA warp
     static constexpr int per_wait = ga <= 8 ? 2 : 1;   // groups per TMEM wait in A1
     static constexpr int gb0 = 2 + ga;
-    static constexpr int threads = 32 * (gb0 + 4);
+    static constexpr int mma_d = gb0 + 4;              // the dz / dB MMA warp
+    static constexpr int du_store = mma_d + 1;         // the du store warp
+    static constexpr int threads = 32 * (du_store + 1);
 };
 constexpr int kGbWarps = 4, kGa0 = 2;
 
@@ -188,14 +190,14 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
     constexpr bool kDbt = BwdCols<K>::dbt;
     constexpr uint32_t kColDz = BwdCols<K>::dz, kColDb = BwdCols<K>::db;
     constexpr int kGaWarps = BwdEpi<K>::ga, kGaGroups = BwdEpi<K>::groups, kGaPerWait = BwdEpi<K>::per_wait;
-    constexpr int kGb0 = BwdEpi<K>::gb0;
+    constexpr int kGb0 = BwdEpi<K>::gb0, kMmaD = BwdEpi<K>::mma_d, kDuSt = BwdEpi<K>::du_store;
     constexpr int NZ = S::NZ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     // dwready / dwfree: per 128-row block (two tap atoms) of the dW tile, so the MMAs of one
     // block overlap the writing of the next and the next item's first block
     __shared__ uint64_t gufull[2], guempty[2], zfull[NZ], zempty[NZ], bfull, bempty, wfull, wempty, dwready[NBLK],
-        dwfree[NBLK], dzfull[2], dzempty[2], dbfree;
+        dwfree[NBLK], dzfull[2], dzempty[2], dbfree, dustaged, dusfree;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,17 +212,19 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         }
         for (int s = 0; s < NZ; ++s) {
             mbar_init(&zfull[s], 1);
-            mbar_init(&zempty[s], 1);
+            mbar_init(&zempty[s], 2);      // the filter and the dB MMAs of the item read z
         }
         for (int bb = 0; bb < NBLK; ++bb) {
             mbar_init(&dwready[bb], kGaWarps);
             mbar_init(&dwfree[bb], 1);
         }
         mbar_init(&bfull, 1);
-        mbar_init(&bempty, 1);
+        mbar_init(&bempty, 2);             // the filter and the dz MMAs read Bp
         mbar_init(&wfull, 1);
         mbar_init(&wempty, kGaWarps);
         mbar_init(&dbfree, kGbWarps);
+        mbar_init(&dustaged, kGaWarps);    // every GA warp has staged its du rows
+        mbar_init(&dusfree, 1);            // the du store has read the staging tile
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_z);
@@ -274,19 +278,16 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             }
         }
     } else if (warp == 1) {
+        // ---- filter MMAs of every item, issued by their own thread (the dz / dB MMAs have another,
+        // on another scheduler: one thread issuing both kinds was the kernel's critical path)
         if (lane == 0) {
             const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
-            const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
-            const uint32_t idesc_db = kDbt ? idesc_bf16(128, 64 * K, true, true) : idesc_bf16(128, a.ndz, true, true);
             const uint32_t bp0 = smem_u32(sm + S::bp);
-            const uint32_t dw0 = smem_u32(sm + S::dw);
             const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
             uint32_t cc = 0;          // B loads consumed
-            uint32_t m = 0;           // chunks whose dB accumulation has started
-            // Filter MMAs: Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows into the z slot),
-            // KS 16-wide steps over the rank, unrolled: this thread shares its scheduler with busy
-            // epilogue warps, and a loop with a run-time trip count per tap cost ~2.5x the issue
-            // time of the unrolled form.
+            // Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows into the z slot), KS 16-wide steps
+            // over the rank, unrolled (the issuing thread shares its scheduler with busy epilogue
+            // warps; a loop with a run-time trip count per tap cost ~2.5x the issue time)
             auto filter_mmas = [&](auto ks, uint32_t z0) {
                 constexpr int KS = decltype(ks)::value;
 #pragma unroll
@@ -296,9 +297,15 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                         umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k),
                                   mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k), idesc_w, k != 0);
             };
-            auto mma1 = [&](uint32_t it) -> bool {
+            ItemPos ipos(i0, a.n_tiles);
+            for (uint32_t it = 0; it < nit && !abort_flag; ++it, ipos.next()) {
                 const int zs = it % NZ;
-                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) return false;
+                if (it == 0 || ipos.tile == 0) {      // a chunk starts: its Bp slice
+                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
+                    ++cc;
+                }
+                if (it > 0 && !mbar_wait(&wempty, (it - 1) & 1, &abort_flag, a.err)) break;   // Wd read
+                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
                 const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
                 // ksteps = ceil(r / 16): 3 or 4 when r > 32, else 1 or 2
@@ -310,23 +317,29 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     else filter_mmas(std::integral_constant<int, 1>{}, z0);
                 }
                 umma_commit(&wfull);
-                return true;
-            };
-            bool ok = nit > 0 && mbar_wait(&bfull, 0, &abort_flag, a.err);
-            if (ok) {
-                cc = 1;
-                ok = mma1(0);
+                umma_commit(&zempty[zs]);
+                if (it + 1 < nit && ipos.last_of_chunk()) umma_commit(&bempty);   // B is reloaded next
             }
+        }
+    } else if (warp == kMmaD) {
+        // ---- dz and dB MMAs of every item
+        if (lane == 0) {
+            const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
+            const uint32_t idesc_db = kDbt ? idesc_bf16(128, 64 * K, true, true) : idesc_bf16(128, a.ndz, true, true);
+            const uint32_t bp0 = smem_u32(sm + S::bp);
+            const uint32_t dw0 = smem_u32(sm + S::dw);
+            const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
+            uint32_t cc = 0;          // B loads consumed
+            uint32_t m = 0;           // chunks whose dB accumulation has started
             ItemPos ipos(i0, a.n_tiles);
-            for (uint32_t it = 0; ok && it < nit && !abort_flag; ++it, ipos.next()) {
+            for (uint32_t it = 0; it < nit && !abort_flag; ++it, ipos.next()) {
                 const bool first = it == 0 || ipos.tile == 0;
-                const bool has_next = it + 1 < nit;
-                const bool next_same = has_next && !ipos.last_of_chunk();
                 const int zs = it % NZ, b = it & 1;
-                if (next_same) {          // the next filter MMA as soon as Wd has been read
-                    if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
-                    if (!mma1(it + 1)) break;
+                if (first) {
+                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
+                    ++cc;
                 }
+                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) break;
                 if (!mbar_wait(&dzempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
                 if (first && m > 0 && !mbar_wait(&dbfree, (m - 1) & 1, &abort_flag, a.err)) break;
                 const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
@@ -369,13 +382,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 if (first) ++m;
                 umma_commit(&dzfull[b]);
                 umma_commit(&zempty[zs]);
-                if (has_next && !next_same) {      // chunk changes: B is reloaded after these MMAs
-                    umma_commit(&bempty);
-                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
-                    ++cc;
-                    if (!mbar_wait(&wempty, it & 1, &abort_flag, a.err)) break;
-                    if (!mma1(it + 1)) break;
-                }
+                if (it + 1 < nit && ipos.last_of_chunk()) umma_commit(&bempty);   // B is reloaded next
             }
         }
     } else if (warp < kGb0) {
@@ -383,7 +390,6 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         const int q = warp & 3;
         const int half = (warp - kGa0) >> 2;   // channel groups kGaGroups*half ..
         const int row = q * 32 + lane;
-        const bool leader = warp == kGa0 && lane == 0;
         const uint32_t lane_base = tbase + (uint32_t(q * 32) << 16);
         uint8_t* dus = sm + S::dust;
         uint8_t* dws = sm + S::dw;
@@ -392,10 +398,12 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
         for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
             const int64_t chunk = ipos.chunk, tile = ipos.tile;
             const int gs = it & 1;
+            // each GA warp goes at its own pace (no barrier among them): a failed wait sets the abort
+            // flag, and every other wait in the kernel then gives up too
             bool ok = mbar_wait(&wfull, it & 1, &abort_flag, a.err) &&
-                      mbar_wait(&gufull[gs], (it >> 1) & 1, &abort_flag, a.err);
-            if (leader) tma_store_wait_read_all();     // the previous du store has read the staging tile
-            if (named_bar_any<2, 32 * kGaWarps>(!ok)) break;
+                      mbar_wait(&gufull[gs], (it >> 1) & 1, &abort_flag, a.err) &&
+                      (it == 0 || mbar_wait(&dusfree, (it - 1) & 1, &abort_flag, a.err));
+            if (!ok) break;
             tc_fence_after();
             const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
             const int32_t n = ta.m0 + row;
@@ -456,13 +464,16 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             tc_fence_before();
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&wempty);
+            if (lane == 0) {
+                mbar_arrive(&wempty);
+                mbar_arrive(&dustaged);
+            }
             // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap).  K <= 3:
             // every tap in one pass (the dB MMA reads every tap, so the blocks are freed together, and
             // each pass costs a barrier and an async-proxy fence); K = 4: block by block (taps 2 bb,
             // 2 bb + 1), each once the MMAs that last read it have finished.
             constexpr int kPasses = kDbt ? 1 : NBLK;
-            bool quit = false;       // uniform over the GA warps
+            bool quit = false;
 #pragma unroll
             for (int ps = 0; ps < kPasses; ++ps) {
                 const int blk0 = kDbt ? 0 : ps, blk1 = kDbt ? NBLK : ps + 1;
@@ -470,13 +481,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
 #pragma unroll
                 for (int bb = blk0; bb < blk1; ++bb)
                     ok = ok && mbar_wait(&dwfree[bb], (it & 1) ^ 1, &abort_flag, a.err);
-                if (named_bar_any<2, 32 * kGaWarps>(!ok)) {
+                if (!ok) {
                     quit = true;
                     break;
-                }
-                if (ps == 0 && leader) {                 // every GA warp has staged its du rows
-                    tma_store_2d_hint(&tm_du, dus, ta.x, ta.y, l2_evict_first());
-                    tma_store_commit();
                 }
 #pragma unroll
                 for (int i = 0; i < kGaGroups; ++i) {
@@ -505,7 +512,22 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             __syncwarp();
             if (lane == 0) mbar_arrive(&guempty[gs]);
         }
-        if (leader) tma_store_wait_all();
+    } else if (warp == kDuSt) {
+        // ---- du store: each item's staged du tile, once every GA warp has written its rows
+        if (lane == 0) {
+            const uint8_t* dus = sm + S::dust;
+            uint32_t it = 0;
+            ItemPos ipos(i0, a.n_tiles);
+            for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
+                if (!mbar_wait(&dustaged, it & 1, &abort_flag, a.err)) break;
+                const TileAt ta = tile_at<CF>(ipos.tile, (int32_t)(ipos.chunk * 64), a.tps, a.seqlen, a.C);
+                tma_store_2d_hint(&tm_du, dus, ta.x, ta.y, l2_evict_first());
+                tma_store_commit();
+                tma_store_wait_read_all();
+                mbar_arrive(&dusfree);
+            }
+            tma_store_wait_all();
+        }
     } else {
         // ---- GB: dz readout (added into the [N, r] fp32 buffer: reduction over chunks) and dB partials
         const int q = warp & 3;
