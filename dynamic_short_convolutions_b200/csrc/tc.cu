@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
 // =====================================================================================
 // lowrank_fwd_kernel<K>: work items (128-token tile m0, 64-channel chunk c0) in contiguous
 // chunk-major runs, one run per CTA, so the chunk's B stays in shared memory.
-//   stage smem (ring of kFwdStages): z tile [128][64] (K-major A) | u tile [136 rows =
-//               m0-8 .. m0+127][64 channels]
+//   rings:      u tiles [136 rows = m0-8 .. m0+127][64 channels] (kFwdU slots) and z tiles
+//               [128][64] (K-major A, kFwdZ slots)
 //   resident:   the chunk's slice of the tap-major Bp (Bp[k, j C + c] = B[k, c K + j], written by
 //               the generator launch) as K atoms [64 r-rows][64] (MN-major B), reloaded when the
 //               chunk changes
@@ -227,9 +227,12 @@ struct FwdArgs {
     int rope_max;            // table rows (positions are clamped below it)
 };
 
-constexpr int kFwdStages = 4;
+// u tiles (DRAM, the epilogue's operand) and z tiles (L2-resident, the MMA's operand) have rings of
+// their own: the u ring is the deeper one (the loads in flight per SM set the forward's throughput;
+// one shared ring of 4 stages left each u load ~3 us of queueing), and the producer issues each z
+// load kFwdZLag items after the u load of the same item.
+constexpr int kFwdU = 6, kFwdZ = 3, kFwdZLag = 2;
 constexpr uint32_t kZBytes = 16384, kUBytes = 136 * 128, kYBytes = 16384;
-constexpr uint32_t kFwdStage = kZBytes + kUBytes;
 constexpr uint32_t kCfUPitch = 136 * 2, kCfYPitch = 128 * 2;   // channel-first tile rows (bytes)
 // Epilogue of lowrank_fwd_kernel<K>: 16 warps in two teams of 8 that take alternate items
 // (ping-pong: one team's arithmetic overlaps the other's TMEM and shared-memory loads; measured
@@ -248,9 +251,12 @@ struct FwdEpi {
 
 template <int K>
 struct FwdSmem {
-    static constexpr uint32_t bres = kFwdStages * kFwdStage;
+    static constexpr uint32_t u0 = 0;
+    static constexpr uint32_t z0 = u0 + kFwdU * kUBytes;
+    static constexpr uint32_t bres = z0 + kFwdZ * kZBytes;
     static constexpr uint32_t ys = bres + K * 8192;
     static constexpr uint32_t total = ys + 2 * kYBytes + 1024;
+    static_assert(z0 % 1024 == 0 && bres % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
 };
 
 // y for 8 channels of one row: wv[j][c] = W_j[t, 8 g + c] (fp32 bits), uj[j] = u[t - j, 8 g .. 8 g + 7].
@@ -317,16 +323,21 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
     constexpr int kFwdGroups = FwdEpi<K>::groups;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ uint64_t full[kFwdStages], empty[kFwdStages], bfull, bempty, tfull[2], tempty[2], yfull[2], yempty[2];
+    __shared__ uint64_t ufull[kFwdU], uempty[kFwdU], zfull[kFwdZ], zempty[kFwdZ], bfull, bempty, tfull[2], tempty[2],
+        yfull[2], yempty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_tiles = a.n_tiles, n_items = n_tiles * (a.C / 64);
     const int64_t i0 = (int64_t)blockIdx.x * a.per_cta, i1 = min(i0 + a.per_cta, n_items);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kFwdStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + FwdEpi<K>::team_warps);
+        for (int s = 0; s < kFwdU; ++s) {
+            mbar_init(&ufull[s], 1);
+            mbar_init(&uempty[s], FwdEpi<K>::team_warps);   // the team of the item read u
+        }
+        for (int s = 0; s < kFwdZ; ++s) {
+            mbar_init(&zfull[s], 1);
+            mbar_init(&zempty[s], 1);                        // the MMA read z
         }
         mbar_init(&bfull, 1);
         mbar_init(&bempty, 1);
@@ -358,27 +369,42 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
         if (lane == 0) {
             const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             int64_t prev = -1;
-            uint32_t cc = 0, it = 0;
-            ItemPos ipos(i0, n_tiles);
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it, ipos.next()) {
-                const int64_t chunk = ipos.chunk, tile = ipos.tile;
-                const int32_t c0 = (int32_t)(chunk * 64);
-                const TileAt ta = tile_at<CF>(tile, c0, a.tps, a.seqlen, a.C);
-                if (chunk != prev) {
-                    if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
-                    mbar_arrive_expect_tx(&bfull, K * 8192);
-                    for (int j = 0; j < K; ++j)
-                        tma_load_2d_hint(sm + S::bres + j * 8192, &tm_b, &bfull, (int32_t)(j * a.C) + c0, 0, keep);
-                    ++cc;
-                    prev = chunk;
+            uint32_t cc = 0;
+            const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
+            ItemPos upos(i0, n_tiles), zpos(i0, n_tiles);
+            // step k: the u tile of item k, then the z tile (and at a chunk start the Bp slice) of item
+            // k - kFwdZLag
+            for (uint32_t k = 0; k < nit + kFwdZLag && !abort_flag; ++k) {
+                if (k < nit) {
+                    const int s = k % kFwdU;
+                    if (!mbar_wait(&uempty[s], ((k / kFwdU) & 1) ^ 1, &abort_flag, a.err)) break;
+                    const TileAt ta = tile_at<CF>(upos.tile, (int32_t)(upos.chunk * 64), a.tps, a.seqlen, a.C);
+                    uint8_t* ut = sm + S::u0 + s * kUBytes;
+                    mbar_arrive_expect_tx(&ufull[s], kUBytes);
+                    if (CF) tma_load_2d_hint(ut, &tm_u, &ufull[s], ta.x - 8, ta.y, stream);
+                    else tma_load_2d_hint(ut, &tm_u, &ufull[s], ta.x, ta.y - 8, stream);
+                    upos.next();
                 }
-                const int s = it % kFwdStages;
-                if (!mbar_wait(&empty[s], ((it / kFwdStages) & 1) ^ 1, &abort_flag, a.err)) break;
-                uint8_t* st = sm + s * kFwdStage;
-                mbar_arrive_expect_tx(&full[s], kFwdStage);
-                tma_load_2d_hint(st, &tm_z, &full[s], 0, ta.m0, keep);
-                if (CF) tma_load_2d_hint(st + kZBytes, &tm_u, &full[s], ta.x - 8, ta.y, stream);
-                else tma_load_2d_hint(st + kZBytes, &tm_u, &full[s], ta.x, ta.y - 8, stream);
+                if (k >= (uint32_t)kFwdZLag) {
+                    const uint32_t it = k - kFwdZLag;
+                    const int64_t chunk = zpos.chunk;
+                    const int32_t c0 = (int32_t)(chunk * 64);
+                    if (chunk != prev) {
+                        if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
+                        mbar_arrive_expect_tx(&bfull, K * 8192);
+                        for (int j = 0; j < K; ++j)
+                            tma_load_2d_hint(sm + S::bres + j * 8192, &tm_b, &bfull, (int32_t)(j * a.C) + c0, 0,
+                                             keep);
+                        ++cc;
+                        prev = chunk;
+                    }
+                    const int s = it % kFwdZ;
+                    if (!mbar_wait(&zempty[s], ((it / kFwdZ) & 1) ^ 1, &abort_flag, a.err)) break;
+                    const TileAt ta = tile_at<CF>(zpos.tile, c0, a.tps, a.seqlen, a.C);
+                    mbar_arrive_expect_tx(&zfull[s], kZBytes);
+                    tma_load_2d_hint(sm + S::z0 + s * kZBytes, &tm_z, &zfull[s], 0, ta.m0, keep);
+                    zpos.next();
+                }
             }
         }
     } else if (warp == 1) {
@@ -396,17 +422,17 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
                     ++cc;
                     prev = chunk;
                 }
-                const int s = it % kFwdStages, b = it & 1;
+                const int s = it % kFwdZ, b = it & 1;
                 if (!mbar_wait(&tempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
-                if (!mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err)) break;
+                if (!mbar_wait(&zfull[s], (it / kFwdZ) & 1, &abort_flag, a.err)) break;
                 tc_fence_after();
-                const uint32_t st = smem_u32(sm + s * kFwdStage);
+                const uint32_t st = smem_u32(sm + S::z0 + s * kZBytes);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)      // ksteps = r / 16 rounded up, at most 4
                     if (k < a.ksteps)
                         umma_bf16(tbase + b * 256, kmajor_desc(st, k), mnmajor_desc(b0, 8192, 16 * k), idesc, k != 0);
                 umma_commit(&tfull[b]);
-                umma_commit(&empty[s]);
+                umma_commit(&zempty[s]);
                 if (last) umma_commit(&bempty);
             }
         }
@@ -438,7 +464,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
         for (int64_t item = i0 + team; item < i1;
              item += FwdEpi<K>::teams, it += FwdEpi<K>::teams, ipos.next(), ipos.next()) {
             const int64_t tile = ipos.tile;
-            const int s = it % kFwdStages, b = it & 1;
+            const int s = it % kFwdU, b = it & 1;
             const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
             const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
             // RoPE: this row's table entries for the thread's channel groups, fetched before the waits
@@ -462,11 +488,11 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             // each warp goes at its own pace (no barrier among the epilogue warps): a failed
             // wait sets the abort flag, and every other wait then gives up too
             const bool ok = mbar_wait(&tfull[b], (it >> 1) & 1, &abort_flag, a.err) &&
-                            mbar_wait(&full[s], (it / kFwdStages) & 1, &abort_flag, a.err) &&
+                            mbar_wait(&ufull[s], (it / kFwdU) & 1, &abort_flag, a.err) &&
                             mbar_wait(&yempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err);
             if (!ok) break;
             tc_fence_after();
-            const uint8_t* us = sm + s * kFwdStage + kZBytes;
+            const uint8_t* us = sm + S::u0 + s * kUBytes;
             uint8_t* ys = sm + S::ys + b * kYBytes;
             const uint32_t taddr = tbase + (uint32_t(q * 32) << 16) + b * 256;
             // NG 8-channel groups per pass: every TMEM and shared-memory load first, then one wait,
@@ -508,7 +534,7 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&tempty[b]);
-                mbar_arrive(&empty[s]);
+                mbar_arrive(&uempty[s]);
                 mbar_arrive(&yfull[b]);
             }
         }
