@@ -136,22 +136,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
         }
     } else {
         if (a.pB) {                              // the side job, before the first accumulator is ready
-            const int CK = a.pC * a.pK;
-            const int64_t total = (int64_t)a.pr * CK, stride = (int64_t)gridDim.x * kEpiThreads;
-            int64_t o = (int64_t)blockIdx.x * kEpiThreads + (threadIdx.x - 64);
-            for (; o + 3 * stride < total; o += 4 * stride) {
-                __nv_bfloat16 v[4];
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int e = (int)(o + x * stride), k = e / CK, rem = e - k * CK, j = rem / a.pC, c = rem - j * a.pC;
-                    v[x] = a.pB[(int64_t)k * CK + c * a.pK + j];
+            // (k, c) pairs in grid-stride order, consecutive threads on consecutive channels: a warp
+            // reads 32 K-element groups of one row of B (contiguous) and writes K runs of 32 channels
+            const int C = a.pC, Kt = a.pK;
+            const int64_t total = (int64_t)a.pr * C, nthr = (int64_t)gridDim.x * kEpiThreads;
+            const int64_t e0 = (int64_t)blockIdx.x * kEpiThreads + (threadIdx.x - 64);
+            const int dk = (int)(nthr / C), dc = (int)(nthr - (int64_t)dk * C);
+            int k = (int)(e0 / C), c = (int)(e0 - (int64_t)k * C);
+            for (int64_t e = e0; e < total; e += nthr) {
+                const __nv_bfloat16* src = a.pB + ((int64_t)k * C + c) * Kt;
+                __nv_bfloat16* dst = a.pBp + (int64_t)k * Kt * C + c;
+                for (int j = 0; j < Kt; ++j) dst[(int64_t)j * C] = src[j];
+                c += dc;
+                k += dk;
+                if (c >= C) {
+                    c -= C;
+                    ++k;
                 }
-#pragma unroll
-                for (int x = 0; x < 4; ++x) a.pBp[o + x * stride] = v[x];
-            }
-            for (; o < total; o += stride) {
-                const int e = (int)o, k = e / CK, rem = e - k * CK, j = rem / a.pC, c = rem - j * a.pC;
-                a.pBp[o] = a.pB[(int64_t)k * CK + c * a.pK + j];
             }
         }
         const int q = warp & 3;                  // TMEM lane quarter of this warp
