@@ -435,6 +435,11 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                         gg[x][j] = CF ? cf_gather8(gt, kCfPitch, g0 + x, row + j)
                                       : *reinterpret_cast<const uint4*>(gt + sw128_off(row + j, g0 + x));
                 tmem_wait_ld();
+                if (gp + 1 == kGaGroups / kGaPerWait) {   // every Wd value is in registers: the next
+                    tc_fence_before();                    // filter MMA may overwrite the TMEM columns
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&wempty);
+                }
 #pragma unroll
                 for (int x = 0; x < kGaPerWait; ++x) {
                     gv[kGaPerWait * gp + x] = gg[x][0];
@@ -461,13 +466,9 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                     else *reinterpret_cast<uint4*>(dus + sw128_off(row, g0 + x)) = dv;
                 }
             }
-            tc_fence_before();
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&wempty);
-                mbar_arrive(&dustaged);
-            }
+            if (lane == 0) mbar_arrive(&dustaged);
             // A2: dw[t, c, j] = g[t, c] u[t - j, c] (bf16 products, one 64-channel atom per tap).  K <= 3:
             // every tap in one pass (the dB MMA reads every tap, so the blocks are freed together, and
             // each pass costs a barrier and an async-proxy fence); K = 4: block by block (taps 2 bb,
