@@ -127,6 +127,24 @@ __device__ __forceinline__ void rope_pairs8v(float (&x)[8], const float4& a, con
 }
 
 // The same on 8 bf16 values packed in a uint4 (rotated in fp32, rounded once back to bf16).
+// The same with the table slice already in registers (a = entries 0..3, b = entries 4..7).
+__device__ __forceinline__ uint4 rope_bf16x8v(const uint4& v, const float4& a, const float4& b, bool inverse) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        x[2 * q] = __uint_as_float(w[q] << 16);
+        x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+    rope_pairs8v(x, a, b, inverse);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        o[q] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
 __device__ __forceinline__ uint4 rope_bf16x8(const uint4& v, const float* __restrict__ cs, bool inverse) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float x[8];
@@ -145,20 +163,43 @@ __device__ __forceinline__ uint4 rope_bf16x8(const uint4& v, const float* __rest
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// out[n, c] = (R^T or R) x[n, c] for the rotated channels c < rope_n of tokens n = first, first + step, ...
-// (bf16, token-major, 8 channels per thread and step; out has row stride rope_n): the block's threads
-// stride over a token's 8-channel groups.  Positions are clamped below rope_max.
+// out[n, c] = (R^T or R) x[n, c] for the rotated channels c < rope_n (bf16, token-major; out has row
+// stride rope_n).  Warp `wid` of `nwarps` takes tokens wid, wid + nwarps, ...: its position (and table
+// row) once per token, its lanes the token's 8-channel groups (two per round, loads first).  Positions
+// are clamped below rope_max.
 __device__ __forceinline__ void rope_rows_bf16(const __nv_bfloat16* __restrict__ x, int64_t x_stride,
-                                               __nv_bfloat16* __restrict__ out, int64_t N, int64_t first,
-                                               int64_t step, int rope_n, int rope_hd, int rope_max,
+                                               __nv_bfloat16* __restrict__ out, int64_t N, int64_t wid,
+                                               int64_t nwarps, int rope_n, int rope_hd, int rope_max,
                                                const float* __restrict__ cs, const int32_t* __restrict__ cu,
                                                int64_t n_docs, int64_t seqlen, bool inverse) {
-    for (int64_t n = first; n < N; n += step) {
-        int64_t pos = n - seg_start(n, cu, n_docs, seqlen);
+    const int lane = threadIdx.x & 31;
+    const int G = rope_n / 8;
+    for (int64_t n = wid; n < N; n += nwarps) {
+        int64_t pos;
+        if (cu == nullptr && N < (int64_t(1) << 31) && seqlen < (int64_t(1) << 31))
+            pos = (int64_t)((uint32_t)n % (uint32_t)seqlen);
+        else
+            pos = n - seg_start(n, cu, n_docs, seqlen);
         pos = pos < rope_max ? pos : rope_max - 1;
-        for (int c = 8 * (int)threadIdx.x; c < rope_n; c += 8 * (int)blockDim.x) {
-            const uint4 v = *reinterpret_cast<const uint4*>(x + n * x_stride + c);
-            *reinterpret_cast<uint4*>(out + n * rope_n + c) = rope_bf16x8(v, cs + pos * rope_hd + c % rope_hd, inverse);
+        const __nv_bfloat16* xr = x + n * x_stride;
+        __nv_bfloat16* orow = out + n * rope_n;
+        const float* crow = cs + pos * rope_hd;
+        for (int g = lane; g < G; g += 64) {
+            const bool two = g + 32 < G;
+            const int c0 = 8 * g, c1 = 8 * (g + 32);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(xr + c0);
+            const float4* t0 = reinterpret_cast<const float4*>(crow + c0 % rope_hd);
+            const float4 a0 = __ldg(t0), b0 = __ldg(t0 + 1);
+            uint4 v1 = make_uint4(0, 0, 0, 0);
+            float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = a1;
+            if (two) {
+                v1 = *reinterpret_cast<const uint4*>(xr + c1);
+                const float4* t1 = reinterpret_cast<const float4*>(crow + c1 % rope_hd);
+                a1 = __ldg(t1);
+                b1 = __ldg(t1 + 1);
+            }
+            *reinterpret_cast<uint4*>(orow + c0) = rope_bf16x8v(v0, a0, b0, inverse);
+            if (two) *reinterpret_cast<uint4*>(orow + c1) = rope_bf16x8v(v1, a1, b1, inverse);
         }
     }
 }

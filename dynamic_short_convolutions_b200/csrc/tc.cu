@@ -468,21 +468,22 @@ __global__ void __launch_bounds__(FwdEpi<K>::threads, 1) lowrank_fwd_kernel(cons
             const int s = it % kFwdU, b = it & 1;
             const int32_t n = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0 + row;
             const int32_t pos = n < a.N ? n - seg_start32(n, a.cu, (int32_t)a.n_docs, (int32_t)a.seqlen) : 0;
-            // RoPE: this row's table entries for the thread's channel groups, fetched before the waits
-            // below so that their latency overlaps them (one 32-byte table slice per group)
+            // RoPE: this row's table entries for the thread's channel groups (32 bytes each, at the
+            // group's offset within its rotary head), fetched before the waits below so that their
+            // latency overlaps them; a chunk lies wholly inside or outside the rotated channels
             constexpr int kRopeG = ROPE ? kFwdGroups : 1;
             float4 rcs[kRopeG][2];
             bool rot = false;
             if constexpr (ROPE) {
-                const int c0 = (int)ipos.chunk * 64 + 8 * kFwdGroups * half;
-                rot = c0 < a.rope_n;         // a chunk lies wholly inside or outside the rotated channels
+                const int c0 = (int)ipos.chunk * 64 + 8 * kFwdGroups * half;   // the thread's first channel
+                rot = c0 < a.rope_n;
                 if (rot) {
-                    const float4* t4 = reinterpret_cast<const float4*>(
-                        a.rope_cs + (int64_t)min(pos, a.rope_max - 1) * a.rope_hd + c0 % a.rope_hd);
+                    const float* crow = a.rope_cs + (int64_t)min(pos, a.rope_max - 1) * a.rope_hd;
 #pragma unroll
                     for (int x = 0; x < kRopeG; ++x) {
-                        rcs[x][0] = __ldg(t4 + 2 * x);
-                        rcs[x][1] = __ldg(t4 + 2 * x + 1);
+                        const float4* t4 = reinterpret_cast<const float4*>(crow + (c0 + 8 * x) % a.rope_hd);
+                        rcs[x][0] = __ldg(t4);
+                        rcs[x][1] = __ldg(t4 + 1);
                     }
                 }
             }

@@ -462,7 +462,8 @@ __global__ void __launch_bounds__(128) rope_rows_kernel(const __nv_bfloat16* __r
                                                         int64_t seqlen) {
     pdl_trigger();
     pdl_wait();
-    rope_rows_bf16(g, C, gr, N, blockIdx.x, gridDim.x, rope_n, rope_hd, rope_max, cs, cu, n_docs, seqlen, true);
+    rope_rows_bf16(g, C, gr, N, (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5),
+                   (int64_t)gridDim.x * (blockDim.x / 32), rope_n, rope_hd, rope_max, cs, cu, n_docs, seqlen, true);
 }
 
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }

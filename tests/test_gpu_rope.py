@@ -63,6 +63,10 @@ CASES = [
     (_case("c2_qkv_150m_lowrank", 2, 300, "rope_c2"), 0, 1536, 64),            # Q and K of the 150M QKV
     (_case("c3_qkv_2b_headwise_gqa", 2, 200, "rope_c3"), 0, 2560, 128),        # Q (16 heads) and K (4 heads)
     (_case("c2_qkv_150m_lowrank", 1, 200, "rope_k4_r64", ksize=4, rank=64), 0, 1536, 64),
+    # rotary heads narrower than a thread's 32 channels, and not dividing them: the table slice
+    # wraps to the next head inside a thread's channel run
+    (_case("c2_qkv_150m_lowrank", 1, 160, "rope_hd16"), 0, 1536, 16),
+    (_case("c2_qkv_150m_lowrank", 1, 160, "rope_hd40"), 0, 640, 40),
     (C["c1_fp32_lowrank"], 0, 32, 16),
 ]
 
