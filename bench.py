@@ -580,17 +580,33 @@ def run_ours(args, rank, world, local_rank):
         d2h += sum(v.numel() * v.element_size() for v in hout.values())
         host.append((hin, hout))
 
+    # Copies run on their own streams (host -> device on one, device -> host on the other, PCIe being
+    # full duplex) and overlap the compute of other layers, as a caller's input pipeline would; events
+    # order each layer's copies against its compute in both directions (a layer's inputs are not
+    # overwritten before its compute has read them, its outputs not before they have been copied out).
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = [{k: torch.cuda.Event() for k in ("in_ready", "done", "out_free")} for _ in layers]
+
     def e2e_step():
-        for (layer, t, plan, A, BW, cu, b), (hin, hout) in zip(layers, host):
-            for k, v in hin.items():
-                t[k].copy_(v, non_blocking=True)
+        for (layer, t, plan, A, BW, cu, b), (hin, hout), e in zip(layers, host, ev):
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(e["done"])                   # the previous step's compute read these inputs
+                for k, v in hin.items():
+                    t[k].copy_(v, non_blocking=True)
+                e["in_ready"].record(s_in)
+            stream.wait_event(e["in_ready"])
+            stream.wait_event(e["out_free"])                 # the previous step's outputs are copied out
             plan.forward(t["u"], t["h"], t.get("A"), t["B"] if "B" in t else t["W"], cu, y=b["y"], z_save=b["z"])
             plan.backward(t["g"], t["u"], t["h"], t.get("A"), t["B"] if "B" in t else t["W"], cu,
                           z_saved=b["z"], out=b["out"])
-            hout["y"].copy_(b["y"], non_blocking=True)
-            for k in ("du", "dh", "dBW", "dA"):
-                if k in hout:
-                    hout[k].copy_(b["out"][k], non_blocking=True)
+            e["done"].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e["done"])
+                hout["y"].copy_(b["y"], non_blocking=True)
+                for k in ("du", "dh", "dBW", "dA"):
+                    if k in hout:
+                        hout[k].copy_(b["out"][k], non_blocking=True)
+                e["out_free"].record(s_out)
 
     for _ in range(max(1, min(args.warmup, 3))):
         e2e_step()
@@ -598,8 +614,15 @@ def run_ours(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(1, min(args.steps, 20))
     e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
     for _ in range(e2e_steps):
         e2e_step()
+    done_in, done_out = torch.cuda.Event(), torch.cuda.Event()
+    done_in.record(s_in)
+    done_out.record(s_out)
+    stream.wait_event(done_in)
+    stream.wait_event(done_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
