@@ -34,6 +34,11 @@ SMALL = [
     (_case("c2_qkv_150m_lowrank", 2, 257, "k2_r64", ksize=2, rank=64), 0),
     (_case("c2_qkv_150m_lowrank", 1, 140, "k1_r64", ksize=1, rank=64), 0),
     (_case("c2_qkv_150m_lowrank", 1, 200, "k4_r8", ksize=4, rank=8), 0),
+    # ranks whose last 16-wide step of the filter MMA is partly padding (r = 24: two steps, r = 48:
+    # three steps of the rank-64 kernels)
+    (_case("c2_qkv_150m_lowrank", 1, 270, "k3_r24", rank=24), 0),
+    (_case("c2_qkv_150m_lowrank", 1, 270, "k3_r48", rank=48), 0),
+    (_case("c2_qkv_150m_lowrank", 1, 200, "k4_r40", ksize=4, rank=40), 0),
     (_case("c2_qkv_150m_lowrank", 1, 130, "odd_channels", layers=(W.Layer("x", 40, 72),)), 0),
     (_case("c3_qkv_2b_headwise_gqa", 1, 150, "hw_k2_hd64", ksize=2, head_dim=64,
            layers=(W.Layer("qkv", 256, 640),)), 0),
