@@ -163,17 +163,17 @@ __device__ __forceinline__ uint4 rope_bf16x8(const uint4& v, const float* __rest
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// out[n, c] = (R^T or R) x[n, c] for the rotated channels c < rope_n (bf16, token-major; out has row
-// stride rope_n).  Warp `wid` of `nwarps` takes tokens wid, wid + nwarps, ...: its position (and table
+// out[n, c] = (R^T or R) x[n, c] for the rotated channels c < rope_n and x[n, c] for rope_n <= c <
+// out_w (bf16, token-major; out has row stride out_w >= rope_n, a multiple of 8).  Warp `wid` of `nwarps` takes tokens wid, wid + nwarps, ...: its position (and table
 // row) once per token, its lanes the token's 8-channel groups (two per round, loads first).  Positions
 // are clamped below rope_max.
 __device__ __forceinline__ void rope_rows_bf16(const __nv_bfloat16* __restrict__ x, int64_t x_stride,
-                                               __nv_bfloat16* __restrict__ out, int64_t N, int64_t wid,
+                                               __nv_bfloat16* __restrict__ out, int out_w, int64_t N, int64_t wid,
                                                int64_t nwarps, int rope_n, int rope_hd, int rope_max,
                                                const float* __restrict__ cs, const int32_t* __restrict__ cu,
                                                int64_t n_docs, int64_t seqlen, bool inverse) {
     const int lane = threadIdx.x & 31;
-    const int G = rope_n / 8;
+    const int Gr = rope_n / 8, G = out_w / 8;
     for (int64_t n = wid; n < N; n += nwarps) {
         int64_t pos;
         if (cu == nullptr && N < (int64_t(1) << 31) && seqlen < (int64_t(1) << 31))
@@ -182,24 +182,29 @@ __device__ __forceinline__ void rope_rows_bf16(const __nv_bfloat16* __restrict__
             pos = n - seg_start(n, cu, n_docs, seqlen);
         pos = pos < rope_max ? pos : rope_max - 1;
         const __nv_bfloat16* xr = x + n * x_stride;
-        __nv_bfloat16* orow = out + n * rope_n;
+        __nv_bfloat16* orow = out + n * out_w;
         const float* crow = cs + pos * rope_hd;
         for (int g = lane; g < G; g += 64) {
             const bool two = g + 32 < G;
             const int c0 = 8 * g, c1 = 8 * (g + 32);
             const uint4 v0 = *reinterpret_cast<const uint4*>(xr + c0);
-            const float4* t0 = reinterpret_cast<const float4*>(crow + c0 % rope_hd);
-            const float4 a0 = __ldg(t0), b0 = __ldg(t0 + 1);
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
+            if (g < Gr) {
+                const float4* t0 = reinterpret_cast<const float4*>(crow + c0 % rope_hd);
+                a0 = __ldg(t0);
+                b0 = __ldg(t0 + 1);
+            }
             uint4 v1 = make_uint4(0, 0, 0, 0);
-            float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = a1;
             if (two) {
                 v1 = *reinterpret_cast<const uint4*>(xr + c1);
-                const float4* t1 = reinterpret_cast<const float4*>(crow + c1 % rope_hd);
-                a1 = __ldg(t1);
-                b1 = __ldg(t1 + 1);
+                if (g + 32 < Gr) {
+                    const float4* t1 = reinterpret_cast<const float4*>(crow + c1 % rope_hd);
+                    a1 = __ldg(t1);
+                    b1 = __ldg(t1 + 1);
+                }
             }
-            *reinterpret_cast<uint4*>(orow + c0) = rope_bf16x8v(v0, a0, b0, inverse);
-            if (two) *reinterpret_cast<uint4*>(orow + c1) = rope_bf16x8v(v1, a1, b1, inverse);
+            *reinterpret_cast<uint4*>(orow + c0) = g < Gr ? rope_bf16x8v(v0, a0, b0, inverse) : v0;
+            if (two) *reinterpret_cast<uint4*>(orow + c1) = g + 32 < Gr ? rope_bf16x8v(v1, a1, b1, inverse) : v1;
         }
     }
 }

@@ -609,8 +609,9 @@ const char* tc_unsupported_reason(const Prob& p, bool bwd) {
     if (p.dtype != 1) return "fp32 storage runs the CUDA-core kernels (no tensor-core rounding of fp32 inputs)";
     if (tensor_map_encoder() == nullptr) return "the driver entry point cuTensorMapEncodeTiled is unavailable";
     if (p.kind == 1) {
-        if (p.rope_n > 0 && (p.layout == 1 || p.rope_hd % 8 != 0))
-            return "head-wise RoPE on the tensor cores needs the token-major layout and rope_head_dim % 8 == 0";
+        if (p.rope_n > 0 && (p.layout == 1 || p.rope_hd % 8 != 0 || p.rope_hd > 256))
+            return "head-wise RoPE on the tensor cores needs the token-major layout and rope_head_dim % 8 == 0, "
+                   "at most 256";
         if (!tc_headwise_supported(p))
             return "head-wise tensor-core kernels need H*K a multiple of 8 up to 128, d a multiple of 8, and "
                    "(token-major) head_dim a power of two in [8, 256] with channels a multiple of 256, or "

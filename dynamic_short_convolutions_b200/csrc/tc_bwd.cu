@@ -80,7 +80,7 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, __nv_bfloat
     pdl_wait();
     if ((int)blockIdx.x >= (int)gridDim.x - rp.nb_rot) {
         const int b = blockIdx.x - (gridDim.x - rp.nb_rot);
-        rope_rows_bf16(rp.g, C, rp.gr, rp.N, (int64_t)b * (blockDim.x / 32) + (threadIdx.x >> 5),
+        rope_rows_bf16(rp.g, C, rp.gr, rp.rope_n, rp.N, (int64_t)b * (blockDim.x / 32) + (threadIdx.x >> 5),
                        (int64_t)rp.nb_rot * (blockDim.x / 32), rp.rope_n, rp.rope_hd, rp.rope_max, rp.cs, rp.cu,
                        rp.n_docs, rp.seqlen, true);
         return;

@@ -9,11 +9,13 @@
 //   du[m, c] = g[m, c] + sum_{j < e(m) - m} wh[m+j, (c/hd)*K + j] g[m+j, c]
 //   dwh[n, q*K + j] = sum_{c in head q} [j <= n - s(n)] g[n, c] u[n-j, c]   (warp shuffles)
 //   dW = h^T dwh,  dh = dwh W^T                                        (tensor cores)
-// The conv kernels are memory-bound CUDA-core kernels: token-major (16-byte loads and stores
-// along C, packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh) and channel-first
+// The conv kernels are memory-bound CUDA-core kernels: token-major (a warp streams consecutive
+// tokens through per-lane cp.async rings in shared memory, 16-byte loads and stores along C,
+// packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh) and channel-first
 // (loads along the token rows of [batch * C, seqlen], a lane's filter taps held across the
 // head's channels, dwh summed per warp and then over the block's warps in order).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -32,10 +34,27 @@ namespace {
 
 using namespace tc;
 
-// A block covers kTokPerBlock tokens x 256 channels: 8 warps, each lane 8 channels (16-byte
-// loads and stores along C) of two consecutive tokens per step; the rows beyond the pair were
-// just read by the block's other warps and come from L1 / L2.
-constexpr int kTokPerBlock = 64;
+// Token-major kernels: a warp streams a run of consecutive tokens over 256 channels, each lane 8
+// channels (16-byte stores along C, packed fp32 FMAs).  The rows of each token -- u; g; the
+// filter taps of the block's heads; with RoPE the table row of the token's position -- come into
+// a shared-memory ring by TMA, a few tokens at a time, so ~8 tokens of every warp are in flight
+// without registers held for them, and rows outside [0, N) read zero through the tensor maps'
+// bounds.  The rows of u (and the backward's pending du rows) sit in rolling register windows,
+// so a row is read and unpacked once; only the K - 1 rows of u before a run (and of g after it)
+// are read twice.
+constexpr int kHwRunFwd = 32, kHwRunBwd = 32;      // tokens per run (one warp, one block)
+constexpr int kHwMaxRopeHd = 256;                  // RoPE table rows of up to 256 floats (1 KB)
+
+// Segment bounds [s, e) of the tokens a warp walks through in increasing order: looked up again
+// (seg_bounds32) only when the walk leaves the current segment.
+struct SegWalk {
+    int32_t s = 0, e = 0;
+    __device__ __forceinline__ int32_t pos(int32_t n, const int32_t* __restrict__ cu, int32_t n_docs, int32_t seqlen,
+                                           int32_t N) {
+        if (n >= e) seg_bounds32(n, cu, n_docs, seqlen, N, s, e);
+        return n - s;
+    }
+};
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
     const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
@@ -50,25 +69,23 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
 }
 
-// acc[0..8) += w * x (8 bf16 in a uint4) on the packed fp32 FMA.
-__device__ __forceinline__ void axpy8(float (&acc)[8], float w, const uint4& x) {
-    const uint32_t* v = reinterpret_cast<const uint32_t*>(&x);
+// acc[0..8) += w * x[0..8) on the packed fp32 FMA.
+__device__ __forceinline__ void axpy8f(float (&acc)[8], float w, const float (&x)[8]) {
 #pragma unroll
-    for (int p = 0; p < 4; ++p) ffma2(acc[2 * p], acc[2 * p + 1], w, w, bf16_lo(v[p]), bf16_hi(v[p]));
+    for (int p = 0; p < 4; ++p) ffma2(acc[2 * p], acc[2 * p + 1], w, w, x[2 * p], x[2 * p + 1]);
 }
 
-// sum_i a[i] b[i] over 8 values given as bf16 (two fp32 lanes, then their sum).
-__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
-    const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
-    const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
+// sum_i a[i] b[i] over 8 values (two fp32 lanes, then their sum).
+__device__ __forceinline__ float dot8f(const float (&a)[8], const float (&b)[8]) {
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) ffma2(s0, s1, bf16_lo(x[p]), bf16_hi(x[p]), bf16_lo(y[p]), bf16_hi(y[p]));
+    for (int p = 0; p < 4; ++p) ffma2(s0, s1, a[2 * p], a[2 * p + 1], b[2 * p], b[2 * p + 1]);
     return s0 + s1;
 }
 
-// The K taps of one head's filter for one token, as floats (8- or 4-byte loads when aligned,
-// which holds for K = 4 and K = 2 since R = H K).
+// The K taps of one head's filter for one token, as floats: 8- or 4-byte loads for K = 4 and
+// K = 2 (aligned since R = H K and the taps boxes start at multiples of 8 columns), else
+// element by element.  p is global (channel-first kernels) or shared memory (token-major).
 template <int K>
 __device__ __forceinline__ void load_taps(const __nv_bfloat16* __restrict__ p, float (&w)[K]) {
     if constexpr (K == 4) {
@@ -87,72 +104,13 @@ __device__ __forceinline__ void load_taps(const __nv_bfloat16* __restrict__ p, f
     }
 }
 
-// A thread takes two consecutive tokens n, n + 1, which share K of their K + 1 rows of u.
+// Sums p[0..K) over the L lanes (a power of two <= 32) that hold one head and stores dst[j]
+// for j < K, masked to 0 for j > pos, when `store`.  For K >= 3 and L >= 4 a reduce-scatter:
+// two exchange steps leave each lane one tap, then a butterfly finishes it (log2(L) + 1
+// shuffles instead of K log2(L)); otherwise a plain butterfly over all K values.  Every lane
+// of the warp takes part in the shuffles.
 template <int K>
-__global__ void __launch_bounds__(256) hw_conv_fwd_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
-                                                          const __nv_bfloat16* __restrict__ wh, int R, int hd,
-                                                          int64_t N, int64_t C, int64_t seqlen,
-                                                          const int32_t* __restrict__ cu, int64_t n_docs,
-                                                          __nv_bfloat16* __restrict__ y,
-                                                          const float* __restrict__ rope_cs, int rope_n, int rope_hd,
-                                                          int rope_max) {
-    pdl_trigger();
-    pdl_wait();
-    const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
-    const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
-    const int q = (int)(c / hd);
-    const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
-    const int64_t n1 = min(N, n0 + kTokPerBlock);
-    for (int64_t n = n0 + 2 * tl; n < n1; n += 16) {
-        const bool two = n + 1 < n1;                     // uniform over the warp
-        // rows n - K + 1 .. n + 1 of u (zero outside [0, N)); the filters of n and n + 1
-        uint4 ur[K + 1];
-        float w[2][K];
-#pragma unroll
-        for (int i = 0; i <= K; ++i) {
-            const int64_t m = n - K + 1 + i;
-            ur[i] = (m >= 0 && m < N) ? *reinterpret_cast<const uint4*>(u + m * us + c) : make_uint4(0, 0, 0, 0);
-        }
-        load_taps<K>(wh + n * R + q * K, w[0]);
-        if (two) load_taps<K>(wh + (n + 1) * R + q * K, w[1]);
-        int32_t pos[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int32_t m = (int32_t)n + (two ? t : 0);
-            pos[t] = m - seg_start32(m, cu, (int32_t)n_docs, (int32_t)seqlen);
-        }
-        // RoPE: the two tokens' table slices, loaded with the rows above
-        const bool rot = rope_cs && c < rope_n;
-        float4 rc[2][2];
-        if (rot) {
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const float4* t4 = reinterpret_cast<const float4*>(
-                    rope_cs + (int64_t)min(pos[t], rope_max - 1) * rope_hd + c % rope_hd);
-                rc[t][0] = __ldg(t4);
-                rc[t][1] = __ldg(t4 + 1);
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            if (t == 1 && !two) break;
-            const int32_t m = (int32_t)n + t;
-            float acc[8];
-            unpack8(ur[K - 1 + t], acc);
-#pragma unroll
-            for (int j = 0; j < K; ++j) axpy8(acc, j <= pos[t] ? w[t][j] : 0.f, ur[K - 1 + t - j]);
-            if (rot) rope_pairs8v(acc, rc[t][0], rc[t][1], false);
-            *reinterpret_cast<uint4*>(y + (int64_t)m * C + c) = pack8(acc);
-        }
-    }
-}
-
-// Sums p[0..K) over the L lanes (a power of two) that hold one head and stores dst[j] for
-// j < K, masked to 0 for j > pos.  For K >= 3 and L >= 4 a reduce-scatter: two exchange
-// steps leave each lane one tap, then a butterfly finishes it (log2(L) + 1 shuffles instead
-// of K log2(L)); otherwise a plain butterfly over all K values.
-template <int K>
-__device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int32_t pos,
+__device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int32_t pos, bool store,
                                                __nv_bfloat16* __restrict__ dst) {
     if constexpr (K >= 3) {
         if (L >= 4) {
@@ -166,81 +124,258 @@ __device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int
             const float s = b2 ? k0 : k1;
             float k = b2 ? k1 : k0;
             k += __shfl_xor_sync(0xffffffffu, s, h2);
-            for (int off = h2 >> 1; off > 0; off >>= 1) k += __shfl_xor_sync(0xffffffffu, k, off);
+#pragma unroll
+            for (int it = 1; it <= 3; ++it) {            // offsets h2 / 2, h2 / 4, h2 / 8 (h2 <= 8)
+                const int off = h2 >> it;
+                if (off > 0) k += __shfl_xor_sync(0xffffffffu, k, off);
+            }
             const int tap = (b1 ? 2 : 0) + (b2 ? 1 : 0);
-            if ((gl & (h2 - 1)) == 0 && tap < K) dst[tap] = __float2bfloat16_rn(tap <= pos ? k : 0.f);
+            if (store && (gl & (h2 - 1)) == 0 && tap < K) dst[tap] = __float2bfloat16_rn(tap <= pos ? k : 0.f);
             return;
         }
     }
 #pragma unroll
     for (int j = 0; j < K; ++j)
-        for (int off = L >> 1; off > 0; off >>= 1) p[j] += __shfl_xor_sync(0xffffffffu, p[j], off);
+#pragma unroll
+        for (int it = 1; it <= 5; ++it) {
+            const int off = L >> it;
+            if (off > 0) p[j] += __shfl_xor_sync(0xffffffffu, p[j], off);
+        }
     const int l = gl & (L - 1);
 #pragma unroll
     for (int j = 0; j < K; ++j)
-        if (j % L == l) dst[j] = __float2bfloat16_rn(j <= pos ? p[j] : 0.f);
+        if (store && j % L == l) dst[j] = __float2bfloat16_rn(j <= pos ? p[j] : 0.f);
 }
 
-// L = head_dim / 8 lanes hold one head's channels (a power of two <= 32, aligned in the warp).
-// A thread takes two consecutive tokens n, n + 1, which share K of their K + 1 rows of g, of u
-// and of the filter: each row is loaded once for both.
+// Rows come in chunks of T stream rows (T a multiple of K, so a row's place in the rolling windows
+// is fixed by its place in the chunk): one TMA box per tensor and chunk, one mbarrier per ring
+// slot, kept Q - 1 chunks ahead of the chunk being computed.  A block is one warp and one run:
+// block b takes channel block b % n_cblk and tokens (b / n_cblk) * run onwards, so everything
+// that depends on the token position is uniform over the block and only the channel offset
+// varies by lane.  Chunks whose rows are all interior (no look-back, look-ahead or end of the
+// tensor among them) run a body without the per-row range tests.
 template <int K>
-__global__ void __launch_bounds__(256) hw_conv_bwd_kernel(const __nv_bfloat16* __restrict__ g,
-                                                          const __nv_bfloat16* __restrict__ u, int64_t us,
-                                                          const __nv_bfloat16* __restrict__ wh, int R, int hd,
-                                                          int64_t N, int64_t C, int64_t seqlen,
-                                                          const int32_t* __restrict__ cu, int64_t n_docs,
-                                                          __nv_bfloat16* __restrict__ du,
-                                                          __nv_bfloat16* __restrict__ dwh,
-                                                          const __nv_bfloat16* __restrict__ gr, int rope_n) {
+struct HwTile {
+    static constexpr int T = K >= 3 ? K : 4;     // stream rows per chunk
+    static constexpr int Q = (12 + T - 1) / T;   // ring slots (chunks)
+};
+
+__host__ __device__ constexpr uint32_t al128(uint32_t x) { return (x + 127u) & ~127u; }
+
+// Forward.  A run covers tokens n0 .. n0 + run - 1; its stream starts K - 1 rows earlier (the
+// taps' reach back).  Chunk: u rows [T][512 B], taps rows [T][taps_box], RoPE table rows
+// [T][rope_hd floats].
+template <int K>
+__global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__ CUtensorMap tm_u,
+                                                         const __grid_constant__ CUtensorMap tm_w, int hd, int32_t N,
+                                                         int64_t C, int32_t seqlen, const int32_t* __restrict__ cu,
+                                                         int32_t n_docs, int n_cblk, __nv_bfloat16* __restrict__ y,
+                                                         const float* __restrict__ rope_cs, int rope_n, int rope_hd,
+                                                         int rope_max, int run, int taps_box, uint32_t* err) {
+    constexpr int T = HwTile<K>::T, Q = HwTile<K>::Q;
+    extern __shared__ __align__(128) uint8_t hw_smem[];
+    __shared__ uint64_t bars[Q];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+        for (int s = 0; s < Q; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        abort_flag = 0;
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_w);
+    }
+    __syncwarp();
     pdl_trigger();
     pdl_wait();
-    const int gl = threadIdx.x & 31, tl = threadIdx.x >> 5;
-    const int64_t c = (int64_t)blockIdx.x * 256 + gl * 8;
-    const int q = (int)(c / hd);
-    const int L = hd >> 3;
-    const int64_t n0 = (int64_t)blockIdx.y * kTokPerBlock;
-    const int64_t n1 = min(N, n0 + kTokPerBlock);
-    // RoPE: the rotated channels' rows of g come from R^T g (gr [N, rope_n]), written beforehand
-    const bool rot = gr != nullptr && c < rope_n;
-    const __nv_bfloat16* gsrc = rot ? gr : g;
-    const int64_t gstride = rot ? rope_n : C;
-    for (int64_t n = n0 + 2 * tl; n < n1; n += 16) {
-        const bool two = n + 1 < n1;                     // uniform over the warp
-        int32_t sb[2], eb[2];
-        seg_bounds32((int32_t)n, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb[0], eb[0]);
-        if (two) seg_bounds32((int32_t)n + 1, cu, (int32_t)n_docs, (int32_t)seqlen, (int32_t)N, sb[1], eb[1]);
-        else { sb[1] = sb[0]; eb[1] = eb[0]; }
-        // rows n .. n + K of g and of the filter, rows n - K + 1 .. n + 1 of u (zero outside [0, N))
-        uint4 gr[K + 1], ur[K + 1];
-        float wr[K + 1][K];
+    const int32_t cb = (int32_t)(blockIdx.x % (uint32_t)n_cblk);
+    const int32_t n0 = (int32_t)(blockIdx.x / (uint32_t)n_cblk) * run;
+    const int32_t c0 = cb * 256, c = c0 + lane * 8;
+    const int q = c / hd, x0 = ((c0 / hd) * K) & ~7;
+    const int len = min(run, N - n0) + K - 1, nch = (len + T - 1) / T;
+    const bool rope_blk = rope_cs != nullptr && c0 < rope_n;      // the block holds rotated channels
+    const bool rot = rope_blk && c < rope_n;
+    const uint32_t tpitch = (uint32_t)taps_box * 2u, toff = al128(T * 512u);
+    const uint32_t rrow = (uint32_t)rope_hd * 4u, roff = toff + al128(T * tpitch);
+    const uint32_t chunk = al128(roff + (rope_cs ? T * rrow : 0u));
+    const int tl = q * K - x0, rl = rot ? (c % rope_hd) : 0;
+    SegWalk walk_in, walk;
+    auto issue = [&](int k) {                        // lane 0
+        if (k >= nch) return;
+        const int32_t row0 = n0 - (K - 1) + k * T;
+        uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
+        uint64_t* bar = &bars[k % Q];
+        mbar_arrive_expect_tx(bar, T * 512u + T * tpitch + (rope_blk ? T * rrow : 0u));
+        tma_load_2d_hint(sl, &tm_u, bar, c0, row0, l2_evict_first());
+        tma_load_2d(sl + toff, &tm_w, bar, x0, row0);
+        if (rope_blk) {
 #pragma unroll
-        for (int i = 0; i <= K; ++i) {                   // every load of the pair first
-            const int64_t mg = n + i, mu = n - K + 1 + i;
-            gr[i] = mg < N ? *reinterpret_cast<const uint4*>(gsrc + mg * gstride + c) : make_uint4(0, 0, 0, 0);
-            ur[i] = (mu >= 0 && mu < N) ? *reinterpret_cast<const uint4*>(u + mu * us + c) : make_uint4(0, 0, 0, 0);
-            if (mg < N) load_taps<K>(wh + mg * R + q * K, wr[i]);
-            else
-#pragma unroll
-                for (int j = 0; j < K; ++j) wr[i][j] = 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            if (t == 1 && !two) break;
-            const int32_t m = (int32_t)n + t;
-            const int32_t pos = m - sb[t], epos = eb[t] - 1 - m;
-            float acc[8];
-            unpack8(gr[t], acc);
-            float part[K];
-#pragma unroll
-            for (int j = 0; j < K; ++j) {
-                axpy8(acc, j <= epos ? wr[t + j][j] : 0.f, gr[t + j]);   // filter of token m+j, tap j
-                part[j] = dot8(gr[t], ur[K - 1 + t - j]);                 // g[m] . u[m-j] over 8 channels
+            for (int t = 0; t < T; ++t) {            // the table row of each token's position
+                const int32_t n = row0 + t;
+                const int32_t p = (n >= n0 && n < N) ? min(walk_in.pos(n, cu, n_docs, seqlen, N), rope_max - 1) : 0;
+                bulk_load(sl + roff + t * rrow, rope_cs + (int64_t)p * rope_hd, rrow, bar);
             }
-            *reinterpret_cast<uint4*>(du + (int64_t)m * C + c) = pack8(acc);
-            head_sum_store<K>(part, L, gl, pos, dwh + (int64_t)m * R + q * K);
         }
+    };
+    if (lane == 0)
+        for (int k = 0; k < Q - 1; ++k) issue(k);
+    __nv_bfloat16* yp = y + (int64_t)n0 * C + c;
+    float win[K][8];                                 // u row of stream index r at win[r mod K]
+    auto body = [&](const uint8_t* sl, int r0, auto full) {
+        constexpr bool FULL = decltype(full)::value;
+#pragma unroll
+        for (int s = 0; s < T; ++s) {
+            const int r = r0 + s;
+            if (!FULL && r >= len) break;
+            unpack8(*reinterpret_cast<const uint4*>(sl + s * 512 + lane * 16), win[s % K]);
+            const int32_t n = n0 - (K - 1) + r;
+            if (!FULL && n < n0) continue;
+            const int32_t pos = walk.pos(n, cu, n_docs, seqlen, N);
+            float w[K];
+            load_taps<K>(reinterpret_cast<const __nv_bfloat16*>(sl + toff + s * tpitch) + tl, w);
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = win[s % K][e];
+#pragma unroll
+            for (int j = 0; j < K; ++j) axpy8f(acc, j <= pos ? w[j] : 0.f, win[(s - j + K) % K]);
+            if (rot) {
+                const float4* t = reinterpret_cast<const float4*>(sl + roff + s * rrow + rl * 4);
+                rope_pairs8v(acc, t[0], t[1], false);
+            }
+            *reinterpret_cast<uint4*>(yp) = pack8(acc);
+            yp += C;
+        }
+    };
+    int k_fail = -1;
+    for (int k = 0; k < nch; ++k) {
+        __syncwarp();                                // slot k - 1, which chunk k + Q - 1 refills, is read
+        if (lane == 0) {
+            fence_async_smem();
+            issue(k + Q - 1);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[k % Q], (uint32_t)(k / Q) & 1u, &abort_flag, err))) {
+            k_fail = k;
+            break;
+        }
+        const uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
+        const int r0 = k * T;
+        if (r0 >= K - 1 && r0 + T <= len) body(sl, r0, std::true_type{});
+        else body(sl, r0, std::false_type{});
     }
+    if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
+        for (int k = k_fail; k < min(nch, k_fail + Q); ++k) mbar_wait_drain(&bars[k % Q], (uint32_t)(k / Q) & 1u);
+}
+
+// Backward.  A run covers tokens n0 .. n_end - 1 (du and dwh rows); its stream runs from
+// n0 - K + 1 (the rows of u that dwh reaches back to) to n_end + K - 2 (the rows of g whose
+// filters reach back into the run).  du is accumulated forward: token n adds wh[n, j] g[n] to
+// the pending du row n - j, which takes the terms of du[m] in the order j = 0 .. K - 1; row
+// n - K + 1 is then complete and stored.  Chunk: g rows, u rows ([T][512 B] each), taps rows.
+// With RoPE the blocks of rotated channels read g from R^T g (tm_gr, written beforehand).
+template <int K>
+__global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__ CUtensorMap tm_g,
+                                                         const __grid_constant__ CUtensorMap tm_gr,
+                                                         const __grid_constant__ CUtensorMap tm_u,
+                                                         const __grid_constant__ CUtensorMap tm_w, int R, int hd,
+                                                         int32_t N, int64_t C, int32_t seqlen,
+                                                         const int32_t* __restrict__ cu, int32_t n_docs, int n_cblk,
+                                                         __nv_bfloat16* __restrict__ du,
+                                                         __nv_bfloat16* __restrict__ dwh, int rope_n, int run,
+                                                         int taps_box, uint32_t* err) {
+    constexpr int T = HwTile<K>::T, Q = HwTile<K>::Q;
+    extern __shared__ __align__(128) uint8_t hw_smem[];
+    __shared__ uint64_t bars[Q];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+        for (int s = 0; s < Q; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        abort_flag = 0;
+        tma_prefetch(&tm_g);
+        tma_prefetch(&tm_gr);
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_w);
+    }
+    __syncwarp();
+    pdl_trigger();
+    pdl_wait();
+    const int32_t cb = (int32_t)(blockIdx.x % (uint32_t)n_cblk);
+    const int32_t n0 = (int32_t)(blockIdx.x / (uint32_t)n_cblk) * run;
+    const int32_t c0 = cb * 256, c = c0 + lane * 8;
+    const int q = c / hd, x0 = ((c0 / hd) * K) & ~7;
+    const int L = hd >> 3, tl = q * K - x0;
+    const int32_t n_end = min(n0 + run, N);
+    const int nb = n_end - n0, len = nb + 2 * (K - 1), nch = (len + T - 1) / T;
+    const CUtensorMap* tg = c0 < rope_n ? &tm_gr : &tm_g;
+    const uint32_t tpitch = (uint32_t)taps_box * 2u, toff = T * 1024u;
+    const uint32_t chunk = al128(toff + T * tpitch);
+    auto issue = [&](int k) {                        // lane 0
+        if (k >= nch) return;
+        const int32_t row0 = n0 - (K - 1) + k * T;
+        uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
+        uint64_t* bar = &bars[k % Q];
+        mbar_arrive_expect_tx(bar, T * 1024u + T * tpitch);
+        tma_load_2d_hint(sl, tg, bar, c0, row0, l2_evict_first());
+        tma_load_2d_hint(sl + T * 512, &tm_u, bar, c0, row0, l2_evict_first());
+        tma_load_2d(sl + toff, &tm_w, bar, x0, row0);
+    };
+    if (lane == 0)
+        for (int k = 0; k < Q - 1; ++k) issue(k);
+    SegWalk walk;
+    __nv_bfloat16* dup = du + (int64_t)n0 * C + c;
+    __nv_bfloat16* dwp = dwh + (int64_t)n0 * R + q * K;
+    float uw[K][8];                                  // u row of stream index r at uw[r mod K]
+    float acc[K][8];                                 // pending du row of stream index r at acc[r mod K]
+    auto body = [&](const uint8_t* sl, int r0, auto full) {
+        constexpr bool FULL = decltype(full)::value;
+#pragma unroll
+        for (int s = 0; s < T; ++s) {
+            const int r = r0 + s;
+            if (!FULL && r >= len) break;
+            const int32_t n = n0 - (K - 1) + r;
+            if (FULL || n < n_end) unpack8(*reinterpret_cast<const uint4*>(sl + (T + s) * 512 + lane * 16), uw[s % K]);
+            if (!FULL && n < n0) continue;
+            const int32_t pos = (FULL || n < N) ? walk.pos(n, cu, n_docs, seqlen, N) : 0;
+            float gf[8], w[K];
+            unpack8(*reinterpret_cast<const uint4*>(sl + s * 512 + lane * 16), gf);
+            load_taps<K>(reinterpret_cast<const __nv_bfloat16*>(sl + toff + s * tpitch) + tl, w);
+            // du: a new row for token n, then token n's term of the pending rows n - 1 .. n - K + 1
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[s % K][e] = gf[e];
+            axpy8f(acc[s % K], w[0], gf);
+#pragma unroll
+            for (int j = 1; j < K; ++j)
+                if (FULL || n - j >= n0) axpy8f(acc[(s - j + K) % K], j <= pos ? w[j] : 0.f, gf);
+            if (FULL || n < n_end) {                 // dwh[n, q K + j] = sum over the head of g[n] . u[n - j]
+                float part[K];
+#pragma unroll
+                for (int j = 0; j < K; ++j) part[j] = dot8f(gf, uw[(s - j + K) % K]);
+                head_sum_store<K>(part, L, lane, pos, true, dwp);
+                dwp += R;
+            }
+            if (FULL || n - (K - 1) >= n0) {         // row n - K + 1 is complete
+                *reinterpret_cast<uint4*>(dup) = pack8(acc[(s + 1) % K]);
+                dup += C;
+            }
+        }
+    };
+    int k_fail = -1;
+    for (int k = 0; k < nch; ++k) {
+        __syncwarp();                                // slot k - 1, which chunk k + Q - 1 refills, is read
+        if (lane == 0) {
+            fence_async_smem();
+            issue(k + Q - 1);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[k % Q], (uint32_t)(k / Q) & 1u, &abort_flag, err))) {
+            k_fail = k;
+            break;
+        }
+        const uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
+        const int r0 = k * T;
+        if (r0 >= 2 * (K - 1) && r0 + T <= K - 1 + nb) body(sl, r0, std::true_type{});
+        else body(sl, r0, std::false_type{});
+    }
+    if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
+        for (int k = k_fail; k < min(nch, k_fail + Q); ++k) mbar_wait_drain(&bars[k % Q], (uint32_t)(k / Q) & 1u);
 }
 
 // ---- channel-first layout: u, y, g, du are [batch * C, seqlen] rows (tokens contiguous) ----
@@ -454,19 +589,31 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __nv_bfloat16
     }
 }
 
-// gr[n, c] = (R^T g)[n, c] for the rotated channels c < rope_n (bf16, token-major), blocks striding over tokens.
+// gr[n, c] = (R^T g)[n, c] for the rotated channels c < rope_n and g[n, c] for rope_n <= c < gr_w
+// (bf16, token-major, rows gr_w wide: whole 256-channel blocks), blocks striding over tokens.
 __global__ void __launch_bounds__(128) rope_rows_kernel(const __nv_bfloat16* __restrict__ g, int64_t C,
-                                                        __nv_bfloat16* __restrict__ gr, int64_t N, int rope_n,
-                                                        int rope_hd, int rope_max, const float* __restrict__ cs,
-                                                        const int32_t* __restrict__ cu, int64_t n_docs,
-                                                        int64_t seqlen) {
+                                                        __nv_bfloat16* __restrict__ gr, int gr_w, int64_t N,
+                                                        int rope_n, int rope_hd, int rope_max,
+                                                        const float* __restrict__ cs, const int32_t* __restrict__ cu,
+                                                        int64_t n_docs, int64_t seqlen) {
     pdl_trigger();
     pdl_wait();
-    rope_rows_bf16(g, C, gr, N, (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5),
+    rope_rows_bf16(g, C, gr, gr_w, N, (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5),
                    (int64_t)gridDim.x * (blockDim.x / 32), rope_n, rope_hd, rope_max, cs, cu, n_docs, seqlen, true);
 }
 
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Width of the R^T g rows the token-major backward reads: the rotated channels rounded up to
+// whole 256-channel blocks (the channels past rope_n copied), so a block reads g from one tensor.
+inline int64_t hw_gr_width(const Prob& p) { return std::min<int64_t>(p.C, (p.rope_n + 255) / 256 * 256); }
+
+// Columns of a block's taps box in wh [N, R]: the K taps of each of its heads, from the first
+// one rounded down to a multiple of 8 columns (TMA copies start on 16-byte boundaries).
+inline int hw_taps_box(const Prob& p) {
+    const int heads = (int)std::max<int64_t>(1, 256 / p.hd);
+    return ((int)p.K * heads + 7 + 7) / 8 * 8;
+}
 
 // Rows of the RoPE table as an int (at least 1; positions are clamped below it).
 inline int rope_rows(const Prob& p) { return (int)std::max<int64_t>(1, std::min<int64_t>(p.rope_max, INT32_MAX)); }
@@ -480,7 +627,7 @@ TcHwLayout tc_hw_layout(const Prob& p) {
     L.wh = off;     off = al256(off + (size_t)p.N * p.R * 2);
     L.dwh = off;    off = al256(off + (size_t)p.N * p.R * 2);
     L.dpart = off;  off = al256(off + (size_t)gen_bwd_splits(p.N, p.d, (int)p.R) * p.d * p.R * 4);
-    L.gr = off;     off = al256(off + (size_t)p.N * p.rope_n * 2);                  // RoPE: R^T g, rotated channels
+    L.gr = off;     off = al256(off + (size_t)p.N * (p.rope_n > 0 ? hw_gr_width(p) : 0) * 2);  // RoPE: R^T g
     L.total = off;
     return L;
 }
@@ -491,8 +638,10 @@ bool tc_headwise_supported(const Prob& p) {
     if (p.K < 1 || p.K > 4) return false;
     if (p.layout == 1) return cf_tiles_ok(p) && p.H < 65536;
     if (p.hd < 8 || p.hd > 256 || (p.hd & (p.hd - 1)) != 0) return false;
-    // one grid row per kTokPerBlock tokens (grid y up to 65535), 32-bit token indices
-    return p.C % 256 == 0 && p.N < int64_t(kTokPerBlock) * 65535;
+    if (p.rope_n > 0 && p.rope_hd > kHwMaxRopeHd) return false;   // one table row per slot
+    // one block per (run, 256-channel block), 32-bit token indices
+    return p.C % 256 == 0 && p.N < (int64_t(1) << 31) - 2 * std::max(kHwRunFwd, kHwRunBwd) &&
+           (p.N / std::min(kHwRunFwd, kHwRunBwd) + 1) * (p.C / 256) < (int64_t(1) << 31);
 }
 
 // Channel-first: 8 tokens per lane in the forward, 4 in the backward (fewer registers for
@@ -500,7 +649,8 @@ bool tc_headwise_supported(const Prob& p) {
 constexpr int kCfFwdV = 8, kCfBwdV = 4;
 
 template <int K>
-static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, cudaStream_t st) {
+static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, uint32_t* err,
+                                 cudaStream_t st) {
     cudaError_t e;
     if (p.layout == 1) {
         const int64_t tps = (p.seqlen + 32 * kCfFwdV - 1) / (32 * kCfFwdV);
@@ -510,17 +660,29 @@ static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, v
             p.N, p.C, p.seqlen, tps, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
         return e;
     }
-    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
-    DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(256), 0, st,
-        static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
-        p.N, p.C, p.seqlen, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y), p.rope_n > 0 ? p.rope_cs : nullptr,
-        (int)p.rope_n, p.rope_n > 0 ? (int)p.rope_hd : 1, rope_rows(p)));
+    const int n_cblk = (int)(p.C / 256);
+    const dim3 grid((unsigned)(n_cblk * ((p.N + kHwRunFwd - 1) / kHwRunFwd)));
+    const bool rope = p.rope_n > 0;
+    const int box = hw_taps_box(p);
+    constexpr uint32_t T = HwTile<K>::T, Q = HwTile<K>::Q;
+    const uint32_t roff = al128(T * 512u) + al128(T * (uint32_t)box * 2u);
+    const int smem = (int)(Q * al128(roff + (rope ? T * (uint32_t)p.rope_hd * 4u : 0u)));
+    e = cudaFuncSetAttribute(hw_conv_fwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tu, tw;
+    if (!make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.C, p.N, p.us * 2, 256, T, false) ||
+        !make_tmap_2d(&tw, wh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.R, p.N, p.R * 2, box, T, false))
+        return cudaErrorInvalidValue;
+    DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_kernel<K>, grid, dim3(32), smem, st, tu, tw, (int)p.hd,
+        (int32_t)p.N, p.C, (int32_t)p.seqlen, p.cu, (int32_t)p.n_docs, n_cblk, static_cast<__nv_bfloat16*>(y),
+        rope ? p.rope_cs : nullptr,
+        (int)p.rope_n, rope ? (int)p.rope_hd : 8, rope_rows(p), kHwRunFwd, box, err));
     return e;
 }
 
 template <int K>
 static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, const void* wh, void* du, void* dwh,
-                                 const void* gr, cudaStream_t st) {
+                                 const void* gr, uint32_t* err, cudaStream_t st) {
     cudaError_t e;
     if (p.layout == 1) {
         const int64_t tps = (p.seqlen + 32 * kCfBwdV - 1) / (32 * kCfBwdV);
@@ -531,12 +693,28 @@ static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, co
             static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
         return e;
     }
-    const dim3 grid((unsigned)(p.C / 256), (unsigned)((p.N + kTokPerBlock - 1) / kTokPerBlock));
-    DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_kernel<K>, grid, dim3(256), 0, st,
-        static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
-        static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, p.cu, p.n_docs,
-        static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh), static_cast<const __nv_bfloat16*>(gr),
-        (int)p.rope_n));
+    const int n_cblk = (int)(p.C / 256);
+    const dim3 grid((unsigned)(n_cblk * ((p.N + kHwRunBwd - 1) / kHwRunBwd)));
+    const int box = hw_taps_box(p);
+    constexpr uint32_t T = HwTile<K>::T, Q = HwTile<K>::Q;
+    const int smem = (int)(Q * al128(T * 1024u + T * (uint32_t)box * 2u));
+    e = cudaFuncSetAttribute(hw_conv_bwd_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tg, tgr, tu, tw;
+    if (!make_tmap_2d(&tg, g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.C, p.N, p.C * 2, 256, T, false) ||
+        !make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.C, p.N, p.us * 2, 256, T, false) ||
+        !make_tmap_2d(&tw, wh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.R, p.N, p.R * 2, box, T, false))
+        return cudaErrorInvalidValue;
+    tgr = tg;
+    if (gr) {
+        const int64_t w = hw_gr_width(p);
+        if (!make_tmap_2d(&tgr, gr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, p.N, w * 2, 256, T, false))
+            return cudaErrorInvalidValue;
+    }
+    DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_kernel<K>, grid, dim3(32), smem, st, tg, tgr, tu, tw,
+        (int)p.R, (int)p.hd, (int32_t)p.N, p.C, (int32_t)p.seqlen, p.cu, (int32_t)p.n_docs, n_cblk,
+        static_cast<__nv_bfloat16*>(du),
+        static_cast<__nv_bfloat16*>(dwh), gr ? (int)p.rope_n : 0, kHwRunBwd, box, err));
     return e;
 }
 
@@ -547,10 +725,10 @@ cudaError_t tc_headwise_forward(const Prob& p, const void* u, const void* h, con
     cudaError_t e = tc_gen_launch(h, p.hs, W, p.N, p.d, (int)p.R, wh, p.R, err, st);
     if (e != cudaSuccess) return e;
     switch (p.K) {
-        case 1: return launch_hw_fwd<1>(p, u, wh, y, st);
-        case 2: return launch_hw_fwd<2>(p, u, wh, y, st);
-        case 3: return launch_hw_fwd<3>(p, u, wh, y, st);
-        default: return launch_hw_fwd<4>(p, u, wh, y, st);
+        case 1: return launch_hw_fwd<1>(p, u, wh, y, err, st);
+        case 2: return launch_hw_fwd<2>(p, u, wh, y, err, st);
+        case 3: return launch_hw_fwd<3>(p, u, wh, y, err, st);
+        default: return launch_hw_fwd<4>(p, u, wh, y, err, st);
     }
 }
 
@@ -572,15 +750,16 @@ cudaError_t tc_headwise_backward(const Prob& p, const void* g, const void* u, co
         gr = tcws + L.gr;
         DC_LAUNCH(kTcPrep, st, e = launch_pdl(rope_rows_kernel, dim3((unsigned)std::min<int64_t>(p.N, 148 * 8)),
                                               dim3(128), 0, st, static_cast<const __nv_bfloat16*>(g), p.C,
-                                              static_cast<__nv_bfloat16*>(gr), p.N, (int)p.rope_n, (int)p.rope_hd,
+                                              static_cast<__nv_bfloat16*>(gr), (int)hw_gr_width(p), p.N,
+                                              (int)p.rope_n, (int)p.rope_hd,
                                               rope_rows(p), p.rope_cs, p.cu, p.n_docs, p.seqlen));
         if (e != cudaSuccess) return e;
     }
     switch (p.K) {
-        case 1: e = launch_hw_bwd<1>(p, g, u, wh, du, dwh, gr, st); break;
-        case 2: e = launch_hw_bwd<2>(p, g, u, wh, du, dwh, gr, st); break;
-        case 3: e = launch_hw_bwd<3>(p, g, u, wh, du, dwh, gr, st); break;
-        default: e = launch_hw_bwd<4>(p, g, u, wh, du, dwh, gr, st); break;
+        case 1: e = launch_hw_bwd<1>(p, g, u, wh, du, dwh, gr, err, st); break;
+        case 2: e = launch_hw_bwd<2>(p, g, u, wh, du, dwh, gr, err, st); break;
+        case 3: e = launch_hw_bwd<3>(p, g, u, wh, du, dwh, gr, err, st); break;
+        default: e = launch_hw_bwd<4>(p, g, u, wh, du, dwh, gr, err, st); break;
     }
     if (e != cudaSuccess) return e;
     return tc_gen_backward(dwh, (int)p.R, h, p.hs, W, p.N, p.d, dh, dW, reinterpret_cast<float*>(tcws + L.dpart),
