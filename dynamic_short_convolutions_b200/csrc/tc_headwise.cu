@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__
         uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
         uint64_t* bar = &bars[k % Q];
         mbar_arrive_expect_tx(bar, T * 512u + T * tpitch + (rope_blk ? T * rrow : 0u));
-        tma_load_2d_hint(sl, &tm_u, bar, c0, row0, l2_evict_first());
+        tma_load_2d(sl, &tm_u, bar, c0, row0);
         tma_load_2d(sl + toff, &tm_w, bar, x0, row0);
         if (rope_blk) {
 #pragma unroll
@@ -314,8 +314,8 @@ __global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__
         uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
         uint64_t* bar = &bars[k % Q];
         mbar_arrive_expect_tx(bar, T * 1024u + T * tpitch);
-        tma_load_2d_hint(sl, tg, bar, c0, row0, l2_evict_first());
-        tma_load_2d_hint(sl + T * 512, &tm_u, bar, c0, row0, l2_evict_first());
+        tma_load_2d(sl, tg, bar, c0, row0);
+        tma_load_2d(sl + T * 512, &tm_u, bar, c0, row0);
         tma_load_2d(sl + toff, &tm_w, bar, x0, row0);
     };
     if (lane == 0)
