@@ -42,7 +42,7 @@ using namespace tc;
 // bounds.  The rows of u (and the backward's pending du rows) sit in rolling register windows,
 // so a row is read and unpacked once; only the K - 1 rows of u before a run (and of g after it)
 // are read twice.
-constexpr int kHwRunFwd = 32, kHwRunBwd = 32;      // tokens per run (one warp, one block)
+constexpr int kHwRunFwd = 16, kHwRunBwd = 32;      // tokens per run (one warp, one block)
 constexpr int kHwMaxRopeHd = 256;                  // RoPE table rows of up to 256 floats (1 KB)
 
 // Segment bounds [s, e) of the tokens a warp walks through in increasing order: looked up again
@@ -153,7 +153,8 @@ __device__ __forceinline__ void head_sum_store(float (&p)[K], int L, int gl, int
 // block b takes channel block b % n_cblk and tokens (b / n_cblk) * run onwards, so everything
 // that depends on the token position is uniform over the block and only the channel offset
 // varies by lane.  Chunks whose rows are all interior (no look-back, look-ahead or end of the
-// tensor among them) run a body without the per-row range tests.
+// tensor among them) run a body without the per-row range tests, and without the taps' segment
+// mask when none of their rows is within K - 1 tokens of a segment start.
 template <int K>
 struct HwTile {
     static constexpr int T = K >= 3 ? K : 4;     // stream rows per chunk
@@ -166,7 +167,7 @@ __host__ __device__ constexpr uint32_t al128(uint32_t x) { return (x + 127u) & ~
 // taps' reach back).  Chunk: u rows [T][512 B], taps rows [T][taps_box], RoPE table rows
 // [T][rope_hd floats].
 template <int K>
-__global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__ CUtensorMap tm_u,
+__global__ void __launch_bounds__(32, 24) hw_conv_fwd_kernel(const __grid_constant__ CUtensorMap tm_u,
                                                          const __grid_constant__ CUtensorMap tm_w, int hd, int32_t N,
                                                          int64_t C, int32_t seqlen, const int32_t* __restrict__ cu,
                                                          int32_t n_docs, int n_cblk, __nv_bfloat16* __restrict__ y,
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__
         for (int k = 0; k < Q - 1; ++k) issue(k);
     __nv_bfloat16* yp = y + (int64_t)n0 * C + c;
     float win[K][8];                                 // u row of stream index r at win[r mod K]
-    auto body = [&](const uint8_t* sl, int r0, auto full) {
-        constexpr bool FULL = decltype(full)::value;
+    auto body = [&](const uint8_t* sl, int r0, auto full, auto masked) {
+        constexpr bool FULL = decltype(full)::value, MASK = decltype(masked)::value;
 #pragma unroll
         for (int s = 0; s < T; ++s) {
             const int r = r0 + s;
@@ -229,14 +230,14 @@ __global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__
             unpack8(*reinterpret_cast<const uint4*>(sl + s * 512 + lane * 16), win[s % K]);
             const int32_t n = n0 - (K - 1) + r;
             if (!FULL && n < n0) continue;
-            const int32_t pos = walk.pos(n, cu, n_docs, seqlen, N);
+            const int32_t pos = MASK ? walk.pos(n, cu, n_docs, seqlen, N) : K;
             float w[K];
             load_taps<K>(reinterpret_cast<const __nv_bfloat16*>(sl + toff + s * tpitch) + tl, w);
             float acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = win[s % K][e];
 #pragma unroll
-            for (int j = 0; j < K; ++j) axpy8f(acc, j <= pos ? w[j] : 0.f, win[(s - j + K) % K]);
+            for (int j = 0; j < K; ++j) axpy8f(acc, (!MASK || j <= pos) ? w[j] : 0.f, win[(s - j + K) % K]);
             if (rot) {
                 const float4* t = reinterpret_cast<const float4*>(sl + roff + s * rrow + rl * 4);
                 rope_pairs8v(acc, t[0], t[1], false);
@@ -258,8 +259,16 @@ __global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__
         }
         const uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
         const int r0 = k * T;
-        if (r0 >= K - 1 && r0 + T <= len) body(sl, r0, std::true_type{});
-        else body(sl, r0, std::false_type{});
+        if (r0 >= K - 1 && r0 + T <= len) {
+            // no row of the chunk within K - 1 of a segment start: the taps need no mask
+            const int32_t nf = n0 - (K - 1) + r0;
+            if (walk.pos(nf, cu, n_docs, seqlen, N) >= K - 1 && nf + T <= walk.e)
+                body(sl, r0, std::true_type{}, std::false_type{});
+            else
+                body(sl, r0, std::true_type{}, std::true_type{});
+        } else {
+            body(sl, r0, std::false_type{}, std::true_type{});
+        }
     }
     if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
         for (int k = k_fail; k < min(nch, k_fail + Q); ++k) mbar_wait_drain(&bars[k % Q], (uint32_t)(k / Q) & 1u);
@@ -272,7 +281,7 @@ __global__ void __launch_bounds__(32) hw_conv_fwd_kernel(const __grid_constant__
 // n - K + 1 is then complete and stored.  Chunk: g rows, u rows ([T][512 B] each), taps rows.
 // With RoPE the blocks of rotated channels read g from R^T g (tm_gr, written beforehand).
 template <int K>
-__global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__ CUtensorMap tm_g,
+__global__ void __launch_bounds__(32, 16) hw_conv_bwd_kernel(const __grid_constant__ CUtensorMap tm_g,
                                                          const __grid_constant__ CUtensorMap tm_gr,
                                                          const __grid_constant__ CUtensorMap tm_u,
                                                          const __grid_constant__ CUtensorMap tm_w, int R, int hd,
@@ -325,8 +334,8 @@ __global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__
     __nv_bfloat16* dwp = dwh + (int64_t)n0 * R + q * K;
     float uw[K][8];                                  // u row of stream index r at uw[r mod K]
     float acc[K][8];                                 // pending du row of stream index r at acc[r mod K]
-    auto body = [&](const uint8_t* sl, int r0, auto full) {
-        constexpr bool FULL = decltype(full)::value;
+    auto body = [&](const uint8_t* sl, int r0, auto full, auto masked) {
+        constexpr bool FULL = decltype(full)::value, MASK = decltype(masked)::value;
 #pragma unroll
         for (int s = 0; s < T; ++s) {
             const int r = r0 + s;
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__
             const int32_t n = n0 - (K - 1) + r;
             if (FULL || n < n_end) unpack8(*reinterpret_cast<const uint4*>(sl + (T + s) * 512 + lane * 16), uw[s % K]);
             if (!FULL && n < n0) continue;
-            const int32_t pos = (FULL || n < N) ? walk.pos(n, cu, n_docs, seqlen, N) : 0;
+            const int32_t pos = !MASK ? K : (FULL || n < N) ? walk.pos(n, cu, n_docs, seqlen, N) : 0;
             float gf[8], w[K];
             unpack8(*reinterpret_cast<const uint4*>(sl + s * 512 + lane * 16), gf);
             load_taps<K>(reinterpret_cast<const __nv_bfloat16*>(sl + toff + s * tpitch) + tl, w);
@@ -344,7 +353,7 @@ __global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__
             axpy8f(acc[s % K], w[0], gf);
 #pragma unroll
             for (int j = 1; j < K; ++j)
-                if (FULL || n - j >= n0) axpy8f(acc[(s - j + K) % K], j <= pos ? w[j] : 0.f, gf);
+                if (FULL || n - j >= n0) axpy8f(acc[(s - j + K) % K], (!MASK || j <= pos) ? w[j] : 0.f, gf);
             if (FULL || n < n_end) {                 // dwh[n, q K + j] = sum over the head of g[n] . u[n - j]
                 float part[K];
 #pragma unroll
@@ -371,8 +380,16 @@ __global__ void __launch_bounds__(32) hw_conv_bwd_kernel(const __grid_constant__
         }
         const uint8_t* sl = hw_smem + (uint32_t)(k % Q) * chunk;
         const int r0 = k * T;
-        if (r0 >= 2 * (K - 1) && r0 + T <= K - 1 + nb) body(sl, r0, std::true_type{});
-        else body(sl, r0, std::false_type{});
+        if (r0 >= 2 * (K - 1) && r0 + T <= K - 1 + nb) {
+            // no row of the chunk within K - 1 of a segment start: the taps need no mask
+            const int32_t nf = n0 - (K - 1) + r0;
+            if (walk.pos(nf, cu, n_docs, seqlen, N) >= K - 1 && nf + T <= walk.e)
+                body(sl, r0, std::true_type{}, std::false_type{});
+            else
+                body(sl, r0, std::true_type{}, std::true_type{});
+        } else {
+            body(sl, r0, std::false_type{}, std::true_type{});
+        }
     }
     if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
         for (int k = k_fail; k < min(nch, k_fail + Q); ++k) mbar_wait_drain(&bars[k % Q], (uint32_t)(k / Q) & 1u);
