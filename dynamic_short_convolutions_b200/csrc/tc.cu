@@ -615,7 +615,7 @@ const char* tc_unsupported_reason(const Prob& p, bool bwd) {
         if (!tc_headwise_supported(p))
             return "head-wise tensor-core kernels need H*K a multiple of 8 up to 128, d a multiple of 8, and "
                    "(token-major) head_dim a power of two in [8, 256] with channels a multiple of 256, or "
-                   "(channel-first) seqlen and u_row_stride multiples of 8";
+                   "(channel-first) seqlen and u_row_stride multiples of 8 and head_dim at most 512";
         return nullptr;
     }
     if (p.r % 8 != 0 || p.r > 64) return "low-rank tensor-core kernels need the rank a multiple of 8 up to 64";

@@ -11,9 +11,9 @@
 //   dW = h^T dwh,  dh = dwh W^T                                        (tensor cores)
 // The conv kernels are memory-bound CUDA-core kernels: token-major (a warp streams consecutive
 // tokens through per-lane cp.async rings in shared memory, 16-byte loads and stores along C,
-// packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh) and channel-first
-// (loads along the token rows of [batch * C, seqlen], a lane's filter taps held across the
-// head's channels, dwh summed per warp and then over the block's warps in order).
+// packed fp32 FMAs, a reduce-scatter over each head's lanes for dwh) and channel-first (a warp
+// streams a head's token rows of [batch * C, seqlen] through a TMA ring, a lane's filter taps held
+// across the head's channels, dwh summed per warp and then over the block's warps in order).
 #include <algorithm>
 #include <type_traits>
 
@@ -396,212 +396,267 @@ __global__ void __launch_bounds__(32, 16) hw_conv_bwd_kernel(const __grid_consta
 }
 
 // ---- channel-first layout: u, y, g, du are [batch * C, seqlen] rows (tokens contiguous) ----
-// A block is 8 warps on one sequence b, tokens t0 .. t0 + 32 V - 1 (V consecutive tokens per
-// lane, one 8- or 16-byte load per row), and one head q; warp w takes channels w, w + 8, ... of
-// the head, so a lane's filter taps stay in registers across the head's channels.  The K - 1
-// tokens before a lane's first come from the previous lane by shuffle (lane 0 loads them), the
-// K - 1 after its last from the next lane (lane 31 loads them).  seqlen is a multiple of 8, so a
-// lane's V tokens are all inside the sequence or all past its end.
+// A warp takes a window of kCfW tokens t0 .. t0 + kCfW - 1 of one sequence b and up to kCfCPW
+// channel rows of one head q; lane l takes tokens t0 + 8 l .. t0 + 8 l + 7, whose filter taps (masked
+// for the segment) stay in registers across the channels.  The rows come kCfCH at a time through
+// a TMA ring in shared memory: the window (box {kCfW, kCfCH}) and 8 tokens beside it (box
+// {8, kCfCH}: before the window for u, after it for g), so each lane finds its K - 1 <= 3
+// neighbours in its row of the chunk.  seqlen is a multiple of 8, so a lane's 8 tokens are all
+// inside the sequence or all past its end (rows past the end read zero).
+constexpr int kCfW = 256;                          // tokens per window (8 per lane)
+constexpr int kCfCH = 2;                           // channel rows per chunk
+constexpr int kCfQ = 4;                            // ring slots (chunks)
+constexpr int kCfCPW = 64;                         // channel rows per warp
+// Chunk layouts (every TMA destination on a 128-byte boundary): forward u window, u 8 before;
+// backward g window, g 8 after, u window, u 8 before.
+constexpr uint32_t kCfFwdUh = kCfCH * 2 * kCfW, kCfFwdChunk = al128(kCfFwdUh + kCfCH * 16);
+constexpr uint32_t kCfBwdGa = kCfCH * 2 * kCfW, kCfBwdU = al128(kCfBwdGa + kCfCH * 16);
+constexpr uint32_t kCfBwdUh = kCfBwdU + kCfCH * 2 * kCfW, kCfBwdChunk = al128(kCfBwdUh + kCfCH * 16);
+static_assert(kCfFwdUh % 128 == 0 && kCfFwdChunk % 128 == 0 && kCfBwdGa % 128 == 0 && kCfBwdU % 128 == 0 &&
+                  kCfBwdUh % 128 == 0 && kCfBwdChunk % 128 == 0,
+              "TMA destinations in shared memory start on 128-byte boundaries");
 
-// V bf16 values of one row, as V / 2 packed pairs.
-template <int V>
-__device__ __forceinline__ void ldrow(const __nv_bfloat16* __restrict__ p, uint32_t (&w)[V / 2]) {
-    if constexpr (V == 8) {
-        const uint4 t = *reinterpret_cast<const uint4*>(p);
-        w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
-    } else {
-        const uint2 t = *reinterpret_cast<const uint2*>(p);
-        w[0] = t.x; w[1] = t.y;
-    }
-}
-template <int V>
-__device__ __forceinline__ void strow(__nv_bfloat16* __restrict__ p, const float (&f)[V]) {
-    if constexpr (V == 8) {
-        *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                                  pack_bf16(f[6], f[7]));
-    } else {
-        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
-    }
-}
-// Element i (0 <= i < 2 P) of P packed bf16 pairs.
-template <int P>
-__device__ __forceinline__ float elem(const uint32_t (&w)[P], int i) {
-    return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-}
-
-// Row values of tokens t - 4 .. t + V - 1 (prev = the 4 before the lane's first) and, for the
-// backward, t + V .. t + V + 3 (next), for a lane whose V tokens start at t.
-template <int V>
-__device__ __forceinline__ void row_halo_prev(const __nv_bfloat16* __restrict__ row, const uint32_t (&cur)[V / 2],
-                                              int lane, int64_t t, bool live, uint32_t (&prev)[2]) {
-    prev[0] = __shfl_up_sync(0xffffffffu, cur[V / 2 - 2], 1);
-    prev[1] = __shfl_up_sync(0xffffffffu, cur[V / 2 - 1], 1);
-    if (lane == 0) {
-        if (live && t >= 4) {
-            const uint2 v = *reinterpret_cast<const uint2*>(row + t - 4);
-            prev[0] = v.x;
-            prev[1] = v.y;
-        } else {
-            prev[0] = prev[1] = 0u;
-        }
-    }
-}
-template <int V>
-__device__ __forceinline__ void row_halo_next(const __nv_bfloat16* __restrict__ row, const uint32_t (&cur)[V / 2],
-                                              int lane, int64_t t, int64_t T, uint32_t (&next)[2]) {
-    next[0] = __shfl_down_sync(0xffffffffu, cur[0], 1);
-    next[1] = __shfl_down_sync(0xffffffffu, cur[1], 1);
-    if (lane == 31) {
-        if (t + V < T) {
-            const uint2 v = *reinterpret_cast<const uint2*>(row + t + V);
-            next[0] = v.x;
-            next[1] = v.y;
-        } else {
-            next[0] = next[1] = 0u;
-        }
-    }
+// 8 bf16 of a row as floats / the 4 before them, from shared memory.
+__device__ __forceinline__ void lds8(const uint8_t* p, float (&f)[8]) { unpack8(*reinterpret_cast<const uint4*>(p), f); }
+__device__ __forceinline__ void lds4(const uint8_t* p, float (&f)[4]) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    f[0] = bf16_lo(v.x);
+    f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y);
+    f[3] = bf16_hi(v.y);
 }
 
 // y[c, t] = u[c, t] + sum_{j <= t - s(t)} wh[t, q K + j] u[c, t - j]  (the same FMA order as the
-// token-major kernel, so both layouts give the same bits).
-template <int K, int V>
-__global__ void __launch_bounds__(256) hw_conv_fwd_cf_kernel(const __nv_bfloat16* __restrict__ u, int64_t us,
-                                                             const __nv_bfloat16* __restrict__ wh, int R, int hd,
-                                                             int64_t N, int64_t C, int64_t T, int64_t tps,
-                                                             const int32_t* __restrict__ cu, int64_t n_docs,
-                                                             __nv_bfloat16* __restrict__ y) {
+// token-major kernel, so both layouts give the same bits).  Blocks: (b, window, head, part).
+template <int K>
+__global__ void __launch_bounds__(32, 24) hw_conv_fwd_cf_kernel(const __grid_constant__ CUtensorMap tm_u,
+                                                                const __grid_constant__ CUtensorMap tm_uh,
+                                                                const __nv_bfloat16* __restrict__ wh, int R, int hd,
+                                                                int64_t C, int64_t T, int64_t tps, int parts, int H,
+                                                                const int32_t* __restrict__ cu, int64_t n_docs,
+                                                                __nv_bfloat16* __restrict__ y, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t hw_smem[];
+    __shared__ uint64_t bars[kCfQ];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+        for (int s = 0; s < kCfQ; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        abort_flag = 0;
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_uh);
+    }
+    __syncwarp();
     pdl_trigger();
     pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t b = blockIdx.x / tps;
-    const int64_t t = (blockIdx.x - b * tps) * (32 * V) + lane * V;
-    const int q = blockIdx.y;
+    int64_t unit = blockIdx.x;
+    const int part = (int)(unit % parts);
+    unit /= parts;
+    const int q = (int)(unit % H);
+    unit /= H;
+    const int64_t win = unit % tps, b = unit / tps;
+    const int64_t t0 = win * kCfW, t = t0 + 8 * lane;
     const bool live = t < T;
+    const int c_begin = q * hd + part * kCfCPW, nrows = min(kCfCPW, hd - part * kCfCPW);
+    const int nch = (nrows + kCfCH - 1) / kCfCH;
     const int64_t n0 = b * T + t;
-    float w[V][K];
-    int32_t pos[V];
+    float wm[8][K];                                  // taps of the lane's tokens, masked for the segment
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
+    for (int i = 0; i < 8; ++i) {
         if (live) {
-            load_taps<K>(wh + (n0 + i) * R + q * K, w[i]);
-            pos[i] = (int32_t)(n0 + i - seg_start(n0 + i, cu, n_docs, T));
+            load_taps<K>(wh + (n0 + i) * R + q * K, wm[i]);
+            const int64_t pos = n0 + i - seg_start(n0 + i, cu, n_docs, T);
+#pragma unroll
+            for (int j = 0; j < K; ++j) wm[i][j] = j <= pos ? wm[i][j] : 0.f;
         } else {
 #pragma unroll
-            for (int j = 0; j < K; ++j) w[i][j] = 0.f;
-            pos[i] = 0;
+            for (int j = 0; j < K; ++j) wm[i][j] = 0.f;
         }
     }
-    for (int c = q * hd + warp; c < (q + 1) * hd; c += 8) {
-        const __nv_bfloat16* urow = u + (b * C + c) * us;
-        uint32_t cur[V / 2], prev[2];
-        if (live) ldrow<V>(urow + t, cur);
-        else
+    auto issue = [&](int k) {                        // lane 0
+        if (k >= nch) return;
+        uint8_t* sl = hw_smem + (uint32_t)(k % kCfQ) * kCfFwdChunk;
+        uint64_t* bar = &bars[k % kCfQ];
+        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfCH);
+        mbar_arrive_expect_tx(bar, kCfCH * (2 * kCfW + 16));
+        tma_load_2d(sl, &tm_u, bar, (int32_t)t0, row0);
+        tma_load_2d(sl + kCfFwdUh, &tm_uh, bar, (int32_t)t0 - 8, row0);
+    };
+    if (lane == 0)
+        for (int k = 0; k < kCfQ - 1; ++k) issue(k);
+    int k_fail = -1;
+    for (int k = 0; k < nch; ++k) {
+        __syncwarp();                                // slot k - 1, which chunk k + kCfQ - 1 refills, is read
+        if (lane == 0) {
+            fence_async_smem();
+            issue(k + kCfQ - 1);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[k % kCfQ], (uint32_t)(k / kCfQ) & 1u, &abort_flag, err))) {
+            k_fail = k;
+            break;
+        }
+        const uint8_t* sl = hw_smem + (uint32_t)(k % kCfQ) * kCfFwdChunk;
 #pragma unroll
-            for (int k = 0; k < V / 2; ++k) cur[k] = 0u;
-        row_halo_prev<V>(urow, cur, lane, t, live, prev);
-        float acc[V];
+        for (int r = 0; r < kCfCH; ++r) {
+            if (k * kCfCH + r >= nrows) break;
+            const uint8_t* row = sl + r * 2 * kCfW;
+            float x[8], xp[4];                       // tokens t .. t + 7 and t - 4 .. t - 1
+            lds8(row + 16 * lane, x);
+            lds4(lane > 0 ? row + 16 * lane - 8 : sl + kCfFwdUh + r * 16 + 8, xp);
+            float acc[8];
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            acc[i] = elem(cur, i);
+            for (int i = 0; i < 8; ++i) {
+                acc[i] = x[i];
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                const float x = i - j >= 0 ? elem(cur, i - j) : elem(prev, 4 + i - j);
-                acc[i] = fmaf(j <= pos[i] ? w[i][j] : 0.f, x, acc[i]);
+                for (int j = 0; j < K; ++j) acc[i] = fmaf(wm[i][j], i - j >= 0 ? x[i - j] : xp[4 + i - j], acc[i]);
+            }
+            if (live) {
+                const int64_t c = c_begin + k * kCfCH + r;
+                *reinterpret_cast<uint4*>(y + (b * C + c) * T + t) = pack8(acc);
             }
         }
-        if (live) strow<V>(y + (b * C + c) * T + t, acc);
     }
+    if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
+        for (int k = k_fail; k < min(nch, k_fail + kCfQ); ++k)
+            mbar_wait_drain(&bars[k % kCfQ], (uint32_t)(k / kCfQ) & 1u);
 }
 
 // du[c, t] = g[c, t] + sum_{j < e(t) - t} wh[t + j, q K + j] g[c, t + j]; dwh[t, q K + j] =
-// sum_{c in q} [j <= t - s(t)] g[c, t] u[c, t - j]: each warp sums its channels in order, then
-// the block sums the 8 warps' partials in order (no atomics).
-template <int K, int V>
-__global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __nv_bfloat16* __restrict__ g,
-                                                             const __nv_bfloat16* __restrict__ u, int64_t us,
+// sum_{c in q} [j <= t - s(t)] g[c, t] u[c, t - j].  A block is (b, window, head): warp w streams
+// the head's channel rows w kCfCPW .. w kCfCPW + kCfCPW - 1, sums its dwh terms over them in
+// order, then the block sums the warps' partials in order (no atomics).
+template <int K>
+__global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __grid_constant__ CUtensorMap tm_g,
+                                                             const __grid_constant__ CUtensorMap tm_ga,
+                                                             const __grid_constant__ CUtensorMap tm_u,
+                                                             const __grid_constant__ CUtensorMap tm_uh,
                                                              const __nv_bfloat16* __restrict__ wh, int R, int hd,
-                                                             int64_t N, int64_t C, int64_t T, int64_t tps,
+                                                             int64_t N, int64_t C, int64_t T, int64_t tps, int H,
                                                              const int32_t* __restrict__ cu, int64_t n_docs,
                                                              __nv_bfloat16* __restrict__ du,
-                                                             __nv_bfloat16* __restrict__ dwh) {
-    __shared__ float red[8][32 * V][K];
+                                                             __nv_bfloat16* __restrict__ dwh, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t hw_smem[];
+    __shared__ uint64_t bars[8][kCfQ];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (lane == 0) {
+        for (int s = 0; s < kCfQ; ++s) mbar_init(&bars[warp][s], 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        tma_prefetch(&tm_g);
+        tma_prefetch(&tm_ga);
+        tma_prefetch(&tm_u);
+        tma_prefetch(&tm_uh);
+    }
+    __syncthreads();
     pdl_trigger();
     pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t b = blockIdx.x / tps;
-    const int64_t tb = (blockIdx.x - b * tps) * (32 * V);
-    const int64_t t = tb + lane * V;
-    const int q = blockIdx.y;
+    const int q = (int)(blockIdx.x % H);
+    const int64_t rest = blockIdx.x / H, win = rest % tps, b = rest / tps;
+    const int64_t t0 = win * kCfW, t = t0 + 8 * lane;
     const bool live = t < T;
+    const int c_begin = q * hd + warp * kCfCPW, nrows = max(0, min(kCfCPW, hd - warp * kCfCPW));
+    const int nch = (nrows + kCfCH - 1) / kCfCH;
     const int64_t n0 = b * T + t;
-    // wf[i][j]: tap j of the filter of token t + i (i < V + K - 1), zero past the sequence end
-    float wf[V + K - 1][K];
-    int32_t pos[V], epos[V];
+    uint8_t* ring = hw_smem + (uint32_t)warp * kCfQ * kCfBwdChunk;
+    // dm[i][j]: tap j of the filter of token t + i + j for du[t + i], zero past the segment end
+    float dm[8][K];
+    {
+        float wf[8 + K - 1][K];
 #pragma unroll
-    for (int i = 0; i < V + K - 1; ++i) {
-        if (live && t + i < T) load_taps<K>(wh + (n0 + i) * R + q * K, wf[i]);
-        else
+        for (int i = 0; i < 8 + K - 1; ++i) {
+            if (live && t + i < T) load_taps<K>(wh + (n0 + i) * R + q * K, wf[i]);
+            else
 #pragma unroll
-            for (int j = 0; j < K; ++j) wf[i][j] = 0.f;
-    }
+                for (int j = 0; j < K; ++j) wf[i][j] = 0.f;
+        }
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-        if (live) {
-            int64_t sb, eb;
-            seg_bounds(n0 + i, cu, n_docs, T, N, sb, eb);
-            pos[i] = (int32_t)(n0 + i - sb);
-            epos[i] = (int32_t)(eb - 1 - (n0 + i));
-        } else {
-            pos[i] = epos[i] = -1;
+        for (int i = 0; i < 8; ++i) {
+            int64_t sb = 0, eb = 0;
+            if (live) seg_bounds(n0 + i, cu, n_docs, T, N, sb, eb);
+            const int64_t epos = eb - 1 - (n0 + i);
+#pragma unroll
+            for (int j = 0; j < K; ++j) dm[i][j] = (live && j <= epos) ? wf[i + j][j] : 0.f;
         }
     }
-    float dacc[V][K];
+    float dacc[8][K];
 #pragma unroll
-    for (int i = 0; i < V; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < K; ++j) dacc[i][j] = 0.f;
-    for (int c = q * hd + warp; c < (q + 1) * hd; c += 8) {
-        const __nv_bfloat16* grow = g + (b * C + c) * T;
-        const __nv_bfloat16* urow = u + (b * C + c) * us;
-        uint32_t gc[V / 2], uc[V / 2], gn[2], up[2];
-        if (live) {
-            ldrow<V>(grow + t, gc);
-            ldrow<V>(urow + t, uc);
-        } else {
-#pragma unroll
-            for (int k = 0; k < V / 2; ++k) gc[k] = uc[k] = 0u;
+    constexpr uint32_t kGa = kCfBwdGa, kU = kCfBwdU, kUh = kCfBwdUh;
+    auto issue = [&](int k) {                        // lane 0
+        if (k >= nch) return;
+        uint8_t* sl = ring + (uint32_t)(k % kCfQ) * kCfBwdChunk;
+        uint64_t* bar = &bars[warp][k % kCfQ];
+        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfCH);
+        mbar_arrive_expect_tx(bar, 2 * kCfCH * (2 * kCfW + 16));
+        tma_load_2d(sl, &tm_g, bar, (int32_t)t0, row0);
+        tma_load_2d(sl + kGa, &tm_ga, bar, (int32_t)t0 + kCfW, row0);
+        tma_load_2d(sl + kU, &tm_u, bar, (int32_t)t0, row0);
+        tma_load_2d(sl + kUh, &tm_uh, bar, (int32_t)t0 - 8, row0);
+    };
+    if (lane == 0)
+        for (int k = 0; k < kCfQ - 1; ++k) issue(k);
+    int k_fail = -1;
+    for (int k = 0; k < nch; ++k) {
+        __syncwarp();                                // slot k - 1, which chunk k + kCfQ - 1 refills, is read
+        if (lane == 0) {
+            fence_async_smem();
+            issue(k + kCfQ - 1);
         }
-        row_halo_next<V>(grow, gc, lane, t, T, gn);
-        row_halo_prev<V>(urow, uc, lane, t, live, up);
-        float acc[V];
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[warp][k % kCfQ], (uint32_t)(k / kCfQ) & 1u, &abort_flag, err))) {
+            k_fail = k;
+            break;
+        }
+        const uint8_t* sl = ring + (uint32_t)(k % kCfQ) * kCfBwdChunk;
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const float gi = elem(gc, i);
-            acc[i] = gi;
+        for (int r = 0; r < kCfCH; ++r) {
+            if (k * kCfCH + r >= nrows) break;
+            const uint8_t* grow = sl + r * 2 * kCfW;
+            const uint8_t* urow = sl + kU + r * 2 * kCfW;
+            float gx[8], gn[4], ux[8], up[4];        // g at t .. t + 7, t + 8 .. t + 11; u at t .. t + 7, t - 4 .. t - 1
+            lds8(grow + 16 * lane, gx);
+            lds4(lane < 31 ? grow + 16 * lane + 16 : sl + kGa + r * 16, gn);
+            lds8(urow + 16 * lane, ux);
+            lds4(lane > 0 ? urow + 16 * lane - 8 : sl + kUh + r * 16 + 8, up);
+            float acc[8];
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                const float gx = i + j < V ? elem(gc, i + j) : elem(gn, i + j - V);
-                acc[i] = fmaf(j <= epos[i] ? wf[i + j][j] : 0.f, gx, acc[i]);
-                const float ux = i - j >= 0 ? elem(uc, i - j) : elem(up, 4 + i - j);
-                dacc[i][j] = fmaf(gi, ux, dacc[i][j]);
+            for (int i = 0; i < 8; ++i) {
+                acc[i] = gx[i];
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    acc[i] = fmaf(dm[i][j], i + j < 8 ? gx[i + j] : gn[i + j - 8], acc[i]);
+                    dacc[i][j] = fmaf(gx[i], i - j >= 0 ? ux[i - j] : up[4 + i - j], dacc[i][j]);
+                }
+            }
+            if (live) {
+                const int64_t c = c_begin + k * kCfCH + r;
+                *reinterpret_cast<uint4*>(du + (b * C + c) * T + t) = pack8(acc);
             }
         }
-        if (live) strow<V>(du + (b * C + c) * T + t, acc);
     }
-#pragma unroll
-    for (int i = 0; i < V; ++i)
-#pragma unroll
-        for (int j = 0; j < K; ++j) red[warp][lane * V + i][j] = dacc[i][j];
+    if (k_fail >= 0 && lane == 0)                    // let the copies already issued land
+        for (int k = k_fail; k < min(nch, k_fail + kCfQ); ++k)
+            mbar_wait_drain(&bars[warp][k % kCfQ], (uint32_t)(k / kCfQ) & 1u);
+    // the warps' dwh partials, summed over the warps in order (the rings are free now)
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * V * K; e += 256) {
-        const int k = e / K, j = e - k * K;
-        const int64_t tt = tb + k;
+    float* red = reinterpret_cast<float*>(hw_smem);  // [nw][kCfW][K]
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < K; ++j) red[((size_t)warp * kCfW + 8 * lane + i) * K + j] = dacc[i][j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < kCfW * K; e += blockDim.x) {
+        const int tk = e / K, j = e - tk * K;
+        const int64_t tt = t0 + tk;
         if (tt >= T) continue;
         float sum = 0.f;
-#pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][k][j];
+        for (int w = 0; w < nw; ++w) sum += red[((size_t)w * kCfW + tk) * K + j];
         const int64_t n = b * T + tt;
-        const int32_t ps = (int32_t)(n - seg_start(n, cu, n_docs, T));
+        const int64_t ps = n - seg_start(n, cu, n_docs, T);
         dwh[n * R + q * K + j] = __float2bfloat16_rn(j <= ps ? sum : 0.f);
     }
 }
@@ -653,7 +708,8 @@ bool tc_headwise_supported(const Prob& p) {
     if (p.dtype != 1 || p.kind != 1) return false;
     if (p.R > 128 || p.R % 8 != 0 || p.d % 8 != 0) return false;
     if (p.K < 1 || p.K > 4) return false;
-    if (p.layout == 1) return cf_tiles_ok(p) && p.H < 65536;
+    if (p.layout == 1) return cf_tiles_ok(p) && p.hd <= 8 * kCfCPW && p.batch * ((p.seqlen + kCfW - 1) / kCfW) * p.H *
+                                                                 ((p.hd + kCfCPW - 1) / kCfCPW) < (int64_t(1) << 31);
     if (p.hd < 8 || p.hd > 256 || (p.hd & (p.hd - 1)) != 0) return false;
     if (p.rope_n > 0 && p.rope_hd > kHwMaxRopeHd) return false;   // one table row per slot
     // one block per (run, 256-channel block), 32-bit token indices
@@ -661,20 +717,25 @@ bool tc_headwise_supported(const Prob& p) {
            (p.N / std::min(kHwRunFwd, kHwRunBwd) + 1) * (p.C / 256) < (int64_t(1) << 31);
 }
 
-// Channel-first: 8 tokens per lane in the forward, 4 in the backward (fewer registers for
-// the look-ahead filters and the dwh partials).
-constexpr int kCfFwdV = 8, kCfBwdV = 4;
 
 template <int K>
 static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, void* y, uint32_t* err,
                                  cudaStream_t st) {
     cudaError_t e;
     if (p.layout == 1) {
-        const int64_t tps = (p.seqlen + 32 * kCfFwdV - 1) / (32 * kCfFwdV);
-        const dim3 grid((unsigned)(p.batch * tps), (unsigned)p.H);
-        DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_cf_kernel<K, kCfFwdV>, grid, dim3(256), 0, st,
-            static_cast<const __nv_bfloat16*>(u), p.us, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd,
-            p.N, p.C, p.seqlen, tps, p.cu, p.n_docs, static_cast<__nv_bfloat16*>(y)));
+        const int64_t tps = (p.seqlen + kCfW - 1) / kCfW;
+        const int parts = (int)((p.hd + kCfCPW - 1) / kCfCPW);
+        const int smem = kCfQ * kCfFwdChunk;
+        e = cudaFuncSetAttribute(hw_conv_fwd_cf_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        CUtensorMap tu, tuh;
+        if (!make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, kCfW, kCfCH, false) ||
+            !make_tmap_2d(&tuh, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, 8, kCfCH, false))
+            return cudaErrorInvalidValue;
+        const dim3 grid((unsigned)(p.batch * tps * p.H * parts));
+        DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_cf_kernel<K>, grid, dim3(32), smem, st, tu, tuh,
+            static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.C, p.seqlen, tps, parts, (int)p.H, p.cu,
+            p.n_docs, static_cast<__nv_bfloat16*>(y), err));
         return e;
     }
     const int n_cblk = (int)(p.C / 256);
@@ -702,12 +763,23 @@ static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, co
                                  const void* gr, uint32_t* err, cudaStream_t st) {
     cudaError_t e;
     if (p.layout == 1) {
-        const int64_t tps = (p.seqlen + 32 * kCfBwdV - 1) / (32 * kCfBwdV);
-        const dim3 grid((unsigned)(p.batch * tps), (unsigned)p.H);
-        DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_cf_kernel<K, kCfBwdV>, grid, dim3(256), 0, st,
-            static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u), p.us,
-            static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, tps, p.cu, p.n_docs,
-            static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh)));
+        const int64_t tps = (p.seqlen + kCfW - 1) / kCfW;
+        const int nw = (int)((p.hd + kCfCPW - 1) / kCfCPW);
+        const int smem = nw * kCfQ * kCfBwdChunk;
+        e = cudaFuncSetAttribute(hw_conv_bwd_cf_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const uint64_t rows = p.batch * p.C;
+        CUtensorMap tg, tga, tu, tuh;
+        if (!make_tmap_2d(&tg, g, BF, p.seqlen, rows, p.seqlen * 2, kCfW, kCfCH, false) ||
+            !make_tmap_2d(&tga, g, BF, p.seqlen, rows, p.seqlen * 2, 8, kCfCH, false) ||
+            !make_tmap_2d(&tu, u, BF, p.seqlen, rows, p.us * 2, kCfW, kCfCH, false) ||
+            !make_tmap_2d(&tuh, u, BF, p.seqlen, rows, p.us * 2, 8, kCfCH, false))
+            return cudaErrorInvalidValue;
+        const dim3 grid((unsigned)(p.batch * tps * p.H));
+        DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_cf_kernel<K>, grid, dim3(32 * nw), smem, st, tg, tga,
+            tu, tuh, static_cast<const __nv_bfloat16*>(wh), (int)p.R, (int)p.hd, p.N, p.C, p.seqlen, tps, (int)p.H,
+            p.cu, p.n_docs, static_cast<__nv_bfloat16*>(du), static_cast<__nv_bfloat16*>(dwh), err));
         return e;
     }
     const int n_cblk = (int)(p.C / 256);

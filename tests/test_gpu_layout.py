@@ -34,6 +34,11 @@ CASES = [
            layers=(W.Layer("qkv", 256, 640),)), 0, None),
     (_case("c3_qkv_2b_headwise_gqa", 1, 520, "cf_hw_k3_hd32", ksize=3, head_dim=32,
            layers=(W.Layer("qkv", 128, 256),)), 0, None),
+    # head rows split over warps: 96 = 64 + 32 rows, and 256 rows on four warps; a third window
+    (_case("c3_qkv_2b_headwise_gqa", 1, 584, "cf_hw_k4_hd96", head_dim=96,
+           layers=(W.Layer("qkv", 128, 384),)), 0, None),
+    (_case("c3_qkv_2b_headwise_gqa", 2, 264, "cf_hw_k4_hd256", head_dim=256,
+           layers=(W.Layer("qkv", 256, 512),)), 0, None),
     # seqlen not a multiple of 8: the generic kernels
     (_case("c2_qkv_150m_lowrank", 2, 130, "cf_odd_T"), 0, None),
     (C["c1_fp32_lowrank"], 0, None),
