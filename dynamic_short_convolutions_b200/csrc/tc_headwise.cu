@@ -398,20 +398,20 @@ __global__ void __launch_bounds__(32, 16) hw_conv_bwd_kernel(const __grid_consta
 // ---- channel-first layout: u, y, g, du are [batch * C, seqlen] rows (tokens contiguous) ----
 // A warp takes a window of kCfW tokens t0 .. t0 + kCfW - 1 of one sequence b and up to kCfCPW
 // channel rows of one head q; lane l takes tokens t0 + 8 l .. t0 + 8 l + 7, whose filter taps (masked
-// for the segment) stay in registers across the channels.  The rows come kCfCH at a time through
-// a TMA ring in shared memory: the window (box {kCfW, kCfCH}) and 8 tokens beside it (box
-// {8, kCfCH}: before the window for u, after it for g), so each lane finds its K - 1 <= 3
+// for the segment) stay in registers across the channels.  The rows come CH at a time through a
+// TMA ring in shared memory: the window (box {kCfW, CH}) and 8 tokens beside it (box {8, CH}:
+// before the window for u, after it for g), so each lane finds its K - 1 <= 3
 // neighbours in its row of the chunk.  seqlen is a multiple of 8, so a lane's 8 tokens are all
 // inside the sequence or all past its end (rows past the end read zero).
 constexpr int kCfW = 256;                          // tokens per window (8 per lane)
-constexpr int kCfCH = 2;                           // channel rows per chunk
+constexpr int kCfFwdCH = 2, kCfBwdCH = 4;          // channel rows per chunk (CH)
 constexpr int kCfQ = 4;                            // ring slots (chunks)
 constexpr int kCfCPW = 64;                         // channel rows per warp
 // Chunk layouts (every TMA destination on a 128-byte boundary): forward u window, u 8 before;
 // backward g window, g 8 after, u window, u 8 before.
-constexpr uint32_t kCfFwdUh = kCfCH * 2 * kCfW, kCfFwdChunk = al128(kCfFwdUh + kCfCH * 16);
-constexpr uint32_t kCfBwdGa = kCfCH * 2 * kCfW, kCfBwdU = al128(kCfBwdGa + kCfCH * 16);
-constexpr uint32_t kCfBwdUh = kCfBwdU + kCfCH * 2 * kCfW, kCfBwdChunk = al128(kCfBwdUh + kCfCH * 16);
+constexpr uint32_t kCfFwdUh = kCfFwdCH * 2 * kCfW, kCfFwdChunk = al128(kCfFwdUh + kCfFwdCH * 16);
+constexpr uint32_t kCfBwdGa = kCfBwdCH * 2 * kCfW, kCfBwdU = al128(kCfBwdGa + kCfBwdCH * 16);
+constexpr uint32_t kCfBwdUh = kCfBwdU + kCfBwdCH * 2 * kCfW, kCfBwdChunk = al128(kCfBwdUh + kCfBwdCH * 16);
 static_assert(kCfFwdUh % 128 == 0 && kCfFwdChunk % 128 == 0 && kCfBwdGa % 128 == 0 && kCfBwdU % 128 == 0 &&
                   kCfBwdUh % 128 == 0 && kCfBwdChunk % 128 == 0,
               "TMA destinations in shared memory start on 128-byte boundaries");
@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(32, 24) hw_conv_fwd_cf_kernel(const __grid_con
     const int64_t t0 = win * kCfW, t = t0 + 8 * lane;
     const bool live = t < T;
     const int c_begin = q * hd + part * kCfCPW, nrows = min(kCfCPW, hd - part * kCfCPW);
-    const int nch = (nrows + kCfCH - 1) / kCfCH;
+    const int nch = (nrows + kCfFwdCH - 1) / kCfFwdCH;
     const int64_t n0 = b * T + t;
     float wm[8][K];                                  // taps of the lane's tokens, masked for the segment
 #pragma unroll
@@ -477,8 +477,8 @@ __global__ void __launch_bounds__(32, 24) hw_conv_fwd_cf_kernel(const __grid_con
         if (k >= nch) return;
         uint8_t* sl = hw_smem + (uint32_t)(k % kCfQ) * kCfFwdChunk;
         uint64_t* bar = &bars[k % kCfQ];
-        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfCH);
-        mbar_arrive_expect_tx(bar, kCfCH * (2 * kCfW + 16));
+        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfFwdCH);
+        mbar_arrive_expect_tx(bar, kCfFwdCH * (2 * kCfW + 16));
         tma_load_2d(sl, &tm_u, bar, (int32_t)t0, row0);
         tma_load_2d(sl + kCfFwdUh, &tm_uh, bar, (int32_t)t0 - 8, row0);
     };
@@ -497,8 +497,8 @@ __global__ void __launch_bounds__(32, 24) hw_conv_fwd_cf_kernel(const __grid_con
         }
         const uint8_t* sl = hw_smem + (uint32_t)(k % kCfQ) * kCfFwdChunk;
 #pragma unroll
-        for (int r = 0; r < kCfCH; ++r) {
-            if (k * kCfCH + r >= nrows) break;
+        for (int r = 0; r < kCfFwdCH; ++r) {
+            if (k * kCfFwdCH + r >= nrows) break;
             const uint8_t* row = sl + r * 2 * kCfW;
             float x[8], xp[4];                       // tokens t .. t + 7 and t - 4 .. t - 1
             lds8(row + 16 * lane, x);
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(32, 24) hw_conv_fwd_cf_kernel(const __grid_con
                 for (int j = 0; j < K; ++j) acc[i] = fmaf(wm[i][j], i - j >= 0 ? x[i - j] : xp[4 + i - j], acc[i]);
             }
             if (live) {
-                const int64_t c = c_begin + k * kCfCH + r;
+                const int64_t c = c_begin + k * kCfFwdCH + r;
                 *reinterpret_cast<uint4*>(y + (b * C + c) * T + t) = pack8(acc);
             }
         }
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __grid_consta
     const int64_t t0 = win * kCfW, t = t0 + 8 * lane;
     const bool live = t < T;
     const int c_begin = q * hd + warp * kCfCPW, nrows = max(0, min(kCfCPW, hd - warp * kCfCPW));
-    const int nch = (nrows + kCfCH - 1) / kCfCH;
+    const int nch = (nrows + kCfBwdCH - 1) / kCfBwdCH;
     const int64_t n0 = b * T + t;
     uint8_t* ring = hw_smem + (uint32_t)warp * kCfQ * kCfBwdChunk;
     // dm[i][j]: tap j of the filter of token t + i + j for du[t + i], zero past the segment end
@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __grid_consta
         if (k >= nch) return;
         uint8_t* sl = ring + (uint32_t)(k % kCfQ) * kCfBwdChunk;
         uint64_t* bar = &bars[warp][k % kCfQ];
-        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfCH);
-        mbar_arrive_expect_tx(bar, 2 * kCfCH * (2 * kCfW + 16));
+        const int32_t row0 = (int32_t)(b * C + c_begin + k * kCfBwdCH);
+        mbar_arrive_expect_tx(bar, 2 * kCfBwdCH * (2 * kCfW + 16));
         tma_load_2d(sl, &tm_g, bar, (int32_t)t0, row0);
         tma_load_2d(sl + kGa, &tm_ga, bar, (int32_t)t0 + kCfW, row0);
         tma_load_2d(sl + kU, &tm_u, bar, (int32_t)t0, row0);
@@ -613,8 +613,8 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __grid_consta
         }
         const uint8_t* sl = ring + (uint32_t)(k % kCfQ) * kCfBwdChunk;
 #pragma unroll
-        for (int r = 0; r < kCfCH; ++r) {
-            if (k * kCfCH + r >= nrows) break;
+        for (int r = 0; r < kCfBwdCH; ++r) {
+            if (k * kCfBwdCH + r >= nrows) break;
             const uint8_t* grow = sl + r * 2 * kCfW;
             const uint8_t* urow = sl + kU + r * 2 * kCfW;
             float gx[8], gn[4], ux[8], up[4];        // g at t .. t + 7, t + 8 .. t + 11; u at t .. t + 7, t - 4 .. t - 1
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(256) hw_conv_bwd_cf_kernel(const __grid_consta
                 }
             }
             if (live) {
-                const int64_t c = c_begin + k * kCfCH + r;
+                const int64_t c = c_begin + k * kCfBwdCH + r;
                 *reinterpret_cast<uint4*>(du + (b * C + c) * T + t) = pack8(acc);
             }
         }
@@ -729,8 +729,8 @@ static cudaError_t launch_hw_fwd(const Prob& p, const void* u, const void* wh, v
         e = cudaFuncSetAttribute(hw_conv_fwd_cf_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         CUtensorMap tu, tuh;
-        if (!make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, kCfW, kCfCH, false) ||
-            !make_tmap_2d(&tuh, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, 8, kCfCH, false))
+        if (!make_tmap_2d(&tu, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, kCfW, kCfFwdCH, false) ||
+            !make_tmap_2d(&tuh, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.seqlen, p.batch * p.C, p.us * 2, 8, kCfFwdCH, false))
             return cudaErrorInvalidValue;
         const dim3 grid((unsigned)(p.batch * tps * p.H * parts));
         DC_LAUNCH(kTcHeadwiseFwd, st, e = launch_pdl(hw_conv_fwd_cf_kernel<K>, grid, dim3(32), smem, st, tu, tuh,
@@ -771,10 +771,10 @@ static cudaError_t launch_hw_bwd(const Prob& p, const void* g, const void* u, co
         const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
         const uint64_t rows = p.batch * p.C;
         CUtensorMap tg, tga, tu, tuh;
-        if (!make_tmap_2d(&tg, g, BF, p.seqlen, rows, p.seqlen * 2, kCfW, kCfCH, false) ||
-            !make_tmap_2d(&tga, g, BF, p.seqlen, rows, p.seqlen * 2, 8, kCfCH, false) ||
-            !make_tmap_2d(&tu, u, BF, p.seqlen, rows, p.us * 2, kCfW, kCfCH, false) ||
-            !make_tmap_2d(&tuh, u, BF, p.seqlen, rows, p.us * 2, 8, kCfCH, false))
+        if (!make_tmap_2d(&tg, g, BF, p.seqlen, rows, p.seqlen * 2, kCfW, kCfBwdCH, false) ||
+            !make_tmap_2d(&tga, g, BF, p.seqlen, rows, p.seqlen * 2, 8, kCfBwdCH, false) ||
+            !make_tmap_2d(&tu, u, BF, p.seqlen, rows, p.us * 2, kCfW, kCfBwdCH, false) ||
+            !make_tmap_2d(&tuh, u, BF, p.seqlen, rows, p.us * 2, 8, kCfBwdCH, false))
             return cudaErrorInvalidValue;
         const dim3 grid((unsigned)(p.batch * tps * p.H));
         DC_LAUNCH(kTcHeadwiseBwd, st, e = launch_pdl(hw_conv_bwd_cf_kernel<K>, grid, dim3(32 * nw), smem, st, tg, tga,
