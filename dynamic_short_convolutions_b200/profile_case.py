@@ -1,12 +1,13 @@
 """One layer of a workload, forward + backward, for profiling a kernel under ncu.
 
     python -m dynamic_short_convolutions_b200.profile_case --config c4_all_linear_2b_block \\
-        --layer 2 --batch 2 [--repeats 2] [--rope]
+        --layer 2 --batch 2 [--repeats 2] [--rope] [--layout channel_first]
 
 runs the layer's forward and backward `repeats` times on seeded inputs (the
 workload's recipe with `batch` sequences of its length), checks the device status
 and prints the problem.  With ``--rope`` the QKV layer of the 150M / 2B
-workloads fuses RoPE after the conv (base 10000).  Meant for captures such as
+workloads fuses RoPE after the conv (base 10000); ``--layout channel_first`` stores
+u, y, g and du as [batch, C, seqlen].  Meant for captures such as
 ``ncu --set full -k regex:lowrank_bwd_kernel -s 1 -c 1 python -m ...``: a
 reduced batch keeps the capture small while the inputs stay above L2.
 """
@@ -23,6 +24,7 @@ def main(argv=None) -> int:
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--repeats", type=int, default=2)
     ap.add_argument("--rope", action="store_true")
+    ap.add_argument("--layout", default="token_major", choices=["token_major", "channel_first"])
     args = ap.parse_args(argv)
     import torch
 
@@ -37,8 +39,13 @@ def main(argv=None) -> int:
     rope = W.ROPE_QKV.get(w0.name) if args.rope and layer.name == "qkv" else None
     table = ops.rope_table(w.seqlen, rope[1], device="cuda") if rope else None
     batch, seqlen = (1, w.tokens) if w.varlen else (w.batch, w.seqlen)
+    cf = args.layout == "channel_first"
+    if cf:                  # u and g stored [batch, C, seqlen]
+        for k in ("u", "g"):
+            t[k] = t[k].reshape(batch, seqlen, layer.channels).transpose(1, 2).contiguous()
     plan = ops.DynConvPlan(kind, W.storage_dtype(w), batch, seqlen, layer.d_model, layer.channels, w.ksize, w.rank,
-                           w.head_dim, device="cuda", rope_channels=rope[0] if rope else 0,
+                           w.head_dim, device="cuda", layout=L.CHANNEL_FIRST if cf else L.TOKEN_MAJOR,
+                           rope_channels=rope[0] if rope else 0,
                            rope_head_dim=rope[1] if rope else 0, rope_table=table)
     BW = t["B"] if kind == L.LOWRANK else t["W"]
     R = w.rank if kind == L.LOWRANK else (layer.channels // w.head_dim) * w.ksize
@@ -53,7 +60,7 @@ def main(argv=None) -> int:
         print("device status", st, L.dynconv_last_error(), file=sys.stderr)
         return 1
     print(f"{w.name} layer {layer.name}: tokens {w.tokens}, d {layer.d_model}, C {layer.channels}, K {w.ksize}, "
-          f"r {w.rank}, head_dim {w.head_dim}, rope {rope}, repeats {args.repeats}")
+          f"r {w.rank}, head_dim {w.head_dim}, rope {rope}, layout {args.layout}, repeats {args.repeats}")
     return 0
 
 
