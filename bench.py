@@ -90,10 +90,10 @@ def layer_flops(w, layer):
 # (kernel, workload) and stored with the SHA-256 of the kernel's source files at capture time: a
 # figure is reported only while those files are unchanged (else traffic is null).
 NCU_TRAFFIC = {
-    ("tc_lowrank_bwd", "c4_all_linear_2b_block"): (550761776, "f9389981e7b57080"),
-    ("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): (197190016, "f9389981e7b57080"),
-    ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): (277363627, "58ce1e3407cfd928"),
-    ("tc_lowrank_bwd", "c5_varlen_packed"): (2186419968, "f9389981e7b57080"),
+    ("tc_lowrank_bwd", "c4_all_linear_2b_block"): (554284474, "2f2485ccebdbbc0b"),
+    ("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): (193070314, "2f2485ccebdbbc0b"),
+    ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): (302766165, "d6fc16bc63cc23d6"),
+    ("tc_lowrank_bwd", "c5_varlen_packed"): (2185422378, "2f2485ccebdbbc0b"),
 }
 KERNEL_SOURCES = {
     "tc_lowrank_bwd": ("tc_bwd.cu", "tc_common.cuh", "common.cuh"),
