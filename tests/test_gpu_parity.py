@@ -42,6 +42,14 @@ SMALL = [
     (_case("c2_qkv_150m_lowrank", 1, 130, "odd_channels", layers=(W.Layer("x", 40, 72),)), 0),
     (_case("c3_qkv_2b_headwise_gqa", 1, 150, "hw_k2_hd64", ksize=2, head_dim=64,
            layers=(W.Layer("qkv", 256, 640),)), 0),
+    # head-wise: K = 3 (taps boxes at odd offsets, chunks of 3 rows), K = 1, heads of 256, 16 and 8
+    # channels (32, 2 and 1 lanes per head), lengths that end runs and chunks part-way
+    (_case("c3_qkv_2b_headwise_gqa", 1, 333, "hw_k3_hd32", ksize=3, head_dim=32,
+           layers=(W.Layer("qkv", 128, 256),)), 0),
+    (_case("c3_qkv_2b_headwise_gqa", 2, 97, "hw_k1_hd256", ksize=1, head_dim=256,
+           layers=(W.Layer("qkv", 128, 2048),)), 0),
+    (_case("c3_qkv_2b_headwise_gqa", 1, 301, "hw_k4_hd16", head_dim=16, layers=(W.Layer("qkv", 64, 256),)), 0),
+    (_case("c3_qkv_2b_headwise_gqa", 3, 45, "hw_k4_hd8", head_dim=8, layers=(W.Layer("qkv", 64, 256),)), 0),
 ]
 
 VARLEN_CU = [0, 1, 3, 6, 10, 15, 115, 400, 700]
@@ -94,6 +102,18 @@ def test_small_parity(case, algo):
 @ALGOS
 def test_varlen_parity(algo):
     w = _varlen_case()
+    layer = w.layers[0]
+    x = W.make_inputs(w, layer)
+    x["cu_seqlens"] = np.array(VARLEN_CU, dtype=np.int32)
+    gpu = _run_or_skip(w, layer, _to_device(x, w), algo)
+    _compare(w, gpu, oracle_all(w, layer, x))
+
+
+@ALGOS
+def test_varlen_parity_headwise(algo):
+    """Packed documents through the head-wise kernels: runs and chunks that cross document
+    starts, documents shorter than K."""
+    w = _case("c3_qkv_2b_headwise_gqa", 1, 700, "hw_varlen", varlen=True, layers=(W.Layer("qkv", 128, 512),))
     layer = w.layers[0]
     x = W.make_inputs(w, layer)
     x["cu_seqlens"] = np.array(VARLEN_CU, dtype=np.int32)
