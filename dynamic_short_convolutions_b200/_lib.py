@@ -29,7 +29,7 @@ TOKEN_MAJOR, CHANNEL_FIRST = 0, 1
 EXPORTS = ("dynconv_workspace_bytes", "dynconv_fwd", "dynconv_fwd_varlen", "dynconv_bwd",
            "dynconv_device_status", "dynconv_last_error", "dynconv_status_string", "dynconv_version",
            "dynconv_profile_enable", "dynconv_profile_read", "dynconv_selftest_umma", "dynconv_fwd_noalloc",
-           "dynconv_decode_step", "dynconv_noalloc_status", "dynconv_query_family")
+           "dynconv_decode_step", "dynconv_noalloc_status", "dynconv_query_family", "dynconv_selftest_wait")
 
 
 class DynConvError(RuntimeError):
@@ -93,6 +93,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.dynconv_profile_read.restype = ctypes.c_int
     lib.dynconv_selftest_umma.argtypes = [ctypes.c_int, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
     lib.dynconv_selftest_umma.restype = ctypes.c_int
+    lib.dynconv_selftest_wait.argtypes = [ctypes.c_uint64, vp, vp, vp]
+    lib.dynconv_selftest_wait.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -200,6 +202,11 @@ def dynconv_profile_read(reset: bool = True):
     arr = (dynconv_profile_entry * 64)()
     n = lib.dynconv_profile_read(arr, 64, int(bool(reset)))
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(min(n, 64))}
+
+
+def dynconv_selftest_wait(limit_ns: int, err_word, out2, stream=None) -> int:
+    """Diagnostic bounded wait that runs out (see include/dynconv_diag.h); returns the status."""
+    return int(load().dynconv_selftest_wait(int(limit_ns), _ptr(err_word), _ptr(out2), _stream(stream, err_word)))
 
 
 def dynconv_selftest_umma(variant: int, A, B, D, N: int, Kd: int, err_word, stream=None) -> int:

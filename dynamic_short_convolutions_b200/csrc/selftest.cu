@@ -117,10 +117,35 @@ __global__ void __launch_bounds__(128) selftest_kernel(const __grid_constant__ C
     }
 }
 
+// A wait that runs out: thread 0 waits, with a limit of limit_ns, on an mbarrier that nothing
+// arrives on; thread 32 (another warp) waits on the same barrier with the kernels' own limit and
+// must give up as soon as thread 0 has (the abort flag).  out[0], out[1] = 1 if the wait
+// returned true, 2 if it gave up; the error word gets kErrWaitTimeout.
+__global__ void __launch_bounds__(64) selftest_wait_kernel(uint64_t limit_ns, uint32_t* err, uint32_t* out) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) out[0] = mbar_wait(&bar, 0, &abort_flag, err, limit_ns) ? 1u : 2u;
+    if (threadIdx.x == 32) out[1] = mbar_wait(&bar, 0, &abort_flag, err) ? 1u : 2u;
+}
+
 }  // namespace
 }  // namespace dynconv
 
 using namespace dynconv;
+
+extern "C" DYNCONV_API dynconv_status dynconv_selftest_wait(uint64_t limit_ns, void* err_word, void* out2,
+                                                            void* stream) {
+    if (!err_word || !out2 || limit_ns == 0 || limit_ns > tc::kWaitNs) return DYNCONV_ERR_INVALID;
+    selftest_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, static_cast<uint32_t*>(err_word),
+                                                                          static_cast<uint32_t*>(out2));
+    return cudaGetLastError() == cudaSuccess ? DYNCONV_OK : DYNCONV_ERR_CUDA;
+}
 
 extern "C" DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const void* A, const void* B, float* D,
                                                             int N, int Kd, void* err_word, void* stream) {

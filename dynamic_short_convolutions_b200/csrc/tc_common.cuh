@@ -66,17 +66,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase of parity `parity` to complete.  Gives up after kWaitNs,
-// or as soon as another thread of the CTA has given up (abort flag): then it
+// Waits for the phase of parity `parity` to complete.  Gives up after limit_ns (kWaitNs
+// unless given), or as soon as another thread of the CTA has given up (abort flag): then it
 // raises kErrWaitTimeout in the device error word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err) {
+                                          uint32_t* err, uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             if (err) atomicOr(err, kErrWaitTimeout);
             return false;

@@ -31,6 +31,17 @@ extern "C" {
 DYNCONV_API dynconv_status dynconv_selftest_umma(int variant, const void *A, const void *B, float *D, int N, int Kd,
                                                  void *err_word, void *stream);
 
+/* A bounded wait that runs out, on purpose and safely: one CTA waits on an
+ * mbarrier that nothing completes, one thread with a limit of limit_ns
+ * nanoseconds (1 .. 2e9) and a thread of another warp with the kernels' own
+ * limit, which must give up as soon as the first has (the CTA's abort flag).
+ * Both waits end; out2 (a device uint32[2]) receives 2, 2 (1 would mean a wait
+ * returned success), and err_word (a device uint32) receives the wait-timeout
+ * bit that dynconv_device_status reports as DYNCONV_ERR_DEVICE_CHECK.  The CUDA
+ * context stays usable.  Asynchronous on `stream`; DYNCONV_ERR_INVALID for null
+ * pointers or a limit outside 1 .. 2e9. */
+DYNCONV_API dynconv_status dynconv_selftest_wait(uint64_t limit_ns, void *err_word, void *out2, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -56,3 +56,36 @@ def test_umma_row_shifted_operand(variant, N, shift):
     print(f"variant {variant} shift {shift}: {'match' if ok else 'MISMATCH'}")
     if variant == 3:
         assert ok
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """A wait on an mbarrier that nothing completes ends after its limit (20 ms), raises the
+    wait-timeout bit, takes the other waiting warp of the CTA down with it through the abort
+    flag, and leaves the context usable: a tensor-core tile computes correctly afterwards."""
+    import time
+
+    from dynamic_short_convolutions_b200 import _lib as L
+
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    out = torch.zeros(2, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    assert L.dynconv_selftest_wait(20_000_000, err, out) == 0
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert out.tolist() == [2, 2]                  # both waits gave up
+    assert int(err[0]) & 2                         # the wait-timeout bit
+    assert 0.015 < elapsed < 1.0                   # the short limit, not the kernels' 2 s
+    # invalid arguments are refused before any launch
+    assert L.STATUS_NAMES[L.dynconv_selftest_wait(0, err, out)] == "DYNCONV_ERR_INVALID"
+    assert L.STATUS_NAMES[L.dynconv_selftest_wait(3_000_000_000, err, out)] == "DYNCONV_ERR_INVALID"
+    # the context still runs work
+    g = torch.Generator(device="cuda").manual_seed(5)
+    A = torch.randn(128, 64, device="cuda", generator=g).bfloat16()
+    B = torch.randn(64, 64, device="cuda", generator=g).bfloat16()
+    D = torch.full((128, 64), float("nan"), device="cuda")
+    err2 = torch.zeros(4, dtype=torch.int32, device="cuda")
+    assert L.dynconv_selftest_umma(0, A, B, D, 64, 64, err2) == 0
+    torch.cuda.synchronize()
+    assert int(err2[0]) == 0
+    torch.testing.assert_close(D.double(), A.double() @ B.double().T, rtol=1e-5, atol=1e-4)
