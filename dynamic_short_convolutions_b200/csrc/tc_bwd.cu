@@ -130,15 +130,19 @@ constexpr uint32_t kSmemTotal = 232448;              // shared memory per CTA (d
 // MMA has read z; three when they fit), one dW tile (K tap atoms of 128 tokens x 64 channels,
 // handed to the MMAs in 128-row blocks of two atoms), the du tile staged for its TMA store, the
 // chunk's Bp slice (rank rounded up to 16 rows per tap), and one fp32 dz box [128 rows][32 ranks]
-// staged for its bulk reduction (rank 64: the two boxes in turn), when it fits (else dz goes
-// through fp32 atomics).
+// staged for its bulk reduction (rank 64: the two boxes in turn); where that does not fit (K = 4
+// at rank 64), a box of 64 rows (the four boxes in turn); with neither, dz goes through fp32
+// atomics.
 template <int K, bool R64>
 struct BwdSmem {
     static constexpr uint32_t gu = 2 * kRowTile;
     static constexpr uint32_t bp_tap = R64 ? 8192 : 4096;
     static constexpr uint32_t stat = 512;                                     // static shared memory
     static constexpr uint32_t base2 = 2 * gu + 2 * kRowTile + K * kAtom128 + kAtom128 + K * bp_tap + 1024 + stat;
-    static constexpr uint32_t dzst_bytes = base2 + kAtom128 <= kSmemTotal ? kAtom128 : 0;
+    static constexpr uint32_t dzst_bytes = base2 + kAtom128 <= kSmemTotal       ? kAtom128
+                                           : base2 + kAtom128 / 2 <= kSmemTotal ? kAtom128 / 2
+                                                                                : 0;
+    static constexpr int dz_rows = dzst_bytes / 128;                             // rows per dz box
     static constexpr int NZ = base2 + kRowTile + dzst_bytes <= kSmemTotal ? 3 : 2;
     static constexpr uint32_t z0 = 2 * gu;
     static constexpr uint32_t dw = z0 + NZ * kRowTile;
@@ -554,38 +558,45 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             const int32_t m0 = tile_at<CF>(tile, 0, a.tps, a.seqlen, a.C).m0;
             const int32_t n = m0 + row;
             if (via_tma) {
-                // one fp32 box [128 rows][32 ranks] at a time through the staging tile, each added into
-                // the [N, r] buffer by one bulk tensor reduction
+                // one fp32 box [dz_rows rows][32 ranks] at a time through the staging tile, each added
+                // into the [N, r] buffer by one bulk tensor reduction; with 64-row boxes the two
+                // warps of the box's rows stage it while the other two wait
+                constexpr int kDzRows = S::dz_rows > 0 ? S::dz_rows : 128;
                 for (int bx = 0; bx * 32 < a.r; ++bx) {
-                    if (bx > 0) {                       // the previous box's reduction has read the tile
-                        if (leader) tma_store_wait_read_all();
-                        named_bar_any<3, 32 * kGbWarps>(false);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 32; c += 16) {
-                        uint32_t v[2][8];
-                        tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c, v[0]);
-                        tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c + 8, v[1]);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int qq = (c + 8 * h) >> 2;
-                            *reinterpret_cast<uint4*>(dzs + sw128_off(row, qq)) =
-                                make_uint4(v[h][0], v[h][1], v[h][2], v[h][3]);
-                            *reinterpret_cast<uint4*>(dzs + sw128_off(row, qq + 1)) =
-                                make_uint4(v[h][4], v[h][5], v[h][6], v[h][7]);
+                    for (int rh = 0; rh < 128 / kDzRows; ++rh) {
+                        if (bx > 0 || rh > 0) {         // the previous box's reduction has read the tile
+                            if (leader) tma_store_wait_read_all();
+                            named_bar_any<3, 32 * kGbWarps>(false);
                         }
-                    }
-                    if ((bx + 1) * 32 >= a.r) {         // every dz column of this buffer has been read
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&dzempty[b]);
-                    }
-                    fence_async_smem();
-                    named_bar_any<3, 32 * kGbWarps>(false);     // every GB warp has staged its dz rows
-                    if (leader) {
-                        tma_reduce_add_2d_hint(&tm_dz, dzs, bx * 32, m0, l2_evict_last());
-                        tma_store_commit();
+                        if (row / kDzRows == rh) {
+                            const int srow = row - rh * kDzRows;
+#pragma unroll
+                            for (int c = 0; c < 32; c += 16) {
+                                uint32_t v[2][8];
+                                tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c, v[0]);
+                                tmem_ld8(lane_base + kColDz + 64 * b + 32 * bx + c + 8, v[1]);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int qq = (c + 8 * h) >> 2;
+                                    *reinterpret_cast<uint4*>(dzs + sw128_off(srow, qq)) =
+                                        make_uint4(v[h][0], v[h][1], v[h][2], v[h][3]);
+                                    *reinterpret_cast<uint4*>(dzs + sw128_off(srow, qq + 1)) =
+                                        make_uint4(v[h][4], v[h][5], v[h][6], v[h][7]);
+                                }
+                            }
+                        }
+                        if ((bx + 1) * 32 >= a.r && rh + 1 == 128 / kDzRows) {   // every dz column is read
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&dzempty[b]);
+                        }
+                        fence_async_smem();
+                        named_bar_any<3, 32 * kGbWarps>(false);     // the box's rows are staged
+                        if (leader) {
+                            tma_reduce_add_2d_hint(&tm_dz, dzs, bx * 32, m0 + rh * kDzRows, l2_evict_last());
+                            tma_store_commit();
+                        }
                     }
                 }
             } else {
@@ -982,6 +993,20 @@ cudaError_t tc_gen_backward(const void* X, int R, const void* h, int64_t hs, con
 
 static inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Rows of the dz box the backward stages for its bulk reductions (BwdSmem<K, R64>::dz_rows).
+static int dz_box_rows(int K, bool r64) {
+    switch (K * 2 + (r64 ? 1 : 0)) {
+        case 2: return BwdSmem<1, false>::dz_rows;
+        case 3: return BwdSmem<1, true>::dz_rows;
+        case 4: return BwdSmem<2, false>::dz_rows;
+        case 5: return BwdSmem<2, true>::dz_rows;
+        case 6: return BwdSmem<3, false>::dz_rows;
+        case 7: return BwdSmem<3, true>::dz_rows;
+        case 8: return BwdSmem<4, false>::dz_rows;
+        default: return BwdSmem<4, true>::dz_rows;
+    }
+}
+
 TcBwdLayout tc_bwd_layout(const Prob& p) {
     TcBwdLayout L{};
     const int sms = 148;   // sizing only; the launch uses at most this many CTAs
@@ -1038,11 +1063,13 @@ cudaError_t tc_lowrank_backward(const Prob& p, const void* g, const void* u, con
     std::memset(&tdz, 0, sizeof(tdz));                 // unused unless dz goes through bulk reductions
     std::memset(&tgr, 0, sizeof(tgr));                 // unused without RoPE
     if (p.rope_n > 0 && !make_tmap_bf16(&tgr, gr, p.rope_n, p.N, p.rope_n, 64, 136)) return cudaErrorInvalidValue;
-    const bool dz_tma = p.r % 32 == 0;
+    const int dz_rows = dz_box_rows((int)p.K, p.r > 32);
+    const bool dz_tma = p.r % 32 == 0 && dz_rows > 0;
     const bool cf = p.layout == 1;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_tmap_bf16(&tz, z, p.r, p.N, p.r, 64, 136) || !make_tmap_bf16(&tbp, bp, p.C * p.K, p.r, p.C * p.K, 64, (uint32_t)((p.r + 15) / 16 * 16)) ||
-        (dz_tma && !make_tmap_2d(&tdz, dz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.r, p.N, p.r * 4, 32, 128, true)))
+        (dz_tma && !make_tmap_2d(&tdz, dz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.r, p.N, p.r * 4, 32,
+                                 (uint32_t)dz_rows, true)))
         return cudaErrorInvalidValue;
     if (cf ? !(make_tmap_2d(&tg, g, BF, p.seqlen, p.batch * p.C, p.seqlen * 2, 136, 64, false) &&
                make_tmap_2d(&tu, u, BF, p.seqlen, p.batch * p.C, p.us * 2, 136, 64, false) &&
