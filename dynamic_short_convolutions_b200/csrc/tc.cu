@@ -110,29 +110,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) gen_kernel(const __grid_constan
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, a.NMMA, false, true);
-            uint32_t it = 0, t = 0;
-            for (int64_t tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++t) {
-                const int b = t & 1;
-                if (!mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+        // the whole warp runs the loop (warp-uniform descriptor arithmetic); one elected lane issues
+        const uint32_t idesc = idesc_bf16(128, a.NMMA, false, true);
+        uint32_t it = 0, t = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++t) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;      // the lanes leave together
+            const int b = t & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, &abort_flag, a.err))) break;
+            tc_fence_after();
+            const uint32_t dcol = tbase + b * a.NMMA;
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, &abort_flag, a.err))) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t dcol = tbase + b * a.NMMA;
-                bool ok = true;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&full[s], ph, &abort_flag, a.err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(sm + s * stage_bytes);
-                    for (int k = 0; k < 4; ++k)
-                        umma_bf16(dcol, kmajor_desc(st, k), mnmajor_desc(st + 16384, 8192, 16 * k), idesc,
-                                  (kb | k) != 0);
+                const uint32_t st = smem_u32(sm + s * stage_bytes);
+                uint64_t da[4], db[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    da[k] = kmajor_desc(st, k);
+                    db[k] = mnmajor_desc(st + 16384, 8192, 16 * k);
+                }
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) umma_bf16(dcol, da[k], db[k], idesc, (kb | k) != 0);
                     umma_commit(&empty[s]);
                 }
-                if (!ok) break;
-                umma_commit(&tfull[b]);
+                __syncwarp();
             }
+            if (!ok) break;
+            if (elect_one()) umma_commit(&tfull[b]);
+            __syncwarp();
         }
     } else {
         if (a.pB) {                              // the side job, before the first accumulator is ready
