@@ -286,112 +286,134 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
             }
         }
     } else if (warp == 1) {
-        // ---- filter MMAs of every item, issued by their own thread (the dz / dB MMAs have another,
-        // on another scheduler: one thread issuing both kinds was the kernel's critical path)
-        if (lane == 0) {
-            const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
-            const uint32_t bp0 = smem_u32(sm + S::bp);
-            const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
-            uint32_t cc = 0;          // B loads consumed
-            // Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows into the z slot), KS 16-wide steps
-            // over the rank, unrolled (the issuing thread shares its scheduler with busy epilogue
-            // warps; a loop with a run-time trip count per tap cost ~2.5x the issue time)
-            auto filter_mmas = [&](auto ks, uint32_t z0) {
-                constexpr int KS = decltype(ks)::value;
+        // ---- filter MMAs of every item, issued by their own warp (the dz / dB MMAs have another,
+        // on another scheduler: one thread issuing both kinds was the kernel's critical path).  The
+        // whole warp runs the loop, so the descriptor arithmetic is warp-uniform; the elected lane
+        // issues the MMAs and commits.
+        const bool leader = elect_one();
+        const uint32_t idesc_w = idesc_bf16(128, 64, false, true);
+        const uint32_t bp0 = smem_u32(sm + S::bp);
+        const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
+        uint32_t cc = 0;          // B loads consumed
+        // Wd_j = z[j : j+128] . Bp_j (K-major A starting j rows into the z slot), KS 16-wide steps
+        // over the rank, unrolled (a loop with a run-time trip count per tap cost ~2.5x the issue time)
+        auto filter_mmas = [&](auto ks, uint32_t z0) {
+            constexpr int KS = decltype(ks)::value;
 #pragma unroll
-                for (int j = 0; j < K; ++j)
+            for (int j = 0; j < K; ++j)
 #pragma unroll
-                    for (int k = 0; k < KS; ++k)
-                        umma_bf16(tbase + 64 * j, kmajor_desc(z0 + 128u * j, k),
-                                  mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k), idesc_w, k != 0);
-            };
-            ItemPos ipos(i0, a.n_tiles);
-            for (uint32_t it = 0; it < nit && !abort_flag; ++it, ipos.next()) {
-                const int zs = it % NZ;
-                if (it == 0 || ipos.tile == 0) {      // a chunk starts: its Bp slice
-                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
-                    ++cc;
+                for (int k = 0; k < KS; ++k) {
+                    const uint64_t da = kmajor_desc(z0 + 128u * j, k);
+                    const uint64_t db = mnmajor_desc(bp0 + j * S::bp_tap, 8192, 16 * k);
+                    if (leader) umma_bf16(tbase + 64 * j, da, db, idesc_w, k != 0);
                 }
-                if (it > 0 && !mbar_wait(&wempty, (it - 1) & 1, &abort_flag, a.err)) break;   // Wd read
-                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) break;
-                tc_fence_after();
-                const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
-                // ksteps = ceil(r / 16): 3 or 4 when r > 32, else 1 or 2
-                if constexpr (R64) {
-                    if (a.ksteps == 4) filter_mmas(std::integral_constant<int, 4>{}, z0);
-                    else filter_mmas(std::integral_constant<int, 3>{}, z0);
-                } else {
-                    if (a.ksteps == 2) filter_mmas(std::integral_constant<int, 2>{}, z0);
-                    else filter_mmas(std::integral_constant<int, 1>{}, z0);
-                }
+        };
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, a.err));
+        };
+        ItemPos ipos(i0, a.n_tiles);
+        for (uint32_t it = 0; it < nit; ++it, ipos.next()) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;      // the lanes leave together
+            const int zs = it % NZ;
+            if (it == 0 || ipos.tile == 0) {      // a chunk starts: its Bp slice
+                if (!wait_all(&bfull, cc & 1)) break;
+                ++cc;
+            }
+            if (it > 0 && !wait_all(&wempty, (it - 1) & 1)) break;   // Wd read
+            if (!wait_all(&zfull[zs], (it / NZ) & 1)) break;
+            tc_fence_after();
+            const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
+            // ksteps = ceil(r / 16): 3 or 4 when r > 32, else 1 or 2
+            if constexpr (R64) {
+                if (a.ksteps == 4) filter_mmas(std::integral_constant<int, 4>{}, z0);
+                else filter_mmas(std::integral_constant<int, 3>{}, z0);
+            } else {
+                if (a.ksteps == 2) filter_mmas(std::integral_constant<int, 2>{}, z0);
+                else filter_mmas(std::integral_constant<int, 1>{}, z0);
+            }
+            if (leader) {
                 umma_commit(&wfull);
                 umma_commit(&zempty[zs]);
                 if (it + 1 < nit && ipos.last_of_chunk()) umma_commit(&bempty);   // B is reloaded next
             }
+            __syncwarp();
         }
     } else if (warp == kMmaD) {
-        // ---- dz and dB MMAs of every item
-        if (lane == 0) {
-            const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
-            const uint32_t idesc_db = kDbt ? idesc_bf16(128, 64 * K, true, true) : idesc_bf16(128, a.ndz, true, true);
-            const uint32_t bp0 = smem_u32(sm + S::bp);
-            const uint32_t dw0 = smem_u32(sm + S::dw);
-            const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
-            uint32_t cc = 0;          // B loads consumed
-            uint32_t m = 0;           // chunks whose dB accumulation has started
-            ItemPos ipos(i0, a.n_tiles);
-            for (uint32_t it = 0; it < nit && !abort_flag; ++it, ipos.next()) {
-                const bool first = it == 0 || ipos.tile == 0;
-                const int zs = it % NZ, b = it & 1;
-                if (first) {
-                    if (!mbar_wait(&bfull, cc & 1, &abort_flag, a.err)) break;
-                    ++cc;
+        // ---- dz and dB MMAs of every item (the whole warp runs the loop; the elected lane issues)
+        const bool leader = elect_one();
+        const uint32_t idesc_dz = idesc_bf16(128, a.ndz, false, false);
+        const uint32_t idesc_db = kDbt ? idesc_bf16(128, 64 * K, true, true) : idesc_bf16(128, a.ndz, true, true);
+        const uint32_t bp0 = smem_u32(sm + S::bp);
+        const uint32_t dw0 = smem_u32(sm + S::dw);
+        const uint32_t nit = i1 > i0 ? (uint32_t)(i1 - i0) : 0u;
+        uint32_t cc = 0;          // B loads consumed
+        uint32_t m = 0;           // chunks whose dB accumulation has started
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, a.err));
+        };
+        ItemPos ipos(i0, a.n_tiles);
+        for (uint32_t it = 0; it < nit; ++it, ipos.next()) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;      // the lanes leave together
+            const bool first = it == 0 || ipos.tile == 0;
+            const int zs = it % NZ, b = it & 1;
+            if (first) {
+                if (!wait_all(&bfull, cc & 1)) break;
+                ++cc;
+            }
+            if (!wait_all(&zfull[zs], (it / NZ) & 1)) break;
+            if (!wait_all(&dzempty[b], ((it >> 1) & 1) ^ 1)) break;
+            if (first && m > 0 && !wait_all(&dbfree, (m - 1) & 1)) break;
+            const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
+            bool blk_ok = true;
+#pragma unroll
+            for (int bb = 0; bb < NBLK; ++bb) {
+                if (!wait_all(&dwready[bb], it & 1)) {
+                    blk_ok = false;
+                    break;
                 }
-                if (!mbar_wait(&zfull[zs], (it / NZ) & 1, &abort_flag, a.err)) break;
-                if (!mbar_wait(&dzempty[b], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
-                if (first && m > 0 && !mbar_wait(&dbfree, (m - 1) & 1, &abort_flag, a.err)) break;
-                const uint32_t z0 = smem_u32(sm + S::z0 + zs * kRowTile);
-                bool blk_ok = true;
+                tc_fence_after();
+                // dz += dW_j . Bp_j^T for the block's taps (both K-major, K = 64 channels)
 #pragma unroll
-                for (int bb = 0; bb < NBLK; ++bb) {
-                    if (!mbar_wait(&dwready[bb], it & 1, &abort_flag, a.err)) {
-                        blk_ok = false;
-                        break;
+                for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t da = kmajor_desc(dw0 + j * kAtom128, k);
+                        const uint64_t db = kmajor_desc(bp0 + j * S::bp_tap, k);
+                        if (leader) umma_bf16(tbase + kColDz + 64 * b, da, db, idesc_dz, (j | k) != 0);
                     }
-                    tc_fence_after();
-                    // dz += dW_j . Bp_j^T for the block's taps (both K-major, K = 64 channels)
+                if constexpr (!kDbt) {
+                    // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
 #pragma unroll
-                    for (int j = 2 * bb; j < 2 * bb + 2 && j < K; ++j)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            umma_bf16(tbase + kColDz + 64 * b, kmajor_desc(dw0 + j * kAtom128, k),
-                                      kmajor_desc(bp0 + j * S::bp_tap, k), idesc_dz, (j | k) != 0);
-                    if constexpr (!kDbt) {
-                        // dB^T[blk] += dW^T . z  (both MN-major, K = 128 tokens)
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            umma_bf16(tbase + kColDb + 64 * bb,
-                                      mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks),
-                                      mnmajor_desc(z0, kRowTile, 16 * ks), idesc_db, !(first && ks == 0));
-                        umma_commit(&dwfree[bb]);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t da = mnmajor_desc(dw0 + 2 * bb * kAtom128, kAtom128, 16 * ks);
+                        const uint64_t db = mnmajor_desc(z0, kRowTile, 16 * ks);
+                        if (leader) umma_bf16(tbase + kColDb + 64 * bb, da, db, idesc_db, !(first && ks == 0));
                     }
+                    if (leader) umma_commit(&dwfree[bb]);
                 }
-                if (!blk_ok) break;
-                if constexpr (kDbt) {
-                    // dB += z^T . dW over every tap at once (A: z tile, MN-major, its second 64-row
-                    // M atom is the next tile and only feeds unused rows; B: the K dW atoms, MN-major)
+                __syncwarp();
+            }
+            if (!blk_ok) break;
+            if constexpr (kDbt) {
+                // dB += z^T . dW over every tap at once (A: z tile, MN-major, its second 64-row
+                // M atom is the next tile and only feeds unused rows; B: the K dW atoms, MN-major)
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tbase + kColDb, mnmajor_desc(z0, kRowTile, 16 * ks),
-                                  mnmajor_desc(dw0, kAtom128, 16 * ks), idesc_db, !(first && ks == 0));
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t da = mnmajor_desc(z0, kRowTile, 16 * ks);
+                    const uint64_t db = mnmajor_desc(dw0, kAtom128, 16 * ks);
+                    if (leader) umma_bf16(tbase + kColDb, da, db, idesc_db, !(first && ks == 0));
+                }
+                if (leader)
 #pragma unroll
                     for (int bb = 0; bb < NBLK; ++bb) umma_commit(&dwfree[bb]);
-                }
-                if (first) ++m;
+            }
+            if (first) ++m;
+            if (leader) {
                 umma_commit(&dzfull[b]);
                 umma_commit(&zempty[zs]);
                 if (it + 1 < nit && ipos.last_of_chunk()) umma_commit(&bempty);   // B is reloaded next
             }
+            __syncwarp();
         }
     } else if (warp < kGb0) {
         // ---- GA: du (A1, staged for a TMA store) and dw (A2) of each item
@@ -824,36 +846,45 @@ __global__ void __launch_bounds__(kThreads, 1) gen_bwd_kernel(const __grid_const
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc_dh = idesc_bf16(128, G::DB, false, false);
-            const uint32_t idesc_dp = idesc_bf16(128, a.ndz, true, true);
-            const uint32_t p0 = smem_u32(pblk);
-            bool ok = mbar_wait(&pfull, 0, &abort_flag, a.err);
-            uint32_t it = 0;
-            for (int64_t tile = t0; ok && tile < t1 && !abort_flag; ++tile, ++it) {
-                const int s = it % NS;
-                if (!mbar_wait(&full[s], (it / NS) & 1, &abort_flag, a.err)) break;
+        // the whole warp runs the loop (warp-uniform descriptor arithmetic); the elected lane issues
+        const bool leader = elect_one();
+        const uint32_t idesc_dh = idesc_bf16(128, G::DB, false, false);
+        const uint32_t idesc_dp = idesc_bf16(128, a.ndz, true, true);
+        const uint32_t p0 = smem_u32(pblk);
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, a.err));
+        };
+        bool ok = wait_all(&pfull, 0);
+        uint32_t it = 0;
+        for (int64_t tile = t0; ok && tile < t1; ++tile, ++it) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;      // the lanes leave together
+            const int s = it % NS;
+            if (!wait_all(&full[s], (it / NS) & 1)) break;
+            tc_fence_after();
+            const uint32_t x0 = smem_u32(sm + s * G::stage), h0 = x0 + XA * kAtom128;
+            if (want_dh) {
+                if (!wait_all(&hempty, (it & 1) ^ 1)) break;
                 tc_fence_after();
-                const uint32_t x0 = smem_u32(sm + s * G::stage), h0 = x0 + XA * kAtom128;
-                if (want_dh) {
-                    if (!mbar_wait(&hempty, (it & 1) ^ 1, &abort_flag, a.err)) break;
-                    tc_fence_after();
-                    // dh = X . P^T: ksteps (R / 16 rounded up, at most 8) 16-wide steps over R, unrolled
+                // dh = X . P^T: ksteps (R / 16 rounded up, at most 8) 16-wide steps over R, unrolled
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        if (k < a.ksteps)
-                            umma_bf16(tbase, kmajor_desc(x0 + (k >> 2) * kAtom128, k & 3),
-                                      kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3), idesc_dh, k != 0);
-                    umma_commit(&hfull);
-                }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16(tbase + G::col_dp, mnmajor_desc(h0, kAtom128, 16 * ks), mnmajor_desc(x0, kAtom128, 16 * ks),
-                              idesc_dp, !(tile == t0 && ks == 0));
-                umma_commit(&empty[s]);
+                for (int k = 0; k < 8; ++k)
+                    if (k < a.ksteps) {
+                        const uint64_t da = kmajor_desc(x0 + (k >> 2) * kAtom128, k & 3);
+                        const uint64_t db = kmajor_desc(p0 + (k >> 2) * G::DB * 128, k & 3);
+                        if (leader) umma_bf16(tbase, da, db, idesc_dh, k != 0);
+                    }
+                if (leader) umma_commit(&hfull);
             }
-            umma_commit(&dpfull);     // every dP MMA of this CTA has completed
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t da = mnmajor_desc(h0, kAtom128, 16 * ks), db = mnmajor_desc(x0, kAtom128, 16 * ks);
+                if (leader) umma_bf16(tbase + G::col_dp, da, db, idesc_dp, !(tile == t0 && ks == 0));
+            }
+            if (leader) umma_commit(&empty[s]);
+            __syncwarp();
         }
+        if (leader) umma_commit(&dpfull);     // every dP MMA of this CTA has completed
+        __syncwarp();
     } else {
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;      // dh columns 64 half ..; dP columns 8 half + 16 i
