@@ -11,7 +11,8 @@
 //                      the [N, C, K] filter lives only in TMEM and registers.
 //
 // Every kernel here is warp-specialised: warp 0 issues TMA loads, warp 1 issues
-// tcgen05.mma (one elected thread) and owns the tensor memory, the remaining warps
+// tcgen05.mma (one thread; in gen_kernel the whole warp runs the issue loop and an elected lane
+// issues) and owns the tensor memory, the remaining warps
 // are the epilogue (thread = token row = TMEM lane).  Shared-memory stages and TMEM
 // accumulators are handed over with mbarriers; every wait is bounded.
 #include <algorithm>

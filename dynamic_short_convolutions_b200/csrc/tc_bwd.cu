@@ -21,16 +21,16 @@
 //       MMA1  Wd_j[t, c] = sum_k z[t+j, k] Bp[k, j C + c]   (the filter of token t+j:
 //             the z tile is loaded with 8 rows of look-ahead and the A operand starts
 //             j rows into it), so du needs no exchange between threads; issued by its own
-//             thread;
+//             warp (the whole warp runs the loop, one elected lane issues);
 //       epi A du (-> staged; a warp of its own issues the TMA store) and dw (-> bf16 tile in
 //             shared memory, 64 channels per tap; all taps at once for K <= 3, blocks of two
 //             taps for K = 4); 16 warps, each paced by mbarriers;
 //       MMA2  dz  = dW Bp_chunk^T      (M = 128 tokens, N = r, K = 64 K)
 //       MMA3  K <= 3: dB += z^T dW     (M = 128 (r rows used), N = 64 K, K = 128 tokens)
 //             K = 4:  dBt += dW^T z    (M = 128 (j, c) rows per block, N = r, K = 128 tokens)
-//             MMA2 and MMA3 are issued by a second thread on another scheduler;
-//       epi B dz -> staged fp32 tile, bulk tensor add into a [N, r] buffer (reduction over
-//             chunks; fp32 atomics when the tile does not fit);
+//             MMA2 and MMA3 are issued by a second warp on another scheduler (likewise);
+//       epi B dz -> staged fp32 tile (128 or 64 rows at a time), bulk tensor add into a [N, r]
+//             buffer (reduction over chunks; fp32 atomics when no tile fits);
 //       epi C at the end of the run: dBt -> per-run partial (reduced in order later).
 //   bwd_finish_kernel  sums the dB partials of each chunk in run order -> dB [r, C K] fp32, and
 //                      converts the fp32 dz to the bf16 operand of the generator backward.
