@@ -255,28 +255,38 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
     pdl_wait();
 
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
-            int64_t prev = -1;
-            uint32_t cc = 0, it = 0;
-            ItemPos ipos(i0, a.n_tiles);
-            for (int64_t item = i0; item < i1 && !abort_flag; ++item, ++it, ipos.next()) {
-                const int64_t chunk = ipos.chunk, tile = ipos.tile;
-                if (chunk != prev) {
-                    if (!mbar_wait(&bempty, (cc & 1) ^ 1, &abort_flag, a.err)) break;
+        // TMA loads: the whole warp runs the loop (warp-uniform coordinates), the elected lane issues
+        const bool leader = elect_one();
+        const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, a.err));
+        };
+        int64_t prev = -1;
+        uint32_t cc = 0, it = 0;
+        ItemPos ipos(i0, a.n_tiles);
+        for (int64_t item = i0; item < i1; ++item, ++it, ipos.next()) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;      // the lanes leave together
+            const int64_t chunk = ipos.chunk, tile = ipos.tile;
+            if (chunk != prev) {
+                if (!wait_all(&bempty, (cc & 1) ^ 1)) break;
+                if (leader) {
                     mbar_arrive_expect_tx(&bfull, K * a.ndz * 128);
                     for (int j = 0; j < K; ++j)
-                        tma_load_2d_hint(sm + S::bp + j * S::bp_tap, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64), 0,
-                                         keep);
-                    ++cc;
-                    prev = chunk;
+                        tma_load_2d_hint(sm + S::bp + j * S::bp_tap, &tm_bp, &bfull, (int32_t)(j * a.C + chunk * 64),
+                                         0, keep);
                 }
-                const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
-                const int zs = it % NZ, gs = it & 1;
-                if (!mbar_wait(&zempty[zs], ((it / NZ) & 1) ^ 1, &abort_flag, a.err)) break;
+                ++cc;
+                prev = chunk;
+            }
+            const TileAt ta = tile_at<CF>(tile, (int32_t)(chunk * 64), a.tps, a.seqlen, a.C);
+            const int zs = it % NZ, gs = it & 1;
+            if (!wait_all(&zempty[zs], ((it / NZ) & 1) ^ 1)) break;
+            if (leader) {
                 mbar_arrive_expect_tx(&zfull[zs], kRowTile);
                 tma_load_2d_hint(sm + S::z0 + zs * kRowTile, &tm_z, &zfull[zs], 0, ta.m0, keep);
-                if (!mbar_wait(&guempty[gs], ((it >> 1) & 1) ^ 1, &abort_flag, a.err)) break;
+            }
+            if (!wait_all(&guempty[gs], ((it >> 1) & 1) ^ 1)) break;
+            if (leader) {
                 uint8_t* gu = sm + gs * S::gu;
                 mbar_arrive_expect_tx(&gufull[gs], S::gu);
                 // RoPE: the conv backward of a rotated chunk reads R^T g, written by the set-up kernel
@@ -284,6 +294,7 @@ __global__ void __launch_bounds__(BwdEpi<K>::threads, 1) lowrank_bwd_kernel(cons
                 if (CF) tma_load_2d_hint(gu + kRowTile, &tm_u, &gufull[gs], ta.x - 8, ta.y, stream);
                 else tma_load_2d_hint(gu + kRowTile, &tm_u, &gufull[gs], ta.x, ta.y - 8, stream);
             }
+            __syncwarp();
         }
     } else if (warp == 1) {
         // ---- filter MMAs of every item, issued by their own warp (the dz / dB MMAs have another,
