@@ -90,10 +90,10 @@ def layer_flops(w, layer):
 # (kernel, workload) and stored with the SHA-256 of the kernel's source files at capture time: a
 # figure is reported only while those files are unchanged (else traffic is null).
 NCU_TRAFFIC = {
-    ("tc_lowrank_bwd", "c4_all_linear_2b_block"): (550760976, "eb37e80a83b4c4a9"),
-    ("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): (196766933, "eb37e80a83b4c4a9"),
+    ("tc_lowrank_bwd", "c4_all_linear_2b_block"): (550760853, "d9ad7f0ee6101c83"),
+    ("tc_lowrank_bwd", "c2_qkv_150m_lowrank"): (192719232, "d9ad7f0ee6101c83"),
     ("tc_headwise_bwd", "c3_qkv_2b_headwise_gqa"): (302353258, "c06e68dc5e1a32cf"),
-    ("tc_lowrank_bwd", "c5_varlen_packed"): (2174687786, "eb37e80a83b4c4a9"),
+    ("tc_lowrank_bwd", "c5_varlen_packed"): (2170718763, "d9ad7f0ee6101c83"),
 }
 KERNEL_SOURCES = {
     "tc_lowrank_bwd": ("tc_bwd.cu", "tc_common.cuh", "common.cuh"),
