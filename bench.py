@@ -501,7 +501,7 @@ def run_ours(args, rank, world, local_rank):
         rope = W.ROPE_QKV.get(w.name) if args.rope and layer.name == "qkv" else None
         table = ops.rope_table(max(seqlen, 1), rope[1], device=dev) if rope else None
         plan = ops.DynConvPlan(kind, dt, batch, seqlen, layer.d_model, layer.channels, w.ksize, w.rank,
-                               w.head_dim, algo=args.algo, device=dev,
+                               w.head_dim, algo=args.algo, device=dev, deterministic=args.deterministic,
                                layout=L.CHANNEL_FIRST if cf else L.TOKEN_MAJOR,
                                rope_channels=rope[0] if rope else 0, rope_head_dim=rope[1] if rope else 0,
                                rope_table=table)
@@ -683,6 +683,7 @@ def run_ours(args, rank, world, local_rank):
                        "varlen": w.varlen, "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (256 MiB write, outside the step events)",
                        "algo": {0: "auto", 1: "simt", 2: "tc"}[args.algo], "layout": args.layout,
+                       "deterministic": bool(args.deterministic),
                        "rope": ({"channels": W.ROPE_QKV[w.name][0], "head_dim": W.ROPE_QKV[w.name][1],
                                  "layers": ["qkv"]} if args.rope and w.name in W.ROPE_QKV else None),
                        "kernel_family": {"fwd": fam[0], "bwd": fam[1], "note": fam[2]}},
@@ -701,6 +702,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--algo", type=int, default=0, help="0 auto, 1 CUDA-core kernels, 2 tensor-core kernels")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="bitwise-repeatable backward (no float atomics; the low-rank one runs the CUDA-core kernels)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="train", choices=["train", "decode"],

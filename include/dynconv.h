@@ -107,7 +107,10 @@ typedef struct {
     int64_t u_row_stride;   /* token-major: elements between tokens of u (0 = channels);
                                channel-first: elements between channels of u (0 = seqlen) */
     int64_t h_row_stride;   /* elements between tokens of h; 0 = d_model */
-    int32_t deterministic;  /* 1: every reduction in a fixed order, no float atomics */
+    int32_t deterministic;  /* 1: every reduction in a fixed order, no float atomics.  The
+                               low-rank backward then runs the CUDA-core kernels, two to three
+                               orders of magnitude slower than the tensor-core backward; the
+                               head-wise backward stays on the tensor-core path at full speed */
     int32_t algo;           /* dynconv_algo */
     int32_t layout;         /* dynconv_layout of u, y, g, du */
     /* Rotary position embedding fused after the conv (0 channels = none): see "RoPE" below. */
