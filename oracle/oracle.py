@@ -24,17 +24,27 @@ HEADWISE = "headwise"
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dynconv_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libdynconv_oracle.so")
+# A prebuilt oracle library to load instead of this directory's build: the mutation
+# tests point it at copies of the C file with one planted mistake each.
+_LIB_OVERRIDE = os.environ.get("DYNCONV_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
 
+def compile_library(src: str, out: str) -> None:
+    """gcc with the oracle's flags: fp64 as written (no fast-math, no FMA contraction), OpenMP."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp",
+                           "-ffp-contract=off", "-fno-fast-math", src, "-o", tmp, "-lm"])
+    os.replace(tmp, out)
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (fp64, no fast-math, no FMA contraction, OpenMP)."""
+    """Compile the oracle (when its library is missing or older than the C file)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp",
-                               "-ffp-contract=off", "-fno-fast-math", _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB_PATH)
+        compile_library(_SRC, _LIB_PATH)
     return _LIB_PATH
 
 

@@ -5,7 +5,8 @@ The pages name RoPE without a variant; the oracle follows the rotation of Su et 
 channel pairs (2i, 2i+1) of each head turn by position * base^(-2i/head_dim).
 These checks pin it to values and properties that do not restate that formula:
   - literal cosines and sines at position 1 (pair 0 turns by exactly 1 rad; for a
-    head of 8 channels the four pairs turn by 1, 0.1, 0.01 and 0.001 rad at base 1e4);
+    head of 8 channels the four pairs turn by 1, 0.1, 0.01 and 0.001 rad at base 1e4;
+    with two heads rotated, each head's pairs turn by the same angles);
   - the relative-position property that defines RoPE: <R_m q, R_n k> depends only
     on m - n;
   - orthogonality (the inverse undoes it, pair norms are kept, the adjoint identity);
@@ -44,6 +45,16 @@ def test_head_of_four_two_pairs():
     # pair 1 of a 4-channel head turns by 1e4^(-1/2) = 0.01 rad: (0, 1) -> (-sin 0.01, cos 0.01)
     np.testing.assert_allclose(y[1], [0.5403023058681398, 0.8414709848078965, -0.009999833334166664,
                                       0.9999500004166653], rtol=0, atol=1e-15)
+
+
+def test_every_head_turns_by_the_same_angles():
+    # two 4-channel heads, both rotated: the pair index restarts in each head, so at
+    # position 1 the second head's pairs turn by 1 and 0.01 rad like the first head's
+    p = _prob(2, 8)
+    x = np.array([[1.0, 0.0, 0.0, 1.0, 1.0, 0.0, 0.0, 1.0]] * 2)
+    y = O.rope(p, x, 8, 4)
+    head = [0.5403023058681398, 0.8414709848078965, -0.009999833334166664, 0.9999500004166653]
+    np.testing.assert_allclose(y[1], head + head, rtol=0, atol=1e-15)
 
 
 def test_relative_position_property():
