@@ -1,4 +1,5 @@
 // api.cu -- the C ABI: argument validation, workspace sizing, kernel-family dispatch.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -52,7 +53,10 @@ dynconv_status make_prob(const dynconv_desc* d, Prob* p) {
     p->dtype = d->dtype;
     p->batch = d->batch;
     p->seqlen = d->seqlen;
-    p->N = d->batch * d->seqlen;
+    if (__builtin_mul_overflow(d->batch, d->seqlen, &p->N)) {
+        set_error("batch * seqlen overflows 64 bits");
+        return DYNCONV_ERR_INVALID;
+    }
     p->d = d->d_model;
     p->C = d->channels;
     p->K = d->ksize;
@@ -86,6 +90,27 @@ dynconv_status make_prob(const dynconv_desc* d, Prob* p) {
     } else {
         if (d->head_dim < 1 || d->channels % d->head_dim) { set_error("head_dim must divide channels"); return DYNCONV_ERR_INVALID; }
         p->r = 0; p->hd = d->head_dim; p->H = d->channels / d->head_dim; p->R = p->H * p->K;
+    }
+    {
+        // Every operand's byte count must fit well inside 64 bits: a product that wrapped
+        // would turn a huge problem into a small or negative one (and the workspace sum
+        // of a few such counts must not wrap either).
+        const int64_t kMaxBytes = int64_t(1) << 56;
+        auto fits = [&](int64_t a, int64_t b, int64_t c) {
+            int64_t t;
+            return !__builtin_mul_overflow(a, b, &t) && !__builtin_mul_overflow(t, c, &t) && t <= kMaxBytes;
+        };
+        const int64_t es = d->dtype == DYNCONV_BF16 ? 2 : 4;
+        const int64_t rows = p->layout == DYNCONV_TOKEN_MAJOR ? p->N : (fits(p->batch, p->C, 1) ? p->batch * p->C : -1);
+        const bool ok = rows >= 0 && fits(rows, p->us, es)         // u, y, g, du
+                        && fits(p->N, p->hs, es)                    // h, dh
+                        && fits(p->N, p->R, 4)                      // per-token generator rows (fp32)
+                        && fits(p->d, p->R, 4)                      // A or W and their fp32 gradients
+                        && fits(p->C, p->K * std::max<int64_t>(p->r, 1), 4);   // B and dB
+        if (!ok) {
+            set_error("sizes overflow: every operand must stay below 2^56 bytes");
+            return DYNCONV_ERR_INVALID;
+        }
     }
     p->cu = nullptr;
     p->n_docs = 0;
@@ -339,6 +364,12 @@ dynconv_status dynconv_query_family(const dynconv_desc* desc, int32_t* fwd_famil
     if (s != DYNCONV_OK) return s;
     const char* rf = tc_unsupported_reason(p, false);
     const char* rb = tc_unsupported_reason(p, true);
+    if (desc->algo == DYNCONV_ALGO_TC && rb) {
+        // the entry points refuse a forced tensor-core run they cannot do (rf implies rb)
+        set_error("desc->algo asks for the tensor-core kernels, which %s refuses: %s",
+                  rf ? "the forward (and the backward)" : "the backward", rf ? rf : rb);
+        return DYNCONV_ERR_UNSUPPORTED;
+    }
     const bool simt = desc->algo == DYNCONV_ALGO_SIMT;
     if (fwd_family) *fwd_family = (!simt && !rf) ? DYNCONV_FAMILY_TENSOR_CORE : DYNCONV_FAMILY_CUDA_CORE;
     if (bwd_family) *bwd_family = (!simt && !rb) ? DYNCONV_FAMILY_TENSOR_CORE : DYNCONV_FAMILY_CUDA_CORE;

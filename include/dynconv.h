@@ -270,7 +270,9 @@ typedef enum { DYNCONV_FAMILY_TENSOR_CORE = 1, DYNCONV_FAMILY_CUDA_CORE = 2 } dy
  * deterministic low-rank mode; dynconv_last_error() then names the reason
  * (else it is "").  Host-only: no device work, no allocation.
  * Returns DYNCONV_ERR_INVALID / _UNSUPPORTED for a descriptor that the entry
- * points would reject. */
+ * points would reject: among them, with DYNCONV_ALGO_TC, one that the
+ * tensor-core kernels of either pass do not cover (dynconv_last_error() names
+ * the pass and the reason). */
 DYNCONV_API dynconv_status dynconv_query_family(const dynconv_desc *desc, int32_t *fwd_family,
                                                 int32_t *bwd_family);
 

@@ -109,3 +109,10 @@ def test_query_family_host_only():
     with pytest.raises(L.DynConvError) as e:
         L.dynconv_query_family(L.make_desc(L.LOWRANK, L.BF16, 1, 64, 64, 64, 5, 16))
     assert e.value.status == 2
+    # a forced tensor-core run the kernels cannot do is refused, as the entry points refuse it
+    with pytest.raises(L.DynConvError) as e:
+        L.dynconv_query_family(L.make_desc(L.LOWRANK, L.F32, 2, 128, 64, 64, 3, 4, algo=L.ALGO_TC))
+    assert e.value.status == 2 and "fp32" in str(e.value)
+    # sizes whose byte counts wrap 64 bits are invalid, not small
+    assert L.dynconv_workspace_bytes(L.make_desc(L.LOWRANK, L.BF16, 3, 1 << 62, 64, 64, 3, 16)) == 0
+    assert "overflow" in L.dynconv_last_error()
