@@ -172,6 +172,7 @@ dynconv_status forward_common(const dynconv_desc* desc, const int32_t* cu, int64
     if (varlen) {
         if (p.batch != 1) { set_error("varlen needs batch == 1"); return DYNCONV_ERR_INVALID; }
         if (n_docs < 1) { set_error("n_docs must be >= 1"); return DYNCONV_ERR_INVALID; }
+        if (p.N > INT32_MAX) { set_error("packed tokens must number below 2^31 (cu_seqlens is int32)"); return DYNCONV_ERR_INVALID; }
         if ((s = check_ptr(cu, "cu_seqlens", true)) != DYNCONV_OK) return s;
         p.cu = cu;
         p.n_docs = n_docs;
@@ -269,6 +270,7 @@ dynconv_status dynconv_bwd(const dynconv_desc* desc, const int32_t* cu_seqlens, 
     if (cu_seqlens) {
         if (p.batch != 1) { set_error("varlen needs batch == 1"); return DYNCONV_ERR_INVALID; }
         if (n_docs < 1) { set_error("n_docs must be >= 1"); return DYNCONV_ERR_INVALID; }
+        if (p.N > INT32_MAX) { set_error("packed tokens must number below 2^31 (cu_seqlens is int32)"); return DYNCONV_ERR_INVALID; }
         if ((s = check_ptr(cu_seqlens, "cu_seqlens", true)) != DYNCONV_OK) return s;
         p.cu = cu_seqlens;
         p.n_docs = n_docs;

@@ -165,7 +165,7 @@ DYNCONV_API dynconv_status dynconv_fwd(const dynconv_desc *desc, const void *u, 
                            void *stream);
 
 /* Forward over packed documents: desc->batch must be 1 and desc->seqlen the
- * total token count N.  cu_seqlens is a DEVICE int32 array [n_docs + 1] with
+ * total token count N (below 2^31).  cu_seqlens is a DEVICE int32 array [n_docs + 1] with
  * cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_docs] = N; the filter never
  * reaches across a document start.  A malformed cu_seqlens is caught by a
  * device pre-check that raises a flag read by dynconv_device_status(); the
