@@ -10,6 +10,10 @@ layer shapes, 2 sequences of 300 tokens, K = 3, r = 32):
     here on the CPU: a dropped tap, a missing document mask, a du tap reading the
     wrong token, a channel chunk missing from the cross-CTA dz reduction, and one
     token tile missing from the dB reduction.  The bar must reject each of these.
+The same for the head-wise generator on the inputs of the GPU case `c3_small`:
+the correct rounding (bf16 taps and dwh operand) passes; a head taking its
+neighbour's taps, a dwh reduction that lost half of a head's channels and a dW
+missing one token tile are rejected.
 The method's formulas are those of "Dynamic Short Convolutions Improve
 Transformers", gist.science technical summary, section "Dynamic Short
 Convolutions" (Mechanism, low-rank Parameterization, residual Placement, causal
@@ -124,3 +128,69 @@ def test_lost_dB_tile_is_rejected(case):
     t = slice(128, 256)
     part = np.einsum("nk,jnc->kcj", z[t], x["g"][None, t] * ush[:, t]).reshape(r, -1)
     assert not _ok("dB", _f32(case["ref"]["dBW"] - part), case["ref"]["dBW"])[0]
+
+
+# ---- head-wise: the inputs of the GPU case `c3_small` (2B head-wise GQA layer shapes,
+# 2 sequences of 200 tokens, K = 4, 24 heads of 128 channels)
+
+@pytest.fixture(scope="module")
+def hcase():
+    w = W.scaled(W.CONFIGS["c3_qkv_2b_headwise_gqa"], 2, 200, name="c3_small")
+    layer = w.layers[0]
+    x = W.make_inputs(w, layer)
+    ref = oracle_all(w, layer, x)
+    N, C, K, hd = w.tokens, layer.channels, w.ksize, w.head_dim
+    H = C // hd
+    cu = [int(v) for v in x["cu_seqlens"]]
+    st = np.zeros(N, dtype=np.int64)
+    for s in range(len(cu) - 1):
+        st[cu[s]:cu[s + 1]] = cu[s]
+    ush = np.zeros((K, N, C))
+    for j in range(K):
+        ok = (np.arange(N) - j) >= st
+        ush[j, ok] = x["u"][np.arange(N)[ok] - j]
+    return dict(x=x, ref=ref, ush=ush, N=N, C=C, K=K, hd=hd, H=H)
+
+
+def _expand(wh, H, K, hd):
+    # wh [N, H*K] (head q, tap j at q*K + j) -> [K, N, H*hd]
+    return np.repeat(wh.reshape(-1, H, K).transpose(2, 0, 1), hd, axis=2)
+
+
+def test_headwise_rounding_of_a_correct_kernel_passes(hcase):
+    x, ref, ush, H, K, hd = hcase["x"], hcase["ref"], hcase["ush"], hcase["H"], hcase["K"], hcase["hd"]
+    # the generator's taps stored in bf16, the conv in fp32, y stored in bf16
+    whb = _bf16(x["h"] @ x["W"])
+    y = _bf16(_f32(x["u"] + np.einsum("jnc,jnc->nc", _expand(whb, H, K, hd), ush)))
+    ok, msg = _ok("y", y, ref["y"])
+    assert ok, msg
+    # dwh summed in fp32 over each head's channels, rounded to bf16 as the generator backward's operand
+    dwh = _f32(np.einsum("jnqc->nqj", (x["g"][None] * ush).reshape(K, -1, H, hd)).reshape(-1, H * K))
+    dwhb = _bf16(dwh)
+    for name, a, b in (("dh", _bf16(dwhb @ x["W"].T), ref["dh"]), ("dW", _f32(x["h"].T @ dwhb), ref["dBW"])):
+        ok, msg = _ok(name, a, b)
+        assert ok, msg
+
+
+def test_headwise_filter_of_the_wrong_head_is_rejected(hcase):
+    x, ush, H, K, hd = hcase["x"], hcase["ush"], hcase["H"], hcase["K"], hcase["hd"]
+    wh = (x["h"] @ x["W"]).reshape(-1, H, K)
+    wrong = np.roll(wh, 1, axis=1).reshape(-1, H * K)           # head q takes head q-1's taps
+    y_bad = x["u"] + np.einsum("jnc,jnc->nc", _expand(wrong, H, K, hd), ush)
+    assert not _ok("y", _bf16(y_bad), hcase["ref"]["y"])[0]
+
+
+def test_headwise_dwh_missing_half_a_head_is_rejected(hcase):
+    # the shuffle reduction over a head's lanes losing its last level: half the channels summed
+    x, ush, H, K, hd = hcase["x"], hcase["ush"], hcase["H"], hcase["K"], hcase["hd"]
+    prod = (x["g"][None] * ush).reshape(K, -1, H, hd)
+    dwh_bad = np.einsum("jnqc->nqj", prod[..., : hd // 2]).reshape(-1, H * K)
+    assert not _ok("dh", _bf16(dwh_bad @ x["W"].T), hcase["ref"]["dh"])[0]
+    assert not _ok("dW", _f32(x["h"].T @ dwh_bad), hcase["ref"]["dBW"])[0]
+
+
+def test_headwise_lost_dW_tile_is_rejected(hcase):
+    x, ush, H, K, hd = hcase["x"], hcase["ush"], hcase["H"], hcase["K"], hcase["hd"]
+    dwh = np.einsum("jnqc->nqj", (x["g"][None] * ush).reshape(K, -1, H, hd)).reshape(-1, H * K)
+    t = slice(128, 256)
+    assert not _ok("dW", _f32(hcase["ref"]["dBW"] - x["h"][t].T @ dwh[t]), hcase["ref"]["dBW"])[0]
