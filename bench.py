@@ -694,7 +694,7 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def main():
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -713,7 +713,11 @@ def main():
                     help="fuse RoPE (base 10000, interleaved pairs) after the conv of the QKV layer (Q and K)")
     ap.add_argument("--layout", default="token_major", choices=["token_major", "channel_first"],
                     help="memory layout of u, y, g, du: [N, C] or [batch, C, seqlen]")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = build_parser().parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

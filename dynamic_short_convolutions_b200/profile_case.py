@@ -17,7 +17,7 @@ import argparse
 import os
 import sys
 
-def main(argv=None) -> int:
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--config", default="c4_all_linear_2b_block")
     ap.add_argument("--layer", type=int, default=0)
@@ -25,7 +25,11 @@ def main(argv=None) -> int:
     ap.add_argument("--repeats", type=int, default=2)
     ap.add_argument("--rope", action="store_true")
     ap.add_argument("--layout", default="token_major", choices=["token_major", "channel_first"])
-    args = ap.parse_args(argv)
+    return ap
+
+
+def main(argv=None) -> int:
+    args = build_parser().parse_args(argv)
     import torch
 
     from . import _lib as L, ops, workloads as W
