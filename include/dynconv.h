@@ -175,7 +175,15 @@ DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const in
                                   const void *u, const void *h, const void *A, const void *B_or_W,
                                   void *y, void *z_save, void *ws, size_t ws_bytes, void *stream);
 
-/* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch).
+/* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch):
+ * the gradients of the Mechanism formula and of the generator map (the same
+ * passages as the forward; "Efficient Training Implementation" asks for fused
+ * kernels in both passes).  With dw[n,c,j] = g[n,c] u[n-j,c] for n-j >= s(n):
+ *   du[m,c] = g[m,c] + sum_j w[m+j,c,j] g[m+j,c]   (taps with m >= s(m+j))
+ *   low-rank:  dz = dw . B^T  [N, r],  dA = h^T dz,  dB = z^T dw,  dh = dz A^T
+ *   head-wise: dwh[n,q,j] = sum_{c in head q} dw[n,c,j],  dW = h^T dwh,  dh = dwh W^T
+ * Every sum over tokens or channels is in fp32.  desc->deterministic = 1 fixes
+ * every reduction order (the low-rank backward then runs the CUDA-core kernels).
  * Channel-first: g, u and du are [batch, C, seqlen] ([C, N] for packed documents).
  *   g        [N, C] upstream gradient dL/dy, dense
  *   z_saved  nullable: the generator output saved by the forward ([N, r] or
@@ -184,6 +192,8 @@ DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const in
  *   dh       nullable [N, d] output dL/dh, dense
  *   dA       [d, r] fp32 output (low-rank; ignored for head-wise)
  *   dB_or_dW [r, C*K] or [d, H*K] fp32 output */
+/* Errors: as dynconv_fwd; with DYNCONV_ALGO_TC, DYNCONV_ERR_UNSUPPORTED where the
+ * tensor-core backward does not cover the descriptor. */
 DYNCONV_API dynconv_status dynconv_bwd(const dynconv_desc *desc, const int32_t *cu_seqlens, int64_t n_docs,
                            const void *g, const void *u, const void *h, const void *A,
                            const void *B_or_W, const void *z_saved, void *du, void *dh, float *dA,
@@ -254,7 +264,7 @@ DYNCONV_API dynconv_status dynconv_decode_step(const dynconv_desc *desc, const v
 /* Synchronises `stream` and reports device-side check failures raised by the
  * calls that used this workspace since the last query (then clears them):
  * DYNCONV_ERR_DEVICE_CHECK for a malformed cu_seqlens or a pipeline wait that
- * ran out of its iteration limit, else DYNCONV_OK. */
+ * ran out of its time limit (2 s), else DYNCONV_OK. */
 DYNCONV_API dynconv_status dynconv_device_status(void *ws, size_t ws_bytes, void *stream);
 
 /* Kernel families (see dynconv_query_family). */
