@@ -177,8 +177,9 @@ DYNCONV_API dynconv_status dynconv_fwd_varlen(const dynconv_desc *desc, const in
 
 /* Backward of dynconv_fwd / dynconv_fwd_varlen (cu_seqlens NULL = dense batch):
  * the gradients of the Mechanism formula and of the generator map (the same
- * passages as the forward; "Efficient Training Implementation" asks for fused
- * kernels in both passes).  With dw[n,c,j] = g[n,c] u[n-j,c] for n-j >= s(n):
+ * passages as the forward).  The training kernels of "Efficient Training
+ * Implementation" keep the filter tensor on chip; the backward keeps the same
+ * rule for w and dw.  With dw[n,c,j] = g[n,c] u[n-j,c] for n-j >= s(n):
  *   du[m,c] = g[m,c] + sum_j w[m+j,c,j] g[m+j,c]   (taps with m >= s(m+j))
  *   low-rank:  dz = dw . B^T  [N, r],  dA = h^T dz,  dB = z^T dw,  dh = dz A^T
  *   head-wise: dwh[n,q,j] = sum_{c in head q} dw[n,c,j],  dW = h^T dwh,  dh = dwh W^T
