@@ -7,9 +7,10 @@ the unmutated copy, built the same way, must pass them all.
 What each mutant breaks is the formula it names: "Dynamic Short Convolutions
 Improve Transformers", gist.science technical summary, section "Dynamic Short
 Convolutions" (Mechanism formula y = u + sum_j w[t,c,j] u[t-j,c]; the low-rank
-and head-wise Parameterization; the residual Placement; per-document causality of
-packed sequences), its gradients, the decode step's rolling state, and the RoPE
-rotation (RoFormer, section 3.4.2) applied after the QKV conv.
+and head-wise Parameterization; the residual Placement), its gradients, this
+library's reading that a filter stays inside its packed document, the decode
+step's rolling state, and the RoPE rotation (RoFormer, section 3.4.2) applied
+after the QKV conv.
 """
 import concurrent.futures
 import os

@@ -16,8 +16,9 @@ neighbour's taps, a dwh reduction that lost half of a head's channels and a dW
 missing one token tile are rejected.
 The method's formulas are those of "Dynamic Short Convolutions Improve
 Transformers", gist.science technical summary, section "Dynamic Short
-Convolutions" (Mechanism, low-rank Parameterization, residual Placement, causal
-per-document filters).
+Convolutions" (Mechanism, low-rank and head-wise Parameterization, residual
+Placement); that a filter stays inside its packed document is this library's
+reading of the causal Mechanism for packed sequences.
 """
 import numpy as np
 import pytest
