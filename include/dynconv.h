@@ -54,8 +54,9 @@
  *     fp32.  The library allocates nothing.
  *   - Stream: `stream` is a cudaStream_t (NULL = legacy default stream).  All
  *     work is enqueued asynchronously on it; nothing synchronises.
- *   - Errors: arguments are validated before any launch; a failed launch
- *     returns DYNCONV_ERR_CUDA.  dynconv_last_error() gives a thread-local
+ *   - Errors: arguments are validated before any launch (a descriptor whose
+ *     operands would pass 2^56 bytes, or whose size products would wrap 64
+ *     bits, is DYNCONV_ERR_INVALID); a failed launch returns DYNCONV_ERR_CUDA.  dynconv_last_error() gives a thread-local
  *     message for the last failure.  Nothing traps on the device.
  */
 #ifndef DYNCONV_H

@@ -7,7 +7,8 @@ and layout from their enums; batch, seqlen >= 0; d_model, channels >= 1; ksize
 1..4; low-rank rank 1..128; head-wise head_dim dividing channels; row strides at
 least the row and, token-major, a multiple of 16 bytes; and every operand's byte
 count below 2^56 without a wrapped product.  An accepted descriptor gets a
-non-zero workspace size and a kernel family for both passes."""
+non-zero workspace size and a kernel family for both passes (or, when it forces
+the tensor-core kernels on a shape they do not cover, DYNCONV_ERR_UNSUPPORTED)."""
 import os
 
 import pytest
